@@ -1,0 +1,243 @@
+"""Python binding of the B200 4-bit FlashAttention library (libhifa4.so).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``csrc/`` behind the C ABI of ``include/hifa4.h``.  PyTorch provides device
+memory and the current stream.  There is no CPU fallback: if the in-tree
+library is missing, every call raises.
+
+Method: "HiFA4: Training-Free 4-bit FlashAttention on Ascend HIF4 NPUs for LLM
+Inference", Abstract paras 1-2 (Smooth-QK, 4-bit QK^T and PV GEMMs, online
+softmax, P-Reordering).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhifa4.so")
+
+NVFP4, MXFP4 = 0, 1
+PREORDER, INCONSISTENT = 0, 1
+BF16, FP16 = 0, 1
+P_PRESCALE_LOG2 = -8
+
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "timeout"}
+_lib = None
+
+ABI_FUNCTIONS = (
+    "hifa4_codes_bytes", "hifa4_scale_bytes", "hifa4_calibrate_smooth_qk", "hifa4_quantize_qkv",
+    "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
+    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_status_string", "hifa4_last_error",
+    "hifa4_device_error",
+)
+
+
+class HiFA4Error(RuntimeError):
+    pass
+
+
+def lib():
+    """Load the in-tree CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise HiFA4Error(f"CUDA library not built: {LIB_PATH} (run __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, i64, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        L.hifa4_codes_bytes.argtypes = [i64, i]; L.hifa4_codes_bytes.restype = sz
+        L.hifa4_scale_bytes.argtypes = [i64, i, i]; L.hifa4_scale_bytes.restype = sz
+        L.hifa4_calibrate_smooth_qk.argtypes = [vp, vp, i, i, i, i, i, i, i, f, i, vp, vp, vp]
+        L.hifa4_quantize_qkv.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, vp, i, vp, vp, vp, vp, vp, vp, vp]
+        L.hifa4_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, vp]
+        L.hifa4_decode_workspace_size.argtypes = [i, i, i, i]; L.hifa4_decode_workspace_size.restype = sz
+        L.hifa4_decode_default_splits.argtypes = [i, i, i, i]; L.hifa4_decode_default_splits.restype = i
+        L.hifa4_attn_decode.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
+                                        ctypes.POINTER(ctypes.c_int), vp, sz, vp, i, vp]
+        L.hifa4_fp4_mma_probe.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, vp]
+        L.hifa4_convert_probe.argtypes = [vp, i64, vp, vp, vp]
+        L.hifa4_status_string.argtypes = [i]; L.hifa4_status_string.restype = ctypes.c_char_p
+        L.hifa4_last_error.argtypes = []; L.hifa4_last_error.restype = ctypes.c_char_p
+        L.hifa4_device_error.argtypes = []; L.hifa4_device_error.restype = ctypes.c_uint
+        for name in ABI_FUNCTIONS:
+            getattr(L, name).restype = getattr(L, name).restype or ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        msg = lib().hifa4_last_error().decode(errors="replace")
+        raise HiFA4Error(f"{what}: {_STATUS.get(st, st)}: {msg}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float16:
+        return FP16
+    raise HiFA4Error(f"unsupported dtype {t.dtype}")
+
+
+def pad128(n: int) -> int:
+    return (n + 127) // 128 * 128
+
+
+def beta_of(fmt: int) -> int:
+    return 16 if fmt == NVFP4 else 32
+
+
+def scale_bytes(rows: int, k: int, fmt: int) -> int:
+    return int(lib().hifa4_scale_bytes(rows, k, fmt))
+
+
+def device_error() -> int:
+    """Synchronizes, returns and clears the device error word (0 = fine)."""
+    return int(lib().hifa4_device_error())
+
+
+# --------------------------------------------------------------- calibrate ---
+def calibrate_smooth_qk(q: torch.Tensor, k: torch.Tensor, n_cal: int, alpha: float = 0.5,
+                        enable: bool = True):
+    """q [B,Hq,T,d], k [B,Hkv,T,d] (cuda, bf16/fp16) -> (s, inv_s) [Hkv,d] float32."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    q = q.contiguous(); k = k.contiguous()
+    s = torch.empty((Hkv, d), device=q.device, dtype=torch.float32)
+    inv = torch.empty_like(s)
+    _check(lib().hifa4_calibrate_smooth_qk(_ptr(q), _ptr(k), _dt(q), B, Hq, Hkv, n_cal, T, d, float(alpha),
+                                           int(bool(enable)), _ptr(s), _ptr(inv), _stream()),
+           "calibrate_smooth_qk")
+    return s, inv
+
+
+# ---------------------------------------------------------------- quantize ---
+@dataclass
+class QuantizedQKV:
+    """4-bit Q-hat, K-hat, V-hat^T in the library layouts (include/hifa4.h)."""
+    q_codes: torch.Tensor
+    q_scales: torch.Tensor
+    k_codes: torch.Tensor
+    k_scales: torch.Tensor
+    vt_codes: torch.Tensor
+    vt_scales: torch.Tensor
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    fmt: int
+
+    @property
+    def Np(self) -> int:
+        return pad128(self.N)
+
+
+def alloc_qkv(B, Hq, Hkv, N, d, fmt, device="cuda") -> QuantizedQKV:
+    Np = pad128(N)
+    u8 = dict(device=device, dtype=torch.uint8)
+    sq = scale_bytes(N, d, fmt)
+    sv = scale_bytes(d, Np, fmt)
+    return QuantizedQKV(
+        torch.empty((B, Hq, Np, d // 2), **u8), torch.empty((B, Hq, sq), **u8),
+        torch.empty((B, Hkv, Np, d // 2), **u8), torch.empty((B, Hkv, sq), **u8),
+        torch.empty((B, Hkv, d, Np // 2), **u8), torch.empty((B, Hkv, sv), **u8),
+        B, Hq, Hkv, N, d, fmt)
+
+
+def quantize_qkv(q, k, v, s=None, inv_s=None, fmt: int = NVFP4, out: QuantizedQKV | None = None):
+    """Fused Smooth-QK scale + block quantization.  q [B,Hq,N,d], k/v [B,Hkv,N,d]."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    q = q.contiguous(); k = k.contiguous(); v = v.contiguous()
+    z = out if out is not None else alloc_qkv(B, Hq, Hkv, N, d, fmt, q.device)
+    _check(lib().hifa4_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hq, Hkv, N, d, _ptr(s), _ptr(inv_s),
+                                    fmt, _ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),
+                                    _ptr(z.vt_codes), _ptr(z.vt_scales), _stream()), "quantize_qkv")
+    return z
+
+
+# --------------------------------------------------------------- attention ---
+def attn_fwd(z: QuantizedQKV, softmax_scale: float | None = None, causal: bool = True, mode: int = PREORDER,
+             block_n: int = 128, out_dtype=torch.bfloat16, return_lse: bool = False, debug: bool = False,
+             out: torch.Tensor | None = None):
+    """4-bit attention forward.  Returns O [B,Hq,N,d] (and lse / debug sums)."""
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(z.d)
+    dev = z.q_codes.device
+    o = out if out is not None else torch.empty((z.B, z.Hq, z.N, z.d), device=dev, dtype=out_dtype)
+    lse = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if return_lse else None
+    lph = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if debug else None
+    lp = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if debug else None
+    _check(lib().hifa4_attn_fwd(_ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),
+                                _ptr(z.vt_codes), _ptr(z.vt_scales), z.B, z.Hq, z.Hkv, z.N, z.d, z.fmt,
+                                float(softmax_scale), int(bool(causal)), int(mode), int(block_n), _ptr(o),
+                                _dt(o), _ptr(lse), _ptr(lph), _ptr(lp), _stream()), "attn_fwd")
+    res = [o]
+    if return_lse:
+        res.append(lse)
+    if debug:
+        res += [lph, lp]
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+# ------------------------------------------------------------------ decode ---
+def decode_workspace_bytes(B, Hq, d, num_splits) -> int:
+    return int(lib().hifa4_decode_workspace_size(B, Hq, d, num_splits))
+
+
+def default_splits(B, Hkv, kv_len, block_n=128) -> int:
+    return int(lib().hifa4_decode_default_splits(B, Hkv, kv_len, block_n))
+
+
+def attn_decode(q: torch.Tensor, s: torch.Tensor | None, cache: QuantizedQKV, kv_len: int | None = None,
+                softmax_scale: float | None = None, mode: int = PREORDER, num_splits: int = 0,
+                workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, out_dtype=torch.bfloat16):
+    """Split-KV decode of q [B,Hq,d] over the 4-bit cache.  Returns (O, splits_used)."""
+    B, Hq, d = q.shape
+    kv = cache.N if kv_len is None else kv_len
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if num_splits == 0:
+        num_splits = default_splits(B, cache.Hkv, kv)
+    ws_bytes = decode_workspace_bytes(B, Hq, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    o = out if out is not None else torch.empty((B, Hq, d), device=q.device, dtype=out_dtype)
+    used = ctypes.c_int(0)
+    q = q.contiguous()
+    _check(lib().hifa4_attn_decode(_ptr(q), _dt(q), _ptr(s), _ptr(cache.k_codes), _ptr(cache.k_scales),
+                                   _ptr(cache.vt_codes), _ptr(cache.vt_scales), B, Hq, cache.Hkv, kv, d,
+                                   cache.fmt, float(softmax_scale), int(mode), 128, int(num_splits),
+                                   ctypes.byref(used), _ptr(workspace), workspace.numel(), _ptr(o), _dt(o),
+                                   _stream()), "attn_decode")
+    return o, used.value
+
+
+# ------------------------------------------------------------- measurement ---
+def fp4_mma_probe(a_codes, a_scales, b_codes, b_scales, n: int, k: int, fmt: int, repeats: int = 1,
+                  ctas: int = 1, out: torch.Tensor | None = None):
+    d = out if out is not None else torch.empty((128, n), device=a_codes.device, dtype=torch.float32)
+    _check(lib().hifa4_fp4_mma_probe(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), n, k, fmt,
+                                     repeats, ctas, _ptr(d), _stream()), "fp4_mma_probe")
+    return d
+
+
+def convert_probe(x: torch.Tensor):
+    x = x.contiguous().float()
+    e2 = torch.empty(x.shape, device=x.device, dtype=torch.uint8)
+    e4 = torch.empty(x.shape, device=x.device, dtype=torch.uint8)
+    _check(lib().hifa4_convert_probe(_ptr(x), x.numel(), _ptr(e2), _ptr(e4), _stream()), "convert_probe")
+    return e2, e4

@@ -1,0 +1,258 @@
+// api.cu -- the C ABI (include/hifa4.h): argument validation, status codes,
+// thread-local error strings, the device error word and TMA descriptor
+// creation.  Kernels live in quantize.cu, attn_fwd.cu, decode.cu, probe.cu.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace hifa4 {
+
+__device__ unsigned int g_device_error = 0;
+
+static thread_local char g_last_error[512] = "";
+
+void set_last_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+}
+
+hifa4_status launch_status(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error("%s: %s", what, cudaGetErrorString(e));
+    return HIFA4_ERR_CUDA;
+  }
+  return HIFA4_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows][inner_bytes] (row pitch inner_bytes), box
+// [box_rows][box_inner], swizzle matching the box row (32/64/128 bytes).
+bool make_tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_inner,
+                  uint32_t box_rows, int swizzle_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner_bytes, rows};
+  cuuint64_t strides[1] = {inner_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+hifa4_status quantize_qkv_launch(const void*, const void*, const void*, int, int, int, int, int, int, const float*,
+                                 const float*, int, uint8_t*, uint8_t*, uint8_t*, uint8_t*, uint8_t*, uint8_t*,
+                                 cudaStream_t);
+hifa4_status calibrate_launch(const void*, const void*, int, int, int, int, int, int, int, float, int, float*, float*,
+                              cudaStream_t);
+hifa4_status attn_fwd_launch(const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*,
+                             const uint8_t*, int, int, int, int, int, int, float, int, int, int, void*, int, float*,
+                             float*, float*, cudaStream_t);
+hifa4_status decode_launch(const void*, int, const float*, const uint8_t*, const uint8_t*, const uint8_t*,
+                           const uint8_t*, int, int, int, int, int, int, float, int, int, int, int*, void*, size_t,
+                           void*, int, cudaStream_t);
+int decode_default_splits(int B, int Hkv, int kv_len, int block_n);
+hifa4_status fp4_mma_probe_launch(const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*, int, int, int, int,
+                                  int, float*, cudaStream_t);
+hifa4_status convert_probe_launch(const float*, int64_t, uint8_t*, uint8_t*, cudaStream_t);
+
+}  // namespace hifa4
+
+using namespace hifa4;
+
+#define HIFA4_REQUIRE(cond, code, ...) \
+  do {                                 \
+    if (!(cond)) {                     \
+      set_last_error(__VA_ARGS__);     \
+      return code;                     \
+    }                                  \
+  } while (0)
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool valid_d(int d) { return d == 64 || d == 128 || d == 256; }
+static bool valid_fmt(int f) { return f == HIFA4_NVFP4 || f == HIFA4_MXFP4; }
+static bool valid_dt(int t) { return t == HIFA4_BF16 || t == HIFA4_FP16; }
+
+extern "C" {
+
+size_t hifa4_codes_bytes(int64_t rows, int k) {
+  if (rows < 0 || k <= 0) return 0;
+  return static_cast<size_t>(pad128(rows)) * static_cast<size_t>(k) / 2;
+}
+
+size_t hifa4_scale_bytes(int64_t rows, int k, hifa4_format fmt) {
+  if (rows < 0 || k <= 0 || !valid_fmt(fmt)) return 0;
+  const int64_t nb = k / beta_of(fmt);
+  const int64_t nkc = (nb + 3) / 4;
+  return static_cast<size_t>(pad128(rows) / 128 * nkc * 512);
+}
+
+hifa4_status hifa4_calibrate_smooth_qk(const void* q, const void* k, hifa4_dtype dt, int B, int Hq, int Hkv,
+                                       int n_cal, int ld_tok, int d, float alpha, int enable, float* s_out,
+                                       float* inv_s_out, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(q && k && s_out && inv_s_out, HIFA4_ERR_INVALID_ARG, "calibrate: null pointer");
+  HIFA4_REQUIRE(valid_dt(dt), HIFA4_ERR_INVALID_ARG, "calibrate: bad dtype %d", (int)dt);
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0, HIFA4_ERR_INVALID_ARG,
+                "calibrate: bad heads B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
+  HIFA4_REQUIRE(n_cal > 0 && n_cal <= ld_tok, HIFA4_ERR_INVALID_ARG, "calibrate: need 0 < n_cal <= ld_tok");
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "calibrate: d=%d not in {64,128,256}", d);
+  HIFA4_REQUIRE(alpha >= 0.0f && alpha <= 1.0f, HIFA4_ERR_INVALID_ARG, "calibrate: alpha outside [0,1]");
+  return calibrate_launch(q, k, dt, B, Hq, Hkv, n_cal, ld_tok, d, alpha, enable, s_out, inv_s_out,
+                          static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hifa4_dtype dt, int B, int Hq,
+                                int Hkv, int N, int d, const float* s, const float* inv_s, hifa4_format fmt,
+                                uint8_t* q_codes, uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales,
+                                uint8_t* vt_codes, uint8_t* vt_scales, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(q && k && v && q_codes && q_scales && k_codes && k_scales && vt_codes && vt_scales,
+                HIFA4_ERR_INVALID_ARG, "quantize_qkv: null pointer");
+  HIFA4_REQUIRE(valid_dt(dt) && valid_fmt(fmt), HIFA4_ERR_INVALID_ARG, "quantize_qkv: bad dtype/format");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0, HIFA4_ERR_INVALID_ARG,
+                "quantize_qkv: bad shape B=%d Hq=%d Hkv=%d N=%d", B, Hq, Hkv, N);
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "quantize_qkv: d=%d not in {64,128,256}", d);
+  HIFA4_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(q_codes) && aligned16(q_scales) &&
+                    aligned16(k_codes) && aligned16(k_scales) && aligned16(vt_codes) && aligned16(vt_scales) &&
+                    (!s || aligned16(s)) && (!inv_s || aligned16(inv_s)),
+                HIFA4_ERR_INVALID_ARG, "quantize_qkv: pointers must be 16-byte aligned");
+  return quantize_qkv_launch(q, k, v, dt, B, Hq, Hkv, N, d, s, inv_s, fmt, q_codes, q_scales, k_codes, k_scales,
+                             vt_codes, vt_scales, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_attn_fwd(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                            const uint8_t* k_scales, const uint8_t* vt_codes, const uint8_t* vt_scales, int B,
+                            int Hq, int Hkv, int N, int d, hifa4_format fmt, float softmax_scale, int causal,
+                            hifa4_norm_mode mode, int block_n, void* o, hifa4_dtype o_dt, float* lse,
+                            float* dbg_l_phat, float* dbg_l_p, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(q_codes && q_scales && k_codes && k_scales && vt_codes && vt_scales && o, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd: null pointer");
+  HIFA4_REQUIRE(valid_fmt(fmt) && valid_dt(o_dt), HIFA4_ERR_INVALID_ARG, "attn_fwd: bad format/dtype");
+  HIFA4_REQUIRE(mode == HIFA4_NORM_PREORDER || mode == HIFA4_NORM_INCONSISTENT, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd: bad normalizer mode");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd: bad shape B=%d Hq=%d Hkv=%d N=%d", B, Hq, Hkv, N);
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "attn_fwd: d=%d not in {64,128,256}", d);
+  HIFA4_REQUIRE(block_n == 0 || block_n == 64 || block_n == 128, HIFA4_ERR_UNSUPPORTED,
+                "attn_fwd: block_n=%d not in {0,64,128}", block_n);
+  HIFA4_REQUIRE(!(d == 256 && block_n == 64), HIFA4_ERR_UNSUPPORTED, "attn_fwd: d=256 needs block_n=128");
+  HIFA4_REQUIRE(softmax_scale > 0.0f, HIFA4_ERR_INVALID_ARG, "attn_fwd: softmax_scale must be > 0");
+  HIFA4_REQUIRE(aligned16(q_codes) && aligned16(q_scales) && aligned16(k_codes) && aligned16(k_scales) &&
+                    aligned16(vt_codes) && aligned16(vt_scales) && aligned16(o),
+                HIFA4_ERR_INVALID_ARG, "attn_fwd: pointers must be 16-byte aligned");
+  HIFA4_REQUIRE(static_cast<int64_t>(B) * Hq * pad128(N) < (int64_t(1) << 31), HIFA4_ERR_UNSUPPORTED,
+                "attn_fwd: problem too large");
+  return attn_fwd_launch(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
+                         softmax_scale, causal, mode, block_n, o, o_dt, lse, dbg_l_phat, dbg_l_p,
+                         static_cast<cudaStream_t>(stream));
+}
+
+size_t hifa4_decode_workspace_size(int B, int Hq, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || d <= 0 || num_splits <= 0) return 0;
+  return static_cast<size_t>(B) * Hq * num_splits * (d + 2) * sizeof(float);
+}
+
+int hifa4_decode_default_splits(int B, int Hkv, int kv_len, int block_n) {
+  return decode_default_splits(B, Hkv, kv_len, block_n);
+}
+
+hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const float* s, const uint8_t* k_codes,
+                               const uint8_t* k_scales, const uint8_t* vt_codes, const uint8_t* vt_scales, int B,
+                               int Hq, int Hkv, int kv_len, int d, hifa4_format fmt, float softmax_scale,
+                               hifa4_norm_mode mode, int block_n, int num_splits, int* num_splits_used,
+                               void* workspace, size_t ws_bytes, void* o, hifa4_dtype o_dt,
+                               hifa4_stream_t stream) {
+  HIFA4_REQUIRE(q && k_codes && k_scales && vt_codes && vt_scales && o && workspace, HIFA4_ERR_INVALID_ARG,
+                "attn_decode: null pointer");
+  HIFA4_REQUIRE(valid_fmt(fmt) && valid_dt(q_dt) && valid_dt(o_dt), HIFA4_ERR_INVALID_ARG,
+                "attn_decode: bad format/dtype");
+  HIFA4_REQUIRE(mode == HIFA4_NORM_PREORDER || mode == HIFA4_NORM_INCONSISTENT, HIFA4_ERR_INVALID_ARG,
+                "attn_decode: bad normalizer mode");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && kv_len > 0, HIFA4_ERR_INVALID_ARG,
+                "attn_decode: bad shape");
+  HIFA4_REQUIRE(d == 128, HIFA4_ERR_UNSUPPORTED, "attn_decode: d=%d (only 128)", d);
+  HIFA4_REQUIRE(Hq / Hkv <= 8, HIFA4_ERR_UNSUPPORTED, "attn_decode: GQA group > 8");
+  HIFA4_REQUIRE(block_n == 0 || block_n == 128, HIFA4_ERR_UNSUPPORTED, "attn_decode: block_n must be 128");
+  HIFA4_REQUIRE(num_splits >= 0, HIFA4_ERR_INVALID_ARG, "attn_decode: num_splits < 0");
+  HIFA4_REQUIRE(softmax_scale > 0.0f, HIFA4_ERR_INVALID_ARG, "attn_decode: softmax_scale must be > 0");
+  HIFA4_REQUIRE(aligned16(q) && aligned16(k_codes) && aligned16(k_scales) && aligned16(vt_codes) &&
+                    aligned16(vt_scales) && aligned16(o) && aligned16(workspace) && (!s || aligned16(s)),
+                HIFA4_ERR_INVALID_ARG, "attn_decode: pointers must be 16-byte aligned");
+  return decode_launch(q, q_dt, s, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, kv_len, d, fmt,
+                       softmax_scale, mode, 128, num_splits, num_splits_used, workspace, ws_bytes, o, o_dt,
+                       static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_fp4_mma_probe(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                                 const uint8_t* b_scales, int n, int k, hifa4_format fmt, int repeats, int ctas,
+                                 float* d_out, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(a_codes && a_scales && b_codes && b_scales && d_out, HIFA4_ERR_INVALID_ARG,
+                "fp4_mma_probe: null pointer");
+  HIFA4_REQUIRE(valid_fmt(fmt) && repeats >= 1 && ctas >= 1 && ctas <= 65535, HIFA4_ERR_INVALID_ARG,
+                "fp4_mma_probe: bad format/repeats/ctas");
+  HIFA4_REQUIRE(aligned16(a_codes) && aligned16(a_scales) && aligned16(b_codes) && aligned16(b_scales),
+                HIFA4_ERR_INVALID_ARG, "fp4_mma_probe: pointers must be 16-byte aligned");
+  return fp4_mma_probe_launch(a_codes, a_scales, b_codes, b_scales, n, k, fmt, repeats, ctas, d_out,
+                              static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_convert_probe(const float* x, int64_t count, uint8_t* e2m1_out, uint8_t* e4m3_out,
+                                 hifa4_stream_t stream) {
+  HIFA4_REQUIRE(x && e2m1_out && e4m3_out && count >= 0, HIFA4_ERR_INVALID_ARG, "convert_probe: bad args");
+  if (count == 0) return HIFA4_OK;
+  return convert_probe_launch(x, count, e2m1_out, e4m3_out, static_cast<cudaStream_t>(stream));
+}
+
+const char* hifa4_status_string(hifa4_status st) {
+  switch (st) {
+    case HIFA4_OK: return "ok";
+    case HIFA4_ERR_INVALID_ARG: return "invalid argument";
+    case HIFA4_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HIFA4_ERR_CUDA: return "CUDA error";
+    case HIFA4_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* hifa4_last_error(void) { return g_last_error; }
+
+unsigned int hifa4_device_error(void) {
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return 0xFFFFFFFFu;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+  const unsigned int zero = 0;
+  cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  return v;
+}
+
+}  // extern "C"

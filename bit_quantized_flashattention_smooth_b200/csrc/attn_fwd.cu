@@ -1,0 +1,557 @@
+// attn_fwd.cu -- 4-bit FlashAttention forward on sm_100a with Smooth-QK'd,
+// block-scaled FP4 operands and P-Reordering.
+//
+// Method: "HiFA4: Training-Free 4-bit FlashAttention on Ascend HIF4 NPUs for
+// LLM Inference", Abstract paras 1-2: QK^T and PV are 4-bit GEMMs, the online
+// softmax keeps a running max m and normalizer l, the attention weights are
+// quantized to P-hat per tile, and under P-Reordering l is accumulated from
+// the same P-hat that feeds the PV GEMM, fused into that GEMM.
+//
+// B200 design (one CTA = one 128-row query tile of one (batch, q head)):
+//   warp 4      TMA producer: Q-hat tile once, then K-hat / V-hat^T tiles and
+//               their tiled scale chunks into an NS-stage ring (mbarriers).
+//   warp 5      MMA issuer (one thread): copies scale chunks shared->TMEM with
+//               tcgen05.cp, issues block-scaled tcgen05.mma for S = Q K^T
+//               into a TMEM S buffer, and for O += P-hat V-hat plus
+//               L += P-hat * ones (the fused normalizer: a 16-row all-ones B
+//               tile, so column 0 of L is sum(P-hat) with the same P-hat
+//               codes and scales as O).  Completion is signalled with
+//               tcgen05.commit onto mbarriers.
+//   warps 0-3   softmax: thread r owns query row r (TMEM lane r).  Per key
+//               tile: tcgen05.ld the S row, online max, P = 2^(S*c - m),
+//               per-block P-hat quantization in registers (cvt to E4M3 /
+//               E2M1), codes stored swizzled into shared memory as the A
+//               operand of the PV MMA, scales into a TMEM-copy chunk; when m
+//               rises, rescale the row of O and L in TMEM (after the previous
+//               PV MMA retired).  Epilogue: O / l, lse, optional debug sums.
+// Key tiles are visited in ascending order (P-hat depends on the running
+// max).  Every wait is bounded (ptx.cuh).
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace hifa4 {
+
+struct AttnParams {
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  const uint8_t* v_sf;
+  int64_t sf_qk_head;   // bytes of one head's Q/K scale matrix
+  int64_t sf_v_head;    // bytes of one head's V^T scale matrix
+  int B, Hq, Hkv, N, Np, G;
+  int num_qtiles;
+  float c_log2;         // softmax_scale * log2(e)
+  int causal;
+  int out_fp16;
+  void* o;
+  float* lse;
+  float* dbg_l_phat;
+  float* dbg_l_p;
+};
+
+template <int D, int BN, int FMT>
+struct AttnCfg {
+  static constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
+  static constexpr int BM = 128;
+  static constexpr int NS = D == 256 ? 2 : 3;               // K/V pipeline stages
+  static constexpr int NSB = D == 256 ? 1 : 2;              // TMEM S buffers
+  static constexpr int QROW = D / 2;                        // bytes per Q/K row
+  static constexpr int PROW = BN / 2;                       // bytes per P-hat / V^T row
+  static constexpr int KSTEPS_S = D / 64;
+  static constexpr int KSTEPS_P = BN / 64;
+  static constexpr int NKC_Q = (D / BETA + 3) / 4;          // scale chunks per Q/K row group
+  static constexpr int NRG_V = (D + 127) / 128;             // 128-row groups of V^T
+  static constexpr int NCH_V = (BN / BETA + 3) / 4;         // V^T scale chunks per tile per row group
+  static constexpr int NKC_P = (BN / BETA + 3) / 4;         // P-hat scale chunks per tile
+  // shared memory layout (byte offsets; operand tiles 1024-aligned)
+  static constexpr int SZ_Q = BM * QROW;
+  static constexpr int SZ_K = BN * QROW;
+  static constexpr int SZ_V = D * PROW;
+  static constexpr int SZ_P = BM * PROW;
+  static constexpr int SZ_ONES = 16 * PROW;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + SZ_Q;
+  static constexpr int OFF_V = OFF_K + NS * SZ_K;
+  static constexpr int OFF_P = OFF_V + NS * SZ_V;
+  static constexpr int OFF_ONES = OFF_P + 2 * SZ_P;
+  static constexpr int OFF_QSF = (OFF_ONES + SZ_ONES + 1023) / 1024 * 1024;
+  static constexpr int OFF_KSF = OFF_QSF + NKC_Q * 512;
+  static constexpr int OFF_VSF = OFF_KSF + NS * NKC_Q * 512;
+  static constexpr int OFF_PSF = OFF_VSF + NS * NRG_V * NCH_V * 512;
+  static constexpr int OFF_ONESF = OFF_PSF + 2 * NKC_P * 512;
+  static constexpr int OFF_BAR = OFF_ONESF + 512;
+  // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
+  // s_full[NSB], s_empty[NSB], p_full[2], p_empty[2], o_ready
+  static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  // TMEM columns
+  static constexpr int TM_S = 0;
+  static constexpr int TM_O = NSB * BN;
+  static constexpr int TM_L = TM_O + D;
+  static constexpr int TM_SFA_Q = TM_L + 16;
+  static constexpr int TM_SFB_K = TM_SFA_Q + 4 * NKC_Q;
+  static constexpr int TM_SFA_P = TM_SFB_K + 4 * NKC_Q;
+  static constexpr int TM_SFB_V = TM_SFA_P + 4 * NKC_P;
+  static constexpr int TM_SFB_1 = TM_SFB_V + 4 * NCH_V * NRG_V;
+  static constexpr int TM_COLS_USED = TM_SFB_1 + 4;
+  static_assert(TM_COLS_USED <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+__device__ __forceinline__ uint32_t swz_chunk(uint32_t r, uint32_t c, uint32_t row_bytes) {
+  // physical 16-byte chunk of logical chunk c in row r under the swizzle that
+  // matches row_bytes (32/64/128); buffers are 1024-byte aligned.
+  return c ^ ((r * row_bytes >> 7) & (row_bytes / 16 - 1));
+}
+
+template <int D, int BN, int FMT, bool PREORDER>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = AttnCfg<D, BN, FMT>;
+  extern __shared__ __align__(1024) unsigned char smem_dyn[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  const uint32_t bar0 = smem_u32(bars);
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + C::NS, B_VFULL = 1 + 2 * C::NS, B_VEMPTY = 1 + 3 * C::NS,
+            B_SFULL = 1 + 4 * C::NS, B_SEMPTY = B_SFULL + C::NSB, B_PFULL = B_SEMPTY + C::NSB,
+            B_PEMPTY = B_PFULL + 2, B_ORDY = B_PEMPTY + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  // ---- work item: heavy (late) query tiles first for causal balance ----
+  const int bhq = blockIdx.x % (p.B * p.Hq);
+  const int qtile = p.num_qtiles - 1 - static_cast<int>(blockIdx.x / (p.B * p.Hq));
+  const int b = bhq / p.Hq, hq = bhq % p.Hq;
+  const int kvbh = b * p.Hkv + hq / p.G;
+  const int row0 = qtile * C::BM;
+  const int kv_end = p.causal ? min(p.N, row0 + C::BM) : p.N;
+  const int nkt = (kv_end + BN - 1) / BN;
+
+  // ---- setup ----
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(B_QFULL), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(BAR(B_KFULL + s), 1);
+      mbar_init(BAR(B_KEMPTY + s), 1);
+      mbar_init(BAR(B_VFULL + s), 1);
+      mbar_init(BAR(B_VEMPTY + s), 1);
+    }
+    for (int s = 0; s < C::NSB; ++s) {
+      mbar_init(BAR(B_SFULL + s), 1);
+      mbar_init(BAR(B_SEMPTY + s), 4);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(B_PFULL + s), 4);
+      mbar_init(BAR(B_PEMPTY + s), 1);
+    }
+    mbar_init(BAR(B_ORDY), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // constant operands of the fused normalizer: 16 rows of E2M1 1.0 (code 2)
+  // and their scale chunk (scale 1.0 for rows 0..15 in every block byte).
+  for (int i = threadIdx.x; i < C::SZ_ONES / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(smem + C::OFF_ONES)[i] = 0x22222222u;
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+    const uint32_t one = FMT == HIFA4_NVFP4 ? 0x38u : 0x7Fu;
+    // word i of the chunk sits at byte 4*i: line (i/4) = row%32, word (i%4) = row/32
+    const int row_of_word = (i >> 2) + 32 * (i & 3);
+    reinterpret_cast<uint32_t*>(smem + C::OFF_ONESF)[i] = row_of_word < 16 ? one * 0x01010101u : 0u;
+  }
+  fence_proxy_async_smem();
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // =============================== TMA producer ===============================
+    if (lane == 0) {
+      const uint8_t* qsf = p.q_sf + static_cast<int64_t>(bhq) * p.sf_qk_head + static_cast<int64_t>(qtile) * C::NKC_Q * 512;
+      mbar_arrive_expect_tx(BAR(B_QFULL), C::SZ_Q + C::NKC_Q * 512);
+      tma_load_2d(sbase + C::OFF_Q, &tm_q, 0, bhq * p.Np + row0, BAR(B_QFULL));
+      bulk_load(sbase + C::OFF_QSF, qsf, C::NKC_Q * 512, BAR(B_QFULL));
+      const int nkc_v_row = p.Np / (4 * C::BETA);  // V^T scale chunks per row group
+      for (int j = 0; j < nkt; ++j) {
+        const int st = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        if (!mbar_wait(BAR(B_KEMPTY + st), ph ^ 1, abort_flag, kErrTimeoutTma)) break;
+        mbar_arrive_expect_tx(BAR(B_KFULL + st), C::SZ_K + C::NKC_Q * 512);
+        tma_load_2d(sbase + C::OFF_K + st * C::SZ_K, &tm_k, 0, kvbh * p.Np + j * BN, BAR(B_KFULL + st));
+        bulk_load(sbase + C::OFF_KSF + st * C::NKC_Q * 512,
+                  p.k_sf + static_cast<int64_t>(kvbh) * p.sf_qk_head + static_cast<int64_t>((j * BN) >> 7) * C::NKC_Q * 512,
+                  C::NKC_Q * 512, BAR(B_KFULL + st));
+        if (!mbar_wait(BAR(B_VEMPTY + st), ph ^ 1, abort_flag, kErrTimeoutTma)) break;
+        mbar_arrive_expect_tx(BAR(B_VFULL + st), C::SZ_V + C::NRG_V * C::NCH_V * 512);
+        tma_load_2d(sbase + C::OFF_V + st * C::SZ_V, &tm_v, j * C::PROW, kvbh * D, BAR(B_VFULL + st));
+        const int chunk0 = (j * BN) / (4 * C::BETA);
+        for (int rg = 0; rg < C::NRG_V; ++rg)
+          bulk_load(sbase + C::OFF_VSF + (st * C::NRG_V + rg) * C::NCH_V * 512,
+                    p.v_sf + static_cast<int64_t>(kvbh) * p.sf_v_head + static_cast<int64_t>(rg * nkc_v_row + chunk0) * 512,
+                    C::NCH_V * 512, BAR(B_VFULL + st));
+      }
+    }
+  } else if (warp == 5) {
+    // ================================ MMA issuer ================================
+    if (lane == 0) {
+      constexpr bool MX = FMT == HIFA4_MXFP4;
+      auto mma = [&](uint32_t d_t, uint64_t a, uint64_t bdesc, uint32_t idesc, uint32_t sfa, uint32_t sfb, uint32_t acc) {
+        if constexpr (MX) mma_mxfp4(d_t, a, bdesc, idesc, sfa, sfb, acc);
+        else mma_nvfp4(d_t, a, bdesc, idesc, sfa, sfb, acc);
+      };
+      bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, kErrTimeoutMma);
+      if (ok) {
+        tc_fence_after();
+        for (int kc = 0; kc < C::NKC_Q; ++kc)
+          tc_cp_32x128b_warpx4(tmem + C::TM_SFA_Q + 4 * kc, make_sf_desc(sbase + C::OFF_QSF + kc * 512));
+        tc_cp_32x128b_warpx4(tmem + C::TM_SFB_1, make_sf_desc(sbase + C::OFF_ONESF));
+      }
+      // S_j = Q K_j^T into S buffer j % NSB
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        const int sb = j % C::NSB;
+        if (!mbar_wait(BAR(B_KFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
+        if (!mbar_wait(BAR(B_SEMPTY + sb), ((j / C::NSB) & 1) ^ 1, abort_flag, kErrTimeoutMma)) return false;
+        tc_fence_after();
+        for (int kc = 0; kc < C::NKC_Q; ++kc)
+          tc_cp_32x128b_warpx4(tmem + C::TM_SFB_K + 4 * kc,
+                               make_sf_desc(sbase + C::OFF_KSF + st * C::NKC_Q * 512 + kc * 512));
+        const uint32_t half_off = (BN == 64 && (j & 1)) ? 2u : 0u;  // rows 64..127 of the K row group
+#pragma unroll
+        for (int ks = 0; ks < C::KSTEPS_S; ++ks) {
+          const uint32_t chunk = MX ? ks / 2 : ks;
+          const uint32_t byte = MX ? 2 * (ks % 2) : 0;
+          const uint64_t a = make_kmajor_desc(sbase + C::OFF_Q + ks * 32, C::QROW);
+          const uint64_t bd = make_kmajor_desc(sbase + C::OFF_K + st * C::SZ_K + ks * 32, C::QROW);
+          const uint32_t idesc = idesc_fp4(128, BN, MX, byte, byte);
+          mma(tmem + C::TM_S + sb * BN, a, bd, idesc, (tmem + C::TM_SFA_Q + 4 * chunk) | (byte << 30),
+              (tmem + C::TM_SFB_K + 4 * chunk + half_off) | (byte << 30), ks > 0 ? 1u : 0u);
+        }
+        tc_commit(BAR(B_SFULL + sb));
+        tc_commit(BAR(B_KEMPTY + st));
+        return true;
+      };
+      // O += P-hat V-hat_j ; L += P-hat ones
+      auto issue_pv = [&](int j) -> bool {
+        const int st = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        const int pb = j & 1;
+        if (!mbar_wait(BAR(B_PFULL + pb), (j >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
+        if (!mbar_wait(BAR(B_VFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
+        tc_fence_after();
+        for (int pc = 0; pc < C::NKC_P; ++pc)
+          tc_cp_32x128b_warpx4(tmem + C::TM_SFA_P + 4 * pc,
+                               make_sf_desc(sbase + C::OFF_PSF + pb * C::NKC_P * 512 + pc * 512));
+        for (int lc = 0; lc < C::NCH_V; ++lc)
+          for (int rg = 0; rg < C::NRG_V; ++rg)
+            tc_cp_32x128b_warpx4(tmem + C::TM_SFB_V + 4 * (lc * C::NRG_V + rg),
+                                 make_sf_desc(sbase + C::OFF_VSF + ((st * C::NRG_V + rg) * C::NCH_V + lc) * 512));
+#pragma unroll
+        for (int ks = 0; ks < C::KSTEPS_P; ++ks) {
+          const int kk = j * BN + ks * 64;                        // first key of this K-step
+          const uint32_t pchunk = MX ? ks / 2 : ks;
+          const uint32_t pbyte = MX ? 2 * (ks % 2) : 0;
+          const uint32_t vchunk = kk / (4 * C::BETA) - (j * BN) / (4 * C::BETA);
+          const uint32_t vbyte = (kk / C::BETA) % 4;
+          const uint64_t a = make_kmajor_desc(sbase + C::OFF_P + pb * C::SZ_P + ks * 32, C::PROW);
+          const uint64_t bv = make_kmajor_desc(sbase + C::OFF_V + st * C::SZ_V + ks * 32, C::PROW);
+          const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+          const uint32_t sfa = (tmem + C::TM_SFA_P + 4 * pchunk) | (pbyte << 30);
+          mma(tmem + C::TM_O, a, bv, idesc_fp4(128, D, MX, pbyte, vbyte), sfa,
+              (tmem + C::TM_SFB_V + 4 * vchunk * C::NRG_V) | (vbyte << 30), acc);
+          const uint64_t b1 = make_kmajor_desc(sbase + C::OFF_ONES + ks * 32, C::PROW);
+          mma(tmem + C::TM_L, a, b1, idesc_fp4(128, 16, MX, pbyte, pbyte), sfa,
+              (tmem + C::TM_SFB_1) | (pbyte << 30), acc);
+        }
+        tc_commit(BAR(B_ORDY));
+        tc_commit(BAR(B_VEMPTY + st));
+        tc_commit(BAR(B_PEMPTY + pb));
+        return true;
+      };
+      if (ok && nkt > 0) ok = issue_s(0);
+      for (int j = 0; ok && j < nkt; ++j) {
+        if (j + 1 < nkt) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
+      }
+      if (!ok) drain_after_abort();
+    }
+  } else {
+    // ================================== softmax ==================================
+    const int r = threadIdx.x;  // 0..127 == TMEM lane
+    const int row = row0 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float c = p.c_log2;
+    float m = -INFINITY;
+    float l_p = 0.0f;
+    const bool want_lp = !PREORDER || p.dbg_l_p != nullptr;
+    constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
+    constexpr float kInvGP = FMT == HIFA4_NVFP4 ? 256.0f : 1.0f;
+    bool ok = true;
+    for (int j = 0; j < nkt && ok; ++j) {
+      const int sb = j % C::NSB;
+      const int pb = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + sb), (j / C::NSB) & 1, abort_flag, kErrTimeoutSoftmax))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[BN];
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32_wait(tmem + lane_base + C::TM_S + sb * BN + cc * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(v[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_SEMPTY + sb));
+      // mask (only tiles that reach past the diagonal or past N need it)
+      const int kbase = j * BN;
+      const bool need_mask = (kbase + BN > p.N) || (p.causal && kbase + BN - 1 > row0);
+      if (need_mask) {
+        const int lim = p.causal ? min(p.N, row + 1) : p.N;
+#pragma unroll
+        for (int k = 0; k < BN; ++k)
+          if (kbase + k >= lim) s[k] = -INFINITY;
+      }
+      float smax = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < BN; ++k) smax = fmaxf(smax, s[k]);
+      const float m_new = fmaxf(m, smax * c);
+      const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);
+      const float neg_m = -m_new;
+      // P = 2^(S*c - m_new); P-hat per block of BETA keys
+      uint32_t codes[BN / 8];
+      uint32_t scw[C::NKC_P];
+#pragma unroll
+      for (int i = 0; i < C::NKC_P; ++i) scw[i] = 0;
+      float psum = 0.0f;
+#pragma unroll
+      for (int blk = 0; blk < BN / C::BETA; ++blk) {
+        float bmax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < C::BETA; ++i) {
+          const int k = blk * C::BETA + i;
+          const float pv = ex2_approx(fmaf(s[k], c, neg_m));
+          s[k] = pv;
+          bmax = fmaxf(bmax, pv);
+        }
+        float mult;
+        uint32_t sc;
+        if constexpr (FMT == HIFA4_NVFP4) {
+          const float t = __fmul_rn(__fdiv_rn(bmax, 6.0f), kInvGP);
+          sc = cvt_e4m3(t);
+          const float sd = __fmul_rn(ue4m3_to_f32(sc), kGP);
+          mult = sc == 0 ? 0.0f : __fdiv_rn(1.0f, sd);
+        } else {
+          const uint32_t ef = (__float_as_uint(bmax) >> 23) & 0xFFu;
+          sc = ef >= 2u ? ef - 2u : 0u;
+          mult = __uint_as_float((254u - sc) << 23);
+        }
+#pragma unroll
+        for (int w = 0; w < C::BETA / 8; ++w) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int k = blk * C::BETA + w * 8 + 2 * q;
+            word |= cvt_e2m1x2(__fmul_rn(s[k + 1], mult), __fmul_rn(s[k], mult)) << (8 * q);
+          }
+          codes[blk * (C::BETA / 8) + w] = word;
+        }
+        scw[blk / 4] |= sc << (8 * (blk % 4));
+        if (want_lp) {
+#pragma unroll
+          for (int i = 0; i < C::BETA; ++i) psum += s[blk * C::BETA + i];
+        }
+      }
+      if (want_lp) l_p = fmaf(alpha, l_p, psum);
+      // the P-hat buffer pb was last read by PV_{j-2}
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(BAR(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, abort_flag,
+                                                        kErrTimeoutSoftmax))) {
+        ok = false;
+        break;
+      }
+      {
+        unsigned char* prow = smem + C::OFF_P + pb * C::SZ_P + r * C::PROW;
+#pragma unroll
+        for (int ch = 0; ch < C::PROW / 16; ++ch) {
+          const uint32_t phys = swz_chunk(r, ch, C::PROW);
+          *reinterpret_cast<uint4*>(prow + phys * 16) =
+              make_uint4(codes[4 * ch], codes[4 * ch + 1], codes[4 * ch + 2], codes[4 * ch + 3]);
+        }
+        unsigned char* psf = smem + C::OFF_PSF + pb * C::NKC_P * 512;
+#pragma unroll
+        for (int pc = 0; pc < C::NKC_P; ++pc)
+          *reinterpret_cast<uint32_t*>(psf + pc * 512 + (r & 31) * 16 + (r >> 5) * 4) = scw[pc];
+      }
+      // rescale the O / L row when the max rose (PV_{j-1} must have retired)
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_ORDY), (j - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t v[16];
+          tmem_ld16_wait(tmem + lane_base + C::TM_O + cc * 16, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+          tmem_st16(tmem + lane_base + C::TM_O + cc * 16, v);
+        }
+        uint32_t lv;
+        tmem_ld1_wait(tmem + lane_base + C::TM_L, lv);
+        tmem_st1(tmem + lane_base + C::TM_L, __float_as_uint(__uint_as_float(lv) * alpha));
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_PFULL + pb));
+      m = m_new;
+    }
+    // ---------------------------------- epilogue ----------------------------------
+    const bool ready = __all_sync(0xffffffffu, ok && nkt > 0 &&
+                                                  mbar_wait(BAR(B_ORDY), (nkt - 1) & 1, abort_flag, kErrTimeoutSoftmax));
+    if (ready) {
+      tc_fence_after();
+      uint32_t lv;
+      tmem_ld1_wait(tmem + lane_base + C::TM_L, lv);
+      const float l_acc = __uint_as_float(lv);           // sum of P-hat in MMA units (P-hat / g_P)
+      const float l_phat = l_acc * kGP;
+      const float l_used = PREORDER ? l_phat : l_p;
+      const float inv_l = 1.0f / l_used;
+      const float o_mul = kGP * inv_l;                    // O_acc is in units of 1/g_P
+      const bool store = row < p.N;
+      const int64_t orow = (static_cast<int64_t>(bhq) * p.N + row) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 16; ++cc) {
+        uint32_t v[16];
+        tmem_ld16_wait(tmem + lane_base + C::TM_O + cc * 16, v);
+        if (store) {
+          uint32_t packed[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float a = __uint_as_float(v[2 * i]) * o_mul, bb = __uint_as_float(v[2 * i + 1]) * o_mul;
+            if (p.out_fp16) {
+              __half2 h = __floats2half2_rn(a, bb);
+              packed[i] = *reinterpret_cast<uint32_t*>(&h);
+            } else {
+              __nv_bfloat162 h = __floats2bfloat162_rn(a, bb);
+              packed[i] = *reinterpret_cast<uint32_t*>(&h);
+            }
+          }
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + orow + cc * 16);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        }
+      }
+      if (store) {
+        const int64_t ri = static_cast<int64_t>(bhq) * p.N + row;
+        if (p.lse) p.lse[ri] = m + log2f(l_used);
+        if (p.dbg_l_phat) p.dbg_l_phat[ri] = l_phat;
+        if (p.dbg_l_p) p.dbg_l_p[ri] = l_p;
+      }
+    }
+  }
+
+  // ---- teardown: every role is done; release TMEM ----
+  if (*abort_flag) drain_after_abort();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host ---
+bool make_tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_inner,
+                  uint32_t box_rows, int swizzle_bytes);
+
+template <int D, int BN, int FMT, bool PRE>
+static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const uint8_t* vc, const AttnParams& p,
+                                  cudaStream_t st) {
+  using C = AttnCfg<D, BN, FMT>;
+  CUtensorMap tq, tk, tv;
+  const uint64_t Np = static_cast<uint64_t>(p.Np);
+  if (!make_tmap_2d(&tq, qc, D / 2, static_cast<uint64_t>(p.B) * p.Hq * Np, D / 2, 128, D / 2) ||
+      !make_tmap_2d(&tk, kc, D / 2, static_cast<uint64_t>(p.B) * p.Hkv * Np, D / 2, BN, D / 2) ||
+      !make_tmap_2d(&tv, vc, Np / 2, static_cast<uint64_t>(p.B) * p.Hkv * D, BN / 2, D, BN / 2)) {
+    set_last_error("cuTensorMapEncodeTiled failed");
+    return HIFA4_ERR_CUDA;
+  }
+  auto kern = attn_fwd_fp4_kernel<D, BN, FMT, PRE>;
+  // The kernel owns all 512 TMEM columns: request enough shared memory that
+  // only one CTA is resident per SM (a second would stall in tcgen05.alloc).
+  const int smem = C::SMEM_BYTES > 116 * 1024 ? C::SMEM_BYTES : 116 * 1024;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * p.num_qtiles;
+  kern<<<grid, 192, smem, st>>>(tq, tk, tv, p);
+  return launch_status("attn_fwd");
+}
+
+template <int D, int BN>
+static hifa4_status launch_attn_fm(int fmt, int mode, const uint8_t* qc, const uint8_t* kc, const uint8_t* vc,
+                                   const AttnParams& p, cudaStream_t st) {
+  if (fmt == HIFA4_NVFP4)
+    return mode == HIFA4_NORM_PREORDER ? launch_attn_t<D, BN, HIFA4_NVFP4, true>(qc, kc, vc, p, st)
+                                       : launch_attn_t<D, BN, HIFA4_NVFP4, false>(qc, kc, vc, p, st);
+  return mode == HIFA4_NORM_PREORDER ? launch_attn_t<D, BN, HIFA4_MXFP4, true>(qc, kc, vc, p, st)
+                                     : launch_attn_t<D, BN, HIFA4_MXFP4, false>(qc, kc, vc, p, st);
+}
+
+hifa4_status attn_fwd_launch(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
+                             const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int N, int d, int fmt,
+                             float softmax_scale, int causal, int mode, int block_n, void* o, int o_dt, float* lse,
+                             float* dbg_l_phat, float* dbg_l_p, cudaStream_t st) {
+  AttnParams p;
+  p.q_sf = qs;
+  p.k_sf = ks;
+  p.v_sf = vs;
+  p.sf_qk_head = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
+  p.Np = static_cast<int>(pad128(N));
+  p.sf_v_head = static_cast<int64_t>(hifa4_scale_bytes(d, p.Np, static_cast<hifa4_format>(fmt)));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.G = Hq / Hkv;
+  p.num_qtiles = p.Np / 128;
+  p.c_log2 = softmax_scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.out_fp16 = o_dt == HIFA4_FP16;
+  p.o = o;
+  p.lse = lse;
+  p.dbg_l_phat = dbg_l_phat;
+  p.dbg_l_p = dbg_l_p;
+  if (block_n == 0) block_n = 128;
+  if (d == 64 && block_n == 64) return launch_attn_fm<64, 64>(fmt, mode, qc, kc, vc, p, st);
+  if (d == 64 && block_n == 128) return launch_attn_fm<64, 128>(fmt, mode, qc, kc, vc, p, st);
+  if (d == 128 && block_n == 64) return launch_attn_fm<128, 64>(fmt, mode, qc, kc, vc, p, st);
+  if (d == 128 && block_n == 128) return launch_attn_fm<128, 128>(fmt, mode, qc, kc, vc, p, st);
+  if (d == 256 && block_n == 128) return launch_attn_fm<256, 128>(fmt, mode, qc, kc, vc, p, st);
+  set_last_error("attn_fwd: unsupported (d=%d, block_n=%d)", d, block_n);
+  return HIFA4_ERR_UNSUPPORTED;
+}
+
+}  // namespace hifa4

@@ -1,0 +1,208 @@
+/*
+ * hifa4.h -- C ABI of the B200 (sm_100a) 4-bit FlashAttention forward with
+ * Smooth-QK and P-Reordering.
+ *
+ * Method: "HiFA4: Training-Free 4-bit FlashAttention on Ascend HIF4 NPUs for
+ * LLM Inference" (arXiv 2607.04302), Abstract paragraphs 1-2: both QK^T and PV
+ * run as 4-bit GEMMs with an online softmax state (running max m, normalizer
+ * l); Smooth-QK rescales post-RoPE Q by s and K by 1/s with calibration-static
+ * per-channel scales; P-Reordering accumulates l from the same quantized
+ * weights P-hat that feed the PV GEMM, fused into that GEMM.  The paper's HIF4
+ * format is replaced by Blackwell's block-scaled E2M1: NVFP4 (one UE4M3 scale
+ * per 16 elements) or MXFP4 (one UE8M0 scale per 32 elements, OCP MX v1.0).
+ *
+ * Conventions for every entry point:
+ *  - All pointers named as device pointers must point to device memory of the
+ *    current CUDA device; the caller owns and allocates all memory.  The
+ *    library never allocates, frees or synchronizes.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Outputs are valid once the stream reaches the call.
+ *  - Argument validation is synchronous and returns HIFA4_ERR_INVALID_ARG or
+ *    HIFA4_ERR_UNSUPPORTED without launching anything; a failed launch
+ *    returns HIFA4_ERR_CUDA.  hifa4_last_error() gives a thread-local detail
+ *    string for the last failing call on the calling thread.
+ *  - Kernels bound every internal wait.  A wait that runs out (a protocol
+ *    error, never expected) ends the kernel early and sets a device error
+ *    word; hifa4_device_error() returns and clears it (it synchronizes the
+ *    device).  No call traps or asserts on the device.
+ *  - Element layouts (N padded to Np = ceil(N/128)*128; pad rows/tokens hold
+ *    zero codes and zero scales):
+ *      Q-hat codes   [B][Hq][Np][d/2]   bytes, element 2i in the low nibble
+ *      K-hat codes   [B][Hkv][Np][d/2]
+ *      V-hat^T codes [B][Hkv][d][Np/2]  channel-major (tokens contiguous)
+ *    Scale layouts are "tiled" per head: for a matrix of R rows (padded to
+ *    128) and nb blocks per row (padded to a multiple of 4), 512-byte chunks
+ *    ordered (row/128, block/4); inside a chunk, the scale of (row r, block b)
+ *    is at byte (r%32)*16 + ((r%128)/32)*4 + (b%4).  hifa4_scale_bytes()
+ *    gives the size of one head's scale matrix; the per-head matrices of a
+ *    tensor are stored back to back in [B][H] order.
+ *  - All pointers must be 16-byte aligned.
+ */
+#ifndef HIFA4_H_
+#define HIFA4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HIFA4_OK = 0,
+  HIFA4_ERR_INVALID_ARG = 1,
+  HIFA4_ERR_UNSUPPORTED = 2,
+  HIFA4_ERR_CUDA = 3,
+  HIFA4_ERR_TIMEOUT = 4
+} hifa4_status;
+
+typedef enum { HIFA4_NVFP4 = 0, HIFA4_MXFP4 = 1 } hifa4_format;
+
+/* P-Reordering (normalizer from P-hat, fused into the PV MMA) or the
+ * inconsistent higher-precision normalizer (from unquantized P). */
+typedef enum { HIFA4_NORM_PREORDER = 0, HIFA4_NORM_INCONSISTENT = 1 } hifa4_norm_mode;
+
+typedef enum { HIFA4_BF16 = 0, HIFA4_FP16 = 1 } hifa4_dtype;
+
+/* P-hat of NVFP4 uses a two-level scale: UE4M3 block scale times the global
+ * prescale 2^HIFA4_NVFP4_P_PRESCALE_LOG2 (a reading: the paper does not define
+ * the HIF4 P-hat scale).  MXFP4 P-hat uses the plain OCP rule. */
+#define HIFA4_NVFP4_P_PRESCALE_LOG2 (-8)
+
+typedef void* hifa4_stream_t; /* a cudaStream_t */
+
+#if defined(__GNUC__)
+#define HIFA4_API __attribute__((visibility("default")))
+#else
+#define HIFA4_API
+#endif
+
+/* ---------------------------------------------------------------- sizes --- */
+
+/* Bytes of one head's codes for `rows` rows of `k` elements (rows padded to
+ * 128): pad128(rows) * k / 2. */
+HIFA4_API size_t hifa4_codes_bytes(int64_t rows, int k);
+
+/* Bytes of one head's tiled scale matrix for `rows` rows of `k` elements
+ * (rows padded to 128, blocks per row padded to a multiple of 4). */
+HIFA4_API size_t hifa4_scale_bytes(int64_t rows, int k, hifa4_format fmt);
+
+/* ------------------------------------------------------- calibration --- */
+
+/* Smooth-QK calibration (paper Abstract para 2: "computed once from a small
+ * offline calibration set"; the formula is a reading).  For kv head h and
+ * channel c: aK = max|K[b,h,t,c]|, aQ = max|Q[b,hq,t,c]| over batches b,
+ * tokens t < n_cal and the G = Hq/Hkv query heads hq of group h;
+ *   s = clamp(aK^alpha / aQ^(1-alpha), 2^-16, 2^16) in fp64 -> fp32,
+ *   inv_s = fl32(1/s); s = inv_s = 1 where enable == 0 or an amax is 0.
+ * q: device [B][Hq][ld_tok][d], k: device [B][Hkv][ld_tok][d] of `dt`;
+ * s_out, inv_s_out: device float [Hkv][d].  Requires 0 < n_cal <= ld_tok,
+ * Hq % Hkv == 0, d in {64, 128, 256}.  Issues two small kernels. */
+HIFA4_API hifa4_status hifa4_calibrate_smooth_qk(const void* q, const void* k, hifa4_dtype dt, int B, int Hq,
+                                       int Hkv, int n_cal, int ld_tok, int d, float alpha,
+                                       int enable, float* s_out, float* inv_s_out,
+                                       hifa4_stream_t stream);
+
+/* -------------------------------------------------- scale + quantize --- */
+
+/* Fused Smooth-QK scale and block quantization (paper Abstract para 2: "only
+ * a fusible element-wise scaling").  q' = fl32(q*s[h(hq),c]) and
+ * k' = fl32(k*inv_s[h,c]) are quantized in blocks along d; V (unscaled) is
+ * quantized in blocks along tokens and written transposed.  Block rule:
+ * NVFP4 amax/6 -> UE4M3 (RNE, saturating) and codes E2M1(x * fl32(1/scale));
+ * MXFP4 E = floor(log2 amax) - 2 and codes E2M1(x * 2^-E).
+ * Inputs (device): q [B][Hq][N][d], k, v [B][Hkv][N][d] of `dt`; s, inv_s
+ * device float [Hkv][d] or NULL (= 1).  Outputs (device): the code and tiled
+ * scale layouts described at the top of this file (q_scales: B*Hq heads of
+ * hifa4_scale_bytes(N, d), k_scales: B*Hkv of hifa4_scale_bytes(N, d),
+ * vt_scales: B*Hkv of hifa4_scale_bytes(d, Np)).  Requires N >= 1,
+ * d in {64, 128, 256}, Hq % Hkv == 0. */
+HIFA4_API hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hifa4_dtype dt, int B,
+                                int Hq, int Hkv, int N, int d, const float* s, const float* inv_s,
+                                hifa4_format fmt, uint8_t* q_codes, uint8_t* q_scales,
+                                uint8_t* k_codes, uint8_t* k_scales, uint8_t* vt_codes,
+                                uint8_t* vt_scales, hifa4_stream_t stream);
+
+/* ------------------------------------------------ attention forward --- */
+
+/* 4-bit FlashAttention forward (paper Abstract paras 1-2).  For each (b, hq)
+ * and 128-row query tile, key tiles of block_n keys are visited in ascending
+ * order: S = Q-hat K-hat^T (block-scaled FP4 MMA, fp32 accumulate), online
+ * softmax in fp32 with P = 2^(S*c - m) (c = softmax_scale*log2 e), P-hat =
+ * per-block quantization of P (NVFP4 with the 2^-8 prescale, or MXFP4),
+ * O += P-hat V-hat (FP4 MMA).  mode PREORDER accumulates l from P-hat inside
+ * the PV MMA (a ones column); mode INCONSISTENT accumulates l from P in fp32.
+ * Output O = acc / l in o_dt, [B][Hq][N][d]; lse (optional, [B][Hq][N]
+ * float) = m + log2(l) in base 2.  dbg_l_phat / dbg_l_p (optional, [B][Hq][N]
+ * float) receive the final normalizers from P-hat and from P (their ratio
+ * minus one is the per-row normalizer error epsilon of Theorem 1).
+ * Inputs are the layouts written by hifa4_quantize_qkv with the same fmt.
+ * causal: top-left aligned (key <= query).  block_n: 0 (default 128), 64 or
+ * 128.  Requires d in {64, 128, 256}, Hq % Hkv == 0, N >= 1. */
+HIFA4_API hifa4_status hifa4_attn_fwd(const uint8_t* q_codes, const uint8_t* q_scales,
+                            const uint8_t* k_codes, const uint8_t* k_scales,
+                            const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
+                            int Hkv, int N, int d, hifa4_format fmt, float softmax_scale,
+                            int causal, hifa4_norm_mode mode, int block_n, void* o,
+                            hifa4_dtype o_dt, float* lse, float* dbg_l_phat, float* dbg_l_p,
+                            hifa4_stream_t stream);
+
+/* ----------------------------------------------------- split-KV decode --- */
+
+/* Workspace bytes for hifa4_attn_decode with `num_splits` splits (per split
+ * and query row: d accumulators plus m and l, fp32). */
+HIFA4_API size_t hifa4_decode_workspace_size(int B, int Hq, int d, int num_splits);
+
+/* Split count chosen by hifa4_attn_decode when num_splits == 0. */
+HIFA4_API int hifa4_decode_default_splits(int B, int Hkv, int kv_len, int block_n);
+
+/* One decode step over a 4-bit KV cache (the cache layouts of
+ * hifa4_quantize_qkv with N = kv_len).  q: device [B][Hq][d] of q_dt,
+ * unscaled; s: device float [Hkv][d] Smooth-QK scales or NULL.  Inside the
+ * kernel each query row is scaled (fl32(q*s)) and quantized by the Q rule.
+ * Keys split into chunks of L = ceil(kv_len/num_splits) rounded up to
+ * block_n; each split runs the prefill recurrence without a mask and writes
+ * (acc, m, l) to `workspace`; a combine kernel merges them:
+ * O = sum 2^(m_s-M) acc_s / sum 2^(m_s-M) l_s.  o: device [B][Hq][d] of o_dt.
+ * num_splits 0 = hifa4_decode_default_splits; *num_splits_used (optional,
+ * host) receives the count of non-empty splits.  Requires d == 128,
+ * Hq/Hkv <= 8, block_n == 0 or 128. */
+HIFA4_API hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const float* s,
+                               const uint8_t* k_codes, const uint8_t* k_scales,
+                               const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
+                               int Hkv, int kv_len, int d, hifa4_format fmt, float softmax_scale,
+                               hifa4_norm_mode mode, int block_n, int num_splits,
+                               int* num_splits_used, void* workspace, size_t ws_bytes, void* o,
+                               hifa4_dtype o_dt, hifa4_stream_t stream);
+
+/* -------------------------------------------------------- measurement --- */
+
+/* One 128 x n block-scaled FP4 product D = A B^T (K-major A [128][k], B [n][k]
+ * in the code/tiled-scale layouts above; d_out device float [128][n]),
+ * repeated `repeats` times into the same accumulator (D = repeats * A B^T)
+ * on each of `ctas` CTAs (CTA 0 writes d_out).  With repeats >> 1 and ctas a
+ * multiple of the SM count this measures the dense FP4 tensor peak.
+ * Requires n in {64, 128, 256}, k a multiple of 128 up to 512. */
+HIFA4_API hifa4_status hifa4_fp4_mma_probe(const uint8_t* a_codes, const uint8_t* a_scales,
+                                 const uint8_t* b_codes, const uint8_t* b_scales, int n, int k,
+                                 hifa4_format fmt, int repeats, int ctas, float* d_out,
+                                 hifa4_stream_t stream);
+
+/* E2M1 / UE4M3 hardware conversion of `count` fp32 values (device): e2m1_out
+ * [count] codes (1 per byte) and e4m3_out [count] saturating E4M3 codes.  Used
+ * to check the written rounding rules against the conversion instructions. */
+HIFA4_API hifa4_status hifa4_convert_probe(const float* x, int64_t count, uint8_t* e2m1_out,
+                                 uint8_t* e4m3_out, hifa4_stream_t stream);
+
+/* ----------------------------------------------------------- errors --- */
+
+HIFA4_API const char* hifa4_status_string(hifa4_status st);
+HIFA4_API const char* hifa4_last_error(void);
+/* Synchronizes the device, returns the device error word and clears it
+ * (0 = no kernel gave up a wait). */
+HIFA4_API unsigned int hifa4_device_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HIFA4_H_ */

@@ -77,6 +77,7 @@ def lib():
         L.or_ue4m3_decode.argtypes = [ctypes.c_uint8]; L.or_ue4m3_decode.restype = d
         L.or_ue8m0_decode.argtypes = [ctypes.c_uint8]; L.or_ue8m0_decode.restype = d
         L.or_mx_exponent.argtypes = [f]; L.or_mx_exponent.restype = i
+        L.or_encode_array.argtypes = [f32p, i64, u8p, u8p]
         L.or_quant_block_nvfp4.argtypes = [f32p, i, f, u8p]; L.or_quant_block_nvfp4.restype = ctypes.c_uint8
         L.or_quant_block_mxfp4.argtypes = [f32p, i, u8p]; L.or_quant_block_mxfp4.restype = ctypes.c_uint8
         L.or_quantize_rows.argtypes = [f32p, i64, i, i, f, u8p, u8p]
@@ -134,6 +135,15 @@ def ue4m3_decode(codes) -> np.ndarray:
 def ue8m0_decode(codes) -> np.ndarray:
     f = lib().or_ue8m0_decode
     return np.array([f(int(c)) for c in np.asarray(codes).ravel()], dtype=np.float64)
+
+
+def encode_array(x):
+    """(E2M1(x), UE4M3(|x|)) element-wise, as uint8 arrays."""
+    x = _f32(x).ravel()
+    e2 = np.zeros(x.size, np.uint8)
+    e4 = np.zeros(x.size, np.uint8)
+    lib().or_encode_array(_p(x, ctypes.c_float), x.size, _p(e2, ctypes.c_uint8), _p(e4, ctypes.c_uint8))
+    return e2, e4
 
 
 def mx_exponent(amax: float) -> int:

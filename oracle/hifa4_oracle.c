@@ -120,6 +120,16 @@ double or_ue8m0_decode(uint8_t code) {
   return ldexp(1.0, (int)code - 127);
 }
 
+/* Element-wise encoders over an array (for comparing with hardware
+ * conversions): e2m1[i] = E2M1(x[i]); e4m3[i] = UE4M3(|x[i]|). */
+void or_encode_array(const float* x, int64_t n, uint8_t* e2m1, uint8_t* e4m3) {
+  #pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    e2m1[i] = or_e2m1_encode(x[i]);
+    e4m3[i] = or_ue4m3_encode(fabsf(x[i]));
+  }
+}
+
 /* ------------------------------------------------------------------------ */
 /* 2. Block quantizers                                                       */
 /* ------------------------------------------------------------------------ */

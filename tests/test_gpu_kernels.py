@@ -1,0 +1,158 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Codes and scales must match bit for bit; outputs must satisfy
+|dO| <= 1e-2 max|O| + 1e-3 elementwise and cosine >= 0.9999."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+h = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    global h
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import bit_quantized_flashattention_smooth_b200 as mod
+    mod.lib()
+    h = mod
+    yield
+    assert h.device_error() == 0, "a kernel gave up a bounded wait"
+
+
+# ------------------------------------------------------------ conversions ---
+def _sweep():
+    rng = np.random.default_rng(0)
+    vals = []
+    for e in range(-14, 10):
+        m = rng.integers(0, 1 << 23, 20000, dtype=np.int64)
+        vals.append((((e + 127) << 23) | m).astype(np.uint32).view(np.float32))
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    mids = ((grid[:-1] + grid[1:]) / 2).astype(np.float32)
+    e4 = oracle.ue4m3_decode(np.arange(127)).astype(np.float32)
+    e4m = ((e4[:-1].astype(np.float64) + e4[1:]) / 2).astype(np.float32)
+    base = np.concatenate(vals + [grid, mids, e4, e4m, np.array([0, 447, 448, 464, 500, 1e30, 2.0 ** -10], np.float32)])
+    nb = np.concatenate([base, np.nextafter(base, np.float32(np.inf)), np.nextafter(base, np.float32(0))])
+    return np.concatenate([nb, -nb]).astype(np.float32)
+
+
+def test_hw_conversions_match_written_rounding():
+    x = _sweep()
+    e2_gpu, e4_gpu = h.convert_probe(torch.from_numpy(x).cuda())
+    e2_ref, e4_ref = oracle.encode_array(x)
+    e2_gpu = U.to_np(e2_gpu).astype(np.uint8)
+    bad = np.nonzero(e2_gpu != e2_ref)[0]
+    assert bad.size == 0, f"E2M1: {bad.size} mismatches e.g. x={x[bad[:8]]} gpu={e2_gpu[bad[:8]]} ref={e2_ref[bad[:8]]}"
+    pos = x >= 0
+    e4_gpu = U.to_np(e4_gpu).astype(np.uint8)
+    bad = np.nonzero((e4_gpu != e4_ref) & pos)[0]
+    assert bad.size == 0, f"E4M3: {bad.size} mismatches e.g. x={x[bad[:8]]} gpu={e4_gpu[bad[:8]]} ref={e4_ref[bad[:8]]}"
+
+
+# --------------------------------------------------------------- FP4 MMA ---
+@pytest.mark.parametrize("fmt", [oracle.NVFP4, oracle.MXFP4])
+@pytest.mark.parametrize("n,k", [(128, 128), (64, 128), (256, 256), (128, 256)])
+def test_fp4_mma_tile_layouts(fmt, n, k):
+    rng = np.random.default_rng(n + k + fmt)
+    beta = oracle.beta_of(fmt)
+    ac = rng.integers(0, 256, (128, k // 2), dtype=np.uint8)
+    bc = rng.integers(0, 256, (n, k // 2), dtype=np.uint8)
+    lo, hi = (0x28, 0x48) if fmt == oracle.NVFP4 else (120, 134)
+    asc = rng.integers(lo, hi, (128, k // beta), dtype=np.uint8)
+    bsc = rng.integers(lo, hi, (n, k // beta), dtype=np.uint8)
+    A = oracle.dequantize_rows(ac, asc, fmt)
+    Bm = oracle.dequantize_rows(bc, bsc, fmt)
+    ref = A @ Bm.T
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    d = h.fp4_mma_probe(dev(ac), dev(oracle.sf_tile(asc)), dev(bc), dev(oracle.sf_tile(bsc)), n, k, fmt, 1, 1)
+    got = U.to_np(d)
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-5 * np.abs(ref).max())
+    d3 = h.fp4_mma_probe(dev(ac), dev(oracle.sf_tile(asc)), dev(bc), dev(oracle.sf_tile(bsc)), n, k, fmt, 3, 2)
+    np.testing.assert_allclose(U.to_np(d3), 3 * ref, rtol=1e-5, atol=3e-5 * np.abs(ref).max())
+
+
+# ---------------------------------------------------- calibrate + quantize ---
+QUANT_CASES = [
+    # B, Hq, Hkv, N, d, fmt, dtype
+    (1, 2, 2, 256, 64, oracle.NVFP4, torch.float16),
+    (1, 4, 2, 200, 128, oracle.NVFP4, torch.bfloat16),
+    (2, 4, 1, 130, 256, oracle.MXFP4, torch.bfloat16),
+    (1, 8, 2, 300, 64, oracle.MXFP4, torch.float16),
+    (1, 2, 2, 1, 128, oracle.NVFP4, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,fmt,dtype", QUANT_CASES)
+def test_calibrate_and_quantize_bit_exact(B, Hq, Hkv, N, d, fmt, dtype):
+    q, k, v = U.synthetic(B, Hq, Hkv, N, d, seed=N + d, dtype=dtype)
+    n_cal = min(N, 64)
+    s_ref, inv_ref = oracle.calibrate(q.float().numpy(), k.float().numpy(), n_cal=n_cal, alpha=0.5)
+    s, inv = h.calibrate_smooth_qk(q.cuda(), k.cuda(), n_cal=n_cal, alpha=0.5)
+    s_g, inv_g = U.to_np(s), U.to_np(inv)
+    np.testing.assert_allclose(s_g, s_ref, rtol=2 ** -22)
+    # quantize with the oracle's scales on both sides, then compare bytes
+    z = h.quantize_qkv(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(s_ref).cuda(),
+                       torch.from_numpy(inv_ref).cuda(), fmt)
+    qz, tiled = U.oracle_quantize(q, k, v, s_ref, inv_ref, fmt)
+    for name in ("q_codes", "k_codes", "vt_codes"):
+        g = U.to_np(getattr(z, name)).astype(np.uint8)
+        assert np.array_equal(g, qz[name]), (name, int(np.sum(g != qz[name])))
+    for name in ("q_sc", "k_sc", "vt_sc"):
+        g = U.to_np(getattr(z, name.replace("_sc", "_scales"))).astype(np.uint8)
+        assert np.array_equal(g, tiled[name]), (name, int(np.sum(g != tiled[name])))
+
+
+# -------------------------------------------------------------- attention ---
+ATTN_CASES = [
+    # B, Hq, Hkv, N, d, causal, BN, fmt, mode, dtype
+    (1, 2, 2, 256, 64, False, 64, oracle.NVFP4, oracle.PREORDER, torch.float16),
+    (1, 2, 2, 256, 64, False, 64, oracle.NVFP4, oracle.INCONSISTENT, torch.float16),
+    (1, 4, 1, 200, 128, True, 128, oracle.NVFP4, oracle.PREORDER, torch.bfloat16),
+    (1, 4, 2, 384, 128, True, 64, oracle.MXFP4, oracle.PREORDER, torch.bfloat16),
+    (1, 2, 2, 300, 64, False, 128, oracle.MXFP4, oracle.INCONSISTENT, torch.bfloat16),
+    (1, 4, 2, 130, 256, True, 128, oracle.NVFP4, oracle.INCONSISTENT, torch.bfloat16),
+    (2, 2, 1, 257, 256, False, 128, oracle.MXFP4, oracle.PREORDER, torch.bfloat16),
+    (1, 2, 2, 1, 128, True, 128, oracle.NVFP4, oracle.PREORDER, torch.bfloat16),
+    (1, 8, 2, 512, 128, True, 128, oracle.NVFP4, oracle.PREORDER, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal,BN,fmt,mode,dtype", ATTN_CASES)
+def test_attention_matches_oracle(B, Hq, Hkv, N, d, causal, BN, fmt, mode, dtype):
+    q, k, v = U.synthetic(B, Hq, Hkv, N, d, seed=7 * N + d, dtype=dtype)
+    s_ref, inv_ref = oracle.calibrate(q.float().numpy(), k.float().numpy(), n_cal=min(N, 64))
+    z = h.quantize_qkv(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(s_ref).cuda(),
+                       torch.from_numpy(inv_ref).cuda(), fmt)
+    qz, _ = U.oracle_quantize(q, k, v, s_ref, inv_ref, fmt)
+    scale = 1.0 / math.sqrt(d)
+    ref = oracle.attention(qz, N, fmt, scale, causal, mode, BN)
+    o, lse, lph, lp = h.attn_fwd(z, scale, causal, mode, BN, out_dtype=dtype, return_lse=True, debug=True)
+    ok, err, bound, cos = U.compare_out(U.to_np(o), ref["O"])
+    assert ok, f"max|dO|={err:.3e} bound={bound:.3e} cos={cos:.6f}"
+    np.testing.assert_allclose(U.to_np(lse), ref["lse"], rtol=1e-3, atol=1e-2)
+    np.testing.assert_allclose(U.to_np(lph), ref["l_phat"], rtol=2e-2)
+    np.testing.assert_allclose(U.to_np(lp), ref["l_p"], rtol=2e-3)
+
+
+def test_theorem1_coherence_on_gpu():
+    """Inconsistent vs P-Reordering outputs differ by one scale per row, equal
+    to l_phat / l_p, with net probability-mass loss (eps < 0)."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 512, 128
+    q, k, v = U.synthetic(B, Hq, Hkv, N, d, seed=99)
+    z = h.quantize_qkv(q.cuda(), k.cuda(), v.cuda(), None, None, oracle.NVFP4)
+    o_r, lph, lp = h.attn_fwd(z, None, True, oracle.PREORDER, 128, out_dtype=torch.float16, debug=True)
+    o_i = h.attn_fwd(z, None, True, oracle.INCONSISTENT, 128, out_dtype=torch.float16)
+    o_r, o_i = U.to_np(o_r).astype(np.float64), U.to_np(o_i).astype(np.float64)
+    ratio = U.to_np(lph) / U.to_np(lp)
+    pred = o_r * ratio[..., None]
+    assert np.max(np.abs(o_i - pred)) <= 2e-3 * np.max(np.abs(o_r)) + 1e-3
+    eps = ratio - 1
+    assert np.median(eps) < 0
