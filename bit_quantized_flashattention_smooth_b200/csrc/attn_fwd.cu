@@ -335,12 +335,17 @@ __global__ void __launch_bounds__(192, 1)
         for (int k = 0; k < BN; ++k)
           if (kbase + k >= lim) s[k] = -INFINITY;
       }
-      float smax = -INFINITY;
+      // x = fl32(S * c) first, then P = 2^(x - m): the row maximum gives
+      // exactly 2^0 = 1, so power-of-two block decisions (the MXFP4 shared
+      // exponent) agree with the written rule.
+      float xmax = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < BN; ++k) smax = fmaxf(smax, s[k]);
-      const float m_new = fmaxf(m, smax * c);
+      for (int k = 0; k < BN; ++k) {
+        s[k] = __fmul_rn(s[k], c);
+        xmax = fmaxf(xmax, s[k]);
+      }
+      const float m_new = fmaxf(m, xmax);
       const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);
-      const float neg_m = -m_new;
       // P = 2^(S*c - m_new); P-hat per block of BETA keys
       uint32_t codes[BN / 8];
       uint32_t scw[C::NKC_P];
@@ -353,7 +358,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int i = 0; i < C::BETA; ++i) {
           const int k = blk * C::BETA + i;
-          const float pv = ex2_approx(fmaf(s[k], c, neg_m));
+          const float pv = ex2_approx(__fsub_rn(s[k], m_new));
           s[k] = pv;
           bmax = fmaxf(bmax, pv);
         }

@@ -51,7 +51,7 @@ def test_hw_conversions_match_written_rounding():
     e2_gpu = U.to_np(e2_gpu).astype(np.uint8)
     bad = np.nonzero(e2_gpu != e2_ref)[0]
     assert bad.size == 0, f"E2M1: {bad.size} mismatches e.g. x={x[bad[:8]]} gpu={e2_gpu[bad[:8]]} ref={e2_ref[bad[:8]]}"
-    pos = x >= 0
+    pos = ~np.signbit(x)   # scales are encoded from |amax| >= +0
     e4_gpu = U.to_np(e4_gpu).astype(np.uint8)
     bad = np.nonzero((e4_gpu != e4_ref) & pos)[0]
     assert bad.size == 0, f"E4M3: {bad.size} mismatches e.g. x={x[bad[:8]]} gpu={e4_gpu[bad[:8]]} ref={e4_ref[bad[:8]]}"
