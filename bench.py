@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark of the 4-bit FlashAttention forward hot path on B200.
+
+One step = one pass of the hot path over one batch of the prefill workload
+(Smooth-QK scale + FP4 quantize of Q, K, V, then the 4-bit attention forward);
+the Smooth-QK calibration is offline and untimed.  The split-KV decode row is
+measured in the same run on its own workload and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Rank 0 prints one JSON line.  Multi-GPU: one process per GPU (torchrun); the
+path has no data exchange, so each rank runs its own batch (weak scaling) and
+the value is all ranks' work over the max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_flashattention_smooth_b200 import workloads as W  # noqa: E402
+
+METRIC = "4-bit attention fwd TFLOPS and % of dense FP4 peak; decode KV GB/s vs HBM"
+FP4_OVER_BF16 = 4.0   # nominal dense ratio: 9 PFLOP/s FP4 / 2.25 PFLOP/s BF16
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    def __init__(self, index: int):
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allmax(x: float, world) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ our arm -----
+def run_prefill(args, rank, world):
+    import bit_quantized_flashattention_smooth_b200 as h
+    w = W.WORKLOADS[args.workload]
+    fmt = h.NVFP4 if args.fmt == "nvfp4" else h.MXFP4
+    mode = h.PREORDER if args.mode == "preorder" else h.INCONSISTENT
+    wr = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})   # each rank its own batch
+    q, k, v = W.make_prefill(wr)
+    dev = torch.device("cuda")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    s, inv = h.calibrate_smooth_qk(qd[:, :, : w.n_cal], kd[:, :, : w.n_cal], w.n_cal)   # offline, untimed
+    z = h.alloc_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, fmt, dev)
+    o = torch.empty((w.B, w.Hq, w.N, w.d), device=dev, dtype=W.torch_dtype(w.dtype))
+    flush = torch.empty(L2_FLUSH_BYTES, device=dev, dtype=torch.uint8)
+    scale = 1.0 / math.sqrt(w.d)
+
+    def step():
+        h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)
+        h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()                       # L2 flush between timed steps (outside the step events)
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)
+        e1.record(stream)
+        h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)
+        e2.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - t_wall
+    clk = clocks.stop() if clocks else None
+    step_ms = sum(a.elapsed_time(c) for a, b, c in ev) / args.steps
+    attn_ms = sum(b.elapsed_time(c) for a, b, c in ev) / args.steps
+    quant_ms = sum(a.elapsed_time(b) for a, b, c in ev) / args.steps
+    dev_err = h.device_error()
+    if dev_err:
+        raise RuntimeError(f"device error word {dev_err:#x}")
+    step_ms_max = allmax(step_ms, world)
+    attn_ms_max = allmax(attn_ms, world)
+    flops = W.prefill_flops(w)
+
+    # ---- end to end through the C ABI with host buffers (pinned) ----
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    n_e2e = max(3, min(args.steps, 200))
+    for _ in range(3):
+        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_s.record(stream)
+    for _ in range(n_e2e):
+        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allmax(e_s.elapsed_time(e_e) / n_e2e, world)
+    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
+    d2h = o.numel() * o.element_size()
+
+    return dict(w=w, fmt=fmt, mode=mode, step_ms=step_ms_max, attn_ms=attn_ms_max, quant_ms=quant_ms,
+                flops=flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clk, wall=wall,
+                launches=4 * args.steps, qd=qd, kd=kd, vd=vd, z=z)
+
+
+def fp4_probe_peak():
+    """Dense FP4 tensor throughput of back-to-back block-scaled MMAs (the
+    repo's fp4_mma_probe): 128x256x256 NVFP4 products on 8 CTAs per SM-wave."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    n, k, reps = 256, 256, 4000
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    ctas = sms
+    ac = torch.randint(0, 256, (128, k // 2), dtype=torch.uint8, device="cuda")
+    bc = torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device="cuda")
+    asc = torch.full((h.scale_bytes(128, k, h.NVFP4),), 0x38, dtype=torch.uint8, device="cuda")
+    bsc = torch.full((h.scale_bytes(n, k, h.NVFP4),), 0x38, dtype=torch.uint8, device="cuda")
+    out = torch.empty((128, n), device="cuda")
+    h.fp4_mma_probe(ac, asc, bc, bsc, n, k, h.NVFP4, 10, ctas, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    h.fp4_mma_probe(ac, asc, bc, bsc, n, k, h.NVFP4, reps, ctas, out)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    return 2.0 * 128 * n * k * reps * ctas / (ms * 1e-3) / 1e12
+
+
+def cpu_baseline(w, fmt, mode, prefill_inputs=None, budget_s=20.0):
+    """The oracle, as it stands, on the host cores: full-workload quantize plus
+    the attention of the last query tile (128 rows, all heads) of batch 0."""
+    import oracle
+    q, k, v = prefill_inputs if prefill_inputs is not None else W.make_prefill(w)
+    qn, kn, vn = q[:1].float().numpy(), k[:1].float().numpy(), v[:1].float().numpy()
+    s, inv = oracle.calibrate(qn, kn, w.n_cal)
+    rows = 128
+    t0 = time.perf_counter()
+    qz = oracle.quantize_qkv(qn, kn, vn, s, inv, fmt)
+    oracle.attention(qz, w.N, fmt, 1 / math.sqrt(w.d), w.causal, mode, w.block_n, rows=(w.N - rows, w.N))
+    dt = time.perf_counter() - t0
+    pairs = sum((i + 1) if w.causal else w.N for i in range(w.N - rows, w.N))
+    flops = 4.0 * w.Hq * w.d * pairs
+    return dict(value=flops / dt / 1e12, unit="TFLOPS", cores=oracle.threads(), kind="oracle",
+                sample=f"batch 0 of {w.name}: oracle quantize of all Q/K/V plus attention of the last "
+                       f"{rows}-row query tile, all {w.Hq} heads ({flops / 1e9:.2f} GFLOP in {dt:.1f} s)")
+
+
+def run_decode(args):
+    """Split-KV decode over the NVFP4 cache of the decode workload; returns
+    achieved KV GB/s (algorithmic cache bytes / kernel time)."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    w = W.WORKLOADS["split_decode"]
+    dev = torch.device("cuda")
+    kv, B, Hkv, Hq, d = w.N, w.B, w.Hkv, w.Hq, w.d
+    q, k, v, qcal, kcal = W.make_decode_device(w, dev)
+    s, inv = h.calibrate_smooth_qk(qcal, kcal, w.n_cal)
+    cache = h.quantize_kv(k, v, inv, h.NVFP4, Hq=Hq)
+    del k, v
+    splits = h.default_splits(B, Hkv, kv)
+    ws = torch.empty(h.decode_workspace_bytes(B, Hq, d, splits), device=dev, dtype=torch.uint8)
+    o = torch.empty((B, Hq, d), device=dev, dtype=torch.bfloat16)
+    flush = torch.empty(L2_FLUSH_BYTES, device=dev, dtype=torch.uint8)
+    for _ in range(3):
+        h.attn_decode(q, s, cache, kv, None, h.PREORDER, splits, ws, o)
+    torch.cuda.synchronize()
+    n = max(5, min(args.steps, 50))
+    tot = 0.0
+    for _ in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        h.attn_decode(q, s, cache, kv, None, h.PREORDER, splits, ws, o)
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    ms = tot / n
+    kv_bytes = (cache.k_codes.numel() + cache.k_scales.numel() + cache.vt_codes.numel() + cache.vt_scales.numel())
+    return dict(ms=ms, bytes=kv_bytes, gbs=kv_bytes / (ms * 1e-3) / 1e9, splits=splits)
+
+
+# ------------------------------------------------------- reference arm ----
+def run_reference(args, rank, world):
+    """The CPU oracle timed on the host cores on bounded samples of the same
+    workload (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    w = W.WORKLOADS[args.workload]
+    fmt = 0 if args.fmt == "nvfp4" else 1
+    mode = 0 if args.mode == "preorder" else 1
+    q, k, v = W.make_prefill(w)
+    qn, kn, vn = q[:1].float().numpy(), k[:1].float().numpy(), v[:1].float().numpy()
+    s, inv = oracle.calibrate(qn, kn, w.n_cal)
+    qz = oracle.quantize_qkv(qn, kn, vn, s, inv, fmt)
+    # one step = attention of `rows` query rows (from the last tile) of all heads
+    total_budget = 90.0
+    rows = 8
+    t0 = time.perf_counter()
+    oracle.attention(qz, w.N, fmt, 1 / math.sqrt(w.d), w.causal, mode, w.block_n, rows=(w.N - rows, w.N))
+    per_row = (time.perf_counter() - t0) / rows
+    rows = int(max(1, min(128, total_budget / max(1, args.steps + args.warmup) / per_row)))
+    for _ in range(args.warmup):
+        oracle.attention(qz, w.N, fmt, 1 / math.sqrt(w.d), w.causal, mode, w.block_n, rows=(w.N - rows, w.N))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attention(qz, w.N, fmt, 1 / math.sqrt(w.d), w.causal, mode, w.block_n, rows=(w.N - rows, w.N))
+    dt = time.perf_counter() - t0
+    pairs = sum((i + 1) if w.causal else w.N for i in range(w.N - rows, w.N))
+    flops = 4.0 * w.Hq * w.d * pairs * args.steps
+    val = flops / dt / 1e12
+    return dict(value=val, ms=dt / args.steps * 1e3,
+                sample=f"per step: oracle attention of the last {rows} query rows of batch 0, all {w.Hq} heads, "
+                       f"of {w.name}")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3_prefill")
+    ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
+    ap.add_argument("--mode", default="preorder", choices=["preorder", "inconsistent"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-probe", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local = dist_setup(args.gpus)
+    w = W.WORKLOADS[args.workload]
+    config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+              "format": args.fmt, "normalizer": args.mode, "block_n": w.block_n,
+              "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}"}
+
+    if args.impl == "reference":
+        ref = run_reference(args, rank, world)
+        if rank == 0:
+            import oracle
+            line = {"metric": METRIC, "value": ref["value"], "unit": "TFLOPS", "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": ref["ms"],
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                    "data": "synthetic", "config": config, "impl": "reference",
+                    "cpu_baseline": {"value": ref["value"], "unit": "TFLOPS", "cores": oracle.threads(),
+                                     "kind": "oracle", "sample": ref["sample"]},
+                    "e2e": {"value": ref["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                            "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+        return
+
+    pk = peaks()
+    res = run_prefill(args, rank, world)
+    value = res["flops"] * world / (res["step_ms"] * 1e-3) / 1e12
+    attn_tflops = res["flops"] / (res["attn_ms"] * 1e-3) / 1e12
+    fp4_peak = pk["bf16"] * FP4_OVER_BF16
+    extra = {}
+    if rank == 0 and not args.no_probe:
+        try:
+            extra["fp4_probe_tflops"] = fp4_probe_peak()
+        except Exception as e:  # measurement only
+            extra["fp4_probe_error"] = str(e)
+    decode = None
+    if not args.no_decode:
+        try:
+            decode = run_decode(args)
+        except Exception as e:
+            decode = {"error": str(e)}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["step_ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp4-e2m1 (fp32 accumulate / softmax)", "data": "synthetic",
+        "config": config,
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_fp4", "achieved": attn_tflops, "peak": fp4_peak,
+                     "unit": "TFLOP/s", "frac": attn_tflops / fp4_peak, "traffic": None,
+                     "peak_note": f"{pk['src']} bf16 burst {pk['bf16']} TFLOP/s x nominal FP4/BF16 ratio 4"},
+        "attn_ms": res["attn_ms"], "quantize_ms": res["quant_ms"],
+        "e2e": {"value": res["flops"] * world / (res["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+    }
+    line.update(extra)
+    if "fp4_probe_tflops" in extra:
+        line["roofline"]["frac_of_probe_peak"] = attn_tflops / extra["fp4_probe_tflops"]
+    if decode is not None:
+        if "gbs" in decode:
+            line["decode"] = {"workload": "split_decode", "kv_gbs": decode["gbs"], "ms": decode["ms"],
+                              "kv_bytes": decode["bytes"], "hbm_peak_gbs": pk["hbm"],
+                              "frac": decode["gbs"] / pk["hbm"], "splits": decode["splits"]}
+        else:
+            line["decode"] = decode
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, res["fmt"], res["mode"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

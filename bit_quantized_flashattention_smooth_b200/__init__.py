@@ -31,6 +31,7 @@ _lib = None
 
 ABI_FUNCTIONS = (
     "hifa4_codes_bytes", "hifa4_scale_bytes", "hifa4_calibrate_smooth_qk", "hifa4_quantize_qkv",
+    "hifa4_quantize_kv",
     "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
@@ -53,6 +54,7 @@ def lib():
         L.hifa4_scale_bytes.argtypes = [i64, i, i]; L.hifa4_scale_bytes.restype = sz
         L.hifa4_calibrate_smooth_qk.argtypes = [vp, vp, i, i, i, i, i, i, i, f, i, vp, vp, vp]
         L.hifa4_quantize_qkv.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, vp, i, vp, vp, vp, vp, vp, vp, vp]
+        L.hifa4_quantize_kv.argtypes = [vp, vp, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp]
         L.hifa4_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, vp]
         L.hifa4_decode_workspace_size.argtypes = [i, i, i, i]; L.hifa4_decode_workspace_size.restype = sz
         L.hifa4_decode_default_splits.argtypes = [i, i, i, i]; L.hifa4_decode_default_splits.restype = i
@@ -166,6 +168,27 @@ def quantize_qkv(q, k, v, s=None, inv_s=None, fmt: int = NVFP4, out: QuantizedQK
     _check(lib().hifa4_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hq, Hkv, N, d, _ptr(s), _ptr(inv_s),
                                     fmt, _ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),
                                     _ptr(z.vt_codes), _ptr(z.vt_scales), _stream()), "quantize_qkv")
+    return z
+
+
+def alloc_kv_cache(B, Hq, Hkv, kv_len, d, fmt, device="cuda") -> QuantizedQKV:
+    """A 4-bit KV cache (no Q buffers)."""
+    Np = pad128(kv_len)
+    u8 = dict(device=device, dtype=torch.uint8)
+    empty = torch.empty(0, **u8)
+    return QuantizedQKV(empty, empty,
+                        torch.empty((B, Hkv, Np, d // 2), **u8), torch.empty((B, Hkv, scale_bytes(kv_len, d, fmt)), **u8),
+                        torch.empty((B, Hkv, d, Np // 2), **u8), torch.empty((B, Hkv, scale_bytes(d, Np, fmt)), **u8),
+                        B, Hq, Hkv, kv_len, d, fmt)
+
+
+def quantize_kv(k, v, inv_s=None, fmt: int = NVFP4, Hq: int | None = None, out: QuantizedQKV | None = None):
+    """Quantize K (scaled by inv_s) and V into a 4-bit KV cache."""
+    B, Hkv, N, d = k.shape
+    k = k.contiguous(); v = v.contiguous()
+    z = out if out is not None else alloc_kv_cache(B, Hq or Hkv, Hkv, N, d, fmt, k.device)
+    _check(lib().hifa4_quantize_kv(_ptr(k), _ptr(v), _dt(k), B, Hkv, N, d, _ptr(inv_s), fmt, _ptr(z.k_codes),
+                                   _ptr(z.k_scales), _ptr(z.vt_codes), _ptr(z.vt_scales), _stream()), "quantize_kv")
     return z
 
 

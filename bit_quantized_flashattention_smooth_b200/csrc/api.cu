@@ -150,6 +150,21 @@ hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hif
                              vt_codes, vt_scales, static_cast<cudaStream_t>(stream));
 }
 
+hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dt, int B, int Hkv, int N, int d,
+                               const float* inv_s, hifa4_format fmt, uint8_t* k_codes, uint8_t* k_scales,
+                               uint8_t* vt_codes, uint8_t* vt_scales, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(k && v && k_codes && k_scales && vt_codes && vt_scales, HIFA4_ERR_INVALID_ARG,
+                "quantize_kv: null pointer");
+  HIFA4_REQUIRE(valid_dt(dt) && valid_fmt(fmt), HIFA4_ERR_INVALID_ARG, "quantize_kv: bad dtype/format");
+  HIFA4_REQUIRE(B > 0 && Hkv > 0 && N > 0, HIFA4_ERR_INVALID_ARG, "quantize_kv: bad shape");
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "quantize_kv: d=%d not in {64,128,256}", d);
+  HIFA4_REQUIRE(aligned16(k) && aligned16(v) && aligned16(k_codes) && aligned16(k_scales) && aligned16(vt_codes) &&
+                    aligned16(vt_scales) && (!inv_s || aligned16(inv_s)),
+                HIFA4_ERR_INVALID_ARG, "quantize_kv: pointers must be 16-byte aligned");
+  return quantize_qkv_launch(nullptr, k, v, dt, B, Hkv, Hkv, N, d, nullptr, inv_s, fmt, nullptr, nullptr, k_codes,
+                             k_scales, vt_codes, vt_scales, static_cast<cudaStream_t>(stream));
+}
+
 hifa4_status hifa4_attn_fwd(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
                             const uint8_t* k_scales, const uint8_t* vt_codes, const uint8_t* vt_scales, int B,
                             int Hq, int Hkv, int N, int d, hifa4_format fmt, float softmax_scale, int causal,

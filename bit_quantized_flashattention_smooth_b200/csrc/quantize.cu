@@ -243,48 +243,57 @@ __global__ void calib_finalize_kernel(float* s, float* inv_s, int n, double alph
 }
 
 // ---------------------------------------------------------- host launchers ---
+// Rows of one tensor (Q with G = Hq/Hkv, or K with G = 1) and V^T.
 template <typename T>
-static hifa4_status launch_quantize(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N,
-                                    int d, const float* s, const float* inv_s, int fmt, uint8_t* qc, uint8_t* qs,
-                                    uint8_t* kc, uint8_t* ks, uint8_t* vc, uint8_t* vs, cudaStream_t st) {
+static void launch_rows(const void* x, int B, int H, int G, int N, int d, const float* scale, int fmt, uint8_t* codes,
+                        uint8_t* sf, cudaStream_t st) {
   const int beta = beta_of(fmt);
   const int Np = static_cast<int>(pad128(N));
   const int wpr = (d / beta + 3) / 4;
-  const int64_t sfq = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
-  const int64_t sfv = static_cast<int64_t>(hifa4_scale_bytes(d, Np, static_cast<hifa4_format>(fmt)));
-  const int G = Hq / Hkv;
-  int64_t tq = static_cast<int64_t>(B) * Hq * Np * wpr, tk = static_cast<int64_t>(B) * Hkv * Np * wpr;
+  const int64_t sfh = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
+  const int64_t total = static_cast<int64_t>(B) * H * Np * wpr;
   const int thr = 256;
-  size_t vsmem = static_cast<size_t>(128) * d * sizeof(T);
-  dim3 vgrid(Np / 128, B * Hkv);
+  const unsigned grid = static_cast<unsigned>((total + thr - 1) / thr);
+  if (fmt == HIFA4_NVFP4)
+    quantize_rows_kernel<HIFA4_NVFP4, T><<<grid, thr, 0, st>>>(static_cast<const T*>(x), H, G, N, Np, d, scale, codes,
+                                                                sf, sfh, total);
+  else
+    quantize_rows_kernel<HIFA4_MXFP4, T><<<grid, thr, 0, st>>>(static_cast<const T*>(x), H, G, N, Np, d, scale, codes,
+                                                                sf, sfh, total);
+}
+
+template <typename T>
+static void launch_v(const void* v, int B, int Hkv, int N, int d, int fmt, uint8_t* vc, uint8_t* vs, cudaStream_t st) {
+  const int Np = static_cast<int>(pad128(N));
+  const int64_t sfv = static_cast<int64_t>(hifa4_scale_bytes(d, Np, static_cast<hifa4_format>(fmt)));
+  const size_t vsmem = static_cast<size_t>(128) * d * sizeof(T);
+  const dim3 vgrid(Np / 128, B * Hkv);
   if (fmt == HIFA4_NVFP4) {
-    quantize_rows_kernel<HIFA4_NVFP4, T><<<(tq + thr - 1) / thr, thr, 0, st>>>(
-        static_cast<const T*>(q), Hq, G, N, Np, d, s, qc, qs, sfq, tq);
-    quantize_rows_kernel<HIFA4_NVFP4, T><<<(tk + thr - 1) / thr, thr, 0, st>>>(
-        static_cast<const T*>(k), Hkv, 1, N, Np, d, inv_s, kc, ks, sfq, tk);
     if (vsmem > 48 * 1024)
       cudaFuncSetAttribute(quantize_v_kernel<HIFA4_NVFP4, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(vsmem));
-    quantize_v_kernel<HIFA4_NVFP4, T><<<vgrid, thr, vsmem, st>>>(static_cast<const T*>(v), N, Np, d, vc, vs, sfv);
+    quantize_v_kernel<HIFA4_NVFP4, T><<<vgrid, 256, vsmem, st>>>(static_cast<const T*>(v), N, Np, d, vc, vs, sfv);
   } else {
-    quantize_rows_kernel<HIFA4_MXFP4, T><<<(tq + thr - 1) / thr, thr, 0, st>>>(
-        static_cast<const T*>(q), Hq, G, N, Np, d, s, qc, qs, sfq, tq);
-    quantize_rows_kernel<HIFA4_MXFP4, T><<<(tk + thr - 1) / thr, thr, 0, st>>>(
-        static_cast<const T*>(k), Hkv, 1, N, Np, d, inv_s, kc, ks, sfq, tk);
     if (vsmem > 48 * 1024)
       cudaFuncSetAttribute(quantize_v_kernel<HIFA4_MXFP4, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(vsmem));
-    quantize_v_kernel<HIFA4_MXFP4, T><<<vgrid, thr, vsmem, st>>>(static_cast<const T*>(v), N, Np, d, vc, vs, sfv);
+    quantize_v_kernel<HIFA4_MXFP4, T><<<vgrid, 256, vsmem, st>>>(static_cast<const T*>(v), N, Np, d, vc, vs, sfv);
   }
-  return launch_status("quantize_qkv");
 }
 
 hifa4_status quantize_qkv_launch(const void* q, const void* k, const void* v, int dt, int B, int Hq, int Hkv, int N,
                                  int d, const float* s, const float* inv_s, int fmt, uint8_t* qc, uint8_t* qs,
                                  uint8_t* kc, uint8_t* ks, uint8_t* vc, uint8_t* vs, cudaStream_t st) {
-  if (dt == HIFA4_BF16)
-    return launch_quantize<__nv_bfloat16>(q, k, v, B, Hq, Hkv, N, d, s, inv_s, fmt, qc, qs, kc, ks, vc, vs, st);
-  return launch_quantize<__half>(q, k, v, B, Hq, Hkv, N, d, s, inv_s, fmt, qc, qs, kc, ks, vc, vs, st);
+  if (dt == HIFA4_BF16) {
+    if (q) launch_rows<__nv_bfloat16>(q, B, Hq, Hq / Hkv, N, d, s, fmt, qc, qs, st);
+    launch_rows<__nv_bfloat16>(k, B, Hkv, 1, N, d, inv_s, fmt, kc, ks, st);
+    launch_v<__nv_bfloat16>(v, B, Hkv, N, d, fmt, vc, vs, st);
+  } else {
+    if (q) launch_rows<__half>(q, B, Hq, Hq / Hkv, N, d, s, fmt, qc, qs, st);
+    launch_rows<__half>(k, B, Hkv, 1, N, d, inv_s, fmt, kc, ks, st);
+    launch_v<__half>(v, B, Hkv, N, d, fmt, vc, vs, st);
+  }
+  return launch_status(q ? "quantize_qkv" : "quantize_kv");
 }
 
 template <typename T>

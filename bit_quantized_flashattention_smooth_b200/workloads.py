@@ -91,6 +91,36 @@ def rope_neox(x: np.ndarray, theta: float, pos0: int = 0) -> np.ndarray:
     return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
 
 
+def rope_torch(x: torch.Tensor, theta: float, pos0: int = 0) -> torch.Tensor:
+    """rope_neox for a float32 torch tensor [..., T, d] on any device."""
+    T, d = x.shape[-2:]
+    half = d // 2
+    inv_freq = theta ** (-torch.arange(half, dtype=torch.float64, device=x.device) * 2.0 / d)
+    ang = torch.arange(pos0, pos0 + T, dtype=torch.float64, device=x.device)[:, None] * inv_freq[None, :]
+    cos, sin = torch.cos(ang).float(), torch.sin(ang).float()
+    x1, x2 = x[..., :half], x[..., half:]
+    return torch.cat([x1 * cos - x2 * sin, x2 * cos + x1 * sin], dim=-1)
+
+
+def make_decode_device(w: Workload, device="cuda"):
+    """The decode recipe drawn on the device with a seeded torch generator (the
+    full-size cache is 2 x 4 GiB of bf16; a host draw would dominate a run).
+    Returns (q [B,Hq,d], k, v [B,Hkv,kv,d], q_cal [B,Hq,n_cal,d], k_cal)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed)
+    kv, B = w.N, w.B
+    k = torch.randn((B, w.Hkv, kv, w.d), generator=g, device=device, dtype=torch.float32)
+    for c in w.outlier_channels:
+        k[..., c] = w.outlier_scale * k[..., c].abs()
+    k = rope_torch(k, w.theta).to(torch_dtype(w.dtype))
+    v = torch.randn((B, w.Hkv, kv, w.d), generator=g, device=device, dtype=torch.float32).to(torch_dtype(w.dtype))
+    q = rope_torch(torch.randn((B, w.Hq, 1, w.d), generator=g, device=device), w.theta, pos0=kv)
+    q_cal = rope_torch(torch.randn((B, w.Hq, w.n_cal, w.d), generator=g, device=device), w.theta)
+    n_cal = min(w.n_cal, kv)
+    return (q[:, :, 0].to(torch_dtype(w.dtype)), k, v, q_cal[:, :, :n_cal].to(torch_dtype(w.dtype)),
+            k[:, :, :n_cal].contiguous())
+
+
 def _draw_k(rng, shape, w: Workload) -> np.ndarray:
     if w.k_dist == "student_t3":
         return rng.standard_t(3, size=shape).astype(np.float32)

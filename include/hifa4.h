@@ -123,6 +123,16 @@ HIFA4_API hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const vo
                                 uint8_t* k_codes, uint8_t* k_scales, uint8_t* vt_codes,
                                 uint8_t* vt_scales, hifa4_stream_t stream);
 
+/* The K / V half of hifa4_quantize_qkv, for building a 4-bit KV cache (the
+ * decode path): k' = fl32(k*inv_s[h,c]) quantized along d and V quantized
+ * along tokens into V-hat^T, with exactly the rules and layouts above.
+ * k, v: device [B][Hkv][N][d] of `dt`; inv_s device float [Hkv][d] or NULL.
+ * Same requirements as hifa4_quantize_qkv. */
+HIFA4_API hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dt, int B, int Hkv, int N,
+                                         int d, const float* inv_s, hifa4_format fmt, uint8_t* k_codes,
+                                         uint8_t* k_scales, uint8_t* vt_codes, uint8_t* vt_scales,
+                                         hifa4_stream_t stream);
+
 /* ------------------------------------------------ attention forward --- */
 
 /* 4-bit FlashAttention forward (paper Abstract paras 1-2).  For each (b, hq)
