@@ -316,12 +316,15 @@ def main():
     ap.add_argument("--workload", default="qwen3_prefill")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--mode", default="preorder", choices=["preorder", "inconsistent"])
+    ap.add_argument("--block-n", type=int, default=0, help="key tile (0 = the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-probe", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_setup(args.gpus)
+    if args.block_n:
+        W.WORKLOADS[args.workload] = W.Workload(**{**W.WORKLOADS[args.workload].__dict__, "block_n": args.block_n})
     w = W.WORKLOADS[args.workload]
     config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
               "format": args.fmt, "normalizer": args.mode, "block_n": w.block_n,

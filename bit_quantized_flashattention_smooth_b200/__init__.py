@@ -33,7 +33,7 @@ ABI_FUNCTIONS = (
     "hifa4_codes_bytes", "hifa4_scale_bytes", "hifa4_calibrate_smooth_qk", "hifa4_quantize_qkv",
     "hifa4_quantize_kv",
     "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
-    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_status_string", "hifa4_last_error",
+    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
 )
 
@@ -62,6 +62,7 @@ def lib():
                                         ctypes.POINTER(ctypes.c_int), vp, sz, vp, i, vp]
         L.hifa4_fp4_mma_probe.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, vp]
         L.hifa4_convert_probe.argtypes = [vp, i64, vp, vp, vp]
+        L.hifa4_div6_probe.argtypes = [ctypes.c_uint32, ctypes.c_uint32, vp, vp, vp]
         L.hifa4_status_string.argtypes = [i]; L.hifa4_status_string.restype = ctypes.c_char_p
         L.hifa4_last_error.argtypes = []; L.hifa4_last_error.restype = ctypes.c_char_p
         L.hifa4_device_error.argtypes = []; L.hifa4_device_error.restype = ctypes.c_uint
@@ -256,6 +257,14 @@ def fp4_mma_probe(a_codes, a_scales, b_codes, b_scales, n: int, k: int, fmt: int
     _check(lib().hifa4_fp4_mma_probe(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), n, k, fmt,
                                      repeats, ctas, _ptr(d), _stream()), "fp4_mma_probe")
     return d
+
+
+def div6_probe(lo_bits: int, hi_bits: int):
+    """(mismatch count, first failing bit pattern) of the fast fl32(a/6)."""
+    cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
+    first = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(lib().hifa4_div6_probe(lo_bits, hi_bits, _ptr(cnt), _ptr(first), _stream()), "div6_probe")
+    return int(cnt.item()), int(first.item()) & 0xFFFFFFFF
 
 
 def convert_probe(x: torch.Tensor):

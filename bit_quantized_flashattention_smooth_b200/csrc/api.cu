@@ -86,6 +86,7 @@ int decode_default_splits(int B, int Hkv, int kv_len, int block_n);
 hifa4_status fp4_mma_probe_launch(const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*, int, int, int, int,
                                   int, float*, cudaStream_t);
 hifa4_status convert_probe_launch(const float*, int64_t, uint8_t*, uint8_t*, cudaStream_t);
+hifa4_status div6_probe_launch(uint32_t, uint32_t, unsigned long long*, uint32_t*, cudaStream_t);
 
 }  // namespace hifa4
 
@@ -246,6 +247,12 @@ hifa4_status hifa4_convert_probe(const float* x, int64_t count, uint8_t* e2m1_ou
   HIFA4_REQUIRE(x && e2m1_out && e4m3_out && count >= 0, HIFA4_ERR_INVALID_ARG, "convert_probe: bad args");
   if (count == 0) return HIFA4_OK;
   return convert_probe_launch(x, count, e2m1_out, e4m3_out, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_div6_probe(uint32_t lo_bits, uint32_t hi_bits, unsigned long long* mismatches,
+                              uint32_t* first_bad, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(mismatches && first_bad && lo_bits <= hi_bits, HIFA4_ERR_INVALID_ARG, "div6_probe: bad args");
+  return div6_probe_launch(lo_bits, hi_bits, mismatches, first_bad, static_cast<cudaStream_t>(stream));
 }
 
 const char* hifa4_status_string(hifa4_status st) {

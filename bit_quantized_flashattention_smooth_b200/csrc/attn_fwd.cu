@@ -58,7 +58,6 @@ struct AttnCfg {
   static constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
   static constexpr int BM = 128;
   static constexpr int NS = D == 256 ? 2 : 3;               // K/V pipeline stages
-  static constexpr int NSB = D == 256 ? 1 : 2;              // TMEM S buffers
   static constexpr int QROW = D / 2;                        // bytes per Q/K row
   static constexpr int PROW = BN / 2;                       // bytes per P-hat / V^T row
   static constexpr int KSTEPS_S = D / 64;
@@ -67,6 +66,15 @@ struct AttnCfg {
   static constexpr int NRG_V = (D + 127) / 128;             // 128-row groups of V^T
   static constexpr int NCH_V = (BN / BETA + 3) / 4;         // V^T scale chunks per tile per row group
   static constexpr int NKC_P = (BN / BETA + 3) / 4;         // P-hat scale chunks per tile
+  // TMEM columns with `nsb` S buffers: S, O, L (16), scale regions.
+  static constexpr int cols(int nsb) {
+    return nsb * BN + D + 16 + 8 * NKC_Q + 4 * NKC_P + 4 * NCH_V * NRG_V + 4;
+  }
+  // Prefer a footprint of 256 columns so that two CTAs share an SM (twice the
+  // softmax warps per scheduler); otherwise own all 512 columns.
+  static constexpr int NSB = cols(2) <= 256 ? 2 : (cols(1) <= 256 ? 1 : (cols(2) <= 512 ? 2 : 1));
+  static constexpr int TMEM_ALLOC = cols(NSB) <= 256 ? 256 : 512;
+  static constexpr int CTAS_PER_SM = TMEM_ALLOC == 256 ? 2 : 1;
   // shared memory layout (byte offsets; operand tiles 1024-aligned)
   static constexpr int SZ_Q = BM * QROW;
   static constexpr int SZ_K = BN * QROW;
@@ -83,7 +91,8 @@ struct AttnCfg {
   static constexpr int OFF_VSF = OFF_KSF + NS * NKC_Q * 512;
   static constexpr int OFF_PSF = OFF_VSF + NS * NRG_V * NCH_V * 512;
   static constexpr int OFF_ONESF = OFF_PSF + 2 * NKC_P * 512;
-  static constexpr int OFF_BAR = OFF_ONESF + 512;
+  static constexpr int OFF_INV = OFF_ONESF + 512;           // 128 floats: 1/scale per UE4M3 code
+  static constexpr int OFF_BAR = OFF_INV + 512;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
   // s_full[NSB], s_empty[NSB], p_full[2], p_empty[2], o_ready
   static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1;
@@ -99,9 +108,46 @@ struct AttnCfg {
   static constexpr int TM_SFB_V = TM_SFA_P + 4 * NKC_P;
   static constexpr int TM_SFB_1 = TM_SFB_V + 4 * NCH_V * NRG_V;
   static constexpr int TM_COLS_USED = TM_SFB_1 + 4;
-  static_assert(TM_COLS_USED <= 512, "TMEM budget");
+  static_assert(TM_COLS_USED <= TMEM_ALLOC, "TMEM budget");
+  // Dynamic shared memory requested: enough that at most CTAS_PER_SM CTAs are
+  // resident (a further CTA would stall in tcgen05.alloc).
+  static constexpr int SMEM_REQ = CTAS_PER_SM == 1 ? (SMEM_BYTES > 116 * 1024 ? SMEM_BYTES : 116 * 1024)
+                                                   : (SMEM_BYTES > 80 * 1024 ? SMEM_BYTES : 80 * 1024);
+  static_assert(CTAS_PER_SM == 1 || SMEM_REQ <= 112 * 1024, "two CTAs per SM must fit");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
+
+// Reductions as shallow trees (3-input max), not dependent chains.
+template <int N>
+__device__ __forceinline__ float tree_max(const float* v) {
+  if constexpr (N == 1) {
+    return v[0];
+  } else if constexpr (N == 2) {
+    return fmaxf(v[0], v[1]);
+  } else {
+    constexpr int M = (N + 2) / 3;
+    float t[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+      const int a = 3 * i;
+      if (a + 2 < N) t[i] = fmax3(v[a], v[a + 1], v[a + 2]);
+      else if (a + 1 < N) t[i] = fmaxf(v[a], v[a + 1]);
+      else t[i] = v[a];
+    }
+    return tree_max<M>(t);
+  }
+}
+template <int N>
+__device__ __forceinline__ float tree_sum(const float* v) {
+  if constexpr (N == 1) {
+    return v[0];
+  } else {
+    float t[N / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) t[i] = v[2 * i] + v[2 * i + 1];
+    return tree_sum<N / 2>(t);
+  }
+}
 
 __device__ __forceinline__ uint32_t swz_chunk(uint32_t r, uint32_t c, uint32_t row_bytes) {
   // physical 16-byte chunk of logical chunk c in row r under the swizzle that
@@ -110,7 +156,7 @@ __device__ __forceinline__ uint32_t swz_chunk(uint32_t r, uint32_t c, uint32_t r
 }
 
 template <int D, int BN, int FMT, bool PREORDER>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D, BN, FMT>;
@@ -167,10 +213,13 @@ __global__ void __launch_bounds__(192, 1)
     // word i of the chunk sits at byte 4*i: line (i/4) = row%32, word (i%4) = row/32
     const int row_of_word = (i >> 2) + 32 * (i & 3);
     reinterpret_cast<uint32_t*>(smem + C::OFF_ONESF)[i] = row_of_word < 16 ? one * 0x01010101u : 0u;
+    // fl32(1 / (UE4M3(i) * g_P)), the P-hat element multiplier of scale code i
+    const float sd = __fmul_rn(ue4m3_to_f32(i), FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f);
+    reinterpret_cast<float*>(smem + C::OFF_INV)[i] = i == 0 ? 0.0f : __fdiv_rn(1.0f, sd);
   }
   fence_proxy_async_smem();
   if (warp == 5) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);
     tmem_relinquish();
   }
   if (warp == 4 && lane == 0) {
@@ -306,6 +355,7 @@ __global__ void __launch_bounds__(192, 1)
     const bool want_lp = !PREORDER || p.dbg_l_p != nullptr;
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
     constexpr float kInvGP = FMT == HIFA4_NVFP4 ? 256.0f : 1.0f;
+    const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
     bool ok = true;
     for (int j = 0; j < nkt && ok; ++j) {
       const int sb = j % C::NSB;
@@ -316,12 +366,15 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       float s[BN];
+      {
+        uint32_t v[BN];
 #pragma unroll
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld32_wait(tmem + lane_base + C::TM_S + sb * BN + cc * 32, v);
+        for (int cc = 0; cc < BN / 32; ++cc)
+          tmem_ld32(tmem + lane_base + C::TM_S + sb * BN + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(v[i]);
+        for (int cc = 0; cc < BN / 32; ++cc) tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
+#pragma unroll
+        for (int i = 0; i < BN; ++i) s[i] = __uint_as_float(v[i]);
       }
       tc_fence_before();
       __syncwarp();
@@ -332,21 +385,22 @@ __global__ void __launch_bounds__(192, 1)
       if (need_mask) {
         const int lim = p.causal ? min(p.N, row + 1) : p.N;
 #pragma unroll
-        for (int k = 0; k < BN; ++k)
-          if (kbase + k >= lim) s[k] = -INFINITY;
+        for (int k = 0; k < BN; ++k) s[k] = (kbase + k >= lim) ? -INFINITY : s[k];
       }
       // x = fl32(S * c) first, then P = 2^(x - m): the row maximum gives
       // exactly 2^0 = 1, so power-of-two block decisions (the MXFP4 shared
       // exponent) agree with the written rule.
-      float xmax = -INFINITY;
+      const float2 c2 = make_float2(c, c);
 #pragma unroll
-      for (int k = 0; k < BN; ++k) {
-        s[k] = __fmul_rn(s[k], c);
-        xmax = fmaxf(xmax, s[k]);
+      for (int k = 0; k < BN; k += 2) {
+        const float2 x = fmul2(make_float2(s[k], s[k + 1]), c2);
+        s[k] = x.x;
+        s[k + 1] = x.y;
       }
-      const float m_new = fmaxf(m, xmax);
+      const float m_new = fmaxf(m, tree_max<BN>(s));
       const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);
-      // P = 2^(S*c - m_new); P-hat per block of BETA keys
+      const float2 negm = make_float2(-m_new, -m_new);
+      // P = 2^(x - m_new); P-hat per block of BETA keys
       uint32_t codes[BN / 8];
       uint32_t scw[C::NKC_P];
 #pragma unroll
@@ -354,41 +408,35 @@ __global__ void __launch_bounds__(192, 1)
       float psum = 0.0f;
 #pragma unroll
       for (int blk = 0; blk < BN / C::BETA; ++blk) {
-        float bmax = 0.0f;
+        float* pb_ = s + blk * C::BETA;
 #pragma unroll
-        for (int i = 0; i < C::BETA; ++i) {
-          const int k = blk * C::BETA + i;
-          const float pv = ex2_approx(__fsub_rn(s[k], m_new));
-          s[k] = pv;
-          bmax = fmaxf(bmax, pv);
+        for (int i = 0; i < C::BETA; i += 2) {
+          const float2 y = fadd2(make_float2(pb_[i], pb_[i + 1]), negm);
+          pb_[i] = ex2_approx(y.x);
+          pb_[i + 1] = ex2_approx(y.y);
         }
+        const float bmax = tree_max<C::BETA>(pb_);
         float mult;
         uint32_t sc;
         if constexpr (FMT == HIFA4_NVFP4) {
-          const float t = __fmul_rn(__fdiv_rn(bmax, 6.0f), kInvGP);
+          const float t = __fmul_rn(div6_rn(bmax), kInvGP);   // fl32(amax/6) / g_P
           sc = cvt_e4m3(t);
-          const float sd = __fmul_rn(ue4m3_to_f32(sc), kGP);
-          mult = sc == 0 ? 0.0f : __fdiv_rn(1.0f, sd);
+          mult = inv_tab[sc];                                  // fl32(1/(scale*g_P)), 0 for scale 0
         } else {
           const uint32_t ef = (__float_as_uint(bmax) >> 23) & 0xFFu;
           sc = ef >= 2u ? ef - 2u : 0u;
           mult = __uint_as_float((254u - sc) << 23);
         }
+        const float2 m2 = make_float2(mult, mult);
 #pragma unroll
         for (int w = 0; w < C::BETA / 8; ++w) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int k = blk * C::BETA + w * 8 + 2 * q;
-            word |= cvt_e2m1x2(__fmul_rn(s[k + 1], mult), __fmul_rn(s[k], mult)) << (8 * q);
-          }
-          codes[blk * (C::BETA / 8) + w] = word;
+          const float* e = pb_ + 8 * w;
+          codes[blk * (C::BETA / 8) + w] =
+              cvt_e2m1x8(fmul2(make_float2(e[0], e[1]), m2), fmul2(make_float2(e[2], e[3]), m2),
+                         fmul2(make_float2(e[4], e[5]), m2), fmul2(make_float2(e[6], e[7]), m2));
         }
         scw[blk / 4] |= sc << (8 * (blk % 4));
-        if (want_lp) {
-#pragma unroll
-          for (int i = 0; i < C::BETA; ++i) psum += s[blk * C::BETA + i];
-        }
+        if (want_lp) psum += tree_sum<C::BETA>(pb_);
       }
       if (want_lp) l_p = fmaf(alpha, l_p, psum);
       // the P-hat buffer pb was last read by PV_{j-2}
@@ -418,12 +466,25 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
 #pragma unroll
-        for (int cc = 0; cc < D / 16; ++cc) {
-          uint32_t v[16];
-          tmem_ld16_wait(tmem + lane_base + C::TM_O + cc * 16, v);
+        for (int cc = 0; cc < D / 64; ++cc) {
+          uint32_t v0[32], v1[32];
+          const uint32_t a0 = tmem + lane_base + C::TM_O + cc * 64;
+          tmem_ld32(a0, v0);
+          tmem_ld32(a0 + 32, v1);
+          tmem_wait_ld_dep(v0);
+          tmem_wait_ld_dep(v1);
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-          tmem_st16(tmem + lane_base + C::TM_O + cc * 16, v);
+          for (int i = 0; i < 32; i += 2) {
+            float2 t0 = fmul2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), a2);
+            float2 t1 = fmul2(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), a2);
+            v0[i] = __float_as_uint(t0.x);
+            v0[i + 1] = __float_as_uint(t0.y);
+            v1[i] = __float_as_uint(t1.x);
+            v1[i + 1] = __float_as_uint(t1.y);
+          }
+          tmem_st32(a0, v0);
+          tmem_st32(a0 + 32, v1);
         }
         uint32_t lv;
         tmem_ld1_wait(tmem + lane_base + C::TM_L, lv);
@@ -486,7 +547,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, 512);
+  if (warp == 5) tmem_dealloc(tmem, C::TMEM_ALLOC);
 }
 
 // ------------------------------------------------------------------ host ---
@@ -506,9 +567,7 @@ static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const ui
     return HIFA4_ERR_CUDA;
   }
   auto kern = attn_fwd_fp4_kernel<D, BN, FMT, PRE>;
-  // The kernel owns all 512 TMEM columns: request enough shared memory that
-  // only one CTA is resident per SM (a second would stall in tcgen05.alloc).
-  const int smem = C::SMEM_BYTES > 116 * 1024 ? C::SMEM_BYTES : 116 * 1024;
+  const int smem = C::SMEM_REQ;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * p.num_qtiles;
   kern<<<grid, 192, smem, st>>>(tq, tk, tv, p);

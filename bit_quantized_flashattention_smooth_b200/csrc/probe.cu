@@ -159,6 +159,25 @@ __global__ void convert_probe_kernel(const float* __restrict__ x, int64_t n, uin
   }
 }
 
+// Every float bit pattern in [lo, hi): count where div6_rn differs from the
+// IEEE quotient; record the smallest failing pattern.
+__global__ void div6_probe_kernel(uint32_t lo, uint32_t hi, unsigned long long* count, uint32_t* first_bad) {
+  for (uint64_t b = lo + static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < hi;
+       b += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    const float a = __uint_as_float(static_cast<uint32_t>(b));
+    if (__float_as_uint(div6_rn(a)) != __float_as_uint(__fdiv_rn(a, 6.0f))) {
+      atomicAdd(count, 1ull);
+      atomicMin(first_bad, static_cast<uint32_t>(b));
+    }
+  }
+}
+
+hifa4_status div6_probe_launch(uint32_t lo, uint32_t hi, unsigned long long* count, uint32_t* first_bad,
+                               cudaStream_t st) {
+  div6_probe_kernel<<<148 * 16, 256, 0, st>>>(lo, hi, count, first_bad);
+  return launch_status("div6_probe");
+}
+
 hifa4_status convert_probe_launch(const float* x, int64_t n, uint8_t* e2m1, uint8_t* e4m3, cudaStream_t st) {
   convert_probe_kernel<<<148 * 8, 256, 0, st>>>(x, n, e2m1, e4m3);
   return launch_status("convert_probe");

@@ -64,11 +64,11 @@ def _lowfreq_pairs(d: int, npairs: int) -> tuple:
 WORKLOADS = {
     "tiny_mha": Workload("tiny_mha", 1, 2, 2, 256, 64, False, "fp16", 0, 64, 64, None,
                          (60, 61, 62, 63), 20.0),
-    "qwen3_prefill": Workload("qwen3_prefill", 1, 32, 8, 4096, 128, True, "bf16", 1, 256, 128, 1e6,
+    "qwen3_prefill": Workload("qwen3_prefill", 1, 32, 8, 4096, 128, True, "bf16", 1, 256, 64, 1e6,
                               _lowfreq_pairs(128, 3), 15.0),
     "gemma2_prefill": Workload("gemma2_prefill", 1, 16, 8, 8192, 256, True, "bf16", 2, 256, 128, 1e4,
                                _lowfreq_pairs(256, 4), 10.0),
-    "long_prefill": Workload("long_prefill", 8, 32, 8, 16384, 128, True, "bf16", 3, 256, 128, 1e6,
+    "long_prefill": Workload("long_prefill", 8, 32, 8, 16384, 128, True, "bf16", 3, 256, 64, 1e6,
                              (), 0.0, "student_t3"),
     "split_decode": Workload("split_decode", 64, 32, 8, 32768, 128, False, "bf16", 4, 256, 128, 1e6,
                              _lowfreq_pairs(128, 3), 15.0, decode=True),

@@ -57,6 +57,18 @@ def test_hw_conversions_match_written_rounding():
     assert bad.size == 0, f"E4M3: {bad.size} mismatches e.g. x={x[bad[:8]]} gpu={e4_gpu[bad[:8]]} ref={e4_ref[bad[:8]]}"
 
 
+def test_fast_div6_is_ieee_division():
+    """The P-hat scale path computes fl32(amax/6) without a division; it must
+    equal IEEE division for zero and every float in [2^-122, 2^20] (quotients
+    that are normal).  Below 2^-122 the scale code is 0 either way: the
+    quotient times 2^8 is under 2^-116, far below half the smallest UE4M3
+    subnormal."""
+    n, first = h.div6_probe(0x02800000, 0x49800000)
+    assert n == 0, f"{n} mismatches, first at bits {first:#x}"
+    n0, _ = h.div6_probe(0, 1)
+    assert n0 == 0
+
+
 # --------------------------------------------------------------- FP4 MMA ---
 @pytest.mark.parametrize("fmt", [oracle.NVFP4, oracle.MXFP4])
 @pytest.mark.parametrize("n,k", [(128, 128), (64, 128), (256, 256), (128, 256)])
