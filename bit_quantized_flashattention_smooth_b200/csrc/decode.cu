@@ -1,22 +1,534 @@
-// decode.cu -- split-KV decode over the 4-bit KV cache (placeholder until the
-// swap-AB tcgen05 decode kernel lands).
+// decode.cu -- split-KV decode over a 4-bit KV cache, and the split combine.
+//
+// Method: the prefill recurrence of "HiFA4: Training-Free 4-bit FlashAttention
+// on Ascend HIF4 NPUs for LLM Inference" (Abstract paras 1-2) for one query
+// per head: Smooth-QK-scaled query quantized to 4 bits, S = Q-hat K-hat^T and
+// O += P-hat V-hat as block-scaled FP4 GEMMs, online softmax, and under
+// P-Reordering the normalizer accumulated from the same P-hat inside the PV
+// GEMM.  Keys are split into chunks that run in parallel and are merged with
+// their log-sum-exp weights.
+//
+// B200 design, one CTA per (batch, kv head, split), "swap AB": the 128 keys of
+// a tile are the M dimension of the MMA and the G query heads of the group
+// (padded to N = 16) are the N dimension, so the tensor core is not wasted on
+// 127 empty query rows:
+//   S^T [128 keys x 16]   = K-hat tile (A, from the cache by TMA) x Q-hat^T (B)
+//   O^T [128 ch   x 16]  += V-hat^T tile (A, channel-major cache) x P-hat^T (B)
+//   L^T [128      x 16]  += ones (A) x P-hat^T (B)      (fused normalizer)
+// The softmax warps hold one key per thread (TMEM lane) and reduce across keys
+// with warp shuffles plus a 4-warp exchange in shared memory.  The kernel is
+// bound by HBM: it streams each K/V tile once through a 3-stage TMA ring.
 #include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace hifa4 {
 
+struct DecodeParams {
+  const void* q;        // [B][Hq][d] bf16/fp16
+  const float* s;       // [Hkv][d] or null
+  const uint8_t* k_sf;
+  const uint8_t* v_sf;
+  int64_t sf_k_head, sf_v_head;
+  int B, Hq, Hkv, G, kv_len, Np, split_len, splits;
+  int q_fp16;
+  float c_log2;
+  float* ws;            // [B][Hq][splits][d+2]: acc (true units), m, l
+};
+
+template <int FMT>
+struct DecCfg {
+  static constexpr int D = 128, BN = 128, NQ = 16;          // head dim, keys per tile, padded queries
+  static constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
+  static constexpr int NS = 3;
+  static constexpr int ROW = 64;                            // bytes per 128-element 4-bit row
+  static constexpr int NKC = (D / BETA + 3) / 4;            // scale chunks per 128 keys / 128 channels
+  static constexpr int SZ_K = BN * ROW, SZ_V = D * ROW, SZ_QB = NQ * ROW, SZ_ONES = 128 * ROW;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + NS * SZ_K;
+  static constexpr int OFF_ONES = OFF_V + NS * SZ_V;
+  static constexpr int OFF_Q = OFF_ONES + SZ_ONES;
+  static constexpr int OFF_P = OFF_Q + SZ_QB;                // 2 buffers
+  static constexpr int OFF_KSF = OFF_P + 2 * SZ_QB;
+  static constexpr int OFF_VSF = OFF_KSF + NS * NKC * 512;
+  static constexpr int OFF_QSF = OFF_VSF + NS * NKC * 512;
+  static constexpr int OFF_PSF = OFF_QSF + NKC * 512;        // 2 buffers
+  static constexpr int OFF_ONESF = OFF_PSF + 2 * NKC * 512;
+  static constexpr int OFF_RED = OFF_ONESF + 512;            // [2][4 warps][16] floats (max), same for sums
+  static constexpr int OFF_INV = OFF_RED + 2 * 2 * 4 * 16 * 4;
+  static constexpr int OFF_BAR = OFF_INV + 512;
+  static constexpr int NBAR = 4 * NS + 2 * 2 + 2 * 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // TMEM columns
+  static constexpr int TM_S = 0;            // 2 x 16
+  static constexpr int TM_O = 32;
+  static constexpr int TM_L = 48;
+  static constexpr int TM_SFK = 64;         // 4 * NKC
+  static constexpr int TM_SFQ = TM_SFK + 4 * NKC;
+  static constexpr int TM_SFV = TM_SFQ + 4 * NKC;
+  static constexpr int TM_SFP = TM_SFV + 4 * NKC;
+  static constexpr int TM_SF1 = TM_SFP + 4 * NKC;
+  static constexpr int TMEM_ALLOC = 128;
+  static_assert(TM_SF1 + 4 <= TMEM_ALLOC, "TMEM budget");
+  static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
+};
+
+__device__ __forceinline__ uint32_t swz64(uint32_t r, uint32_t c) { return c ^ ((r >> 1) & 3); }
+
+template <int FMT, bool PREORDER>
+__global__ void __launch_bounds__(192, 2)
+    attn_decode_fp4_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                           const DecodeParams p) {
+  using C = DecCfg<FMT>;
+  constexpr bool MX = FMT == HIFA4_MXFP4;
+  extern __shared__ __align__(1024) unsigned char smem_dyn[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  const int B_KFULL = 0, B_KEMPTY = C::NS, B_VFULL = 2 * C::NS, B_VEMPTY = 3 * C::NS, B_SFULL = 4 * C::NS,
+            B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2, B_PEMPTY = B_PFULL + 2, B_ORDY = B_PEMPTY + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+
+  const int sp = blockIdx.x % p.splits;
+  const int bh = blockIdx.x / p.splits;      // b * Hkv + h
+  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  const int k_begin = sp * p.split_len;
+  const int k_end = min(p.kv_len, k_begin + p.split_len);
+  const int ntile = (k_end - k_begin + C::BN - 1) / C::BN;
+  const float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;
+
+  // ---------------------------------------------------------------- setup ---
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(BAR(B_KFULL + s), 1);
+      mbar_init(BAR(B_KEMPTY + s), 1);
+      mbar_init(BAR(B_VFULL + s), 1);
+      mbar_init(BAR(B_VEMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(B_SFULL + s), 1);
+      mbar_init(BAR(B_SEMPTY + s), 4);
+      mbar_init(BAR(B_PFULL + s), 4);
+      mbar_init(BAR(B_PEMPTY + s), 1);
+    }
+    mbar_init(BAR(B_ORDY), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // ones A operand (128 rows of E2M1 1.0) and its scale chunk (1.0 on every row)
+  for (int i = threadIdx.x; i < C::SZ_ONES / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(smem + C::OFF_ONES)[i] = 0x22222222u;
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+    reinterpret_cast<uint32_t*>(smem + C::OFF_ONESF)[i] = (FMT == HIFA4_NVFP4 ? 0x38u : 0x7Fu) * 0x01010101u;
+    const float sd = __fmul_rn(ue4m3_to_f32(i), kGP);
+    reinterpret_cast<float*>(smem + C::OFF_INV)[i] = i == 0 ? 0.0f : __fdiv_rn(1.0f, sd);
+  }
+  // the query rows of this group: fl32(q * s) quantized along d (B operand,
+  // 16 rows, rows >= G are zero) and its scale chunk(s)
+  for (int i = threadIdx.x; i < (C::SZ_QB + C::NKC * 512) / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(smem + (i < C::SZ_QB / 4 ? C::OFF_Q : C::OFF_QSF - C::SZ_QB))[i] = 0u;
+  __syncthreads();
+  if (warp == 0) {
+    const int nblk = p.G * (C::D / C::BETA);
+    for (int t = lane; t < nblk; t += 32) {
+      const int g = t / (C::D / C::BETA), blk = t % (C::D / C::BETA);
+      const int hq = h * p.G + g;
+      float v[C::BETA];
+      for (int i = 0; i < C::BETA; ++i) {
+        const int c = blk * C::BETA + i;
+        const int64_t off = (static_cast<int64_t>(b) * p.Hq + hq) * C::D + c;
+        float x = p.q_fp16 ? __half2float(reinterpret_cast<const __half*>(p.q)[off])
+                           : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.q)[off]);
+        v[i] = p.s ? __fmul_rn(x, p.s[h * C::D + c]) : x;
+      }
+      float amax = 0.0f;
+      for (int i = 0; i < C::BETA; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      uint32_t sc;
+      float mult;
+      if constexpr (FMT == HIFA4_NVFP4) {
+        sc = cvt_e4m3(__fdiv_rn(amax, 6.0f));
+        mult = sc == 0 ? 0.0f : __fdiv_rn(1.0f, ue4m3_to_f32(sc));
+      } else {
+        const uint32_t ef = (__float_as_uint(amax) >> 23) & 0xFFu;
+        sc = ef >= 2u ? ef - 2u : 0u;
+        mult = __uint_as_float((254u - sc) << 23);
+      }
+      for (int i = 0; i < C::BETA; i += 2) {
+        uint32_t byte = cvt_e2m1x2(__fmul_rn(v[i + 1], mult), __fmul_rn(v[i], mult));
+        if (FMT == HIFA4_NVFP4 && sc == 0) byte = 0;
+        const int kb = (blk * C::BETA + i) / 2;   // byte in the 64-byte row
+        smem[C::OFF_Q + g * C::ROW + swz64(g, kb >> 4) * 16 + (kb & 15)] = static_cast<unsigned char>(byte);
+      }
+      smem[C::OFF_QSF + (blk / 4) * 512 + g * 16 + (blk % 4)] = static_cast<unsigned char>(sc);
+    }
+  }
+  fence_proxy_async_smem();
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      const int nkc_v_row = p.Np / (4 * C::BETA);
+      for (int j = 0; j < ntile; ++j) {
+        const int st = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        const int key0 = k_begin + j * C::BN;
+        if (!mbar_wait(BAR(B_KEMPTY + st), ph ^ 1, abort_flag, kErrTimeoutTma)) break;
+        mbar_arrive_expect_tx(BAR(B_KFULL + st), C::SZ_K + C::NKC * 512);
+        tma_load_2d(sbase + C::OFF_K + st * C::SZ_K, &tm_k, 0, bh * p.Np + key0, BAR(B_KFULL + st));
+        bulk_load(sbase + C::OFF_KSF + st * C::NKC * 512,
+                  p.k_sf + bh * p.sf_k_head + static_cast<int64_t>(key0 >> 7) * C::NKC * 512, C::NKC * 512,
+                  BAR(B_KFULL + st));
+        if (!mbar_wait(BAR(B_VEMPTY + st), ph ^ 1, abort_flag, kErrTimeoutTma)) break;
+        mbar_arrive_expect_tx(BAR(B_VFULL + st), C::SZ_V + C::NKC * 512);
+        tma_load_2d(sbase + C::OFF_V + st * C::SZ_V, &tm_v, key0 / 2, bh * C::D, BAR(B_VFULL + st));
+        bulk_load(sbase + C::OFF_VSF + st * C::NKC * 512,
+                  p.v_sf + bh * p.sf_v_head + static_cast<int64_t>(key0 / (4 * C::BETA)) * 512, C::NKC * 512,
+                  BAR(B_VFULL + st));
+        (void)nkc_v_row;
+      }
+    }
+  } else if (warp == 5) {
+    // ================================= MMA issuer =================================
+    if (lane == 0) {
+      auto mma = [&](uint32_t d_t, uint64_t a, uint64_t bd, uint32_t idesc, uint32_t sfa, uint32_t sfb, uint32_t acc) {
+        if constexpr (MX) mma_mxfp4(d_t, a, bd, idesc, sfa, sfb, acc);
+        else mma_nvfp4(d_t, a, bd, idesc, sfa, sfb, acc);
+      };
+      bool ok = true;
+      tc_fence_after();
+      for (int kc = 0; kc < C::NKC; ++kc)
+        tc_cp_32x128b_warpx4(tmem + C::TM_SFQ + 4 * kc, make_sf_desc(sbase + C::OFF_QSF + kc * 512));
+      tc_cp_32x128b_warpx4(tmem + C::TM_SF1, make_sf_desc(sbase + C::OFF_ONESF));
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        const int sb = j & 1;
+        if (!mbar_wait(BAR(B_KFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
+        if (!mbar_wait(BAR(B_SEMPTY + sb), ((j >> 1) & 1) ^ 1, abort_flag, kErrTimeoutMma)) return false;
+        tc_fence_after();
+        for (int kc = 0; kc < C::NKC; ++kc)
+          tc_cp_32x128b_warpx4(tmem + C::TM_SFK + 4 * kc, make_sf_desc(sbase + C::OFF_KSF + (st * C::NKC + kc) * 512));
+#pragma unroll
+        for (int ks = 0; ks < C::D / 64; ++ks) {
+          const uint32_t chunk = MX ? ks / 2 : ks, byte = MX ? 2 * (ks % 2) : 0;
+          mma(tmem + C::TM_S + sb * C::NQ, make_kmajor_desc(sbase + C::OFF_K + st * C::SZ_K + ks * 32, C::ROW),
+              make_kmajor_desc(sbase + C::OFF_Q + ks * 32, C::ROW), idesc_fp4(128, C::NQ, MX, byte, byte),
+              (tmem + C::TM_SFK + 4 * chunk) | (byte << 30), (tmem + C::TM_SFQ + 4 * chunk) | (byte << 30),
+              ks > 0 ? 1u : 0u);
+        }
+        tc_commit(BAR(B_SFULL + sb));
+        tc_commit(BAR(B_KEMPTY + st));
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int st = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        const int pb = j & 1;
+        if (!mbar_wait(BAR(B_PFULL + pb), (j >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
+        if (!mbar_wait(BAR(B_VFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
+        tc_fence_after();
+        for (int kc = 0; kc < C::NKC; ++kc) {
+          tc_cp_32x128b_warpx4(tmem + C::TM_SFV + 4 * kc, make_sf_desc(sbase + C::OFF_VSF + (st * C::NKC + kc) * 512));
+          tc_cp_32x128b_warpx4(tmem + C::TM_SFP + 4 * kc, make_sf_desc(sbase + C::OFF_PSF + (pb * C::NKC + kc) * 512));
+        }
+#pragma unroll
+        for (int ks = 0; ks < C::BN / 64; ++ks) {
+          const uint32_t chunk = MX ? ks / 2 : ks, byte = MX ? 2 * (ks % 2) : 0;
+          const uint64_t bp = make_kmajor_desc(sbase + C::OFF_P + pb * C::SZ_QB + ks * 32, C::ROW);
+          const uint32_t sfp = (tmem + C::TM_SFP + 4 * chunk) | (byte << 30);
+          const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+          mma(tmem + C::TM_O, make_kmajor_desc(sbase + C::OFF_V + st * C::SZ_V + ks * 32, C::ROW), bp,
+              idesc_fp4(128, C::NQ, MX, byte, byte), (tmem + C::TM_SFV + 4 * chunk) | (byte << 30), sfp, acc);
+          mma(tmem + C::TM_L, make_kmajor_desc(sbase + C::OFF_ONES + ks * 32, C::ROW), bp,
+              idesc_fp4(128, C::NQ, MX, byte, byte), (tmem + C::TM_SF1) | (byte << 30), sfp, acc);
+        }
+        tc_commit(BAR(B_ORDY));
+        tc_commit(BAR(B_VEMPTY + st));
+        tc_commit(BAR(B_PEMPTY + pb));
+        return true;
+      };
+      if (ntile > 0) ok = issue_s(0);
+      for (int j = 0; ok && j < ntile; ++j) {
+        if (j + 1 < ntile) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
+      }
+      if (!ok) drain_after_abort();
+    }
+  } else {
+    // ================================== softmax ==================================
+    // thread t = key t of the tile = TMEM lane t; columns = the group's queries
+    const int t = threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
+    float m[C::NQ], lp[C::NQ];
+#pragma unroll
+    for (int q = 0; q < C::NQ; ++q) {
+      m[q] = -INFINITY;
+      lp[q] = 0.0f;
+    }
+    const bool want_lp = !PREORDER;
+    bool ok = true;
+    for (int j = 0; j < ntile && ok; ++j) {
+      const int sb = j & 1, pb = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + sb), (j >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[16];
+      tmem_ld16_wait(tmem + lane_base + C::TM_S + sb * C::NQ, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_SEMPTY + sb));
+      const bool valid = k_begin + j * C::BN + t < k_end;
+      float x[C::NQ];
+#pragma unroll
+      for (int q = 0; q < C::NQ; ++q) x[q] = valid && q < p.G ? __fmul_rn(__uint_as_float(v[q]), p.c_log2) : -INFINITY;
+      // tile max per query: warp shuffle, then across the 4 warps
+      float* rbuf = red + (j & 1) * 2 * 4 * 16;
+#pragma unroll
+      for (int q = 0; q < C::NQ; ++q) {
+        float mx = x[q];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == q) rbuf[warp * 16 + q] = mx;
+      }
+      named_bar_sync(1, 128);
+      float alpha[C::NQ], mnew[C::NQ];
+#pragma unroll
+      for (int q = 0; q < C::NQ; ++q) {
+        const float tm = fmaxf(fmaxf(rbuf[q], rbuf[16 + q]), fmaxf(rbuf[32 + q], rbuf[48 + q]));
+        mnew[q] = fmaxf(m[q], tm);
+        alpha[q] = (mnew[q] == m[q]) ? 1.0f : ex2_approx(m[q] - mnew[q]);
+      }
+      // P-hat buffer pb was last read by PV_{j-2}
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(BAR(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, abort_flag,
+                                                        kErrTimeoutSoftmax))) {
+        ok = false;
+        break;
+      }
+      unsigned char* pbuf = smem + C::OFF_P + pb * C::SZ_QB;
+      unsigned char* psf = smem + C::OFF_PSF + pb * C::NKC * 512;
+      float psum[C::NQ];
+#pragma unroll
+      for (int q = 0; q < C::NQ; ++q) {
+        const float pr = (q < p.G) ? ex2_approx(__fsub_rn(x[q], mnew[q])) : 0.0f;
+        psum[q] = pr;
+        // block amax over BETA consecutive keys (lanes)
+        float bm = pr;
+#pragma unroll
+        for (int o = C::BETA / 2; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        uint32_t sc;
+        float mult;
+        if constexpr (FMT == HIFA4_NVFP4) {
+          sc = cvt_e4m3(__fmul_rn(div6_rn(bm), 256.0f));
+          mult = inv_tab[sc];
+        } else {
+          const uint32_t ef = (__float_as_uint(bm) >> 23) & 0xFFu;
+          sc = ef >= 2u ? ef - 2u : 0u;
+          mult = __uint_as_float((254u - sc) << 23);
+        }
+        const float y = __fmul_rn(pr, mult);
+        const float y_odd = __shfl_down_sync(0xffffffffu, y, 1);
+        if ((t & 1) == 0) {
+          const uint32_t byte = cvt_e2m1x2(y_odd, y);
+          const int kb = t >> 1;
+          pbuf[q * C::ROW + swz64(q, kb >> 4) * 16 + (kb & 15)] = static_cast<unsigned char>(byte);
+        }
+        if ((t % C::BETA) == 0) {
+          const int blk = t / C::BETA;
+          psf[(blk / 4) * 512 + q * 16 + (blk % 4)] = static_cast<unsigned char>(sc);
+        }
+      }
+      if (want_lp) {
+        float* sbuf = rbuf + 4 * 16;
+#pragma unroll
+        for (int q = 0; q < C::NQ; ++q) {
+          float sm = psum[q];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+          if (lane == q) sbuf[warp * 16 + q] = sm;
+        }
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int q = 0; q < C::NQ; ++q)
+          lp[q] = fmaf(alpha[q], lp[q], (sbuf[q] + sbuf[16 + q]) + (sbuf[32 + q] + sbuf[48 + q]));
+      }
+      // rescale O^T and L^T columns whose max rose (after PV_{j-1} retired)
+      bool any = false;
+#pragma unroll
+      for (int q = 0; q < C::NQ; ++q) any |= alpha[q] != 1.0f;
+      if (j > 0 && any) {
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_ORDY), (j - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t o[16], l[16];
+        tmem_ld16_wait(tmem + lane_base + C::TM_O, o);
+        tmem_ld16_wait(tmem + lane_base + C::TM_L, l);
+#pragma unroll
+        for (int q = 0; q < C::NQ; ++q) {
+          o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
+          l[q] = __float_as_uint(__uint_as_float(l[q]) * alpha[q]);
+        }
+        tmem_st16(tmem + lane_base + C::TM_O, o);
+        tmem_st16(tmem + lane_base + C::TM_L, l);
+        tmem_wait_st();
+      }
+#pragma unroll
+      for (int q = 0; q < C::NQ; ++q) m[q] = mnew[q];
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_PFULL + pb));
+    }
+    // ------------------------------------------------------------- epilogue ---
+    const bool ready = __all_sync(0xffffffffu, ok && ntile > 0 &&
+                                                  mbar_wait(BAR(B_ORDY), (ntile - 1) & 1, abort_flag, kErrTimeoutSoftmax));
+    if (ready) {
+      tc_fence_after();
+      uint32_t o[16], l[16];
+      tmem_ld16_wait(tmem + lane_base + C::TM_O, o);
+      tmem_ld16_wait(tmem + lane_base + C::TM_L, l);
+      const int c = t;  // TMEM lane = output channel
+      for (int q = 0; q < p.G; ++q) {
+        const int hq = h * p.G + q;
+        float* w = p.ws + ((static_cast<int64_t>(b) * p.Hq + hq) * p.splits + sp) * (C::D + 2);
+        w[c] = __uint_as_float(o[q]) * kGP;
+        if (c == 0) {
+          w[C::D] = m[q];
+          w[C::D + 1] = PREORDER ? __uint_as_float(l[q]) * kGP : lp[q];
+        }
+      }
+    }
+  }
+  if (*abort_flag) drain_after_abort();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, C::TMEM_ALLOC);
+}
+
+// Merge the splits of each (b, hq): O = sum w_s acc_s / sum w_s l_s with
+// w_s = 2^(m_s - max m).  One warp per query row, d = 128 (4 channels/lane).
+__global__ void decode_combine_kernel(const float* __restrict__ ws, int rows, int splits, int d, void* o, int o_fp16) {
+  const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float* base = ws + static_cast<int64_t>(row) * splits * (d + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, base[s * (d + 2) + d]);
+  float den = 0.0f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < splits; ++s) {
+    const float* w = base + s * (d + 2);
+    const float ms = w[d];
+    if (ms == -INFINITY) continue;
+    const float wt = exp2f(ms - M);
+    den = fmaf(wt, w[d + 1], den);
+    for (int i = 0; i < 4; ++i) acc[i] = fmaf(wt, w[lane * 4 + i], acc[i]);
+  }
+  const float inv = 1.0f / den;
+  for (int i = 0; i < 4; ++i) {
+    const int64_t off = static_cast<int64_t>(row) * d + lane * 4 + i;
+    if (o_fp16) reinterpret_cast<__half*>(o)[off] = __float2half_rn(acc[i] * inv);
+    else reinterpret_cast<__nv_bfloat16*>(o)[off] = __float2bfloat16_rn(acc[i] * inv);
+  }
+}
+
+bool make_tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_inner,
+                  uint32_t box_rows, int swizzle_bytes);
+
 int decode_default_splits(int B, int Hkv, int kv_len, int block_n) {
+  // enough CTAs for several waves over 148 SMs (2 resident each), each split
+  // keeping at least 16 key tiles to amortize the per-CTA setup
   const int tiles = (kv_len + block_n - 1) / block_n;
   int splits = 1;
-  while (static_cast<int64_t>(B) * Hkv * splits < 2 * 148 && splits * 2 <= tiles) splits *= 2;
+  while (static_cast<int64_t>(B) * Hkv * splits < 8 * 148 * 2 && (tiles / (splits * 2)) >= 16) splits *= 2;
   return splits;
 }
 
-hifa4_status decode_launch(const void*, int, const float*, const uint8_t*, const uint8_t*, const uint8_t*,
-                           const uint8_t*, int, int, int, int, int, int, float, int, int, int, int*, void*, size_t,
-                           void*, int, cudaStream_t) {
-  set_last_error("attn_decode: not built yet");
-  return HIFA4_ERR_UNSUPPORTED;
+template <int FMT, bool PRE>
+static hifa4_status launch_decode_t(const uint8_t* kc, const uint8_t* vc, const DecodeParams& p, cudaStream_t st) {
+  using C = DecCfg<FMT>;
+  CUtensorMap tk, tv;
+  const uint64_t Np = static_cast<uint64_t>(p.Np);
+  if (!make_tmap_2d(&tk, kc, C::D / 2, static_cast<uint64_t>(p.B) * p.Hkv * Np, C::D / 2, C::BN, C::D / 2) ||
+      !make_tmap_2d(&tv, vc, Np / 2, static_cast<uint64_t>(p.B) * p.Hkv * C::D, C::BN / 2, C::D, C::BN / 2)) {
+    set_last_error("cuTensorMapEncodeTiled failed");
+    return HIFA4_ERR_CUDA;
+  }
+  auto kern = attn_decode_fp4_kernel<FMT, PRE>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  kern<<<static_cast<unsigned>(p.B) * p.Hkv * p.splits, 192, C::SMEM_BYTES, st>>>(tk, tv, p);
+  return launch_status("attn_decode");
+}
+
+hifa4_status decode_launch(const void* q, int q_dt, const float* s, const uint8_t* kc, const uint8_t* ks,
+                           const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int kv_len, int d, int fmt,
+                           float softmax_scale, int mode, int block_n, int num_splits, int* num_splits_used,
+                           void* workspace, size_t ws_bytes, void* o, int o_dt, cudaStream_t st) {
+  if (num_splits == 0) num_splits = decode_default_splits(B, Hkv, kv_len, block_n);
+  const int tiles = (kv_len + block_n - 1) / block_n;
+  if (num_splits > tiles) num_splits = tiles;
+  const int split_len = ((kv_len + num_splits - 1) / num_splits + block_n - 1) / block_n * block_n;
+  const int used = (kv_len + split_len - 1) / split_len;
+  if (ws_bytes < static_cast<size_t>(B) * Hq * used * (d + 2) * sizeof(float)) {
+    set_last_error("attn_decode: workspace too small (%zu bytes)", ws_bytes);
+    return HIFA4_ERR_INVALID_ARG;
+  }
+  DecodeParams p;
+  p.q = q;
+  p.s = s;
+  p.k_sf = ks;
+  p.v_sf = vs;
+  p.Np = static_cast<int>(pad128(kv_len));
+  p.sf_k_head = static_cast<int64_t>(hifa4_scale_bytes(kv_len, d, static_cast<hifa4_format>(fmt)));
+  p.sf_v_head = static_cast<int64_t>(hifa4_scale_bytes(d, p.Np, static_cast<hifa4_format>(fmt)));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.kv_len = kv_len;
+  p.split_len = split_len;
+  p.splits = used;
+  p.q_fp16 = q_dt == HIFA4_FP16;
+  p.c_log2 = softmax_scale * 1.4426950408889634f;
+  p.ws = static_cast<float*>(workspace);
+  hifa4_status r;
+  if (fmt == HIFA4_NVFP4)
+    r = mode == HIFA4_NORM_PREORDER ? launch_decode_t<HIFA4_NVFP4, true>(kc, vc, p, st)
+                                    : launch_decode_t<HIFA4_NVFP4, false>(kc, vc, p, st);
+  else
+    r = mode == HIFA4_NORM_PREORDER ? launch_decode_t<HIFA4_MXFP4, true>(kc, vc, p, st)
+                                    : launch_decode_t<HIFA4_MXFP4, false>(kc, vc, p, st);
+  if (r != HIFA4_OK) return r;
+  const int rows = B * Hq;
+  decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(p.ws, rows, used, d, o, o_dt == HIFA4_FP16);
+  if (num_splits_used) *num_splits_used = used;
+  return launch_status("decode_combine");
 }
 
 }  // namespace hifa4

@@ -168,3 +168,36 @@ def test_theorem1_coherence_on_gpu():
     assert np.max(np.abs(o_i - pred)) <= 2e-3 * np.max(np.abs(o_r)) + 1e-3
     eps = ratio - 1
     assert np.median(eps) < 0
+
+
+# ----------------------------------------------------------------- decode ---
+DECODE_CASES = [
+    # B, Hq, Hkv, kv_len, fmt, mode, splits, q dtype
+    (2, 8, 2, 1000, oracle.NVFP4, oracle.PREORDER, 3, torch.bfloat16),
+    (2, 8, 2, 1000, oracle.NVFP4, oracle.INCONSISTENT, 1, torch.bfloat16),
+    (1, 8, 1, 777, oracle.MXFP4, oracle.PREORDER, 4, torch.float16),
+    (3, 4, 2, 2048, oracle.MXFP4, oracle.INCONSISTENT, 0, torch.bfloat16),
+    (1, 2, 2, 129, oracle.NVFP4, oracle.PREORDER, 2, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,kv,fmt,mode,splits,qdt", DECODE_CASES)
+def test_decode_matches_oracle(B, Hq, Hkv, kv, fmt, mode, splits, qdt):
+    d = 128
+    _, k, v = U.synthetic(B, Hq, Hkv, kv, d, seed=kv + Hq, dtype=torch.bfloat16)
+    g = np.random.Generator(np.random.PCG64(kv))
+    q = torch.from_numpy(g.standard_normal((B, Hq, d), dtype=np.float32)).to(qdt)
+    qcal = torch.from_numpy(g.standard_normal((B, Hq, 64, d), dtype=np.float32)).to(torch.bfloat16)
+    s_ref, inv_ref = oracle.calibrate(qcal.float().numpy(), k[:, :, :64].float().numpy(), n_cal=64)
+    cache = h.quantize_kv(k.cuda(), v.cuda(), torch.from_numpy(inv_ref).cuda(), fmt, Hq=Hq)
+    # cache bytes equal the oracle's
+    qz, tiled = U.oracle_quantize(torch.zeros((B, Hkv, kv, d)), k, v, np.ones_like(s_ref), inv_ref, fmt)
+    assert np.array_equal(U.to_np(cache.k_codes).astype(np.uint8), qz["k_codes"])
+    assert np.array_equal(U.to_np(cache.vt_codes).astype(np.uint8), qz["vt_codes"])
+    assert np.array_equal(U.to_np(cache.k_scales).astype(np.uint8), tiled["k_sc"])
+    assert np.array_equal(U.to_np(cache.vt_scales).astype(np.uint8), tiled["vt_sc"])
+    o, used = h.attn_decode(q.cuda(), torch.from_numpy(s_ref).cuda(), cache, kv, 1 / math.sqrt(d), mode, splits,
+                            out_dtype=torch.float32 if False else torch.bfloat16)
+    ref = oracle.decode(q.float().numpy(), s_ref, qz, kv, fmt, 1 / math.sqrt(d), mode, 128, num_splits=used)
+    ok, err, bound, cos = U.compare_out(U.to_np(o), ref["O"])
+    assert ok, f"splits={used} max|dO|={err:.3e} bound={bound:.3e} cos={cos:.6f}"
