@@ -33,6 +33,7 @@ ABI_FUNCTIONS = (
     "hifa4_codes_bytes", "hifa4_scale_bytes", "hifa4_calibrate_smooth_qk", "hifa4_quantize_qkv",
     "hifa4_quantize_kv",
     "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
+    "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
     "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
 )
@@ -60,6 +61,9 @@ def lib():
         L.hifa4_decode_default_splits.argtypes = [i, i, i, i]; L.hifa4_decode_default_splits.restype = i
         L.hifa4_attn_decode.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
                                         ctypes.POINTER(ctypes.c_int), vp, sz, vp, i, vp]
+        L.hifa4_decode_noalloc_max_bytes.argtypes = []; L.hifa4_decode_noalloc_max_bytes.restype = sz
+        L.hifa4_attn_decode_noalloc.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
+                                                ctypes.POINTER(ctypes.c_int), vp, i, vp]
         L.hifa4_fp4_mma_probe.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, vp]
         L.hifa4_convert_probe.argtypes = [vp, i64, vp, vp, vp]
         L.hifa4_div6_probe.argtypes = [ctypes.c_uint32, ctypes.c_uint32, vp, vp, vp]
@@ -247,6 +251,26 @@ def attn_decode(q: torch.Tensor, s: torch.Tensor | None, cache: QuantizedQKV, kv
                                    cache.fmt, float(softmax_scale), int(mode), 128, int(num_splits),
                                    ctypes.byref(used), _ptr(workspace), workspace.numel(), _ptr(o), _dt(o),
                                    _stream()), "attn_decode")
+    return o, used.value
+
+
+def attn_decode_noalloc(q: torch.Tensor, s: torch.Tensor | None, cache: QuantizedQKV, kv_len: int | None = None,
+                        softmax_scale: float | None = None, mode: int = PREORDER, num_splits: int = 0,
+                        out: torch.Tensor | None = None, out_dtype=torch.bfloat16):
+    """Split-KV decode that allocates nothing on the device: the split partials
+    live in the library's own scratch (for callers that may not allocate).
+    Returns (O, splits_used)."""
+    B, Hq, d = q.shape
+    kv = cache.N if kv_len is None else kv_len
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    o = out if out is not None else torch.empty((B, Hq, d), device=q.device, dtype=out_dtype)
+    used = ctypes.c_int(0)
+    q = q.contiguous()
+    _check(lib().hifa4_attn_decode_noalloc(_ptr(q), _dt(q), _ptr(s), _ptr(cache.k_codes), _ptr(cache.k_scales),
+                                           _ptr(cache.vt_codes), _ptr(cache.vt_scales), B, Hq, cache.Hkv, kv, d,
+                                           cache.fmt, float(softmax_scale), int(mode), 128, int(num_splits),
+                                           ctypes.byref(used), _ptr(o), _dt(o), _stream()), "attn_decode_noalloc")
     return o, used.value
 
 

@@ -532,3 +532,90 @@ hifa4_status decode_launch(const void* q, int q_dt, const float* s, const uint8_
 }
 
 }  // namespace hifa4
+
+// ---------------------------------------------------------------------------
+// Decode without any device allocation by the caller.
+//
+// Some callers cannot call cudaMalloc: an inference-server plugin or a custom
+// operator that is handed only its input and output buffers by the host
+// framework (whose caching allocator owns all device memory), or a latency-
+// critical serving loop where an allocation may block or synchronize the
+// device.  hifa4_attn_decode_noalloc serves them: the split partials live in a
+// library-owned scratch array in device global memory, declared below.  Every
+// GPU that loads this library holds this array until the process exits.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
+
+// The scratch itself.  In host code this symbol is only a host-side stand-in
+// for the device array: its device address must come from
+// cudaGetSymbolAddress on the device in question (see scratch_for_current).
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch on the current device, looked up once per
+// device (the first call on a device does this lookup).
+hifa4_status scratch_for_current(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    hifa4::set_last_error("attn_decode_noalloc: no usable current CUDA device");
+    return HIFA4_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      hifa4::set_last_error("attn_decode_noalloc: cudaGetSymbolAddress failed on device %d: %s", dev,
+                            cudaGetErrorString(e));
+      return HIFA4_ERR_CUDA;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return HIFA4_OK;
+}
+
+}  // namespace
+
+extern "C" HIFA4_API size_t hifa4_decode_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
+
+extern "C" HIFA4_API hifa4_status hifa4_attn_decode_noalloc(
+    const void* q, hifa4_dtype q_dt, const float* s, const uint8_t* k_codes, const uint8_t* k_scales,
+    const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq, int Hkv, int kv_len, int d, hifa4_format fmt,
+    float softmax_scale, hifa4_norm_mode mode, int block_n, int num_splits, int* num_splits_used, void* o,
+    hifa4_dtype o_dt, hifa4_stream_t stream) {
+  // Size of the split partials this call needs, computed as the decode does.
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || kv_len <= 0 || d <= 0 || num_splits < 0) {
+    hifa4::set_last_error("attn_decode_noalloc: bad shape");
+    return HIFA4_ERR_INVALID_ARG;
+  }
+  const int bn = 128;
+  int splits = num_splits == 0 ? hifa4::decode_default_splits(B, Hkv, kv_len, bn) : num_splits;
+  const int tiles = (kv_len + bn - 1) / bn;
+  if (splits > tiles) splits = tiles;
+  const int split_len = ((kv_len + splits - 1) / splits + bn - 1) / bn * bn;
+  const int used = (kv_len + split_len - 1) / split_len;
+  const size_t need = static_cast<size_t>(B) * Hq * used * (static_cast<size_t>(d) + 2) * sizeof(float);
+  if (need > kNoAllocScratchBytes) {
+    hifa4::set_last_error(
+        "attn_decode_noalloc: this call needs %zu bytes of split scratch but the library-owned scratch holds at "
+        "most %zu bytes; lower num_splits or the batch, or use hifa4_attn_decode with a caller workspace",
+        need, kNoAllocScratchBytes);
+    return HIFA4_ERR_INVALID_ARG;
+  }
+  void* scratch = nullptr;
+  hifa4_status st = scratch_for_current(&scratch);
+  if (st != HIFA4_OK) return st;
+  // Every split writes all of its partials before the combine reads them, so
+  // the scratch needs no clearing between calls.
+  return hifa4_attn_decode(q, q_dt, s, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, kv_len, d, fmt,
+                           softmax_scale, mode, block_n, num_splits, num_splits_used, scratch, kNoAllocScratchBytes, o,
+                           o_dt, stream);
+}

@@ -185,6 +185,33 @@ HIFA4_API hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const 
                                int* num_splits_used, void* workspace, size_t ws_bytes, void* o,
                                hifa4_dtype o_dt, hifa4_stream_t stream);
 
+/* Decode for callers that cannot allocate device memory.  (The paper has no
+ * counterpart; this is a deployment convenience of this library.)  Callers
+ * such as an inference-server plugin or a framework custom operator that is
+ * handed only its input and output buffers (the host framework's allocator
+ * owns all device memory), or a latency-critical serving loop where a device
+ * allocation may block or synchronize, cannot provide the workspace that
+ * hifa4_attn_decode needs.  This entry point takes the same arguments minus
+ * the workspace and keeps the split partials in a library-owned scratch array
+ * in device global memory of hifa4_decode_noalloc_max_bytes() (16 MiB), which
+ * every GPU that loads the library holds until the process exits.  It calls
+ * no allocation routine.  A call needing more scratch than that (B * Hq *
+ * splits_used * (d + 2) * 4 bytes) returns HIFA4_ERR_INVALID_ARG with the
+ * sizes in hifa4_last_error().  The first call on a device looks up the
+ * scratch's device address for that device (a CUDA runtime query), so make
+ * that first call before any stream capture.  All calls on a device share
+ * the one scratch array: calls that overlap on the GPU (concurrent streams)
+ * race on it and must be serialized by the caller.  The scratch keeps the last
+ * call's contents; nothing in it needs to start at zero. */
+HIFA4_API size_t hifa4_decode_noalloc_max_bytes(void);
+HIFA4_API hifa4_status hifa4_attn_decode_noalloc(const void* q, hifa4_dtype q_dt, const float* s,
+                                                 const uint8_t* k_codes, const uint8_t* k_scales,
+                                                 const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
+                                                 int Hkv, int kv_len, int d, hifa4_format fmt, float softmax_scale,
+                                                 hifa4_norm_mode mode, int block_n, int num_splits,
+                                                 int* num_splits_used, void* o, hifa4_dtype o_dt,
+                                                 hifa4_stream_t stream);
+
 /* -------------------------------------------------------- measurement --- */
 
 /* One 128 x n block-scaled FP4 product D = A B^T (K-major A [128][k], B [n][k]
