@@ -412,19 +412,23 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
 #pragma unroll
         for (int i = 0; i < C::BETA; i += 2) {
           const float2 y = fadd2(make_float2(pb_[i], pb_[i + 1]), negm);
-          pb_[i] = ex2_approx(y.x);
-          pb_[i + 1] = ex2_approx(y.y);
+          pb_[i] = y.x;
+          pb_[i + 1] = y.y;
         }
-        const float bmax = tree_max<C::BETA>(pb_);
         float mult;
         uint32_t sc;
         if constexpr (FMT == HIFA4_NVFP4) {
+#pragma unroll
+          for (int i = 0; i < C::BETA; ++i) pb_[i] = ex2_approx(pb_[i]);
+          const float bmax = tree_max<C::BETA>(pb_);
           const float t = __fmul_rn(div6_rn(bmax), kInvGP);   // fl32(amax/6) / g_P
           sc = cvt_e4m3(t);
           mult = inv_tab[sc];                                  // fl32(1/(scale*g_P)), 0 for scale 0
         } else {
-          const uint32_t ef = (__float_as_uint(bmax) >> 23) & 0xFFu;
-          sc = ef >= 2u ? ef - 2u : 0u;
+          // the shared exponent follows from the block maximum of y exactly
+          sc = mx_scale_from_ymax(tree_max<C::BETA>(pb_));
+#pragma unroll
+          for (int i = 0; i < C::BETA; ++i) pb_[i] = ex2_approx(pb_[i]);
           mult = __uint_as_float((254u - sc) << 23);
         }
         const float2 m2 = make_float2(mult, mult);

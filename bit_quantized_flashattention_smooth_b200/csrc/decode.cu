@@ -333,20 +333,24 @@ __global__ void __launch_bounds__(192, 2)
       float psum[C::NQ];
 #pragma unroll
       for (int q = 0; q < C::NQ; ++q) {
-        const float pr = (q < p.G) ? ex2_approx(__fsub_rn(x[q], mnew[q])) : 0.0f;
+        const float yq = (q < p.G) ? __fsub_rn(x[q], mnew[q]) : -INFINITY;
+        const float pr = ex2_approx(yq);
         psum[q] = pr;
-        // block amax over BETA consecutive keys (lanes)
-        float bm = pr;
-#pragma unroll
-        for (int o = C::BETA / 2; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
         uint32_t sc;
         float mult;
         if constexpr (FMT == HIFA4_NVFP4) {
+          // block amax over BETA consecutive keys (lanes)
+          float bm = pr;
+#pragma unroll
+          for (int o = C::BETA / 2; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
           sc = cvt_e4m3(__fmul_rn(div6_rn(bm), 256.0f));
           mult = inv_tab[sc];
         } else {
-          const uint32_t ef = (__float_as_uint(bm) >> 23) & 0xFFu;
-          sc = ef >= 2u ? ef - 2u : 0u;
+          // shared exponent from the block maximum of y (exact, see ptx.cuh)
+          float ym = yq;
+#pragma unroll
+          for (int o = C::BETA / 2; o > 0; o >>= 1) ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, o));
+          sc = mx_scale_from_ymax(ym);
           mult = __uint_as_float((254u - sc) << 23);
         }
         const float y = __fmul_rn(pr, mult);

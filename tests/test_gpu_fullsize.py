@@ -1,0 +1,105 @@
+"""GPU parity at the full sizes of the five workloads, in the launch
+configuration bench.py times (key tile = the workload's block_n).
+
+Quantized codes and scales are compared bit for bit (whole tensors where the
+oracle finishes in seconds, else whole batch slices); attention outputs on
+sampled query rows (first and last query tiles, all heads), which the oracle
+computes row by row; decode outputs on sampled batches."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_quantized_flashattention_smooth_b200 import workloads as W
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+h = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    global h
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import bit_quantized_flashattention_smooth_b200 as mod
+    mod.lib()
+    h = mod
+    yield
+    assert h.device_error() == 0
+
+
+def _prefill_case(name, fmt, mode, row_ranges, batches=None):
+    w = W.WORKLOADS[name]
+    q, k, v = W.make_prefill(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    s, inv = h.calibrate_smooth_qk(qd[:, :, : w.n_cal], kd[:, :, : w.n_cal], w.n_cal)
+    s_ref, inv_ref = oracle.calibrate(q[:, :, : w.n_cal].float().numpy(), k[:, :, : w.n_cal].float().numpy(),
+                                      w.n_cal)
+    np.testing.assert_allclose(U.to_np(s), s_ref, rtol=2 ** -22)
+    z = h.quantize_qkv(qd, kd, vd, torch.from_numpy(s_ref).cuda(), torch.from_numpy(inv_ref).cuda(), fmt)
+    scale = 1.0 / math.sqrt(w.d)
+    o, lph, lp = h.attn_fwd(z, scale, w.causal, mode, w.block_n, out_dtype=W.torch_dtype(w.dtype), debug=True)
+    o, lph, lp = U.to_np(o), U.to_np(lph), U.to_np(lp)
+    for b in (batches or range(w.B)):
+        qz, tiled = U.oracle_quantize(q[b:b + 1], k[b:b + 1], v[b:b + 1], s_ref, inv_ref, fmt)
+        for name_ in ("q_codes", "k_codes", "vt_codes"):
+            assert np.array_equal(U.to_np(getattr(z, name_)[b:b + 1]).astype(np.uint8), qz[name_]), name_
+        for name_ in ("q_sc", "k_sc", "vt_sc"):
+            g = U.to_np(getattr(z, name_.replace("_sc", "_scales"))[b:b + 1]).astype(np.uint8)
+            assert np.array_equal(g, tiled[name_]), name_
+        for (r0, r1) in row_ranges:
+            ref = oracle.attention(qz, w.N, fmt, scale, w.causal, mode, w.block_n, rows=(r0, r1))
+            ok, err, bound, cos = U.compare_out(o[b:b + 1, :, r0:r1], ref["O"][:, :, r0:r1])
+            assert ok, f"{name} b={b} rows {r0}:{r1}: max|dO|={err:.3e} bound={bound:.3e} cos={cos:.6f}"
+            np.testing.assert_allclose(lph[b:b + 1, :, r0:r1], ref["l_phat"][:, :, r0:r1], rtol=2e-2)
+            np.testing.assert_allclose(lp[b:b + 1, :, r0:r1], ref["l_p"][:, :, r0:r1], rtol=2e-3)
+    return o, lph, lp
+
+
+@pytest.mark.parametrize("mode", [oracle.PREORDER, oracle.INCONSISTENT])
+def test_tiny_mha_full(mode):
+    _prefill_case("tiny_mha", oracle.NVFP4, mode, [(0, 256)])
+
+
+@pytest.mark.parametrize("fmt", [oracle.NVFP4, oracle.MXFP4])
+def test_qwen3_prefill_full(fmt):
+    _, lph, lp = _prefill_case("qwen3_prefill", fmt, oracle.PREORDER, [(0, 128), (4096 - 128, 4096)])
+    # Theorem 1 on the full workload: net probability-mass loss
+    eps = lph / lp - 1
+    assert np.median(eps) < 0
+
+
+@pytest.mark.parametrize("mode", [oracle.PREORDER, oracle.INCONSISTENT])
+def test_gemma2_prefill_full(mode):
+    _prefill_case("gemma2_prefill", oracle.NVFP4, mode, [(0, 64), (8192 - 64, 8192)])
+
+
+def test_long_prefill_full():
+    _prefill_case("long_prefill", oracle.NVFP4, oracle.PREORDER, [(16384 - 32, 16384)], batches=[0, 7])
+
+
+def test_split_decode_full():
+    w = W.WORKLOADS["split_decode"]
+    q, k, v, qcal, kcal = W.make_decode_device(w)
+    s, inv = h.calibrate_smooth_qk(qcal, kcal, w.n_cal)
+    cache = h.quantize_kv(k, v, inv, h.NVFP4, Hq=w.Hq)
+    scale = 1.0 / math.sqrt(w.d)
+    o, used = h.attn_decode(q, s, cache, w.N, scale, h.PREORDER, 0)
+    o = U.to_np(o)
+    s_np, inv_np = U.to_np(s), U.to_np(inv)
+    for b in (0, w.B - 1):
+        kb, vb = k[b:b + 1].cpu().float().numpy(), v[b:b + 1].cpu().float().numpy()
+        # the cache is the K/V half of the quantizer (Q is a dummy here)
+        cz = oracle.quantize_qkv(np.zeros_like(kb), kb, vb, None, inv_np, h.NVFP4)
+        cz_t = oracle.tile_scales(cz)
+        assert np.array_equal(U.to_np(cache.k_codes[b:b + 1]).astype(np.uint8), cz["k_codes"])
+        assert np.array_equal(U.to_np(cache.vt_codes[b:b + 1]).astype(np.uint8), cz["vt_codes"])
+        assert np.array_equal(U.to_np(cache.k_scales[b:b + 1]).astype(np.uint8), cz_t["k_sc"])
+        assert np.array_equal(U.to_np(cache.vt_scales[b:b + 1]).astype(np.uint8), cz_t["vt_sc"])
+        ref = oracle.decode(U.to_np(q[b:b + 1]), s_np, cz, w.N, h.NVFP4, scale, h.PREORDER, 128, num_splits=used)
+        ok, err, bound, cos = U.compare_out(o[b:b + 1], ref["O"])
+        assert ok, f"decode b={b}: max|dO|={err:.3e} bound={bound:.3e} cos={cos:.6f}"
