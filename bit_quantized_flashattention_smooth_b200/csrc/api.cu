@@ -217,7 +217,8 @@ hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const float* s, 
   HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && kv_len > 0, HIFA4_ERR_INVALID_ARG,
                 "attn_decode: bad shape");
   HIFA4_REQUIRE(d == 128, HIFA4_ERR_UNSUPPORTED, "attn_decode: d=%d (only 128)", d);
-  HIFA4_REQUIRE(Hq / Hkv <= 8, HIFA4_ERR_UNSUPPORTED, "attn_decode: GQA group > 8");
+  HIFA4_REQUIRE(Hq / Hkv == 1 || Hq / Hkv == 2 || Hq / Hkv == 4 || Hq / Hkv == 8, HIFA4_ERR_UNSUPPORTED,
+                "attn_decode: GQA group %d not in {1,2,4,8}", Hq / Hkv);
   HIFA4_REQUIRE(block_n == 0 || block_n == 128, HIFA4_ERR_UNSUPPORTED, "attn_decode: block_n must be 128");
   HIFA4_REQUIRE(num_splits >= 0, HIFA4_ERR_INVALID_ARG, "attn_decode: num_splits < 0");
   HIFA4_REQUIRE(softmax_scale > 0.0f, HIFA4_ERR_INVALID_ARG, "attn_decode: softmax_scale must be > 0");

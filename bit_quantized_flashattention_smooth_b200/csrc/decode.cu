@@ -58,30 +58,32 @@ struct DecCfg {
   static constexpr int OFF_QSF = OFF_VSF + NS * NKC * 512;
   static constexpr int OFF_PSF = OFF_QSF + NKC * 512;        // 2 buffers
   static constexpr int OFF_ONESF = OFF_PSF + 2 * NKC * 512;
-  static constexpr int OFF_RED = OFF_ONESF + 512;            // [2][4 warps][16] floats (max), same for sums
-  static constexpr int OFF_INV = OFF_RED + 2 * 2 * 4 * 16 * 4;
+  static constexpr int OFF_RED = OFF_ONESF + 512;            // [2 parities][max | sum][4 warps][8] floats
+  static constexpr int OFF_INV = OFF_RED + 2 * 2 * 4 * 8 * 4;
   static constexpr int OFF_BAR = OFF_INV + 512;
-  static constexpr int NBAR = 4 * NS + 2 * 2 + 2 * 2 + 1;
+  // k_full/k_empty/v_full/v_empty [NS], s_full, s_empty, p_full/p_empty [2], o_full/o_empty [2]
+  static constexpr int NBAR = 4 * NS + 2 + 4 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  // TMEM columns
-  static constexpr int TM_S = 0;            // 2 x 16
-  static constexpr int TM_O = 32;
+  // TMEM columns: S (one buffer), per-tile O and L partials (two buffers each), scales
+  static constexpr int TM_S = 0;
+  static constexpr int TM_O = 16;
   static constexpr int TM_L = 48;
-  static constexpr int TM_SFK = 64;         // 4 * NKC
+  static constexpr int TM_SFK = 80;
   static constexpr int TM_SFQ = TM_SFK + 4 * NKC;
   static constexpr int TM_SFV = TM_SFQ + 4 * NKC;
   static constexpr int TM_SFP = TM_SFV + 4 * NKC;
   static constexpr int TM_SF1 = TM_SFP + 4 * NKC;
   static constexpr int TMEM_ALLOC = 128;
   static_assert(TM_SF1 + 4 <= TMEM_ALLOC, "TMEM budget");
-  static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
+  static_assert(SMEM_BYTES * 3 <= 227 * 1024, "three CTAs per SM");
 };
 
 __device__ __forceinline__ uint32_t swz64(uint32_t r, uint32_t c) { return c ^ ((r >> 1) & 3); }
 
-template <int FMT, bool PREORDER>
-__global__ void __launch_bounds__(192, 2)
+// G = query heads per kv head (1, 2, 4 or 8); the MMA N dimension is 16.
+template <int FMT, bool PREORDER, int G>
+__global__ void __launch_bounds__(192, 3)
     attn_decode_fp4_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                            const DecodeParams p) {
   using C = DecCfg<FMT>;
@@ -93,7 +95,8 @@ __global__ void __launch_bounds__(192, 2)
   const uint32_t bar0 = sbase + C::OFF_BAR;
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
   const int B_KFULL = 0, B_KEMPTY = C::NS, B_VFULL = 2 * C::NS, B_VEMPTY = 3 * C::NS, B_SFULL = 4 * C::NS,
-            B_SEMPTY = B_SFULL + 2, B_PFULL = B_SEMPTY + 2, B_PEMPTY = B_PFULL + 2, B_ORDY = B_PEMPTY + 2;
+            B_SEMPTY = B_SFULL + 1, B_PFULL = B_SEMPTY + 1, B_PEMPTY = B_PFULL + 2, B_OFULL = B_PEMPTY + 2,
+            B_OEMPTY = B_OFULL + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
@@ -114,13 +117,14 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(BAR(B_VFULL + s), 1);
       mbar_init(BAR(B_VEMPTY + s), 1);
     }
+    mbar_init(BAR(B_SFULL), 1);
+    mbar_init(BAR(B_SEMPTY), 4);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(BAR(B_SFULL + s), 1);
-      mbar_init(BAR(B_SEMPTY + s), 4);
       mbar_init(BAR(B_PFULL + s), 4);
       mbar_init(BAR(B_PEMPTY + s), 1);
+      mbar_init(BAR(B_OFULL + s), 1);
+      mbar_init(BAR(B_OEMPTY + s), 4);
     }
-    mbar_init(BAR(B_ORDY), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -134,14 +138,14 @@ __global__ void __launch_bounds__(192, 2)
   }
   // the query rows of this group: fl32(q * s) quantized along d (B operand,
   // 16 rows, rows >= G are zero) and its scale chunk(s)
-  for (int i = threadIdx.x; i < (C::SZ_QB + C::NKC * 512) / 4; i += blockDim.x)
-    reinterpret_cast<uint32_t*>(smem + (i < C::SZ_QB / 4 ? C::OFF_Q : C::OFF_QSF - C::SZ_QB))[i] = 0u;
+  for (int i = threadIdx.x; i < C::SZ_QB / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(smem + C::OFF_Q)[i] = 0u;
+  for (int i = threadIdx.x; i < C::NKC * 128; i += blockDim.x) reinterpret_cast<uint32_t*>(smem + C::OFF_QSF)[i] = 0u;
   __syncthreads();
   if (warp == 0) {
-    const int nblk = p.G * (C::D / C::BETA);
-    for (int t = lane; t < nblk; t += 32) {
+    constexpr int NBLK = G * (C::D / C::BETA);
+    for (int t = lane; t < NBLK; t += 32) {
       const int g = t / (C::D / C::BETA), blk = t % (C::D / C::BETA);
-      const int hq = h * p.G + g;
+      const int hq = h * G + g;
       float v[C::BETA];
       for (int i = 0; i < C::BETA; ++i) {
         const int c = blk * C::BETA + i;
@@ -188,7 +192,6 @@ __global__ void __launch_bounds__(192, 2)
   if (warp == 4) {
     // ================================ TMA producer ================================
     if (lane == 0) {
-      const int nkc_v_row = p.Np / (4 * C::BETA);
       for (int j = 0; j < ntile; ++j) {
         const int st = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
@@ -205,7 +208,6 @@ __global__ void __launch_bounds__(192, 2)
         bulk_load(sbase + C::OFF_VSF + st * C::NKC * 512,
                   p.v_sf + bh * p.sf_v_head + static_cast<int64_t>(key0 / (4 * C::BETA)) * 512, C::NKC * 512,
                   BAR(B_VFULL + st));
-        (void)nkc_v_row;
       }
     }
   } else if (warp == 5) {
@@ -220,33 +222,36 @@ __global__ void __launch_bounds__(192, 2)
       for (int kc = 0; kc < C::NKC; ++kc)
         tc_cp_32x128b_warpx4(tmem + C::TM_SFQ + 4 * kc, make_sf_desc(sbase + C::OFF_QSF + kc * 512));
       tc_cp_32x128b_warpx4(tmem + C::TM_SF1, make_sf_desc(sbase + C::OFF_ONESF));
+      // S^T_j = K-hat_j Q-hat^T into the single S buffer
       auto issue_s = [&](int j) -> bool {
         const int st = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
-        const int sb = j & 1;
         if (!mbar_wait(BAR(B_KFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
-        if (!mbar_wait(BAR(B_SEMPTY + sb), ((j >> 1) & 1) ^ 1, abort_flag, kErrTimeoutMma)) return false;
+        if (!mbar_wait(BAR(B_SEMPTY), (j & 1) ^ 1, abort_flag, kErrTimeoutMma)) return false;
         tc_fence_after();
         for (int kc = 0; kc < C::NKC; ++kc)
           tc_cp_32x128b_warpx4(tmem + C::TM_SFK + 4 * kc, make_sf_desc(sbase + C::OFF_KSF + (st * C::NKC + kc) * 512));
 #pragma unroll
         for (int ks = 0; ks < C::D / 64; ++ks) {
           const uint32_t chunk = MX ? ks / 2 : ks, byte = MX ? 2 * (ks % 2) : 0;
-          mma(tmem + C::TM_S + sb * C::NQ, make_kmajor_desc(sbase + C::OFF_K + st * C::SZ_K + ks * 32, C::ROW),
+          mma(tmem + C::TM_S, make_kmajor_desc(sbase + C::OFF_K + st * C::SZ_K + ks * 32, C::ROW),
               make_kmajor_desc(sbase + C::OFF_Q + ks * 32, C::ROW), idesc_fp4(128, C::NQ, MX, byte, byte),
               (tmem + C::TM_SFK + 4 * chunk) | (byte << 30), (tmem + C::TM_SFQ + 4 * chunk) | (byte << 30),
               ks > 0 ? 1u : 0u);
         }
-        tc_commit(BAR(B_SFULL + sb));
+        tc_commit(BAR(B_SFULL));
         tc_commit(BAR(B_KEMPTY + st));
         return true;
       };
+      // this tile's partials O_j^T = V-hat_j^T P-hat_j^T and L_j^T = ones P-hat_j^T
+      // into a fresh buffer (no accumulation across tiles in TMEM)
       auto issue_pv = [&](int j) -> bool {
         const int st = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
         const int pb = j & 1;
         if (!mbar_wait(BAR(B_PFULL + pb), (j >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
         if (!mbar_wait(BAR(B_VFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
+        if (!mbar_wait(BAR(B_OEMPTY + pb), ((j >> 1) & 1) ^ 1, abort_flag, kErrTimeoutMma)) return false;
         tc_fence_after();
         for (int kc = 0; kc < C::NKC; ++kc) {
           tc_cp_32x128b_warpx4(tmem + C::TM_SFV + 4 * kc, make_sf_desc(sbase + C::OFF_VSF + (st * C::NKC + kc) * 512));
@@ -257,13 +262,13 @@ __global__ void __launch_bounds__(192, 2)
           const uint32_t chunk = MX ? ks / 2 : ks, byte = MX ? 2 * (ks % 2) : 0;
           const uint64_t bp = make_kmajor_desc(sbase + C::OFF_P + pb * C::SZ_QB + ks * 32, C::ROW);
           const uint32_t sfp = (tmem + C::TM_SFP + 4 * chunk) | (byte << 30);
-          const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
-          mma(tmem + C::TM_O, make_kmajor_desc(sbase + C::OFF_V + st * C::SZ_V + ks * 32, C::ROW), bp,
-              idesc_fp4(128, C::NQ, MX, byte, byte), (tmem + C::TM_SFV + 4 * chunk) | (byte << 30), sfp, acc);
-          mma(tmem + C::TM_L, make_kmajor_desc(sbase + C::OFF_ONES + ks * 32, C::ROW), bp,
-              idesc_fp4(128, C::NQ, MX, byte, byte), (tmem + C::TM_SF1) | (byte << 30), sfp, acc);
+          mma(tmem + C::TM_O + pb * C::NQ, make_kmajor_desc(sbase + C::OFF_V + st * C::SZ_V + ks * 32, C::ROW), bp,
+              idesc_fp4(128, C::NQ, MX, byte, byte), (tmem + C::TM_SFV + 4 * chunk) | (byte << 30), sfp,
+              ks > 0 ? 1u : 0u);
+          mma(tmem + C::TM_L + pb * C::NQ, make_kmajor_desc(sbase + C::OFF_ONES + ks * 32, C::ROW), bp,
+              idesc_fp4(128, C::NQ, MX, byte, byte), (tmem + C::TM_SF1) | (byte << 30), sfp, ks > 0 ? 1u : 0u);
         }
-        tc_commit(BAR(B_ORDY));
+        tc_commit(BAR(B_OFULL + pb));
         tc_commit(BAR(B_VEMPTY + st));
         tc_commit(BAR(B_PEMPTY + pb));
         return true;
@@ -277,48 +282,71 @@ __global__ void __launch_bounds__(192, 2)
     }
   } else {
     // ================================== softmax ==================================
-    // thread t = key t of the tile = TMEM lane t; columns = the group's queries
+    // thread t = key t of the tile (TMEM lane t) for the scores, and output
+    // channel t for the PV partials; columns = the group's G queries
     const int t = threadIdx.x;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
-    float m[C::NQ], lp[C::NQ];
+    float m[G], lp[G], acc[G], lacc[G], alpha_prev[G];
 #pragma unroll
-    for (int q = 0; q < C::NQ; ++q) {
+    for (int q = 0; q < G; ++q) {
       m[q] = -INFINITY;
       lp[q] = 0.0f;
+      acc[q] = 0.0f;
+      lacc[q] = 0.0f;
+      alpha_prev[q] = 0.0f;
     }
-    const bool want_lp = !PREORDER;
+    // fold the partials of tile jj (already complete or about to be) into the
+    // register accumulators, scaled by that tile's alpha
+    auto fold = [&](int jj) -> bool {
+      const int ob = jj & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_OFULL + ob), (jj >> 1) & 1, abort_flag, kErrTimeoutSoftmax)))
+        return false;
+      tc_fence_after();
+      uint32_t o[16], l[16];
+      tmem_ld16_wait(tmem + lane_base + C::TM_O + ob * C::NQ, o);
+      tmem_ld16_wait(tmem + lane_base + C::TM_L + ob * C::NQ, l);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_OEMPTY + ob));
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        acc[q] = fmaf(alpha_prev[q], acc[q], __uint_as_float(o[q]));
+        lacc[q] = fmaf(alpha_prev[q], lacc[q], __uint_as_float(l[q]));
+      }
+      return true;
+    };
     bool ok = true;
     for (int j = 0; j < ntile && ok; ++j) {
-      const int sb = j & 1, pb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + sb), (j >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+      const int pb = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL), j & 1, abort_flag, kErrTimeoutSoftmax))) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t v[16];
-      tmem_ld16_wait(tmem + lane_base + C::TM_S + sb * C::NQ, v);
+      tmem_ld16_wait(tmem + lane_base + C::TM_S, v);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_SEMPTY + sb));
+      if (lane == 0) mbar_arrive(BAR(B_SEMPTY));
       const bool valid = k_begin + j * C::BN + t < k_end;
-      float x[C::NQ];
+      float x[G];
 #pragma unroll
-      for (int q = 0; q < C::NQ; ++q) x[q] = valid && q < p.G ? __fmul_rn(__uint_as_float(v[q]), p.c_log2) : -INFINITY;
+      for (int q = 0; q < G; ++q) x[q] = valid ? __fmul_rn(__uint_as_float(v[q]), p.c_log2) : -INFINITY;
       // tile max per query: warp shuffle, then across the 4 warps
-      float* rbuf = red + (j & 1) * 2 * 4 * 16;
+      float* rbuf = red + (j & 1) * 2 * 4 * 8;
 #pragma unroll
-      for (int q = 0; q < C::NQ; ++q) {
+      for (int q = 0; q < G; ++q) {
         float mx = x[q];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == q) rbuf[warp * 16 + q] = mx;
+        if (lane == q) rbuf[warp * 8 + q] = mx;
       }
       named_bar_sync(1, 128);
-      float alpha[C::NQ], mnew[C::NQ];
+      float alpha[G], mnew[G];
 #pragma unroll
-      for (int q = 0; q < C::NQ; ++q) {
-        const float tm = fmaxf(fmaxf(rbuf[q], rbuf[16 + q]), fmaxf(rbuf[32 + q], rbuf[48 + q]));
+      for (int q = 0; q < G; ++q) {
+        const float tm = fmaxf(fmaxf(rbuf[q], rbuf[8 + q]), fmaxf(rbuf[16 + q], rbuf[24 + q]));
         mnew[q] = fmaxf(m[q], tm);
         alpha[q] = (mnew[q] == m[q]) ? 1.0f : ex2_approx(m[q] - mnew[q]);
       }
@@ -330,10 +358,10 @@ __global__ void __launch_bounds__(192, 2)
       }
       unsigned char* pbuf = smem + C::OFF_P + pb * C::SZ_QB;
       unsigned char* psf = smem + C::OFF_PSF + pb * C::NKC * 512;
-      float psum[C::NQ];
+      float psum[G];
 #pragma unroll
-      for (int q = 0; q < C::NQ; ++q) {
-        const float yq = (q < p.G) ? __fsub_rn(x[q], mnew[q]) : -INFINITY;
+      for (int q = 0; q < G; ++q) {
+        const float yq = __fsub_rn(x[q], mnew[q]);
         const float pr = ex2_approx(yq);
         psum[q] = pr;
         uint32_t sc;
@@ -365,65 +393,58 @@ __global__ void __launch_bounds__(192, 2)
           psf[(blk / 4) * 512 + q * 16 + (blk % 4)] = static_cast<unsigned char>(sc);
         }
       }
-      if (want_lp) {
-        float* sbuf = rbuf + 4 * 16;
+      if constexpr (G < C::NQ) {
+        // rows G..15 of the P-hat tile stay zero (written once per buffer)
+        if (j < 2) {
+          for (int i = t; i < (C::NQ - G) * C::ROW / 4; i += 128)
+            reinterpret_cast<uint32_t*>(pbuf + G * C::ROW)[i] = 0u;
+          for (int i = t; i < (C::NQ - G) * C::NKC; i += 128) {
+            const int r = G + i / C::NKC, kc = i % C::NKC;
+            *reinterpret_cast<uint32_t*>(psf + kc * 512 + r * 16) = 0u;
+          }
+        }
+      }
+      if constexpr (!PREORDER) {
+        float* sbuf = rbuf + 4 * 8;
 #pragma unroll
-        for (int q = 0; q < C::NQ; ++q) {
+        for (int q = 0; q < G; ++q) {
           float sm = psum[q];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
-          if (lane == q) sbuf[warp * 16 + q] = sm;
+          if (lane == q) sbuf[warp * 8 + q] = sm;
         }
         named_bar_sync(1, 128);
 #pragma unroll
-        for (int q = 0; q < C::NQ; ++q)
-          lp[q] = fmaf(alpha[q], lp[q], (sbuf[q] + sbuf[16 + q]) + (sbuf[32 + q] + sbuf[48 + q]));
+        for (int q = 0; q < G; ++q)
+          lp[q] = fmaf(alpha[q], lp[q], (sbuf[q] + sbuf[8 + q]) + (sbuf[16 + q] + sbuf[24 + q]));
       }
-      // rescale O^T and L^T columns whose max rose (after PV_{j-1} retired)
-      bool any = false;
-#pragma unroll
-      for (int q = 0; q < C::NQ; ++q) any |= alpha[q] != 1.0f;
-      if (j > 0 && any) {
-        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_ORDY), (j - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t o[16], l[16];
-        tmem_ld16_wait(tmem + lane_base + C::TM_O, o);
-        tmem_ld16_wait(tmem + lane_base + C::TM_L, l);
-#pragma unroll
-        for (int q = 0; q < C::NQ; ++q) {
-          o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
-          l[q] = __float_as_uint(__uint_as_float(l[q]) * alpha[q]);
-        }
-        tmem_st16(tmem + lane_base + C::TM_O, o);
-        tmem_st16(tmem + lane_base + C::TM_L, l);
-        tmem_wait_st();
-      }
-#pragma unroll
-      for (int q = 0; q < C::NQ; ++q) m[q] = mnew[q];
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_PFULL + pb));
+      // the previous tile's partials are complete by now: fold them in
+      if (j > 0 && !fold(j - 1)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        m[q] = mnew[q];
+        alpha_prev[q] = alpha[q];
+      }
     }
     // ------------------------------------------------------------- epilogue ---
-    const bool ready = __all_sync(0xffffffffu, ok && ntile > 0 &&
-                                                  mbar_wait(BAR(B_ORDY), (ntile - 1) & 1, abort_flag, kErrTimeoutSoftmax));
+    const bool ready = __all_sync(0xffffffffu, ok && ntile > 0) && fold(ntile - 1);
     if (ready) {
-      tc_fence_after();
-      uint32_t o[16], l[16];
-      tmem_ld16_wait(tmem + lane_base + C::TM_O, o);
-      tmem_ld16_wait(tmem + lane_base + C::TM_L, l);
       const int c = t;  // TMEM lane = output channel
-      for (int q = 0; q < p.G; ++q) {
-        const int hq = h * p.G + q;
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        const int hq = h * G + q;
         float* w = p.ws + ((static_cast<int64_t>(b) * p.Hq + hq) * p.splits + sp) * (C::D + 2);
-        w[c] = __uint_as_float(o[q]) * kGP;
+        w[c] = acc[q] * kGP;
         if (c == 0) {
           w[C::D] = m[q];
-          w[C::D + 1] = PREORDER ? __uint_as_float(l[q]) * kGP : lp[q];
+          w[C::D + 1] = PREORDER ? lacc[q] * kGP : lp[q];
         }
       }
     }
@@ -474,7 +495,7 @@ int decode_default_splits(int B, int Hkv, int kv_len, int block_n) {
   return splits;
 }
 
-template <int FMT, bool PRE>
+template <int FMT, bool PRE, int G>
 static hifa4_status launch_decode_t(const uint8_t* kc, const uint8_t* vc, const DecodeParams& p, cudaStream_t st) {
   using C = DecCfg<FMT>;
   CUtensorMap tk, tv;
@@ -484,7 +505,7 @@ static hifa4_status launch_decode_t(const uint8_t* kc, const uint8_t* vc, const 
     set_last_error("cuTensorMapEncodeTiled failed");
     return HIFA4_ERR_CUDA;
   }
-  auto kern = attn_decode_fp4_kernel<FMT, PRE>;
+  auto kern = attn_decode_fp4_kernel<FMT, PRE, G>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   kern<<<static_cast<unsigned>(p.B) * p.Hkv * p.splits, 192, C::SMEM_BYTES, st>>>(tk, tv, p);
   return launch_status("attn_decode");
@@ -521,13 +542,23 @@ hifa4_status decode_launch(const void* q, int q_dt, const float* s, const uint8_
   p.q_fp16 = q_dt == HIFA4_FP16;
   p.c_log2 = softmax_scale * 1.4426950408889634f;
   p.ws = static_cast<float*>(workspace);
-  hifa4_status r;
-  if (fmt == HIFA4_NVFP4)
-    r = mode == HIFA4_NORM_PREORDER ? launch_decode_t<HIFA4_NVFP4, true>(kc, vc, p, st)
-                                    : launch_decode_t<HIFA4_NVFP4, false>(kc, vc, p, st);
-  else
-    r = mode == HIFA4_NORM_PREORDER ? launch_decode_t<HIFA4_MXFP4, true>(kc, vc, p, st)
-                                    : launch_decode_t<HIFA4_MXFP4, false>(kc, vc, p, st);
+  hifa4_status r = HIFA4_ERR_UNSUPPORTED;
+  const bool pre = mode == HIFA4_NORM_PREORDER;
+#define HIFA4_DEC_G(GG)                                                                          \
+  if (p.G == GG) {                                                                               \
+    if (fmt == HIFA4_NVFP4)                                                                      \
+      r = pre ? launch_decode_t<HIFA4_NVFP4, true, GG>(kc, vc, p, st)                            \
+              : launch_decode_t<HIFA4_NVFP4, false, GG>(kc, vc, p, st);                          \
+    else                                                                                         \
+      r = pre ? launch_decode_t<HIFA4_MXFP4, true, GG>(kc, vc, p, st)                            \
+              : launch_decode_t<HIFA4_MXFP4, false, GG>(kc, vc, p, st);                          \
+  }
+  HIFA4_DEC_G(1)
+  HIFA4_DEC_G(2)
+  HIFA4_DEC_G(4)
+  HIFA4_DEC_G(8)
+#undef HIFA4_DEC_G
+  if (r == HIFA4_ERR_UNSUPPORTED) set_last_error("attn_decode: GQA group %d not in {1,2,4,8}", p.G);
   if (r != HIFA4_OK) return r;
   const int rows = B * Hq;
   decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(p.ws, rows, used, d, o, o_dt == HIFA4_FP16);

@@ -176,7 +176,7 @@ HIFA4_API int hifa4_decode_default_splits(int B, int Hkv, int kv_len, int block_
  * O = sum 2^(m_s-M) acc_s / sum 2^(m_s-M) l_s.  o: device [B][Hq][d] of o_dt.
  * num_splits 0 = hifa4_decode_default_splits; *num_splits_used (optional,
  * host) receives the count of non-empty splits.  Requires d == 128,
- * Hq/Hkv <= 8, block_n == 0 or 128. */
+ * Hq/Hkv in {1, 2, 4, 8}, block_n == 0 or 128. */
 HIFA4_API hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const float* s,
                                const uint8_t* k_codes, const uint8_t* k_scales,
                                const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
