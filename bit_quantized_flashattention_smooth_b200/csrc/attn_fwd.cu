@@ -8,16 +8,18 @@
 // the same P-hat that feeds the PV GEMM, fused into that GEMM.
 //
 // B200 design (one CTA = one 128-row query tile of one (batch, q head)):
-//   warp 4      TMA producer: Q-hat tile once, then K-hat / V-hat^T tiles and
+//   warp 8      TMA producer: Q-hat tile once, then K-hat / V-hat^T tiles and
 //               their tiled scale chunks into an NS-stage ring (mbarriers).
-//   warp 5      MMA issuer (one thread): copies scale chunks shared->TMEM with
+//   warp 9      MMA issuer (one thread): copies scale chunks shared->TMEM with
 //               tcgen05.cp, issues block-scaled tcgen05.mma for S = Q K^T
 //               into a TMEM S buffer, and for O += P-hat V-hat plus
 //               L += P-hat * ones (the fused normalizer: a 16-row all-ones B
 //               tile, so column 0 of L is sum(P-hat) with the same P-hat
 //               codes and scales as O).  Completion is signalled with
 //               tcgen05.commit onto mbarriers.
-//   warps 0-3   softmax: thread r owns query row r (TMEM lane r).  Per key
+//   warps 0-7   softmax: two warpgroups share each query row r (TMEM lane
+//               r), each with half of the key columns and half of O; the
+//               row max is exchanged in shared memory.  Per key
 //               tile: tcgen05.ld the S row, online max, P = 2^(S*c - m),
 //               per-block P-hat quantization in registers (cvt to E4M3 /
 //               E2M1), codes stored swizzled into shared memory as the A
@@ -92,10 +94,12 @@ struct AttnCfg {
   static constexpr int OFF_PSF = OFF_VSF + NS * NRG_V * NCH_V * 512;
   static constexpr int OFF_ONESF = OFF_PSF + 2 * NKC_P * 512;
   static constexpr int OFF_INV = OFF_ONESF + 512;           // 128 floats: 1/scale per UE4M3 code
-  static constexpr int OFF_BAR = OFF_INV + 512;
+  static constexpr int OFF_XM = OFF_INV + 512;              // row-max exchange [2][2][128] floats
+  static constexpr int OFF_LP = OFF_XM + 2048;              // normalizer exchange [2][128] floats
+  static constexpr int OFF_BAR = OFF_LP + 1024;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
   // s_full[NSB], s_empty[NSB], p_full[2], p_empty[2], o_ready
-  static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1;
+  static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1 + 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   // TMEM columns
@@ -156,7 +160,7 @@ __device__ __forceinline__ uint32_t swz_chunk(uint32_t r, uint32_t c, uint32_t r
 }
 
 template <int D, int BN, int FMT, bool PREORDER>
-__global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
+__global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D, BN, FMT>;
@@ -170,7 +174,7 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
   const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + C::NS, B_VFULL = 1 + 2 * C::NS, B_VEMPTY = 1 + 3 * C::NS,
             B_SFULL = 1 + 4 * C::NS, B_SEMPTY = B_SFULL + C::NSB, B_PFULL = B_SEMPTY + C::NSB,
-            B_PEMPTY = B_PFULL + 2, B_ORDY = B_PEMPTY + 2;
+            B_PEMPTY = B_PFULL + 2, B_ORDY = B_PEMPTY + 2, B_XM = B_ORDY + 1, B_EP1 = B_XM + 1, B_EP2 = B_EP1 + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -194,13 +198,16 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     }
     for (int s = 0; s < C::NSB; ++s) {
       mbar_init(BAR(B_SFULL + s), 1);
-      mbar_init(BAR(B_SEMPTY + s), 4);
+      mbar_init(BAR(B_SEMPTY + s), 8);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(BAR(B_PFULL + s), 4);
+      mbar_init(BAR(B_PFULL + s), 8);
       mbar_init(BAR(B_PEMPTY + s), 1);
     }
     mbar_init(BAR(B_ORDY), 1);
+    mbar_init(BAR(B_XM), 256);    // row-max exchange between the two column halves
+    mbar_init(BAR(B_EP1), 128);   // epilogue: half 1 -> half 0
+    mbar_init(BAR(B_EP2), 128);   // epilogue: half 0 -> half 1
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -218,11 +225,11 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     reinterpret_cast<float*>(smem + C::OFF_INV)[i] = i == 0 ? 0.0f : __fdiv_rn(1.0f, sd);
   }
   fence_proxy_async_smem();
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -232,7 +239,7 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // =============================== TMA producer ===============================
     if (lane == 0) {
       const uint8_t* qsf = p.q_sf + static_cast<int64_t>(bhq) * p.sf_qk_head + static_cast<int64_t>(qtile) * C::NKC_Q * 512;
@@ -259,7 +266,7 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
                     C::NCH_V * 512, BAR(B_VFULL + st));
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ================================ MMA issuer ================================
     if (lane == 0) {
       constexpr bool MX = FMT == HIFA4_MXFP4;
@@ -346,9 +353,17 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     }
   } else {
     // ================================== softmax ==================================
-    const int r = threadIdx.x;  // 0..127 == TMEM lane
+    // Two warpgroups share each query row: thread (hw, r) owns TMEM lane r,
+    // key columns [hw*BN/2, (hw+1)*BN/2) of S and P-hat, and output columns
+    // [hw*D/2, (hw+1)*D/2) of O.  The row maximum is exchanged through
+    // shared memory once per key tile.
+    constexpr int HB = BN / 2;                       // key columns per thread
+    constexpr int HD = D / 2;                        // output columns per thread
+    constexpr int NBH = HB / C::BETA;                // P-hat blocks per thread
+    const int hw = warp >> 2;                        // column half
+    const int r = threadIdx.x & 127;                 // row == TMEM lane
     const int row = row0 + r;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c = p.c_log2;
     float m = -INFINITY;
     float l_p = 0.0f;
@@ -356,6 +371,7 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
     constexpr float kInvGP = FMT == HIFA4_NVFP4 ? 256.0f : 1.0f;
     const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
+    float* xm = reinterpret_cast<float*>(smem + C::OFF_XM);  // [2 parities][2 halves][128]
     bool ok = true;
     for (int j = 0; j < nkt && ok; ++j) {
       const int sb = j % C::NSB;
@@ -365,49 +381,54 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
         break;
       }
       tc_fence_after();
-      float s[BN];
+      float s[HB];
       {
-        uint32_t v[BN];
+        uint32_t v[HB];
 #pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc)
-          tmem_ld32(tmem + lane_base + C::TM_S + sb * BN + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
+        for (int cc = 0; cc < HB / 32; ++cc)
+          tmem_ld32(tmem + lane_base + C::TM_S + sb * BN + hw * HB + cc * 32,
+                    *reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
 #pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc) tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
+        for (int cc = 0; cc < HB / 32; ++cc) tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
 #pragma unroll
-        for (int i = 0; i < BN; ++i) s[i] = __uint_as_float(v[i]);
+        for (int i = 0; i < HB; ++i) s[i] = __uint_as_float(v[i]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_SEMPTY + sb));
       // mask (only tiles that reach past the diagonal or past N need it)
-      const int kbase = j * BN;
-      const bool need_mask = (kbase + BN > p.N) || (p.causal && kbase + BN - 1 > row0);
+      const int kbase = j * BN + hw * HB;
+      const bool need_mask = (j * BN + BN > p.N) || (p.causal && j * BN + BN - 1 > row0);
       if (need_mask) {
         const int lim = p.causal ? min(p.N, row + 1) : p.N;
 #pragma unroll
-        for (int k = 0; k < BN; ++k) s[k] = (kbase + k >= lim) ? -INFINITY : s[k];
+        for (int k = 0; k < HB; ++k) s[k] = (kbase + k >= lim) ? -INFINITY : s[k];
       }
       // x = fl32(S * c) first, then P = 2^(x - m): the row maximum gives
-      // exactly 2^0 = 1, so power-of-two block decisions (the MXFP4 shared
-      // exponent) agree with the written rule.
+      // exactly 2^0 = 1, as the written rule does.
       const float2 c2 = make_float2(c, c);
 #pragma unroll
-      for (int k = 0; k < BN; k += 2) {
+      for (int k = 0; k < HB; k += 2) {
         const float2 x = fmul2(make_float2(s[k], s[k + 1]), c2);
         s[k] = x.x;
         s[k + 1] = x.y;
       }
-      const float m_new = fmaxf(m, tree_max<BN>(s));
+      float* xb = xm + (j & 1) * 256;
+      xb[hw * 128 + r] = tree_max<HB>(s);
+      mbar_arrive(BAR(B_XM));     // release: this thread's max is visible to waiters
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_XM), j & 1, abort_flag, kErrTimeoutSoftmax))) {
+        ok = false;
+        break;
+      }
+      const float m_new = fmaxf(m, fmaxf(xb[r], xb[128 + r]));
       const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);
       const float2 negm = make_float2(-m_new, -m_new);
       // P = 2^(x - m_new); P-hat per block of BETA keys
-      uint32_t codes[BN / 8];
-      uint32_t scw[C::NKC_P];
-#pragma unroll
-      for (int i = 0; i < C::NKC_P; ++i) scw[i] = 0;
+      uint32_t codes[HB / 8];
+      uint32_t scb[NBH];
       float psum = 0.0f;
 #pragma unroll
-      for (int blk = 0; blk < BN / C::BETA; ++blk) {
+      for (int blk = 0; blk < NBH; ++blk) {
         float* pb_ = s + blk * C::BETA;
 #pragma unroll
         for (int i = 0; i < C::BETA; i += 2) {
@@ -439,7 +460,7 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
               cvt_e2m1x8(fmul2(make_float2(e[0], e[1]), m2), fmul2(make_float2(e[2], e[3]), m2),
                          fmul2(make_float2(e[4], e[5]), m2), fmul2(make_float2(e[6], e[7]), m2));
         }
-        scw[blk / 4] |= sc << (8 * (blk % 4));
+        scb[blk] = sc;
         if (want_lp) psum += tree_sum<C::BETA>(pb_);
       }
       if (want_lp) l_p = fmaf(alpha, l_p, psum);
@@ -452,47 +473,46 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
       {
         unsigned char* prow = smem + C::OFF_P + pb * C::SZ_P + r * C::PROW;
 #pragma unroll
-        for (int ch = 0; ch < C::PROW / 16; ++ch) {
-          const uint32_t phys = swz_chunk(r, ch, C::PROW);
+        for (int ch = 0; ch < HB / 32; ++ch) {
+          const uint32_t phys = swz_chunk(r, hw * (HB / 32) + ch, C::PROW);
           *reinterpret_cast<uint4*>(prow + phys * 16) =
               make_uint4(codes[4 * ch], codes[4 * ch + 1], codes[4 * ch + 2], codes[4 * ch + 3]);
         }
-        unsigned char* psf = smem + C::OFF_PSF + pb * C::NKC_P * 512;
+        unsigned char* psf = smem + C::OFF_PSF + pb * C::NKC_P * 512 + (r & 31) * 16 + (r >> 5) * 4;
 #pragma unroll
-        for (int pc = 0; pc < C::NKC_P; ++pc)
-          *reinterpret_cast<uint32_t*>(psf + pc * 512 + (r & 31) * 16 + (r >> 5) * 4) = scw[pc];
+        for (int blk = 0; blk < NBH; ++blk) {
+          const int gb = hw * NBH + blk;                       // block index within the tile
+          psf[(gb / 4) * 512 + (gb % 4)] = static_cast<unsigned char>(scb[blk]);
+        }
       }
-      // rescale the O / L row when the max rose (PV_{j-1} must have retired)
+      // rescale this half of the O row (and L) when the max rose, after
+      // PV_{j-1} retired
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
         if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_ORDY), (j - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc) {
-          uint32_t v0[32], v1[32];
-          const uint32_t a0 = tmem + lane_base + C::TM_O + cc * 64;
+        for (int cc = 0; cc < HD / 32; ++cc) {
+          uint32_t v0[32];
+          const uint32_t a0 = tmem + lane_base + C::TM_O + hw * HD + cc * 32;
           tmem_ld32(a0, v0);
-          tmem_ld32(a0 + 32, v1);
           tmem_wait_ld_dep(v0);
-          tmem_wait_ld_dep(v1);
-          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            float2 t0 = fmul2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), a2);
-            float2 t1 = fmul2(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), a2);
+            const float2 t0 = fmul2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), a2);
             v0[i] = __float_as_uint(t0.x);
             v0[i + 1] = __float_as_uint(t0.y);
-            v1[i] = __float_as_uint(t1.x);
-            v1[i + 1] = __float_as_uint(t1.y);
           }
           tmem_st32(a0, v0);
-          tmem_st32(a0 + 32, v1);
         }
-        uint32_t lv;
-        tmem_ld1_wait(tmem + lane_base + C::TM_L, lv);
-        tmem_st1(tmem + lane_base + C::TM_L, __float_as_uint(__uint_as_float(lv) * alpha));
+        if (hw == 0) {
+          uint32_t lv;
+          tmem_ld1_wait(tmem + lane_base + C::TM_L, lv);
+          tmem_st1(tmem + lane_base + C::TM_L, __float_as_uint(__uint_as_float(lv) * alpha));
+        }
         tmem_wait_st();
       }
       fence_proxy_async_smem();
@@ -502,6 +522,15 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
       m = m_new;
     }
     // ---------------------------------- epilogue ----------------------------------
+    // the two halves' partial sums of P (same recurrence) add up to l_p
+    float* lpx = reinterpret_cast<float*>(smem + C::OFF_LP);
+    if (hw == 1) {
+      lpx[r] = l_p;
+      mbar_arrive(BAR(B_EP1));
+    } else {
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(BAR(B_EP1), 0, abort_flag, kErrTimeoutSoftmax));
+      l_p += lpx[r];
+    }
     const bool ready = __all_sync(0xffffffffu, ok && nkt > 0 &&
                                                   mbar_wait(BAR(B_ORDY), (nkt - 1) & 1, abort_flag, kErrTimeoutSoftmax));
     if (ready) {
@@ -510,26 +539,37 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
       tmem_ld1_wait(tmem + lane_base + C::TM_L, lv);
       const float l_acc = __uint_as_float(lv);           // sum of P-hat in MMA units (P-hat / g_P)
       const float l_phat = l_acc * kGP;
-      const float l_used = PREORDER ? l_phat : l_p;
-      const float inv_l = 1.0f / l_used;
-      const float o_mul = kGP * inv_l;                    // O_acc is in units of 1/g_P
       const bool store = row < p.N;
-      const int64_t orow = (static_cast<int64_t>(bhq) * p.N + row) * D;
+      const int64_t orow = (static_cast<int64_t>(bhq) * p.N + row) * D + hw * HD;
+      // INCONSISTENT: only half 0 holds the full l_p; share it
+      float l_used = l_phat;
+      if constexpr (!PREORDER) {
+        // half 1 needs the full l_p of its row for the output scale
+        if (hw == 0) {
+          lpx[128 + r] = l_p;
+          mbar_arrive(BAR(B_EP2));
+          l_used = l_p;
+        } else {
+          if (!mbar_wait(BAR(B_EP2), 0, abort_flag, kErrTimeoutSoftmax)) atomicOr(&g_device_error, kErrTimeoutSoftmax);
+          l_used = lpx[128 + r];
+        }
+      }
+      const float o_mul = kGP / l_used;                   // O_acc is in units of 1/g_P
 #pragma unroll
-      for (int cc = 0; cc < D / 16; ++cc) {
+      for (int cc = 0; cc < HD / 16; ++cc) {
         uint32_t v[16];
-        tmem_ld16_wait(tmem + lane_base + C::TM_O + cc * 16, v);
+        tmem_ld16_wait(tmem + lane_base + C::TM_O + hw * HD + cc * 16, v);
         if (store) {
           uint32_t packed[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float a = __uint_as_float(v[2 * i]) * o_mul, bb = __uint_as_float(v[2 * i + 1]) * o_mul;
             if (p.out_fp16) {
-              __half2 h = __floats2half2_rn(a, bb);
-              packed[i] = *reinterpret_cast<uint32_t*>(&h);
+              __half2 hh = __floats2half2_rn(a, bb);
+              packed[i] = *reinterpret_cast<uint32_t*>(&hh);
             } else {
-              __nv_bfloat162 h = __floats2bfloat162_rn(a, bb);
-              packed[i] = *reinterpret_cast<uint32_t*>(&h);
+              __nv_bfloat162 hh = __floats2bfloat162_rn(a, bb);
+              packed[i] = *reinterpret_cast<uint32_t*>(&hh);
             }
           }
           uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + orow + cc * 16);
@@ -537,7 +577,7 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
       }
-      if (store) {
+      if (store && hw == 0) {
         const int64_t ri = static_cast<int64_t>(bhq) * p.N + row;
         if (p.lse) p.lse[ri] = m + log2f(l_used);
         if (p.dbg_l_phat) p.dbg_l_phat[ri] = l_phat;
@@ -551,7 +591,7 @@ __global__ void __launch_bounds__(192, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, C::TMEM_ALLOC);
+  if (warp == 9) tmem_dealloc(tmem, C::TMEM_ALLOC);
 }
 
 // ------------------------------------------------------------------ host ---
@@ -574,7 +614,7 @@ static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const ui
   const int smem = C::SMEM_REQ;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * p.num_qtiles;
-  kern<<<grid, 192, smem, st>>>(tq, tk, tv, p);
+  kern<<<grid, 320, smem, st>>>(tq, tk, tv, p);
   return launch_status("attn_fwd");
 }
 

@@ -62,7 +62,7 @@ struct DecCfg {
   static constexpr int OFF_INV = OFF_RED + 2 * 2 * 4 * 8 * 4;
   static constexpr int OFF_BAR = OFF_INV + 512;
   // k_full/k_empty/v_full/v_empty [NS], s_full, s_empty, p_full/p_empty [2], o_full/o_empty [2]
-  static constexpr int NBAR = 4 * NS + 2 + 4 + 4;
+  static constexpr int NBAR = 4 * NS + 2 + 4 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // TMEM columns: S (one buffer), per-tile O and L partials (two buffers each), scales
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(192, 3)
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
   const int B_KFULL = 0, B_KEMPTY = C::NS, B_VFULL = 2 * C::NS, B_VEMPTY = 3 * C::NS, B_SFULL = 4 * C::NS,
             B_SEMPTY = B_SFULL + 1, B_PFULL = B_SEMPTY + 1, B_PEMPTY = B_PFULL + 2, B_OFULL = B_PEMPTY + 2,
-            B_OEMPTY = B_OFULL + 2;
+            B_OEMPTY = B_OFULL + 2, B_RED = B_OEMPTY + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
@@ -125,6 +125,7 @@ __global__ void __launch_bounds__(192, 3)
       mbar_init(BAR(B_OFULL + s), 1);
       mbar_init(BAR(B_OEMPTY + s), 4);
     }
+    mbar_init(BAR(B_RED), 128);    // cross-warp reductions of the softmax warps
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -342,7 +343,12 @@ __global__ void __launch_bounds__(192, 3)
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         if (lane == q) rbuf[warp * 8 + q] = mx;
       }
-      named_bar_sync(1, 128);
+      // exchange round 2j (the sums of the inconsistent mode use round 2j+1)
+      mbar_arrive(BAR(B_RED));
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_RED), PREORDER ? (j & 1) : 0, abort_flag, kErrTimeoutSoftmax))) {
+        ok = false;
+        break;
+      }
       float alpha[G], mnew[G];
 #pragma unroll
       for (int q = 0; q < G; ++q) {
@@ -413,7 +419,11 @@ __global__ void __launch_bounds__(192, 3)
           for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
           if (lane == q) sbuf[warp * 8 + q] = sm;
         }
-        named_bar_sync(1, 128);
+        mbar_arrive(BAR(B_RED));
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_RED), 1, abort_flag, kErrTimeoutSoftmax))) {
+          ok = false;
+          break;
+        }
 #pragma unroll
         for (int q = 0; q < G; ++q)
           lp[q] = fmaf(alpha[q], lp[q], (sbuf[q] + sbuf[8 + q]) + (sbuf[16 + q] + sbuf[24 + q]));
