@@ -194,7 +194,7 @@ def run_prefill(args, rank, world):
 
     return dict(w=w, fmt=fmt, mode=mode, step_ms=step_ms_max, attn_ms=attn_ms_max, quant_ms=quant_ms,
                 flops=flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clk, wall=wall,
-                launches=4 * args.steps, qd=qd, kd=kd, vd=vd, z=z)
+                launches=2 * args.steps, qd=qd, kd=kd, vd=vd, z=z)
 
 
 def fp4_probe_peak():

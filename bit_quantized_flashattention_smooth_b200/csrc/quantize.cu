@@ -84,14 +84,10 @@ __device__ __forceinline__ uint32_t quant_block(const float (&v)[BETA], uint32_t
 // of a row.  x: [BH][N][d] rows of head bh; rows N..Np-1 are zero padding.
 // Head bh uses smoothing scale row (bh % H) / G of `scale` ([Hkv][d]).
 template <int FMT, typename T>
-__global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ x, int H, int G, int N,
-                                                            int Np, int d, const float* __restrict__ scale,
-                                                            uint8_t* __restrict__ codes,
-                                                            uint8_t* __restrict__ sf, int64_t sf_head_bytes,
-                                                            int64_t total_words) {
+__device__ __forceinline__ void quantize_row_word(const T* __restrict__ x, int H, int G, int N, int Np, int d,
+                                                  const float* __restrict__ scale, uint8_t* __restrict__ codes,
+                                                  uint8_t* __restrict__ sf, int64_t sf_head_bytes, int64_t idx) {
   constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
-  int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= total_words) return;
   const int nb = d / BETA;
   const int wpr = (nb + 3) / 4;
   const int w = static_cast<int>(idx % wpr);
@@ -138,41 +134,47 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
     }
     sc_word |= sc << (8 * blk);
   }
-  const int nkc = wpr;
-  *reinterpret_cast<uint32_t*>(sf + bh * sf_head_bytes + sf_word_offset(t, w, nkc)) = sc_word;
+  *reinterpret_cast<uint32_t*>(sf + bh * sf_head_bytes + sf_word_offset(t, w, wpr)) = sc_word;
 }
 
-// V: one CTA per (128-token tile, head).  The tile is staged in shared memory
-// (coalesced 16-byte loads), then one thread per (channel, scale word)
-// quantizes 4 blocks of tokens and writes 4*BETA/2 contiguous code bytes of
-// the channel-major V^T row plus one scale word.
+// V: one CTA per (128-token tile, head, 64-channel group).  The tile is staged
+// in shared memory with coalesced 16-byte loads; then one thread per (channel,
+// scale word) quantizes 4 blocks of tokens and writes 4*BETA/2 contiguous code
+// bytes of the channel-major V^T row plus one scale word.
+constexpr int kVCh = 64;   // channels per V CTA
 template <int FMT, typename T>
-__global__ void __launch_bounds__(256) quantize_v_kernel(const T* __restrict__ v, int N, int Np, int d,
-                                                         uint8_t* __restrict__ vt_codes,
-                                                         uint8_t* __restrict__ vt_sf, int64_t sf_head_bytes) {
+__device__ __forceinline__ void quantize_v_tile(const T* __restrict__ v, int N, int Np, int d,
+                                                uint8_t* __restrict__ vt_codes, uint8_t* __restrict__ vt_sf,
+                                                int64_t sf_head_bytes, int tile, T* tile_smem) {
   constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  T* tile = reinterpret_cast<T*>(smem_raw);  // [128][d]
-  const int t0 = blockIdx.x * 128;
-  const int64_t bh = blockIdx.y;
-  const int vec_per_row = d / 8;
-  for (int i = threadIdx.x; i < 128 * vec_per_row; i += blockDim.x) {
-    int r = i / vec_per_row, cv = i % vec_per_row;
+  const int ncg = d / kVCh;
+  const int cg = tile % ncg;
+  const int64_t bhx = tile / ncg;          // head * (Np / 128) + token tile
+  const int ntt = Np / 128;
+  const int t0 = static_cast<int>(bhx % ntt) * 128;
+  const int64_t head = bhx / ntt;
+  const int c_base = cg * kVCh;
+  constexpr int VEC = kVCh / 8;   // 16-byte vectors per token row
+  for (int i = threadIdx.x; i < 128 * VEC; i += blockDim.x) {
+    const int r = i / VEC, cv = i % VEC;
     uint4 u = make_uint4(0, 0, 0, 0);
-    if (t0 + r < N) u = *reinterpret_cast<const uint4*>(v + (bh * N + t0 + r) * static_cast<int64_t>(d) + cv * 8);
-    *reinterpret_cast<uint4*>(tile + r * d + cv * 8) = u;
+    if (t0 + r < N)
+      u = *reinterpret_cast<const uint4*>(v + (head * N + t0 + r) * static_cast<int64_t>(d) + c_base + cv * 8);
+    *reinterpret_cast<uint4*>(tile_smem + r * kVCh + cv * 8) = u;
   }
   __syncthreads();
   const int words_per_ch = 128 / (4 * BETA);
   const int nkc = Np / (4 * BETA);
-  // rows d..127 of a 128-row scale group are padding (d = 64): zero them
-  for (int task = threadIdx.x; task < (128 - min(d, 128)) * words_per_ch; task += blockDim.x) {
-    const int c = d + task % (128 - d), w = task / (128 - d);
-    const int block4 = (t0 / (4 * BETA)) + w;
-    *reinterpret_cast<uint32_t*>(vt_sf + bh * sf_head_bytes + sf_word_offset(c, block4, nkc)) = 0u;
+  if (cg == 0 && d < 128) {
+    // rows d..127 of the 128-row scale group are padding (d = 64): zero them
+    for (int task = threadIdx.x; task < (128 - d) * words_per_ch; task += blockDim.x) {
+      const int c = d + task % (128 - d), w = task / (128 - d);
+      *reinterpret_cast<uint32_t*>(vt_sf + head * sf_head_bytes + sf_word_offset(c, t0 / (4 * BETA) + w, nkc)) = 0u;
+    }
   }
-  for (int task = threadIdx.x; task < d * words_per_ch; task += blockDim.x) {
-    const int c = task % d, w = task / d;
+  for (int task = threadIdx.x; task < kVCh * words_per_ch; task += blockDim.x) {
+    const int cl = task % kVCh, w = task / kVCh;
+    const int c = c_base + cl;
     uint32_t sc_word = 0;
     uint32_t out[4 * BETA / 8];
 #pragma unroll
@@ -180,24 +182,55 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const T* __restrict__ v
       float val[BETA];
 #pragma unroll
       for (int i = 0; i < BETA; ++i) {
-        int tt = w * 4 * BETA + blk * BETA + i;
+        const int tt = w * 4 * BETA + blk * BETA + i;
         if constexpr (std::is_same<T, __nv_bfloat16>::value)
-          val[i] = __bfloat162float(tile[tt * d + c]);
+          val[i] = __bfloat162float(tile_smem[tt * kVCh + cl]);
         else
-          val[i] = __half2float(tile[tt * d + c]);
+          val[i] = __half2float(tile_smem[tt * kVCh + cl]);
       }
       uint32_t packed[BETA / 8];
-      uint32_t sc = quant_block<FMT, BETA>(val, packed);
+      const uint32_t sc = quant_block<FMT, BETA>(val, packed);
 #pragma unroll
       for (int j = 0; j < BETA / 8; ++j) out[blk * (BETA / 8) + j] = packed[j];
       sc_word |= sc << (8 * blk);
     }
-    uint8_t* dst = vt_codes + (bh * d + c) * static_cast<int64_t>(Np / 2) + (t0 + w * 4 * BETA) / 2;
+    uint8_t* dst = vt_codes + (head * d + c) * static_cast<int64_t>(Np / 2) + (t0 + w * 4 * BETA) / 2;
 #pragma unroll
     for (int j = 0; j < 4 * BETA / 8; j += 4)
       *reinterpret_cast<uint4*>(dst + 4 * j) = make_uint4(out[j], out[j + 1], out[j + 2], out[j + 3]);
-    const int block4 = (t0 / (4 * BETA)) + w;
-    *reinterpret_cast<uint32_t*>(vt_sf + bh * sf_head_bytes + sf_word_offset(c, block4, nkc)) = sc_word;
+    *reinterpret_cast<uint32_t*>(vt_sf + head * sf_head_bytes + sf_word_offset(c, t0 / (4 * BETA) + w, nkc)) =
+        sc_word;
+  }
+}
+
+// One launch for the whole step: CTAs [0, nq) quantize Q rows, [nq, nq+nk)
+// K rows, the rest V tiles.
+struct QuantArgs {
+  const void *q, *k, *v;
+  const float *s, *inv_s;
+  uint8_t *qc, *qs, *kc, *ks, *vc, *vs;
+  int B, Hq, Hkv, N, Np, d;
+  int64_t sf_qk_head, sf_v_head, q_words, k_words;
+  int nq_ctas, nk_ctas;
+};
+
+template <int FMT, typename T>
+__global__ void __launch_bounds__(256) quantize_qkv_kernel(const QuantArgs a) {
+  __shared__ __align__(16) T tile_smem[128 * kVCh];
+  const int bid = blockIdx.x;
+  if (bid < a.nq_ctas) {
+    const int64_t idx = static_cast<int64_t>(bid) * blockDim.x + threadIdx.x;
+    if (idx < a.q_words)
+      quantize_row_word<FMT, T>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.d, a.s, a.qc, a.qs,
+                                a.sf_qk_head, idx);
+  } else if (bid < a.nq_ctas + a.nk_ctas) {
+    const int64_t idx = static_cast<int64_t>(bid - a.nq_ctas) * blockDim.x + threadIdx.x;
+    if (idx < a.k_words)
+      quantize_row_word<FMT, T>(static_cast<const T*>(a.k), a.Hkv, 1, a.N, a.Np, a.d, a.inv_s, a.kc, a.ks,
+                                a.sf_qk_head, idx);
+  } else {
+    quantize_v_tile<FMT, T>(static_cast<const T*>(a.v), a.N, a.Np, a.d, a.vc, a.vs, a.sf_v_head,
+                            bid - a.nq_ctas - a.nk_ctas, tile_smem);
   }
 }
 
@@ -243,56 +276,30 @@ __global__ void calib_finalize_kernel(float* s, float* inv_s, int n, double alph
 }
 
 // ---------------------------------------------------------- host launchers ---
-// Rows of one tensor (Q with G = Hq/Hkv, or K with G = 1) and V^T.
 template <typename T>
-static void launch_rows(const void* x, int B, int H, int G, int N, int d, const float* scale, int fmt, uint8_t* codes,
-                        uint8_t* sf, cudaStream_t st) {
-  const int beta = beta_of(fmt);
-  const int Np = static_cast<int>(pad128(N));
-  const int wpr = (d / beta + 3) / 4;
-  const int64_t sfh = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
-  const int64_t total = static_cast<int64_t>(B) * H * Np * wpr;
-  const int thr = 256;
-  const unsigned grid = static_cast<unsigned>((total + thr - 1) / thr);
-  if (fmt == HIFA4_NVFP4)
-    quantize_rows_kernel<HIFA4_NVFP4, T><<<grid, thr, 0, st>>>(static_cast<const T*>(x), H, G, N, Np, d, scale, codes,
-                                                                sf, sfh, total);
-  else
-    quantize_rows_kernel<HIFA4_MXFP4, T><<<grid, thr, 0, st>>>(static_cast<const T*>(x), H, G, N, Np, d, scale, codes,
-                                                                sf, sfh, total);
+static void launch_quant(const QuantArgs& a, int fmt, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(a.nq_ctas + a.nk_ctas + (a.Np / 128) * (a.B * a.Hkv) * (a.d / kVCh));
+  if (fmt == HIFA4_NVFP4) quantize_qkv_kernel<HIFA4_NVFP4, T><<<grid, 256, 0, st>>>(a);
+  else quantize_qkv_kernel<HIFA4_MXFP4, T><<<grid, 256, 0, st>>>(a);
 }
 
-template <typename T>
-static void launch_v(const void* v, int B, int Hkv, int N, int d, int fmt, uint8_t* vc, uint8_t* vs, cudaStream_t st) {
-  const int Np = static_cast<int>(pad128(N));
-  const int64_t sfv = static_cast<int64_t>(hifa4_scale_bytes(d, Np, static_cast<hifa4_format>(fmt)));
-  const size_t vsmem = static_cast<size_t>(128) * d * sizeof(T);
-  const dim3 vgrid(Np / 128, B * Hkv);
-  if (fmt == HIFA4_NVFP4) {
-    if (vsmem > 48 * 1024)
-      cudaFuncSetAttribute(quantize_v_kernel<HIFA4_NVFP4, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(vsmem));
-    quantize_v_kernel<HIFA4_NVFP4, T><<<vgrid, 256, vsmem, st>>>(static_cast<const T*>(v), N, Np, d, vc, vs, sfv);
-  } else {
-    if (vsmem > 48 * 1024)
-      cudaFuncSetAttribute(quantize_v_kernel<HIFA4_MXFP4, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(vsmem));
-    quantize_v_kernel<HIFA4_MXFP4, T><<<vgrid, 256, vsmem, st>>>(static_cast<const T*>(v), N, Np, d, vc, vs, sfv);
-  }
-}
-
+// q == nullptr quantizes only K and V (a KV cache).
 hifa4_status quantize_qkv_launch(const void* q, const void* k, const void* v, int dt, int B, int Hq, int Hkv, int N,
                                  int d, const float* s, const float* inv_s, int fmt, uint8_t* qc, uint8_t* qs,
                                  uint8_t* kc, uint8_t* ks, uint8_t* vc, uint8_t* vs, cudaStream_t st) {
-  if (dt == HIFA4_BF16) {
-    if (q) launch_rows<__nv_bfloat16>(q, B, Hq, Hq / Hkv, N, d, s, fmt, qc, qs, st);
-    launch_rows<__nv_bfloat16>(k, B, Hkv, 1, N, d, inv_s, fmt, kc, ks, st);
-    launch_v<__nv_bfloat16>(v, B, Hkv, N, d, fmt, vc, vs, st);
-  } else {
-    if (q) launch_rows<__half>(q, B, Hq, Hq / Hkv, N, d, s, fmt, qc, qs, st);
-    launch_rows<__half>(k, B, Hkv, 1, N, d, inv_s, fmt, kc, ks, st);
-    launch_v<__half>(v, B, Hkv, N, d, fmt, vc, vs, st);
-  }
+  QuantArgs a;
+  a.q = q; a.k = k; a.v = v; a.s = s; a.inv_s = inv_s;
+  a.qc = qc; a.qs = qs; a.kc = kc; a.ks = ks; a.vc = vc; a.vs = vs;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.N = N; a.Np = static_cast<int>(pad128(N)); a.d = d;
+  const int wpr = (d / beta_of(fmt) + 3) / 4;
+  a.sf_qk_head = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
+  a.sf_v_head = static_cast<int64_t>(hifa4_scale_bytes(d, a.Np, static_cast<hifa4_format>(fmt)));
+  a.q_words = q ? static_cast<int64_t>(B) * Hq * a.Np * wpr : 0;
+  a.k_words = static_cast<int64_t>(B) * Hkv * a.Np * wpr;
+  a.nq_ctas = static_cast<int>((a.q_words + 255) / 256);
+  a.nk_ctas = static_cast<int>((a.k_words + 255) / 256);
+  if (dt == HIFA4_BF16) launch_quant<__nv_bfloat16>(a, fmt, st);
+  else launch_quant<__half>(a, fmt, st);
   return launch_status(q ? "quantize_qkv" : "quantize_kv");
 }
 
