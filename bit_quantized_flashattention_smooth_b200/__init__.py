@@ -34,7 +34,7 @@ ABI_FUNCTIONS = (
     "hifa4_quantize_kv",
     "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
-    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_status_string", "hifa4_last_error",
+    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
 )
 
@@ -67,6 +67,7 @@ def lib():
         L.hifa4_fp4_mma_probe.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, vp]
         L.hifa4_convert_probe.argtypes = [vp, i64, vp, vp, vp]
         L.hifa4_div6_probe.argtypes = [ctypes.c_uint32, ctypes.c_uint32, vp, vp, vp]
+        L.hifa4_exp2_poly_probe.argtypes = [vp, i64, vp, vp]
         L.hifa4_status_string.argtypes = [i]; L.hifa4_status_string.restype = ctypes.c_char_p
         L.hifa4_last_error.argtypes = []; L.hifa4_last_error.restype = ctypes.c_char_p
         L.hifa4_device_error.argtypes = []; L.hifa4_device_error.restype = ctypes.c_uint
@@ -289,6 +290,14 @@ def div6_probe(lo_bits: int, hi_bits: int):
     first = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     _check(lib().hifa4_div6_probe(lo_bits, hi_bits, _ptr(cnt), _ptr(first), _stream()), "div6_probe")
     return int(cnt.item()), int(first.item()) & 0xFFFFFFFF
+
+
+def exp2_poly_probe(y: torch.Tensor) -> torch.Tensor:
+    """The prefill kernel's FMA-pipe 2^y (for y <= 0) applied element-wise."""
+    y = y.contiguous().float()
+    out = torch.empty_like(y)
+    _check(lib().hifa4_exp2_poly_probe(_ptr(y), y.numel(), _ptr(out), _stream()), "exp2_poly_probe")
+    return out
 
 
 def convert_probe(x: torch.Tensor):

@@ -87,6 +87,7 @@ hifa4_status fp4_mma_probe_launch(const uint8_t*, const uint8_t*, const uint8_t*
                                   int, float*, cudaStream_t);
 hifa4_status convert_probe_launch(const float*, int64_t, uint8_t*, uint8_t*, cudaStream_t);
 hifa4_status div6_probe_launch(uint32_t, uint32_t, unsigned long long*, uint32_t*, cudaStream_t);
+hifa4_status exp2_poly_probe_launch(const float*, int64_t, float*, cudaStream_t);
 
 }  // namespace hifa4
 
@@ -254,6 +255,11 @@ hifa4_status hifa4_div6_probe(uint32_t lo_bits, uint32_t hi_bits, unsigned long 
                               uint32_t* first_bad, hifa4_stream_t stream) {
   HIFA4_REQUIRE(mismatches && first_bad && lo_bits <= hi_bits, HIFA4_ERR_INVALID_ARG, "div6_probe: bad args");
   return div6_probe_launch(lo_bits, hi_bits, mismatches, first_bad, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_exp2_poly_probe(const float* y, int64_t count, float* out, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(count >= 0 && (count == 0 || (y && out)), HIFA4_ERR_INVALID_ARG, "exp2_poly_probe: bad args");
+  return exp2_poly_probe_launch(y, count, out, static_cast<cudaStream_t>(stream));
 }
 
 const char* hifa4_status_string(hifa4_status st) {

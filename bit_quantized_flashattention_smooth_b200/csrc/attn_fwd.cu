@@ -7,27 +7,27 @@
 // quantized to P-hat per tile, and under P-Reordering l is accumulated from
 // the same P-hat that feeds the PV GEMM, fused into that GEMM.
 //
-// B200 design (one CTA = one 128-row query tile of one (batch, q head)):
-//   warp 8      TMA producer: Q-hat tile once, then K-hat / V-hat^T tiles and
+// B200 design (one CTA = one 128-row query tile of one (batch, q head)),
+// with NH = 1 or 2 softmax warpgroups per row (1 for 64-key tiles, 2 for
+// 128-key tiles; W = 4 * NH softmax warps):
+//   warp W      TMA producer: Q-hat tile once, then K-hat / V-hat^T tiles and
 //               their tiled scale chunks into an NS-stage ring (mbarriers).
-//   warp 9      MMA issuer (one thread): copies scale chunks shared->TMEM with
+//   warp W+1    MMA issuer (one thread): copies scale chunks shared->TMEM with
 //               tcgen05.cp, issues block-scaled tcgen05.mma for S = Q K^T
 //               into a TMEM S buffer, and for O += P-hat V-hat plus
 //               L += P-hat * ones (the fused normalizer: a 16-row all-ones B
 //               tile, so column 0 of L is sum(P-hat) with the same P-hat
 //               codes and scales as O).  Completion is signalled with
 //               tcgen05.commit onto mbarriers.
-//   warps 0-7   softmax: two warpgroups share each query row r (TMEM lane
-//               r), each with half of the key columns and half of O; the
-//               row max is exchanged in shared memory.  Per key
-//               tile: tcgen05.ld the S row, online max, P = 2^(S*c - m),
-//               per-block P-hat quantization in registers (cvt to E4M3 /
-//               E2M1), codes stored swizzled into shared memory as the A
-//               operand of the PV MMA, scales into a TMEM-copy chunk; when m
-//               rises, rescale the row of O and L in TMEM (after the previous
-//               PV MMA retired).  Epilogue: O / l, lse, optional debug sums.
-// Key tiles are visited in ascending order (P-hat depends on the running
-// max).  Every wait is bounded (ptx.cuh).
+//   warps 0..W-1 softmax: thread (h, r) owns TMEM lane r (query row r) and
+//               the h-th of NH column slices of S, P-hat and O; with NH = 2
+//               the row max is exchanged in shared memory.  Per key tile:
+//               tcgen05.ld the S row, block maxima, online max, block scales,
+//               P = 2^(S*c - m) and its E2M1 codes in registers, codes stored
+//               swizzled into shared memory as the A operand of the PV MMA,
+//               scales into a TMEM-copy chunk; when m rises, rescale the row
+//               of O and L in TMEM (after the previous PV MMA retired).
+//               Epilogue: O / l, lse, optional debug sums.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -35,6 +35,17 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+
+// Tuning knobs (measured on the 32-head, 4096-token causal prefill):
+// element pairs (of every eight pairs) whose 2^y runs on the FMA pipe (-1: 0 for
+// 64-key tiles, 2 for 128-key tiles), and softmax warpgroups per row for
+// 64-key tiles.
+#ifndef HIFA4_POLY_PAIRS
+#define HIFA4_POLY_PAIRS -1
+#endif
+#ifndef HIFA4_ATTN_NH_BN64
+#define HIFA4_ATTN_NH_BN64 1
+#endif
 
 namespace hifa4 {
 
@@ -59,6 +70,12 @@ template <int D, int BN, int FMT>
 struct AttnCfg {
   static constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
   static constexpr int BM = 128;
+  // softmax warpgroups per query row: 2 split each row's key columns (and O
+  // columns) between two warpgroups, 1 gives each thread a whole row
+  static constexpr int NH = BN == 64 ? HIFA4_ATTN_NH_BN64 : 2;
+  static constexpr int WARP_TMA = 4 * NH;
+  static constexpr int WARP_MMA = 4 * NH + 1;
+  static constexpr int NTHREADS = 32 * (4 * NH + 2);
   static constexpr int NS = D == 256 ? 2 : 3;               // K/V pipeline stages
   static constexpr int QROW = D / 2;                        // bytes per Q/K row
   static constexpr int PROW = BN / 2;                       // bytes per P-hat / V^T row
@@ -160,7 +177,7 @@ __device__ __forceinline__ uint32_t swz_chunk(uint32_t r, uint32_t c, uint32_t r
 }
 
 template <int D, int BN, int FMT, bool PREORDER>
-__global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
+__global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D, BN, FMT>;
@@ -198,16 +215,16 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     }
     for (int s = 0; s < C::NSB; ++s) {
       mbar_init(BAR(B_SFULL + s), 1);
-      mbar_init(BAR(B_SEMPTY + s), 8);
+      mbar_init(BAR(B_SEMPTY + s), 4 * C::NH);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(BAR(B_PFULL + s), 8);
+      mbar_init(BAR(B_PFULL + s), 4 * C::NH);
       mbar_init(BAR(B_PEMPTY + s), 1);
     }
     mbar_init(BAR(B_ORDY), 1);
-    mbar_init(BAR(B_XM), 256);    // row-max exchange between the two column halves
-    mbar_init(BAR(B_EP1), 128);   // epilogue: half 1 -> half 0
-    mbar_init(BAR(B_EP2), 128);   // epilogue: half 0 -> half 1
+    mbar_init(BAR(B_XM), 8);      // row-max exchange between two column halves (one arrival per warp)
+    mbar_init(BAR(B_EP1), 4);     // epilogue: half 1 -> half 0
+    mbar_init(BAR(B_EP2), 4);     // epilogue: half 0 -> half 1
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -225,11 +242,11 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     reinterpret_cast<float*>(smem + C::OFF_INV)[i] = i == 0 ? 0.0f : __fdiv_rn(1.0f, sd);
   }
   fence_proxy_async_smem();
-  if (warp == 9) {
+  if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == C::WARP_TMA && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -239,7 +256,7 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == C::WARP_TMA) {
     // =============================== TMA producer ===============================
     if (lane == 0) {
       const uint8_t* qsf = p.q_sf + static_cast<int64_t>(bhq) * p.sf_qk_head + static_cast<int64_t>(qtile) * C::NKC_Q * 512;
@@ -266,7 +283,7 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
                     C::NCH_V * 512, BAR(B_VFULL + st));
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == C::WARP_MMA) {
     // ================================ MMA issuer ================================
     if (lane == 0) {
       constexpr bool MX = FMT == HIFA4_MXFP4;
@@ -357,8 +374,8 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     // key columns [hw*BN/2, (hw+1)*BN/2) of S and P-hat, and output columns
     // [hw*D/2, (hw+1)*D/2) of O.  The row maximum is exchanged through
     // shared memory once per key tile.
-    constexpr int HB = BN / 2;                       // key columns per thread
-    constexpr int HD = D / 2;                        // output columns per thread
+    constexpr int HB = BN / C::NH;                   // key columns per thread
+    constexpr int HD = D / C::NH;                    // output columns per thread
     constexpr int NBH = HB / C::BETA;                // P-hat blocks per thread
     const int hw = warp >> 2;                        // column half
     const int r = threadIdx.x & 127;                 // row == TMEM lane
@@ -370,6 +387,8 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     const bool want_lp = !PREORDER || p.dbg_l_p != nullptr;
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
     constexpr float kInvGP = FMT == HIFA4_NVFP4 ? 256.0f : 1.0f;
+    // pairs (of every eight) whose 2^y runs on the FMA pipe instead of MUFU
+    constexpr int kPolyPairs = HIFA4_POLY_PAIRS >= 0 ? HIFA4_POLY_PAIRS : (BN == 128 ? 2 : 0);
     const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
     float* xm = reinterpret_cast<float*>(smem + C::OFF_XM);  // [2 parities][2 halves][128]
     bool ok = true;
@@ -383,13 +402,16 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
       tc_fence_after();
       float s[HB];
       {
+        // load and wait in one asm statement each (the destination registers
+        // fill asynchronously)
         uint32_t v[HB];
+        const uint32_t sa = tmem + lane_base + C::TM_S + sb * BN + hw * HB;
+        if constexpr (HB == 64) {
+          tmem_ld64_wait(sa, v);
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < HB / 32; ++cc)
-          tmem_ld32(tmem + lane_base + C::TM_S + sb * BN + hw * HB + cc * 32,
-                    *reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
-#pragma unroll
-        for (int cc = 0; cc < HB / 32; ++cc) tmem_wait_ld_dep(*reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
+          for (int cc = 0; cc < HB / 32; ++cc) tmem_ld32_wait(sa + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * cc));
+        }
 #pragma unroll
         for (int i = 0; i < HB; ++i) s[i] = __uint_as_float(v[i]);
       }
@@ -404,64 +426,70 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
 #pragma unroll
         for (int k = 0; k < HB; ++k) s[k] = (kbase + k >= lim) ? -INFINITY : s[k];
       }
-      // x = fl32(S * c) first, then P = 2^(x - m): the row maximum gives
-      // exactly 2^0 = 1, as the written rule does.
-      const float2 c2 = make_float2(c, c);
+      // Block maxima of S; c > 0, so the maximum of x = fl32(S * c) over a
+      // block is fl32(max S * c) and needs no pass over x.
+      float bms[NBH];
 #pragma unroll
-      for (int k = 0; k < HB; k += 2) {
-        const float2 x = fmul2(make_float2(s[k], s[k + 1]), c2);
-        s[k] = x.x;
-        s[k + 1] = x.y;
+      for (int blk = 0; blk < NBH; ++blk) bms[blk] = tree_max<C::BETA>(s + blk * C::BETA);
+      float m_new;
+      if constexpr (C::NH == 2) {
+        float* xb = xm + (j & 1) * 256;
+        xb[hw * 128 + r] = __fmul_rn(tree_max<NBH>(bms), c);
+        __syncwarp();             // the warp's stores are ordered before lane 0's release
+        if (lane == 0) mbar_arrive(BAR(B_XM));
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_XM), j & 1, abort_flag, kErrTimeoutSoftmax))) {
+          ok = false;
+          break;
+        }
+        m_new = fmaxf(m, fmaxf(xb[r], xb[128 + r]));
+      } else {
+        m_new = fmaxf(m, __fmul_rn(tree_max<NBH>(bms), c));
       }
-      float* xb = xm + (j & 1) * 256;
-      xb[hw * 128 + r] = tree_max<HB>(s);
-      mbar_arrive(BAR(B_XM));     // release: this thread's max is visible to waiters
-      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_XM), j & 1, abort_flag, kErrTimeoutSoftmax))) {
-        ok = false;
-        break;
-      }
-      const float m_new = fmaxf(m, fmaxf(xb[r], xb[128 + r]));
       const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);
-      const float2 negm = make_float2(-m_new, -m_new);
-      // P = 2^(x - m_new); P-hat per block of BETA keys
-      uint32_t codes[HB / 8];
+      // Block scales first, from y_max = fl32(x_max - m) of each block: the
+      // maximum of P over the block is 2^(y_max) (2^y is monotonic), and the
+      // MXFP4 exponent follows from y_max exactly.
+      float mult[NBH];
       uint32_t scb[NBH];
-      float psum = 0.0f;
 #pragma unroll
       for (int blk = 0; blk < NBH; ++blk) {
-        float* pb_ = s + blk * C::BETA;
-#pragma unroll
-        for (int i = 0; i < C::BETA; i += 2) {
-          const float2 y = fadd2(make_float2(pb_[i], pb_[i + 1]), negm);
-          pb_[i] = y.x;
-          pb_[i + 1] = y.y;
-        }
-        float mult;
-        uint32_t sc;
+        const float ym = __fadd_rn(__fmul_rn(bms[blk], c), -m_new);
         if constexpr (FMT == HIFA4_NVFP4) {
-#pragma unroll
-          for (int i = 0; i < C::BETA; ++i) pb_[i] = ex2_approx(pb_[i]);
-          const float bmax = tree_max<C::BETA>(pb_);
-          const float t = __fmul_rn(div6_rn(bmax), kInvGP);   // fl32(amax/6) / g_P
-          sc = cvt_e4m3(t);
-          mult = inv_tab[sc];                                  // fl32(1/(scale*g_P)), 0 for scale 0
+          const float t = __fmul_rn(div6_rn(ex2_approx(ym)), kInvGP);   // fl32(amax/6) / g_P
+          scb[blk] = cvt_e4m3(t);
+          mult[blk] = inv_tab[scb[blk]];                                  // fl32(1/(scale*g_P)), 0 for scale 0
         } else {
-          // the shared exponent follows from the block maximum of y exactly
-          sc = mx_scale_from_ymax(tree_max<C::BETA>(pb_));
-#pragma unroll
-          for (int i = 0; i < C::BETA; ++i) pb_[i] = ex2_approx(pb_[i]);
-          mult = __uint_as_float((254u - sc) << 23);
+          scb[blk] = mx_scale_from_ymax(ym);
+          mult[blk] = __uint_as_float((254u - scb[blk]) << 23);
         }
-        const float2 m2 = make_float2(mult, mult);
+      }
+      // P = 2^(S*c - m) element by element (MUFU ex2 for most pairs, the
+      // FMA-pipe polynomial for kPolyPairs of every eight pairs), then the E2M1
+      // codes of P * mult.
+      uint32_t codes[HB / 8];
+      float psum = 0.0f;
+      const float2 c2 = make_float2(c, c);
+      const float2 nm2 = make_float2(-m_new, -m_new);
 #pragma unroll
-        for (int w = 0; w < C::BETA / 8; ++w) {
-          const float* e = pb_ + 8 * w;
-          codes[blk * (C::BETA / 8) + w] =
-              cvt_e2m1x8(fmul2(make_float2(e[0], e[1]), m2), fmul2(make_float2(e[2], e[3]), m2),
-                         fmul2(make_float2(e[4], e[5]), m2), fmul2(make_float2(e[6], e[7]), m2));
+      for (int w = 0; w < HB / 8; ++w) {
+        const int blk = (8 * w) / C::BETA;
+        const float2 m2 = make_float2(mult[blk], mult[blk]);
+        float2 e[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = 8 * w + 2 * q;
+          const float2 y = ffma2(make_float2(s[i], s[i + 1]), c2, nm2);
+          const int pair16 = (i % 16) / 2;
+          float2 pp;
+          if (pair16 < kPolyPairs) {
+            pp = exp2_poly2(y);
+          } else {
+            pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+          }
+          if (want_lp) psum += pp.x + pp.y;
+          e[q] = fmul2(pp, m2);
         }
-        scb[blk] = sc;
-        if (want_lp) psum += tree_sum<C::BETA>(pb_);
+        codes[w] = cvt_e2m1x8(e[0], e[1], e[2], e[3]);
       }
       if (want_lp) l_p = fmaf(alpha, l_p, psum);
       // the P-hat buffer pb was last read by PV_{j-2}
@@ -498,8 +526,7 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
         for (int cc = 0; cc < HD / 32; ++cc) {
           uint32_t v0[32];
           const uint32_t a0 = tmem + lane_base + C::TM_O + hw * HD + cc * 32;
-          tmem_ld32(a0, v0);
-          tmem_wait_ld_dep(v0);
+          tmem_ld32_wait(a0, v0);
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const float2 t0 = fmul2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), a2);
@@ -524,15 +551,25 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     // ---------------------------------- epilogue ----------------------------------
     // the two halves' partial sums of P (same recurrence) add up to l_p
     float* lpx = reinterpret_cast<float*>(smem + C::OFF_LP);
-    if (hw == 1) {
-      lpx[r] = l_p;
-      mbar_arrive(BAR(B_EP1));
-    } else {
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(BAR(B_EP1), 0, abort_flag, kErrTimeoutSoftmax));
-      l_p += lpx[r];
+    if constexpr (C::NH == 2) {
+      if (hw == 1) {
+        lpx[r] = l_p;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_EP1));
+      } else {
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(BAR(B_EP1), 0, abort_flag, kErrTimeoutSoftmax));
+        l_p += lpx[r];
+      }
     }
+    // O and L are final once the last PV MMA retired.  Its completion is
+    // awaited on the P-hat buffer's barrier, whose earlier phases are all
+    // known to be complete here (the P-hat waits above); the o_ready barrier
+    // may lag by two phases when the last tiles needed no rescale, and a
+    // parity wait cannot tell phase k from phase k-2.
+    const int jl = nkt - 1;
     const bool ready = __all_sync(0xffffffffu, ok && nkt > 0 &&
-                                                  mbar_wait(BAR(B_ORDY), (nkt - 1) & 1, abort_flag, kErrTimeoutSoftmax));
+                                                  mbar_wait(BAR(B_PEMPTY + (jl & 1)), (jl >> 1) & 1, abort_flag,
+                                                            kErrTimeoutSoftmax));
     if (ready) {
       tc_fence_after();
       uint32_t lv;
@@ -543,11 +580,14 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
       const int64_t orow = (static_cast<int64_t>(bhq) * p.N + row) * D + hw * HD;
       // INCONSISTENT: only half 0 holds the full l_p; share it
       float l_used = l_phat;
-      if constexpr (!PREORDER) {
+      if constexpr (!PREORDER && C::NH == 1) {
+        l_used = l_p;
+      } else if constexpr (!PREORDER) {
         // half 1 needs the full l_p of its row for the output scale
         if (hw == 0) {
           lpx[128 + r] = l_p;
-          mbar_arrive(BAR(B_EP2));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(B_EP2));
           l_used = l_p;
         } else {
           if (!mbar_wait(BAR(B_EP2), 0, abort_flag, kErrTimeoutSoftmax)) atomicOr(&g_device_error, kErrTimeoutSoftmax);
@@ -591,7 +631,7 @@ __global__ void __launch_bounds__(320, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, C::TMEM_ALLOC);
+  if (warp == C::WARP_MMA) tmem_dealloc(tmem, C::TMEM_ALLOC);
 }
 
 // ------------------------------------------------------------------ host ---
@@ -614,7 +654,7 @@ static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const ui
   const int smem = C::SMEM_REQ;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * p.num_qtiles;
-  kern<<<grid, 320, smem, st>>>(tq, tk, tv, p);
+  kern<<<grid, C::NTHREADS, smem, st>>>(tq, tk, tv, p);
   return launch_status("attn_fwd");
 }
 

@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(192, 3)
       mbar_init(BAR(B_OFULL + s), 1);
       mbar_init(BAR(B_OEMPTY + s), 4);
     }
-    mbar_init(BAR(B_RED), 128);    // cross-warp reductions of the softmax warps
+    mbar_init(BAR(B_RED), 4);      // cross-warp reductions of the softmax warps (one arrival per warp)
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -344,7 +344,8 @@ __global__ void __launch_bounds__(192, 3)
         if (lane == q) rbuf[warp * 8 + q] = mx;
       }
       // exchange round 2j (the sums of the inconsistent mode use round 2j+1)
-      mbar_arrive(BAR(B_RED));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_RED));
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_RED), PREORDER ? (j & 1) : 0, abort_flag, kErrTimeoutSoftmax))) {
         ok = false;
         break;
@@ -419,7 +420,8 @@ __global__ void __launch_bounds__(192, 3)
           for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
           if (lane == q) sbuf[warp * 8 + q] = sm;
         }
-        mbar_arrive(BAR(B_RED));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_RED));
         if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_RED), 1, abort_flag, kErrTimeoutSoftmax))) {
           ok = false;
           break;

@@ -183,4 +183,19 @@ hifa4_status convert_probe_launch(const float* x, int64_t n, uint8_t* e2m1, uint
   return launch_status("convert_probe");
 }
 
+__global__ void exp2_poly_probe_kernel(const float* __restrict__ y, int64_t n, float* __restrict__ out) {
+  for (int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); i < n;
+       i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float y1 = i + 1 < n ? y[i + 1] : 0.0f;
+    const float2 r = exp2_poly2(make_float2(y[i], y1));
+    out[i] = r.x;
+    if (i + 1 < n) out[i + 1] = r.y;
+  }
+}
+hifa4_status exp2_poly_probe_launch(const float* y, int64_t n, float* out, cudaStream_t st) {
+  if (n == 0) return HIFA4_OK;
+  exp2_poly_probe_kernel<<<148 * 4, 256, 0, st>>>(y, n, out);
+  return launch_status("exp2_poly_probe");
+}
+
 }  // namespace hifa4

@@ -238,6 +238,13 @@ HIFA4_API hifa4_status hifa4_convert_probe(const float* x, int64_t count, uint8_
 HIFA4_API hifa4_status hifa4_div6_probe(uint32_t lo_bits, uint32_t hi_bits, unsigned long long* mismatches,
                                         uint32_t* first_bad, hifa4_stream_t stream);
 
+/* The FMA-pipe 2^y the prefill kernel uses for part of each P tile (range
+ * reduction to the nearest integer plus a degree-4 polynomial, see ptx.cuh),
+ * applied to `count` fp32 values y <= 0 (device in, device out).  Lets a test
+ * hold its relative error to the fitted bound and check the y <= -127 -> 0
+ * and y = 0 -> 1 edges. */
+HIFA4_API hifa4_status hifa4_exp2_poly_probe(const float* y, int64_t count, float* out, hifa4_stream_t stream);
+
 /* ----------------------------------------------------------- errors --- */
 
 HIFA4_API const char* hifa4_status_string(hifa4_status st);

@@ -67,7 +67,8 @@ def test_tiny_mha_full(mode):
 
 @pytest.mark.parametrize("fmt", [oracle.NVFP4, oracle.MXFP4])
 def test_qwen3_prefill_full(fmt):
-    _, lph, lp = _prefill_case("qwen3_prefill", fmt, oracle.PREORDER, [(0, 128), (4096 - 128, 4096)])
+    _, lph, lp = _prefill_case("qwen3_prefill", fmt, oracle.PREORDER,
+                               [(0, 128), (640, 768), (2048 + 64, 2048 + 192), (4096 - 128, 4096)])
     # Theorem 1 on the full workload: net probability-mass loss
     eps = lph / lp - 1
     assert np.median(eps) < 0
@@ -103,3 +104,23 @@ def test_split_decode_full():
         ref = oracle.decode(U.to_np(q[b:b + 1]), s_np, cz, w.N, h.NVFP4, scale, h.PREORDER, 128, num_splits=used)
         ok, err, bound, cos = U.compare_out(o[b:b + 1], ref["O"])
         assert ok, f"decode b={b}: max|dO|={err:.3e} bound={bound:.3e} cos={cos:.6f}"
+
+
+@pytest.mark.parametrize("name,fmt", [("qwen3_prefill", oracle.NVFP4), ("qwen3_prefill", oracle.MXFP4),
+                                      ("gemma2_prefill", oracle.NVFP4)])
+def test_prefill_repeatable(name, fmt):
+    """Every output bit equal over repeated launches of the bench
+    configuration: the kernel has no order-dependent arithmetic, so a flipped
+    bit means a pipeline race (a buffer read before it was filled or after it
+    was reused)."""
+    w = W.WORKLOADS[name]
+    q, k, v = W.make_prefill(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    s, inv = h.calibrate_smooth_qk(qd[:, :, : w.n_cal], kd[:, :, : w.n_cal], w.n_cal)
+    z = h.quantize_qkv(qd, kd, vd, s, inv, fmt)
+    scale = 1.0 / math.sqrt(w.d)
+    o0 = h.attn_fwd(z, scale, w.causal, oracle.PREORDER, w.block_n, out_dtype=W.torch_dtype(w.dtype))
+    for _ in range(20):
+        o1 = h.attn_fwd(z, scale, w.causal, oracle.PREORDER, w.block_n, out_dtype=W.torch_dtype(w.dtype))
+        diff = (o1.view(torch.int16) != o0.view(torch.int16))
+        assert not bool(diff.any()), f"{name}: {int(diff.sum())} output elements changed between launches"
