@@ -29,6 +29,7 @@
 //               of O and L in TMEM (after the previous PV MMA retired).
 //               Epilogue: O / l, lse, optional debug sums.
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -45,6 +46,10 @@
 #endif
 #ifndef HIFA4_ATTN_NH_BN64
 #define HIFA4_ATTN_NH_BN64 1
+#endif
+// with one softmax warpgroup per row: a correction warpgroup rescales O
+#ifndef HIFA4_ATTN_CORR
+#define HIFA4_ATTN_CORR 0
 #endif
 
 namespace hifa4 {
@@ -73,9 +78,12 @@ struct AttnCfg {
   // softmax warpgroups per query row: 2 split each row's key columns (and O
   // columns) between two warpgroups, 1 gives each thread a whole row
   static constexpr int NH = BN == 64 ? HIFA4_ATTN_NH_BN64 : 2;
-  static constexpr int WARP_TMA = 4 * NH;
-  static constexpr int WARP_MMA = 4 * NH + 1;
-  static constexpr int NTHREADS = 32 * (4 * NH + 2);
+  // correction warps (4, one per TMEM lane quadrant) rescale the O rows
+  // when the running max rises, off the softmax warps' path
+  static constexpr int CORR = (NH == 1 && HIFA4_ATTN_CORR) ? 1 : 0;
+  static constexpr int WARP_TMA = 4 * NH + 4 * CORR;
+  static constexpr int WARP_MMA = WARP_TMA + 1;
+  static constexpr int NTHREADS = 32 * (WARP_MMA + 1);
   static constexpr int NS = D == 256 ? 2 : 3;               // K/V pipeline stages
   static constexpr int QROW = D / 2;                        // bytes per Q/K row
   static constexpr int PROW = BN / 2;                       // bytes per P-hat / V^T row
@@ -111,12 +119,14 @@ struct AttnCfg {
   static constexpr int OFF_PSF = OFF_VSF + NS * NRG_V * NCH_V * 512;
   static constexpr int OFF_ONESF = OFF_PSF + 2 * NKC_P * 512;
   static constexpr int OFF_INV = OFF_ONESF + 512;           // 128 floats: 1/scale per UE4M3 code
-  static constexpr int OFF_XM = OFF_INV + 512;              // row-max exchange [2][2][128] floats
+  static constexpr int OFF_LOG = OFF_INV + 512;             // 128 floats: log2 of the above
+  static constexpr int OFF_XM = OFF_LOG + 512;              // row-max exchange [2][2][128] floats, or
+                                                            // the correction warps' alpha [3][128]
   static constexpr int OFF_LP = OFF_XM + 2048;              // normalizer exchange [2][128] floats
   static constexpr int OFF_BAR = OFF_LP + 1024;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
   // s_full[NSB], s_empty[NSB], p_full[2], p_empty[2], o_ready
-  static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1 + 3;
+  static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1 + 3 + 24;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   // TMEM columns
@@ -176,6 +186,38 @@ __device__ __forceinline__ uint32_t swz_chunk(uint32_t r, uint32_t c, uint32_t r
   return c ^ ((r * row_bytes >> 7) & (row_bytes / 16 - 1));
 }
 
+// Scale this warp's 32 TMEM lanes of an HD-column O slice (and, with_l, the
+// L column) by alpha: chunks of at most 64 columns, one TMEM round trip each,
+// L riding along with the first.  The caller waits for the stores.
+template <int HD>
+__device__ __forceinline__ void rescale_o_rows(uint32_t a0, uint32_t al, bool with_l_slice, float alpha) {
+  constexpr int RC = HD < 64 ? HD : 64;
+  static_assert(RC == 32 || RC == 64, "O slice chunks of 32 or 64 columns");
+  const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+  for (int cc = 0; cc < HD / RC; ++cc) {
+    uint32_t v[RC];
+    uint32_t lv = 0;
+    const bool with_l = with_l_slice && cc == 0;
+    if (with_l) {
+      if constexpr (RC == 64) tmem_ld64_and1_wait(a0 + cc * RC, v, al, lv);
+      else tmem_ld32_and1_wait(a0 + cc * RC, v, al, lv);
+    } else {
+      if constexpr (RC == 64) tmem_ld64_wait(a0 + cc * RC, v);
+      else tmem_ld32_wait(a0 + cc * RC, v);
+    }
+#pragma unroll
+    for (int i = 0; i < RC; i += 2) {
+      const float2 t0 = fmul2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), a2);
+      v[i] = __float_as_uint(t0.x);
+      v[i + 1] = __float_as_uint(t0.y);
+    }
+    if constexpr (RC == 64) tmem_st64(a0 + cc * RC, v);
+    else tmem_st32(a0 + cc * RC, v);
+    if (with_l) tmem_st1(al, __float_as_uint(__uint_as_float(lv) * alpha));
+  }
+}
+
 template <int D, int BN, int FMT, bool PREORDER>
 __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -191,7 +233,9 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
   const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + C::NS, B_VFULL = 1 + 2 * C::NS, B_VEMPTY = 1 + 3 * C::NS,
             B_SFULL = 1 + 4 * C::NS, B_SEMPTY = B_SFULL + C::NSB, B_PFULL = B_SEMPTY + C::NSB,
-            B_PEMPTY = B_PFULL + 2, B_ORDY = B_PEMPTY + 2, B_XM = B_ORDY + 1, B_EP1 = B_XM + 1, B_EP2 = B_EP1 + 1;
+            B_PEMPTY = B_PFULL + 2, B_ORDY = B_PEMPTY + 2, B_XM = B_ORDY + 1, B_EP1 = B_XM + 1, B_EP2 = B_EP1 + 1,
+            B_AF = B_EP2 + 1,   // [quadrant][4]: softmax warp -> correction warp, alpha of tile j ready
+            B_OC = B_AF + 16;   // [quadrant][2]: correction warp -> MMA, O rescaled for PV_j
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -221,10 +265,10 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       mbar_init(BAR(B_PFULL + s), 4 * C::NH);
       mbar_init(BAR(B_PEMPTY + s), 1);
     }
-    mbar_init(BAR(B_ORDY), 1);
     mbar_init(BAR(B_XM), 8);      // row-max exchange between two column halves (one arrival per warp)
     mbar_init(BAR(B_EP1), 4);     // epilogue: half 1 -> half 0
     mbar_init(BAR(B_EP2), 4);     // epilogue: half 0 -> half 1
+    for (int i = 0; i < 24; ++i) mbar_init(BAR(B_AF + i), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -239,7 +283,9 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     reinterpret_cast<uint32_t*>(smem + C::OFF_ONESF)[i] = row_of_word < 16 ? one * 0x01010101u : 0u;
     // fl32(1 / (UE4M3(i) * g_P)), the P-hat element multiplier of scale code i
     const float sd = __fmul_rn(ue4m3_to_f32(i), FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f);
-    reinterpret_cast<float*>(smem + C::OFF_INV)[i] = i == 0 ? 0.0f : __fdiv_rn(1.0f, sd);
+    const float inv = i == 0 ? 0.0f : __fdiv_rn(1.0f, sd);
+    reinterpret_cast<float*>(smem + C::OFF_INV)[i] = inv;
+    reinterpret_cast<float*>(smem + C::OFF_LOG)[i] = i == 0 ? -INFINITY : log2f(inv);
   }
   fence_proxy_async_smem();
   if (warp == C::WARP_MMA) {
@@ -330,6 +376,15 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         const uint32_t ph = (j / C::NS) & 1;
         const int pb = j & 1;
         if (!mbar_wait(BAR(B_PFULL + pb), (j >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
+        if constexpr (C::CORR) {
+          // O (and L) rescaled for this tile's max by every lane quadrant
+          // (tile j >= 1 is phase (j-1)/2 of barrier (j-1)%2: the correction
+          // warps run at most two tiles ahead of this wait)
+          if (j > 0)
+            for (int q = 0; q < 4; ++q)
+              if (!mbar_wait(BAR(B_OC + 2 * q + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, kErrTimeoutMma))
+                return false;
+        }
         if (!mbar_wait(BAR(B_VFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
         tc_fence_after();
         for (int pc = 0; pc < C::NKC_P; ++pc)
@@ -356,7 +411,6 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
           mma(tmem + C::TM_L, a, b1, idesc_fp4(128, 16, MX, pbyte, pbyte), sfa,
               (tmem + C::TM_SFB_1) | (pbyte << 30), acc);
         }
-        tc_commit(BAR(B_ORDY));
         tc_commit(BAR(B_VEMPTY + st));
         tc_commit(BAR(B_PEMPTY + pb));
         return true;
@@ -367,6 +421,42 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         if (ok) ok = issue_pv(j);
       }
       if (!ok) drain_after_abort();
+    }
+  } else if (C::CORR && warp >= 4) {
+    // ================================ correction ================================
+    // Warp 4+q owns TMEM lanes [32q, 32q+32).  For every key tile j >= 1 it
+    // takes alpha_j = 2^(m_{j-1} - m_j) of its rows from the softmax warp of
+    // the same quadrant and, when any of them is below 1, scales those rows of
+    // O and L after PV_{j-1} retired; PV_j waits for it.
+    const int q = warp - 4;
+    const int r = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const float* xa = reinterpret_cast<const float*>(smem + C::OFF_XM);
+    bool ok = true;
+    for (int j = 1; j < nkt && ok; ++j) {
+      // tile j's alpha is phase (j-1)/4 of barrier (j-1)%4 of this quadrant
+      // (the softmax warp runs at most two tiles ahead: its tile j+3 waits for
+      // PV_{j+1}, which waits for this warp's tile j+1)
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_AF + 4 * q + ((j - 1) & 3)), ((j - 1) >> 2) & 1, abort_flag,
+                                             kErrTimeoutSoftmax))) {
+        ok = false;
+        break;
+      }
+      const float alpha = xa[(j % 3) * 128 + r];
+      if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+        // PV_{j-1} retired (its P-hat buffer's earlier phase is known complete)
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PEMPTY + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag,
+                                               kErrTimeoutSoftmax))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        rescale_o_rows<D>(tmem + lane_base + C::TM_O, tmem + lane_base + C::TM_L, true, alpha);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_OC + 2 * q + ((j - 1) & 1)));
     }
   } else {
     // ================================== softmax ==================================
@@ -390,6 +480,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     // pairs (of every eight) whose 2^y runs on the FMA pipe instead of MUFU
     constexpr int kPolyPairs = HIFA4_POLY_PAIRS >= 0 ? HIFA4_POLY_PAIRS : (BN == 128 ? 2 : 0);
     const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
+    const float* log_tab = reinterpret_cast<const float*>(smem + C::OFF_LOG);
     float* xm = reinterpret_cast<float*>(smem + C::OFF_XM);  // [2 parities][2 halves][128]
     bool ok = true;
     for (int j = 0; j < nkt && ok; ++j) {
@@ -446,6 +537,13 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         m_new = fmaxf(m, __fmul_rn(tree_max<NBH>(bms), c));
       }
       const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);
+      if constexpr (C::CORR) {
+        if (j > 0) {
+          reinterpret_cast<float*>(smem + C::OFF_XM)[(j % 3) * 128 + r] = alpha;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(B_AF + 4 * (warp & 3) + ((j - 1) & 3)));
+        }
+      }
       // Block scales first, from y_max = fl32(x_max - m) of each block: the
       // maximum of P over the block is 2^(y_max) (2^y is monotonic), and the
       // MXFP4 exponent follows from y_max exactly.
@@ -470,27 +568,51 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       float psum = 0.0f;
       const float2 c2 = make_float2(c, c);
       const float2 nm2 = make_float2(-m_new, -m_new);
+      // one straight-line body per choice of the running sum of P (a branch
+      // per element would split the block the compiler schedules)
+      auto quant_tile = [&](auto lp_tag) {
+        constexpr bool LP = decltype(lp_tag)::value;
+        float2 acc = make_float2(0.0f, 0.0f);
+        // Without the sum of P, the multiplier folds into the exponent:
+        // P * mult = 2^(S*c - m + log2 mult), one packed FMA per pair.
+        float lnb[NBH];
+        if constexpr (!LP) {
 #pragma unroll
-      for (int w = 0; w < HB / 8; ++w) {
-        const int blk = (8 * w) / C::BETA;
-        const float2 m2 = make_float2(mult[blk], mult[blk]);
-        float2 e[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int i = 8 * w + 2 * q;
-          const float2 y = ffma2(make_float2(s[i], s[i + 1]), c2, nm2);
-          const int pair16 = (i % 16) / 2;
-          float2 pp;
-          if (pair16 < kPolyPairs) {
-            pp = exp2_poly2(y);
-          } else {
-            pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+          for (int blk = 0; blk < NBH; ++blk) {
+            const float lm = FMT == HIFA4_NVFP4 ? log_tab[scb[blk]] : static_cast<float>(127 - static_cast<int>(scb[blk]));
+            lnb[blk] = lm - m_new;
           }
-          if (want_lp) psum += pp.x + pp.y;
-          e[q] = fmul2(pp, m2);
         }
-        codes[w] = cvt_e2m1x8(e[0], e[1], e[2], e[3]);
-      }
+#pragma unroll
+        for (int w = 0; w < HB / 8; ++w) {
+          const int blk = (8 * w) / C::BETA;
+          const float2 m2 = make_float2(mult[blk], mult[blk]);
+          const float2 nb2 = LP ? nm2 : make_float2(lnb[blk], lnb[blk]);
+          float2 e[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i = 8 * w + 2 * q;
+            const float2 y = ffma2(make_float2(s[i], s[i + 1]), c2, nb2);
+            const int pair16 = (i % 16) / 2;
+            float2 pp;
+            if (pair16 < kPolyPairs) {
+              pp = exp2_poly2(y);
+            } else {
+              pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+            }
+            if constexpr (LP) {
+              acc = fadd2(acc, pp);
+              e[q] = fmul2(pp, m2);
+            } else {
+              e[q] = pp;
+            }
+          }
+          codes[w] = cvt_e2m1x8(e[0], e[1], e[2], e[3]);
+        }
+        if constexpr (LP) psum = acc.x + acc.y;
+      };
+      if (want_lp) quant_tile(std::true_type{});
+      else quant_tile(std::false_type{});
       if (want_lp) l_p = fmaf(alpha, l_p, psum);
       // the P-hat buffer pb was last read by PV_{j-2}
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(BAR(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, abort_flag,
@@ -513,36 +635,20 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
           psf[(gb / 4) * 512 + (gb % 4)] = static_cast<unsigned char>(scb[blk]);
         }
       }
-      // rescale this half of the O row (and L) when the max rose, after
-      // PV_{j-1} retired
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_ORDY), (j - 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+      // rescale this slice of the O row (and L) when the max rose, after
+      // PV_{j-1} retired (awaited on its P-hat buffer's barrier, whose earlier
+      // phase, PV_{j-3}, completed before this tile's P-hat stores)
+      if (!C::CORR && j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PEMPTY + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag,
+                                               kErrTimeoutSoftmax))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-        for (int cc = 0; cc < HD / 32; ++cc) {
-          uint32_t v0[32];
-          const uint32_t a0 = tmem + lane_base + C::TM_O + hw * HD + cc * 32;
-          tmem_ld32_wait(a0, v0);
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 t0 = fmul2(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), a2);
-            v0[i] = __float_as_uint(t0.x);
-            v0[i + 1] = __float_as_uint(t0.y);
-          }
-          tmem_st32(a0, v0);
-        }
-        if (hw == 0) {
-          uint32_t lv;
-          tmem_ld1_wait(tmem + lane_base + C::TM_L, lv);
-          tmem_st1(tmem + lane_base + C::TM_L, __float_as_uint(__uint_as_float(lv) * alpha));
-        }
+        rescale_o_rows<HD>(tmem + lane_base + C::TM_O + hw * HD, tmem + lane_base + C::TM_L, hw == 0, alpha);
         tmem_wait_st();
       }
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();   // the P-hat codes and scales are read by the MMA (async proxy)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_PFULL + pb));
