@@ -34,7 +34,7 @@ ABI_FUNCTIONS = (
     "hifa4_quantize_kv",
     "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
-    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_status_string", "hifa4_last_error",
+    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
 )
 
@@ -68,6 +68,8 @@ def lib():
         L.hifa4_convert_probe.argtypes = [vp, i64, vp, vp, vp]
         L.hifa4_div6_probe.argtypes = [ctypes.c_uint32, ctypes.c_uint32, vp, vp, vp]
         L.hifa4_exp2_poly_probe.argtypes = [vp, i64, vp, vp]
+        L.hifa4_bf16_attn_fwd.argtypes = [vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp]
+        L.hifa4_bf16_transpose_v.argtypes = [vp, i, i, i, i, vp, vp]
         L.hifa4_status_string.argtypes = [i]; L.hifa4_status_string.restype = ctypes.c_char_p
         L.hifa4_last_error.argtypes = []; L.hifa4_last_error.restype = ctypes.c_char_p
         L.hifa4_device_error.argtypes = []; L.hifa4_device_error.restype = ctypes.c_uint
@@ -290,6 +292,29 @@ def div6_probe(lo_bits: int, hi_bits: int):
     first = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     _check(lib().hifa4_div6_probe(lo_bits, hi_bits, _ptr(cnt), _ptr(first), _stream()), "div6_probe")
     return int(cnt.item()), int(first.item()) & 0xFFFFFFFF
+
+
+def bf16_transpose_v(v: torch.Tensor) -> torch.Tensor:
+    """V [B, Hkv, N, d] bf16 -> V^T [B, Hkv, d, N] (the BF16 kernel's layout)."""
+    v = v.contiguous()
+    B, H, N, d = v.shape
+    vt = torch.empty((B, H, d, N), device=v.device, dtype=torch.bfloat16)
+    _check(lib().hifa4_bf16_transpose_v(_ptr(v), B, H, N, d, _ptr(vt), _stream()), "bf16_transpose_v")
+    return vt
+
+
+def bf16_attn_fwd(q: torch.Tensor, k: torch.Tensor, vt: torch.Tensor, softmax_scale: float | None = None,
+                  causal: bool = True, return_lse: bool = False, out: torch.Tensor | None = None):
+    """Plain BF16 attention (the unquantized baseline).  q [B,Hq,N,d], k [B,Hkv,N,d], vt [B,Hkv,d,N] bf16."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    o = out if out is not None else torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32) if return_lse else None
+    _check(lib().hifa4_bf16_attn_fwd(_ptr(q), _ptr(k), _ptr(vt), B, Hq, Hkv, N, d, float(softmax_scale), int(causal),
+                                     _ptr(o), _ptr(lse) if lse is not None else None, _stream()), "bf16_attn_fwd")
+    return (o, lse) if return_lse else o
 
 
 def exp2_poly_probe(y: torch.Tensor) -> torch.Tensor:

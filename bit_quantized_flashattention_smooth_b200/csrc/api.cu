@@ -88,6 +88,9 @@ hifa4_status fp4_mma_probe_launch(const uint8_t*, const uint8_t*, const uint8_t*
 hifa4_status convert_probe_launch(const float*, int64_t, uint8_t*, uint8_t*, cudaStream_t);
 hifa4_status div6_probe_launch(uint32_t, uint32_t, unsigned long long*, uint32_t*, cudaStream_t);
 hifa4_status exp2_poly_probe_launch(const float*, int64_t, float*, cudaStream_t);
+hifa4_status bf16_attn_launch(const void*, const void*, const void*, int, int, int, int, int, float, int, void*, float*,
+                              cudaStream_t);
+hifa4_status transpose_v_bf16_launch(const void*, int, int, int, int, void*, cudaStream_t);
 
 }  // namespace hifa4
 
@@ -255,6 +258,25 @@ hifa4_status hifa4_div6_probe(uint32_t lo_bits, uint32_t hi_bits, unsigned long 
                               uint32_t* first_bad, hifa4_stream_t stream) {
   HIFA4_REQUIRE(mismatches && first_bad && lo_bits <= hi_bits, HIFA4_ERR_INVALID_ARG, "div6_probe: bad args");
   return div6_probe_launch(lo_bits, hi_bits, mismatches, first_bad, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_bf16_attn_fwd(const void* q, const void* k, const void* vt, int B, int Hq, int Hkv, int N, int d,
+                                 float softmax_scale, int causal, void* o, float* lse, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(q && k && vt && o, HIFA4_ERR_INVALID_ARG, "bf16_attn_fwd: null pointer");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0 && N % 8 == 0, HIFA4_ERR_INVALID_ARG,
+                "bf16_attn_fwd: bad shape B=%d Hq=%d Hkv=%d N=%d (N a multiple of 8)", B, Hq, Hkv, N);
+  HIFA4_REQUIRE(d == 64 || d == 128, HIFA4_ERR_UNSUPPORTED, "bf16_attn_fwd: d=%d not in {64,128}", d);
+  HIFA4_REQUIRE(softmax_scale > 0.0f, HIFA4_ERR_INVALID_ARG, "bf16_attn_fwd: softmax_scale must be > 0");
+  HIFA4_REQUIRE(aligned16(q) && aligned16(k) && aligned16(vt) && aligned16(o), HIFA4_ERR_INVALID_ARG,
+                "bf16_attn_fwd: pointers must be 16-byte aligned");
+  HIFA4_REQUIRE(static_cast<int64_t>(B) * Hq * N < (int64_t(1) << 31), HIFA4_ERR_UNSUPPORTED,
+                "bf16_attn_fwd: problem too large");
+  return bf16_attn_launch(q, k, vt, B, Hq, Hkv, N, d, softmax_scale, causal, o, lse, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_bf16_transpose_v(const void* v, int B, int Hkv, int N, int d, void* vt, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(v && vt && B >= 0 && Hkv > 0 && N >= 0 && d > 0, HIFA4_ERR_INVALID_ARG, "bf16_transpose_v: bad args");
+  return transpose_v_bf16_launch(v, B, Hkv, N, d, vt, static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_exp2_poly_probe(const float* y, int64_t count, float* out, hifa4_stream_t stream) {

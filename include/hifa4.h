@@ -238,6 +238,25 @@ HIFA4_API hifa4_status hifa4_convert_probe(const float* x, int64_t count, uint8_
 HIFA4_API hifa4_status hifa4_div6_probe(uint32_t lo_bits, uint32_t hi_bits, unsigned long long* mismatches,
                                         uint32_t* first_bad, hifa4_stream_t stream);
 
+/* ------------------------------------------------- BF16 reference --- */
+
+/* Plain BF16 FlashAttention forward, the unquantized baseline the 4-bit path
+ * is measured against (no Smooth-QK, no quantization; P rounded to bf16 for
+ * the PV MMA, l summed in fp32 over the unrounded P).  All device pointers:
+ *   q  [B, Hq, N, d] bf16, k [B, Hkv, N, d] bf16,
+ *   vt [B, Hkv, d, N] bf16 (V transposed, see hifa4_bf16_transpose_v),
+ *   o  [B, Hq, N, d] bf16 (written), lse [B, Hq, N] f32 base-2 log-sum-exp
+ *   (m + log2 l of the scores times softmax_scale * log2 e) or NULL.
+ * d in {64, 128}; N a multiple of 8; Hq a multiple of Hkv (GQA); causal is
+ * top-left aligned.  Pointers 16-byte aligned.  Asynchronous on `stream`. */
+HIFA4_API hifa4_status hifa4_bf16_attn_fwd(const void* q, const void* k, const void* vt, int B, int Hq, int Hkv,
+                                           int N, int d, float softmax_scale, int causal, void* o, float* lse,
+                                           hifa4_stream_t stream);
+
+/* V [B, Hkv, N, d] bf16 -> vt [B, Hkv, d, N] bf16 (device, no overlap). */
+HIFA4_API hifa4_status hifa4_bf16_transpose_v(const void* v, int B, int Hkv, int N, int d, void* vt,
+                                              hifa4_stream_t stream);
+
 /* The FMA-pipe 2^y the prefill kernel uses for part of each P tile (range
  * reduction to the nearest integer plus a degree-4 polynomial, see ptx.cuh),
  * applied to `count` fp32 values y <= 0 (device in, device out).  Lets a test
