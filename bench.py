@@ -88,18 +88,26 @@ class ClockSampler:
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun env).  backend "gloo" runs the same
+    plumbing on CPU (tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return rank, world, local
+
+
+def _coll_device():
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
 
 
 def barrier(world):
@@ -109,12 +117,24 @@ def barrier(world):
 
 
 def allmax(x: float, world) -> float:
+    """Max over ranks (device time of a multi-GPU step is the slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=_coll_device(), dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, ms_per_rank: float, world: int) -> float:
+    """Whole-job throughput: the units all ranks processed (each its own batch,
+    no exchange) over the max-over-ranks time, per second."""
+    return units_per_rank * world / (allmax(ms_per_rank, world) * 1e-3)
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch of the workload."""
+    return seed + 1000 * rank
 
 
 # ------------------------------------------------------------ our arm -----
@@ -123,7 +143,7 @@ def run_prefill(args, rank, world):
     w = W.WORKLOADS[args.workload]
     fmt = h.NVFP4 if args.fmt == "nvfp4" else h.MXFP4
     mode = h.PREORDER if args.mode == "preorder" else h.INCONSISTENT
-    wr = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})   # each rank its own batch
+    wr = W.Workload(**{**w.__dict__, "seed": rank_seed(w.seed, rank)})   # each rank its own batch
     q, k, v = W.make_prefill(wr)
     dev = torch.device("cuda")
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
@@ -194,7 +214,112 @@ def run_prefill(args, rank, world):
 
     return dict(w=w, fmt=fmt, mode=mode, step_ms=step_ms_max, attn_ms=attn_ms_max, quant_ms=quant_ms,
                 flops=flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clk, wall=wall,
-                launches=2 * args.steps, qd=qd, kd=kd, vd=vd, z=z)
+                launches=2 * args.steps, qd=qd, kd=kd, vd=vd, z=z, o=o, s=s, inv=inv)
+
+
+def time_ms(fn, n=30):
+    """Mean device time of fn over n launches after 3 warm-ups, L2 flushed
+    before each (CUDA events on the current stream)."""
+    flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    return tot / n
+
+
+def exact_attention_rows(q, k, v, causal, scale, heads):
+    """fp32 softmax attention of the given heads on the unquantized inputs
+    (the 'exact BF16 attention' the 4-bit output is compared with)."""
+    B, Hq, N, d = q.shape
+    G = Hq // k.shape[1]
+    mask = torch.ones(N, N, dtype=torch.bool, device=q.device).tril() if causal else None
+    out = []
+    for hh in heads:
+        sc = (q[0, hh].float() @ k[0, hh // G].float().T) * scale
+        if mask is not None:
+            sc = sc.masked_fill(~mask, float("-inf"))
+        out.append(torch.softmax(sc, dim=-1) @ v[0, hh // G].float())
+    return torch.stack(out)
+
+
+def comparisons(res):
+    """Outside the timed region: the in-house BF16 kernel and the cuDNN BF16
+    attention on the same (unsmoothed, unquantized) inputs, the deviation of
+    the 4-bit output from exact attention, and the normalizer error eps of
+    both modes (Theorem 1)."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    w, z = res["w"], res["z"]
+    qd, kd, vd = res["qd"], res["kd"], res["vd"]
+    scale = 1.0 / math.sqrt(w.d)
+    out = {}
+    qb, kb, vb = qd.to(torch.bfloat16), kd.to(torch.bfloat16), vd.to(torch.bfloat16)
+    attn_ms = res["attn_ms"]
+    if w.d in (64, 128) and w.N % 8 == 0:
+        vt = h.bf16_transpose_v(vb)
+        ob = h.bf16_attn_fwd(qb, kb, vt, scale, w.causal)
+        ms = time_ms(lambda: h.bf16_attn_fwd(qb, kb, vt, scale, w.causal, out=ob))
+        out["bf16_inhouse"] = {"ms": ms, "tflops": res["flops"] / (ms * 1e-3) / 1e12,
+                               "fp4_speedup": ms / attn_ms, "kernel": "attn_fwd_bf16 (tcgen05 kind::f16)"}
+    try:
+        import torch.nn.functional as F
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        G = w.Hq // w.Hkv
+        kk, vv = kb.repeat_interleave(G, dim=1), vb.repeat_interleave(G, dim=1)
+        with sdpa_kernel(SDPBackend.CUDNN_ATTENTION):
+            ms = time_ms(lambda: F.scaled_dot_product_attention(qb, kk, vv, is_causal=w.causal, scale=scale))
+        out["bf16_cudnn_sdpa"] = {"ms": ms, "tflops": res["flops"] / (ms * 1e-3) / 1e12,
+                                  "fp4_speedup": ms / attn_ms, "note": "library kernel, context only"}
+        del kk, vv
+    except Exception as e:  # context only
+        out["bf16_cudnn_sdpa"] = {"error": str(e)[:120]}
+    # deviation from exact attention (4 heads of batch 0)
+    heads = list(range(min(4, w.Hq)))
+    ex = exact_attention_rows(qd, kd, vd, w.causal, scale, heads)
+    o4 = res["o"][0, heads].float()
+    out["deviation_from_exact"] = {"heads": heads, "max_abs_rel": float((o4 - ex).abs().max() / ex.abs().max()),
+                                   "cosine": float(torch.nn.functional.cosine_similarity(o4.flatten(), ex.flatten(), dim=0))}
+    if "bf16_inhouse" in out:
+        obf = ob[0, heads].float()
+        out["deviation_from_exact"]["bf16_inhouse_max_abs_rel"] = float((obf - ex).abs().max() / ex.abs().max())
+    # normalizer error: eps_row = l_Phat / l_P - 1; under P-Reordering the
+    # output divides by l_Phat itself, under the inconsistent mode by l_P, so
+    # O_incons / O_preorder - 1 equals eps row by row (coherent scaling)
+    o_pre, lph, lp = h.attn_fwd(z, scale, w.causal, h.PREORDER, w.block_n, out_dtype=torch.float16 if w.dtype == "fp16" else torch.bfloat16, debug=True)
+    o_inc = h.attn_fwd(z, scale, w.causal, h.INCONSISTENT, w.block_n, out_dtype=o_pre.dtype)
+    eps = (lph / lp - 1.0).flatten()
+    a, b = o_inc[0, heads].float().flatten(1), o_pre[0, heads].float().flatten(1)
+    scale_err = ((a * b).sum(1) / (b * b).sum(1) - 1.0)
+    out["epsilon"] = {"median": float(eps.median()), "p10": float(eps.quantile(0.1)) if eps.numel() < 1 << 24 else None,
+                      "frac_rows_negative": float((eps < 0).float().mean()),
+                      "preorder_output_scale_error": 0.0,
+                      "inconsistent_output_scale_error_median_over_heads": float(scale_err.median())}
+    return out
+
+
+def traffic_record(kernel, workload, fmt, block_n):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+    one ncu capture, from profiles/traffic.json, if the kernel source still has
+    the hash recorded with it (else None: the counters are stale)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "bit_quantized_flashattention_smooth_b200", "csrc", kernel.replace("_fp4", "") + ".cu")
+    if not os.path.exists(path) or not os.path.exists(src):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    for rec in json.load(open(path)):
+        if (rec.get("kernel") == kernel and rec.get("workload") == workload and rec.get("format") == fmt and
+                rec.get("block_n") == block_n and rec.get("source_sha256_16") == digest):
+            return rec["bytes_per_launch"]
+    return None
 
 
 def fp4_probe_peak():
@@ -307,6 +432,49 @@ def run_reference(args, rank, world):
                        f"of {w.name}")
 
 
+def profile_target(args, launches: int = 5):
+    """A short run of one kernel for an ncu capture: inputs built, then
+    `launches` launches of the target (skip the first with -s in ncu)."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    w = W.WORKLOADS[args.workload]
+    fmt = h.NVFP4 if args.fmt == "nvfp4" else h.MXFP4
+    mode = h.PREORDER if args.mode == "preorder" else h.INCONSISTENT
+    dev = torch.device("cuda")
+    if args.profile == "decode":
+        wd = W.WORKLOADS["split_decode"]
+        q, k, v, qcal, kcal = W.make_decode_device(wd, dev)
+        s, inv = h.calibrate_smooth_qk(qcal, kcal, wd.n_cal)
+        cache = h.quantize_kv(k, v, inv, h.NVFP4, Hq=wd.Hq)
+        del k, v
+        splits = h.default_splits(wd.B, wd.Hkv, wd.N)
+        ws = torch.empty(h.decode_workspace_bytes(wd.B, wd.Hq, wd.d, splits), device=dev, dtype=torch.uint8)
+        o = torch.empty((wd.B, wd.Hq, wd.d), device=dev, dtype=torch.bfloat16)
+        fn = lambda: h.attn_decode(q, s, cache, wd.N, None, h.PREORDER, splits, ws, o)  # noqa: E731
+    else:
+        q, k, v = W.make_prefill(w)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        s, inv = h.calibrate_smooth_qk(qd[:, :, : w.n_cal], kd[:, :, : w.n_cal], w.n_cal)
+        z = h.quantize_qkv(qd, kd, vd, s, inv, fmt)
+        scale = 1.0 / math.sqrt(w.d)
+        if args.profile == "quantize":
+            fn = lambda: h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)  # noqa: E731
+        elif args.profile == "attn":
+            o = torch.empty((w.B, w.Hq, w.N, w.d), device=dev, dtype=W.torch_dtype(w.dtype))
+            fn = lambda: h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)  # noqa: E731
+        else:
+            qb, kb = qd.to(torch.bfloat16), kd.to(torch.bfloat16)
+            vt = h.bf16_transpose_v(vd.to(torch.bfloat16))
+            ob = torch.empty_like(qb)
+            fn = lambda: h.bf16_attn_fwd(qb, kb, vt, scale, w.causal, out=ob)  # noqa: E731
+    for _ in range(launches):
+        fn()
+    torch.cuda.synchronize()
+    if h.device_error():
+        raise RuntimeError("device error word set")
+    print(json.dumps({"profile": args.profile, "workload": w.name if args.profile != "decode" else "split_decode",
+                      "launches": launches}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -320,6 +488,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-probe", action="store_true")
+    ap.add_argument("--no-compare", action="store_true", help="skip the BF16 / exact / epsilon comparisons")
+    ap.add_argument("--profile", choices=["attn", "quantize", "decode", "bf16"], default=None,
+                    help="run only this kernel a few times (for an ncu capture) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_setup(args.gpus)
@@ -329,6 +500,10 @@ def main():
     config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
               "format": args.fmt, "normalizer": args.mode, "block_n": w.block_n,
               "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}"}
+
+    if args.profile:
+        profile_target(args)
+        return
 
     if args.impl == "reference":
         ref = run_reference(args, rank, world)
@@ -343,11 +518,14 @@ def main():
                     "e2e": {"value": ref["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0,
                             "d2h_bytes_per_step": 0}}
             print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
         return
 
     pk = peaks()
     res = run_prefill(args, rank, world)
-    value = res["flops"] * world / (res["step_ms"] * 1e-3) / 1e12
+    value = weak_scaling_value(res["flops"], res["step_ms"], world) / 1e12
     attn_tflops = res["flops"] / (res["attn_ms"] * 1e-3) / 1e12
     fp4_peak = pk["bf16"] * FP4_OVER_BF16
     extra = {}
@@ -386,6 +564,24 @@ def main():
                               "frac": decode["gbs"] / pk["hbm"], "splits": decode["splits"]}
         else:
             line["decode"] = decode
+    line["tokens_per_s"] = w.B * w.N * world / (res["step_ms"] * 1e-3)
+    # the softmax's own ceiling: every score needs one 2^x, and the MUFU unit
+    # gives 16 per clock per SM (at the median SM clock seen while timing)
+    clk_mhz = (res["clocks"] or {}).get("sm_mhz") or 1965.0
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n_exp = W.exp_count(w)
+    line["roofline_softmax"] = {"bound": "alu", "unit": "exp2/s", "achieved": n_exp / (res["attn_ms"] * 1e-3),
+                                "peak": 16.0 * sms * clk_mhz * 1e6, "exp2_per_launch": n_exp,
+                                "frac": n_exp / (res["attn_ms"] * 1e-3) / (16.0 * sms * clk_mhz * 1e6),
+                                "note": "MUFU ex2 ceiling: 16/clk/SM x SMs x median SM clock"}
+    tr = traffic_record("attn_fwd_fp4", w.name, args.fmt, w.block_n)
+    if tr is not None:
+        line["roofline"]["traffic"] = tr
+    if rank == 0 and not args.no_compare:
+        try:
+            line["comparisons"] = comparisons(res)
+        except Exception as e:  # measurement only
+            line["comparisons"] = {"error": str(e)[:200]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, res["fmt"], res["mode"])
     if rank == 0:

@@ -173,6 +173,11 @@ def attended_pairs(N: int, causal: bool) -> int:
     return N * (N + 1) // 2 if causal else N * N
 
 
+def exp_count(w: Workload) -> float:
+    """2^x evaluations of the softmax: one per attended query-key pair."""
+    return float(w.B * w.Hq * attended_pairs(w.N, w.causal))
+
+
 def prefill_flops(w: Workload, N: int | None = None, B: int | None = None) -> float:
     """4 * B * Hq * d * (attended query-key pairs): QK^T and PV multiply-adds."""
     N = w.N if N is None else N
