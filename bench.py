@@ -48,7 +48,9 @@ class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
 
     def __init__(self, index: int):
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        import tempfile
+        log_dir = os.environ.get("HIFA4_CLOCK_LOG_DIR", tempfile.gettempdir())
+        self.path = os.path.join(log_dir, f"hifa4_clocks_rank{index}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"

@@ -19,8 +19,8 @@
  *   [NVFP4] NVIDIA NVFP4: 16 E2M1 elements share one unsigned E4M3 scale.
  *
  * The pages never define HIF4, the Smooth-QK scale formula, the P-hat scale,
- * or epsilon; the readings taken here are listed in the design doc and restated in
- * the comment of each function.
+ * or epsilon; the reading taken for each is stated in the comment of the
+ * function that implements it.
  *
  * Arithmetic: everything that is not a 4-bit/8-bit format decision is done in
  * double precision.  Format decisions (block amax, scale, element rounding)
