@@ -47,94 +47,132 @@ __device__ __forceinline__ void load8<__half>(const __half* p, float (&f)[8]) {
 
 // Quantize one block of BETA fp32 values in place into packed codes
 // (BETA/2 bytes, element 2i in the low nibble) and return the scale code.
+// inv_tab[c] = fl32(1 / UE4M3(c)) (0 for c = 0), in shared memory.
 template <int FMT, int BETA>
-__device__ __forceinline__ uint32_t quant_block(const float (&v)[BETA], uint32_t (&packed)[BETA / 8]) {
-  float amax = 0.0f;
+__device__ __forceinline__ uint32_t quant_block(const float (&v)[BETA], uint32_t (&packed)[BETA / 8],
+                                                const float* inv_tab) {
+  float amax = fmaxf(fabsf(v[0]), fabsf(v[1]));
 #pragma unroll
-  for (int i = 0; i < BETA; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  for (int i = 2; i + 1 < BETA; i += 2) amax = fmax3(amax, fabsf(v[i]), fabsf(v[i + 1]));
   float mult;
   uint32_t sc;
+  uint32_t keep = 0xFFFFFFFFu;
   if constexpr (FMT == HIFA4_NVFP4) {
-    float t = __fdiv_rn(amax, 6.0f);
+    // fl32(amax/6): the reciprocal-and-residual form is IEEE-exact on
+    // [2^-122, 2^20] (checked on the GPU); below, both give scale code 0
+    const float t = amax <= 1048576.0f ? div6_rn(amax) : __fdiv_rn(amax, 6.0f);
     sc = cvt_e4m3(t);
-    float sd = ue4m3_to_f32(sc);
-    mult = (sc == 0) ? 0.0f : __fdiv_rn(1.0f, sd);
+    mult = inv_tab[sc];
+    if (sc == 0) keep = 0u;                             // scale 0: every code 0 (no -0 codes)
   } else {
-    uint32_t ef = (__float_as_uint(amax) >> 23) & 0xFFu;
+    const uint32_t ef = (__float_as_uint(amax) >> 23) & 0xFFu;
     sc = ef >= 2u ? ef - 2u : 0u;                       // E + 127, E = floor(log2 amax) - 2
     mult = __uint_as_float((254u - sc) << 23);          // 2^-E
   }
+  const float2 m2 = make_float2(mult, mult);
 #pragma unroll
   for (int w = 0; w < BETA / 8; ++w) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float lo = __fmul_rn(v[8 * w + 2 * j], mult);
-      float hi = __fmul_rn(v[8 * w + 2 * j + 1], mult);
-      uint32_t byte = cvt_e2m1x2(hi, lo);
-      if (FMT == HIFA4_NVFP4 && sc == 0) byte = 0;
-      word |= byte << (8 * j);
-    }
-    packed[w] = word;
+    const float* e = v + 8 * w;
+    packed[w] = keep & cvt_e2m1x8(fmul2(make_float2(e[0], e[1]), m2), fmul2(make_float2(e[2], e[3]), m2),
+                                  fmul2(make_float2(e[4], e[5]), m2), fmul2(make_float2(e[6], e[7]), m2));
   }
   return sc;
 }
 
-// One thread per (row, scale word): a word covers up to 4 consecutive blocks
-// of a row.  x: [BH][N][d] rows of head bh; rows N..Np-1 are zero padding.
-// Head bh uses smoothing scale row (bh % H) / G of `scale` ([Hkv][d]).
-template <int FMT, typename T>
-__device__ __forceinline__ void quantize_row_word(const T* __restrict__ x, int H, int G, int N, int Np, int d,
+// Rows of Q or K, one lane per block: D/BETA lanes cover a row, so each
+// 16-byte load instruction of a warp touches a few whole 128-byte lines
+// instead of one line per lane, and the code bytes of a row are written by
+// consecutive lanes.  kLpbUnroll row groups per lane are loaded before any is
+// quantized.  Rows are flattened (head, token); tokens N..Np-1 are zero
+// padding; head bh uses smoothing row (bh % H) / G of `scale`.
+template <int FMT>
+struct LpbCfg {
+  static constexpr int kUnroll = FMT == HIFA4_NVFP4 ? 2 : 1;
+};
+
+template <int FMT, int D>
+struct RowTile {
+  static constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
+  static constexpr int U = LpbCfg<FMT>::kUnroll;
+  static constexpr int LPR = D / BETA;     // lanes (= blocks) per row
+  static constexpr int RPW = 32 / LPR;     // rows per warp and row group
+  static constexpr int ROWS = 8 * U * RPW; // rows per 256-thread CTA; divides 128
+  static_assert(128 % ROWS == 0, "a CTA's rows stay inside one head");
+};
+
+// CTA `cta` of a tensor with `heads` heads of Np (padded) rows: head
+// cta / (Np / ROWS), rows [chunk * ROWS, +ROWS).  Index arithmetic per CTA,
+// none per lane beyond shifts.
+template <int FMT, typename T, int D>
+__device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H, int G, int N, int Np,
                                                   const float* __restrict__ scale, uint8_t* __restrict__ codes,
-                                                  uint8_t* __restrict__ sf, int64_t sf_head_bytes, int64_t idx) {
-  constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
-  const int nb = d / BETA;
-  const int wpr = (nb + 3) / 4;
-  const int w = static_cast<int>(idx % wpr);
-  const int64_t rowg = idx / wpr;
-  const int t = static_cast<int>(rowg % Np);
-  const int64_t bh = rowg / Np;
-  const int kvh = static_cast<int>(bh % H) / G;
-  const int nbw = min(4, nb - 4 * w);
-  uint32_t sc_word = 0;
-  for (int blk = 0; blk < nbw; ++blk) {
-    const int c0 = (4 * w + blk) * BETA;
-    float v[BETA];
-    if (t < N) {
-      const T* src = x + (bh * N + t) * static_cast<int64_t>(d) + c0;
+                                                  uint8_t* __restrict__ sf, int64_t sf_head_bytes, int cta,
+                                                  const float* inv_tab) {
+  using R = RowTile<FMT, D>;
+  constexpr int BETA = R::BETA, U = R::U, LPR = R::LPR, RPW = R::RPW;
+  constexpr int WPR = (LPR + 3) / 4;       // scale words per row
+  const int cpt = Np / R::ROWS;
+  const int bh = cta / cpt;
+  const int chunk = cta - bh * cpt;
+  const int kvh = (bh % H) / G;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lb = lane % LPR;
+  const T* xh = x + static_cast<int64_t>(bh) * N * D + lb * BETA;
+  const float* srow = scale != nullptr ? scale + kvh * D + lb * BETA : nullptr;
+  float v[U][BETA];
+  int tok[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    tok[u] = chunk * R::ROWS + (warp * U + u) * RPW + lane / LPR;
+    if (tok[u] < N) {
+      const T* src = xh + static_cast<int64_t>(tok[u]) * D;
 #pragma unroll
       for (int i = 0; i < BETA / 8; ++i) {
         float f[8];
         load8<T>(src + 8 * i, f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[8 * i + j] = f[j];
-      }
-      if (scale != nullptr) {
-        const float4* s4 = reinterpret_cast<const float4*>(scale + static_cast<int64_t>(kvh) * d + c0);
-#pragma unroll
-        for (int i = 0; i < BETA / 4; ++i) {
-          float4 s = s4[i];
-          v[4 * i + 0] = __fmul_rn(v[4 * i + 0], s.x);
-          v[4 * i + 1] = __fmul_rn(v[4 * i + 1], s.y);
-          v[4 * i + 2] = __fmul_rn(v[4 * i + 2], s.z);
-          v[4 * i + 3] = __fmul_rn(v[4 * i + 3], s.w);
-        }
+        for (int j = 0; j < 8; ++j) v[u][8 * i + j] = f[j];
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < BETA; ++i) v[i] = 0.0f;
+      for (int i = 0; i < BETA; ++i) v[u][i] = 0.0f;
+    }
+  }
+  uint8_t* ch = codes + (static_cast<int64_t>(bh) * Np) * (D / 2) + lb * (BETA / 2);
+  uint8_t* sh = sf + static_cast<int64_t>(bh) * sf_head_bytes;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int t = tok[u];
+    if (srow != nullptr && t < N) {
+      const float4* s4 = reinterpret_cast<const float4*>(srow);
+#pragma unroll
+      for (int i = 0; i < BETA / 4; ++i) {
+        const float4 sv = s4[i];
+        const float2 p0 = fmul2(make_float2(v[u][4 * i + 0], v[u][4 * i + 1]), make_float2(sv.x, sv.y));
+        const float2 p1 = fmul2(make_float2(v[u][4 * i + 2], v[u][4 * i + 3]), make_float2(sv.z, sv.w));
+        v[u][4 * i + 0] = p0.x;
+        v[u][4 * i + 1] = p0.y;
+        v[u][4 * i + 2] = p1.x;
+        v[u][4 * i + 3] = p1.y;
+      }
     }
     uint32_t packed[BETA / 8];
-    uint32_t sc = quant_block<FMT, BETA>(v, packed);
-    uint8_t* dst = codes + (bh * Np + t) * static_cast<int64_t>(d / 2) + c0 / 2;
+    const uint32_t sc = quant_block<FMT, BETA>(v[u], packed, inv_tab);
+    uint8_t* dst = ch + static_cast<int64_t>(t) * (D / 2);
     if constexpr (BETA == 16) {
       *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
     } else {
       *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
-    sc_word |= sc << (8 * blk);
+    uint8_t* sfw = sh + sf_word_offset(t, lb / 4, WPR);
+    sfw[lb % 4] = static_cast<uint8_t>(sc);
+    if constexpr (LPR < 4) {
+      // the rest of the row's only scale word holds no block: zero it
+      if (lb == LPR - 1)
+#pragma unroll
+        for (int bb = LPR; bb < 4; ++bb) sfw[bb] = 0;   // lb / 4 == 0: the same word
+    }
   }
-  *reinterpret_cast<uint32_t*>(sf + bh * sf_head_bytes + sf_word_offset(t, w, wpr)) = sc_word;
 }
 
 // V: one CTA per (128-token tile, head, 64-channel group).  The tile is staged
@@ -145,7 +183,7 @@ constexpr int kVCh = 64;   // channels per V CTA
 template <int FMT, typename T>
 __device__ __forceinline__ void quantize_v_tile(const T* __restrict__ v, int N, int Np, int d,
                                                 uint8_t* __restrict__ vt_codes, uint8_t* __restrict__ vt_sf,
-                                                int64_t sf_head_bytes, int tile, T* tile_smem) {
+                                                int64_t sf_head_bytes, int tile, T* tile_smem, const float* inv_tab) {
   constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
   const int ncg = d / kVCh;
   const int cg = tile % ncg;
@@ -172,65 +210,62 @@ __device__ __forceinline__ void quantize_v_tile(const T* __restrict__ v, int N, 
       *reinterpret_cast<uint32_t*>(vt_sf + head * sf_head_bytes + sf_word_offset(c, t0 / (4 * BETA) + w, nkc)) = 0u;
     }
   }
-  for (int task = threadIdx.x; task < kVCh * words_per_ch; task += blockDim.x) {
-    const int cl = task % kVCh, w = task / kVCh;
+  // one task per (channel, token block): all threads busy, codes and the
+  // scale byte written per block
+  for (int task = threadIdx.x; task < kVCh * (128 / BETA); task += blockDim.x) {
+    const int cl = task % kVCh, blk = task / kVCh;
     const int c = c_base + cl;
-    uint32_t sc_word = 0;
-    uint32_t out[4 * BETA / 8];
+    float val[BETA];
 #pragma unroll
-    for (int blk = 0; blk < 4; ++blk) {
-      float val[BETA];
-#pragma unroll
-      for (int i = 0; i < BETA; ++i) {
-        const int tt = w * 4 * BETA + blk * BETA + i;
-        if constexpr (std::is_same<T, __nv_bfloat16>::value)
-          val[i] = __bfloat162float(tile_smem[tt * kVCh + cl]);
-        else
-          val[i] = __half2float(tile_smem[tt * kVCh + cl]);
-      }
-      uint32_t packed[BETA / 8];
-      const uint32_t sc = quant_block<FMT, BETA>(val, packed);
-#pragma unroll
-      for (int j = 0; j < BETA / 8; ++j) out[blk * (BETA / 8) + j] = packed[j];
-      sc_word |= sc << (8 * blk);
+    for (int i = 0; i < BETA; ++i) {
+      const int tt = blk * BETA + i;
+      if constexpr (std::is_same<T, __nv_bfloat16>::value)
+        val[i] = __bfloat162float(tile_smem[tt * kVCh + cl]);
+      else
+        val[i] = __half2float(tile_smem[tt * kVCh + cl]);
     }
-    uint8_t* dst = vt_codes + (head * d + c) * static_cast<int64_t>(Np / 2) + (t0 + w * 4 * BETA) / 2;
-#pragma unroll
-    for (int j = 0; j < 4 * BETA / 8; j += 4)
-      *reinterpret_cast<uint4*>(dst + 4 * j) = make_uint4(out[j], out[j + 1], out[j + 2], out[j + 3]);
-    *reinterpret_cast<uint32_t*>(vt_sf + head * sf_head_bytes + sf_word_offset(c, t0 / (4 * BETA) + w, nkc)) =
-        sc_word;
+    uint32_t packed[BETA / 8];
+    const uint32_t sc = quant_block<FMT, BETA>(val, packed, inv_tab);
+    uint8_t* dst = vt_codes + (head * d + c) * static_cast<int64_t>(Np / 2) + (t0 + blk * BETA) / 2;
+    if constexpr (BETA == 16) {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    } else {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+    const int gb = t0 / BETA + blk;                   // block index along the row
+    vt_sf[head * sf_head_bytes + sf_word_offset(c, gb / 4, nkc) + (gb % 4)] = static_cast<uint8_t>(sc);
   }
 }
 
-// One launch for the whole step: CTAs [0, nq) quantize Q rows, [nq, nq+nk)
-// K rows, the rest V tiles.
+// One launch for the whole step: CTAs [0, nv) quantize V tiles, the next nq
+// Q rows, the rest K rows.
 struct QuantArgs {
   const void *q, *k, *v;
   const float *s, *inv_s;
   uint8_t *qc, *qs, *kc, *ks, *vc, *vs;
   int B, Hq, Hkv, N, Np, d;
-  int64_t sf_qk_head, sf_v_head, q_words, k_words;
-  int nq_ctas, nk_ctas;
+  int64_t sf_qk_head, sf_v_head, q_rows, k_rows;
+  int nq_ctas, nk_ctas, nv_ctas;
 };
 
-template <int FMT, typename T>
-__global__ void __launch_bounds__(256) quantize_qkv_kernel(const QuantArgs a) {
+template <int FMT, typename T, int D>
+__global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a) {
   __shared__ __align__(16) T tile_smem[128 * kVCh];
-  const int bid = blockIdx.x;
-  if (bid < a.nq_ctas) {
-    const int64_t idx = static_cast<int64_t>(bid) * blockDim.x + threadIdx.x;
-    if (idx < a.q_words)
-      quantize_row_word<FMT, T>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.d, a.s, a.qc, a.qs,
-                                a.sf_qk_head, idx);
-  } else if (bid < a.nq_ctas + a.nk_ctas) {
-    const int64_t idx = static_cast<int64_t>(bid - a.nq_ctas) * blockDim.x + threadIdx.x;
-    if (idx < a.k_words)
-      quantize_row_word<FMT, T>(static_cast<const T*>(a.k), a.Hkv, 1, a.N, a.Np, a.d, a.inv_s, a.kc, a.ks,
-                                a.sf_qk_head, idx);
-  } else {
+  __shared__ float inv_tab[128];
+  if (FMT == HIFA4_NVFP4 && threadIdx.x < 128)
+    inv_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __fdiv_rn(1.0f, ue4m3_to_f32(threadIdx.x));
+  __syncthreads();
+  // V tiles first (the longest CTAs start early), then Q rows, then K rows
+  const int bid = static_cast<int>(blockIdx.x) - a.nv_ctas;
+  if (bid < 0) {
     quantize_v_tile<FMT, T>(static_cast<const T*>(a.v), a.N, a.Np, a.d, a.vc, a.vs, a.sf_v_head,
-                            bid - a.nq_ctas - a.nk_ctas, tile_smem);
+                            static_cast<int>(blockIdx.x), tile_smem, inv_tab);
+  } else if (bid < a.nq_ctas) {
+    quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.s, a.qc, a.qs,
+                                 a.sf_qk_head, bid, inv_tab);
+  } else if (bid < a.nq_ctas + a.nk_ctas) {
+    quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.k), a.Hkv, 1, a.N, a.Np, a.inv_s, a.kc, a.ks,
+                                 a.sf_qk_head, bid - a.nq_ctas, inv_tab);
   }
 }
 
@@ -276,11 +311,17 @@ __global__ void calib_finalize_kernel(float* s, float* inv_s, int n, double alph
 }
 
 // ---------------------------------------------------------- host launchers ---
+template <typename T, int D>
+static void launch_quant_d(const QuantArgs& a, int fmt, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(a.nq_ctas + a.nk_ctas + a.nv_ctas);
+  if (fmt == HIFA4_NVFP4) quantize_qkv_kernel<HIFA4_NVFP4, T, D><<<grid, 256, 0, st>>>(a);
+  else quantize_qkv_kernel<HIFA4_MXFP4, T, D><<<grid, 256, 0, st>>>(a);
+}
 template <typename T>
 static void launch_quant(const QuantArgs& a, int fmt, cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>(a.nq_ctas + a.nk_ctas + (a.Np / 128) * (a.B * a.Hkv) * (a.d / kVCh));
-  if (fmt == HIFA4_NVFP4) quantize_qkv_kernel<HIFA4_NVFP4, T><<<grid, 256, 0, st>>>(a);
-  else quantize_qkv_kernel<HIFA4_MXFP4, T><<<grid, 256, 0, st>>>(a);
+  if (a.d == 64) launch_quant_d<T, 64>(a, fmt, st);
+  else if (a.d == 128) launch_quant_d<T, 128>(a, fmt, st);
+  else launch_quant_d<T, 256>(a, fmt, st);
 }
 
 // q == nullptr quantizes only K and V (a KV cache).
@@ -291,13 +332,17 @@ hifa4_status quantize_qkv_launch(const void* q, const void* k, const void* v, in
   a.q = q; a.k = k; a.v = v; a.s = s; a.inv_s = inv_s;
   a.qc = qc; a.qs = qs; a.kc = kc; a.ks = ks; a.vc = vc; a.vs = vs;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.N = N; a.Np = static_cast<int>(pad128(N)); a.d = d;
-  const int wpr = (d / beta_of(fmt) + 3) / 4;
   a.sf_qk_head = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
   a.sf_v_head = static_cast<int64_t>(hifa4_scale_bytes(d, a.Np, static_cast<hifa4_format>(fmt)));
-  a.q_words = q ? static_cast<int64_t>(B) * Hq * a.Np * wpr : 0;
-  a.k_words = static_cast<int64_t>(B) * Hkv * a.Np * wpr;
-  a.nq_ctas = static_cast<int>((a.q_words + 255) / 256);
-  a.nk_ctas = static_cast<int>((a.k_words + 255) / 256);
+  a.q_rows = q ? static_cast<int64_t>(B) * Hq * a.Np : 0;
+  a.k_rows = static_cast<int64_t>(B) * Hkv * a.Np;
+  // 8 warps per CTA, each kUnroll row groups of 32 / (d / BETA) rows
+  const int lpr = d / beta_of(fmt);
+  const int rows_per_cta = 8 * (32 / lpr) * (fmt == HIFA4_NVFP4 ? LpbCfg<HIFA4_NVFP4>::kUnroll
+                                                                 : LpbCfg<HIFA4_MXFP4>::kUnroll);
+  a.nq_ctas = static_cast<int>(a.q_rows / rows_per_cta);    // Np is a multiple of 128, rows_per_cta divides 128
+  a.nk_ctas = static_cast<int>(a.k_rows / rows_per_cta);
+  a.nv_ctas = (a.Np / 128) * (a.B * a.Hkv) * (a.d / kVCh);
   if (dt == HIFA4_BF16) launch_quant<__nv_bfloat16>(a, fmt, st);
   else launch_quant<__half>(a, fmt, st);
   return launch_status(q ? "quantize_qkv" : "quantize_kv");
