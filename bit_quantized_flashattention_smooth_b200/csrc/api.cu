@@ -265,7 +265,7 @@ hifa4_status hifa4_bf16_attn_fwd(const void* q, const void* k, const void* vt, i
   HIFA4_REQUIRE(q && k && vt && o, HIFA4_ERR_INVALID_ARG, "bf16_attn_fwd: null pointer");
   HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0 && N % 8 == 0, HIFA4_ERR_INVALID_ARG,
                 "bf16_attn_fwd: bad shape B=%d Hq=%d Hkv=%d N=%d (N a multiple of 8)", B, Hq, Hkv, N);
-  HIFA4_REQUIRE(d == 64 || d == 128, HIFA4_ERR_UNSUPPORTED, "bf16_attn_fwd: d=%d not in {64,128}", d);
+  HIFA4_REQUIRE(d == 64 || d == 128 || d == 256, HIFA4_ERR_UNSUPPORTED, "bf16_attn_fwd: d=%d not in {64,128,256}", d);
   HIFA4_REQUIRE(softmax_scale > 0.0f, HIFA4_ERR_INVALID_ARG, "bf16_attn_fwd: softmax_scale must be > 0");
   HIFA4_REQUIRE(aligned16(q) && aligned16(k) && aligned16(vt) && aligned16(o), HIFA4_ERR_INVALID_ARG,
                 "bf16_attn_fwd: pointers must be 16-byte aligned");

@@ -54,7 +54,7 @@ struct Bf16Cfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int TM_S = 0;
   static constexpr int TM_O = BN;
-  static constexpr int TMEM_ALLOC = BN + D <= 128 ? 128 : 256;
+  static constexpr int TMEM_ALLOC = BN + D <= 128 ? 128 : (BN + D <= 256 ? 256 : 512);
   static constexpr int CTAS_PER_SM = 512 / TMEM_ALLOC > 2 ? 2 : 512 / TMEM_ALLOC;
   static_assert(SMEM_BYTES * CTAS_PER_SM <= 226 * 1024, "shared memory for the resident CTAs");
 };
@@ -353,7 +353,9 @@ hifa4_status bf16_attn_launch(const void* q, const void* k, const void* vt, int 
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   if (B == 0 || N == 0) return HIFA4_OK;
-  return d == 64 ? launch_bf16_t<64>(q, k, vt, p, st) : launch_bf16_t<128>(q, k, vt, p, st);
+  if (d == 64) return launch_bf16_t<64>(q, k, vt, p, st);
+  if (d == 128) return launch_bf16_t<128>(q, k, vt, p, st);
+  return launch_bf16_t<256>(q, k, vt, p, st);
 }
 
 hifa4_status transpose_v_bf16_launch(const void* v, int B, int Hkv, int N, int d, void* vt, cudaStream_t st) {

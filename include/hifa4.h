@@ -247,7 +247,7 @@ HIFA4_API hifa4_status hifa4_div6_probe(uint32_t lo_bits, uint32_t hi_bits, unsi
  *   vt [B, Hkv, d, N] bf16 (V transposed, see hifa4_bf16_transpose_v),
  *   o  [B, Hq, N, d] bf16 (written), lse [B, Hq, N] f32 base-2 log-sum-exp
  *   (m + log2 l of the scores times softmax_scale * log2 e) or NULL.
- * d in {64, 128}; N a multiple of 8; Hq a multiple of Hkv (GQA); causal is
+ * d in {64, 128, 256}; N a multiple of 8; Hq a multiple of Hkv (GQA); causal is
  * top-left aligned.  Pointers 16-byte aligned.  Asynchronous on `stream`. */
 HIFA4_API hifa4_status hifa4_bf16_attn_fwd(const void* q, const void* k, const void* vt, int B, int Hq, int Hkv,
                                            int N, int d, float softmax_scale, int causal, void* o, float* lse,

@@ -47,6 +47,7 @@ def _reference(q, k, v, causal, scale):
     (1, 2, 2, 256, 64, False),      # the tiny MHA shape
     (1, 4, 2, 200, 128, True),      # GQA, ragged last query and key tiles
     (2, 2, 1, 136, 64, True),       # two batches, one row past a query tile
+    (1, 4, 2, 320, 256, True),      # d = 256 (one CTA per SM), ragged
     (1, 32, 8, 4096, 128, True),    # the 32-head 4096-token causal prefill
 ])
 def test_bf16_attention_matches_fp32_reference(B, Hq, Hkv, N, d, causal):
