@@ -34,7 +34,7 @@ ABI_FUNCTIONS = (
     "hifa4_quantize_kv",
     "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
-    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_status_string", "hifa4_last_error",
+    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
 )
 
@@ -70,6 +70,7 @@ def lib():
         L.hifa4_exp2_poly_probe.argtypes = [vp, i64, vp, vp]
         L.hifa4_bf16_attn_fwd.argtypes = [vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp]
         L.hifa4_bf16_transpose_v.argtypes = [vp, i, i, i, i, vp, vp]
+        L.hifa4_wait_timeout_probe.argtypes = [vp, vp]
         L.hifa4_status_string.argtypes = [i]; L.hifa4_status_string.restype = ctypes.c_char_p
         L.hifa4_last_error.argtypes = []; L.hifa4_last_error.restype = ctypes.c_char_p
         L.hifa4_device_error.argtypes = []; L.hifa4_device_error.restype = ctypes.c_uint
@@ -292,6 +293,14 @@ def div6_probe(lo_bits: int, hi_bits: int):
     first = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     _check(lib().hifa4_div6_probe(lo_bits, hi_bits, _ptr(cnt), _ptr(first), _stream()), "div6_probe")
     return int(cnt.item()), int(first.item()) & 0xFFFFFFFF
+
+
+def wait_timeout_probe():
+    """Run the bounded-wait failure path once; returns (wait succeeded, abort flag)."""
+    st = torch.zeros(2, dtype=torch.int32, device="cuda")
+    _check(lib().hifa4_wait_timeout_probe(_ptr(st), _stream()), "wait_timeout_probe")
+    torch.cuda.synchronize()
+    return bool(st[0].item()), int(st[1].item())
 
 
 def bf16_transpose_v(v: torch.Tensor) -> torch.Tensor:

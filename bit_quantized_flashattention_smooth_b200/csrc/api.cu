@@ -88,6 +88,7 @@ hifa4_status fp4_mma_probe_launch(const uint8_t*, const uint8_t*, const uint8_t*
 hifa4_status convert_probe_launch(const float*, int64_t, uint8_t*, uint8_t*, cudaStream_t);
 hifa4_status div6_probe_launch(uint32_t, uint32_t, unsigned long long*, uint32_t*, cudaStream_t);
 hifa4_status exp2_poly_probe_launch(const float*, int64_t, float*, cudaStream_t);
+hifa4_status wait_timeout_probe_launch(unsigned int*, cudaStream_t);
 hifa4_status bf16_attn_launch(const void*, const void*, const void*, int, int, int, int, int, float, int, void*, float*,
                               cudaStream_t);
 hifa4_status transpose_v_bf16_launch(const void*, int, int, int, int, void*, cudaStream_t);
@@ -277,6 +278,11 @@ hifa4_status hifa4_bf16_attn_fwd(const void* q, const void* k, const void* vt, i
 hifa4_status hifa4_bf16_transpose_v(const void* v, int B, int Hkv, int N, int d, void* vt, hifa4_stream_t stream) {
   HIFA4_REQUIRE(v && vt && B >= 0 && Hkv > 0 && N >= 0 && d > 0, HIFA4_ERR_INVALID_ARG, "bf16_transpose_v: bad args");
   return transpose_v_bf16_launch(v, B, Hkv, N, d, vt, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_wait_timeout_probe(unsigned int* status, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(status != nullptr, HIFA4_ERR_INVALID_ARG, "wait_timeout_probe: null status");
+  return wait_timeout_probe_launch(status, static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_exp2_poly_probe(const float* y, int64_t count, float* out, hifa4_stream_t stream) {

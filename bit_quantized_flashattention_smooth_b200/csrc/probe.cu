@@ -198,4 +198,29 @@ hifa4_status exp2_poly_probe_launch(const float* y, int64_t n, float* out, cudaS
   return launch_status("exp2_poly_probe");
 }
 
+// The failure path of the bounded mbarrier wait, exercised on purpose: one
+// warp waits on a barrier that nothing arrives at.  The wait gives up after
+// its time limit, raises the abort flag and ORs kErrTimeoutOther into the
+// device error word; the kernel then returns normally (no trap, no hang).
+// status[0] = 1 if the wait (wrongly) succeeded, status[1] = abort flag.
+__global__ void wait_timeout_probe_kernel(unsigned int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(smem_u32(&bar), 0, &abort_flag, kErrTimeoutOther);
+  if (threadIdx.x == 0) {
+    status[0] = ok ? 1u : 0u;
+    status[1] = static_cast<unsigned int>(abort_flag);
+  }
+}
+hifa4_status wait_timeout_probe_launch(unsigned int* status, cudaStream_t st) {
+  wait_timeout_probe_kernel<<<1, 32, 0, st>>>(status);
+  return launch_status("wait_timeout_probe");
+}
+
 }  // namespace hifa4

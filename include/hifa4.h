@@ -264,6 +264,14 @@ HIFA4_API hifa4_status hifa4_bf16_transpose_v(const void* v, int B, int Hkv, int
  * and y = 0 -> 1 edges. */
 HIFA4_API hifa4_status hifa4_exp2_poly_probe(const float* y, int64_t count, float* out, hifa4_stream_t stream);
 
+/* The kernels' failure path, exercised: one warp waits on an mbarrier that
+ * nothing arrives at.  The bounded wait gives up after its limit (2 s), sets
+ * its CTA's abort flag and the timeout bit 8 of the device error word, and the
+ * kernel returns.  status (device, 2 words): [0] = 1 if the wait succeeded
+ * (it must not), [1] = the abort flag.  The context stays usable; read and
+ * clear the error word with hifa4_device_error(). */
+HIFA4_API hifa4_status hifa4_wait_timeout_probe(unsigned int* status, hifa4_stream_t stream);
+
 /* ----------------------------------------------------------- errors --- */
 
 HIFA4_API const char* hifa4_status_string(hifa4_status st);

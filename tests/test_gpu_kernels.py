@@ -89,6 +89,19 @@ def test_exp2_polynomial_error_bound():
     assert np.all(out[yd < -126.0] < 2.0 ** -126) and np.all(out >= 0.0)
 
 
+def test_bounded_wait_gives_up_and_reports():
+    """A wait that nothing completes ends after its limit with the abort flag
+    and the timeout bit set, the kernel returns, and the context stays usable
+    (no trap, no hang)."""
+    assert h.device_error() == 0
+    ok, flag = h.wait_timeout_probe()
+    assert not ok and flag == 1
+    assert h.device_error() & 8           # read and cleared
+    assert h.device_error() == 0
+    n, _ = h.div6_probe(0x3F800000, 0x3F801000)
+    assert n == 0
+
+
 # --------------------------------------------------------------- FP4 MMA ---
 @pytest.mark.parametrize("fmt", [oracle.NVFP4, oracle.MXFP4])
 @pytest.mark.parametrize("n,k", [(128, 128), (64, 128), (256, 256), (128, 256)])
