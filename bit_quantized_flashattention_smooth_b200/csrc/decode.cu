@@ -44,7 +44,7 @@ template <int FMT>
 struct DecCfg {
   static constexpr int D = 128, BN = 128, NQ = 16;          // head dim, keys per tile, padded queries
   static constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
-  static constexpr int NS = 3;
+  static constexpr int NS = 2;                               // two stages, four CTAs per SM
   static constexpr int ROW = 64;                            // bytes per 128-element 4-bit row
   static constexpr int NKC = (D / BETA + 3) / 4;            // scale chunks per 128 keys / 128 channels
   static constexpr int SZ_K = BN * ROW, SZ_V = D * ROW, SZ_QB = NQ * ROW, SZ_ONES = 128 * ROW;
@@ -76,14 +76,14 @@ struct DecCfg {
   static constexpr int TM_SF1 = TM_SFP + 4 * NKC;
   static constexpr int TMEM_ALLOC = 128;
   static_assert(TM_SF1 + 4 <= TMEM_ALLOC, "TMEM budget");
-  static_assert(SMEM_BYTES * 3 <= 227 * 1024, "three CTAs per SM");
+  static_assert(SMEM_BYTES * 4 <= 227 * 1024, "four CTAs per SM");
 };
 
 __device__ __forceinline__ uint32_t swz64(uint32_t r, uint32_t c) { return c ^ ((r >> 1) & 3); }
 
 // G = query heads per kv head (1, 2, 4 or 8); the MMA N dimension is 16.
 template <int FMT, bool PREORDER, int G>
-__global__ void __launch_bounds__(192, 3)
+__global__ void __launch_bounds__(192, 4)
     attn_decode_fp4_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                            const DecodeParams p) {
   using C = DecCfg<FMT>;
@@ -499,11 +499,11 @@ bool make_tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner_bytes, uint6
                   uint32_t box_rows, int swizzle_bytes);
 
 int decode_default_splits(int B, int Hkv, int kv_len, int block_n) {
-  // enough CTAs for several waves over 148 SMs (2 resident each), each split
-  // keeping at least 16 key tiles to amortize the per-CTA setup
+  // about three waves of CTAs over 148 SMs (4 resident each), each split
+  // keeping at least 16 key tiles to amortize the per-CTA setup and the combine
   const int tiles = (kv_len + block_n - 1) / block_n;
   int splits = 1;
-  while (static_cast<int64_t>(B) * Hkv * splits < 8 * 148 * 2 && (tiles / (splits * 2)) >= 16) splits *= 2;
+  while (static_cast<int64_t>(B) * Hkv * splits < 3 * 148 * 4 && (tiles / (splits * 2)) >= 16) splits *= 2;
   return splits;
 }
 
