@@ -1,0 +1,258 @@
+"""Model check of the prefill kernel's mbarrier protocol on the CPU.
+
+The roles of one CTA of attn_fwd_fp4_kernel (TMA producer, MMA issuer, the
+softmax warps) are replayed as cooperative processes.  The model carries:
+- mbarriers with arrival counts and phase parity;
+- TMA copies that complete asynchronously;
+- tensor-core MMAs that complete in issue order;
+- tcgen05.commit arrivals once every earlier MMA has completed.
+
+A random scheduler interleaves the processes, and every wait is a parity wait
+exactly as the kernel issues it.  The checks are:
+- every wait returns only after the phase it is meant to see has completed
+  (a parity wait that returns one lap early is the bug class this test
+  guards against);
+- every shared buffer (S in TMEM, P-hat in shared memory, O) is read and
+  overwritten in the right order;
+- every schedule finishes, so there is no deadlock.
+
+The waits, counts and parities below restate the kernel's; keep them in step
+with csrc/attn_fwd.cu.
+"""
+import random
+
+import pytest
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+BLOCKED = "blocked"
+
+
+class Barrier:
+    def __init__(self, name, count):
+        self.name, self.count, self.pending, self.phase = name, count, 0, 0
+
+    def arrive(self):
+        self.pending += 1
+        if self.pending == self.count:
+            self.pending = 0
+            self.phase += 1
+
+    def parity_ready(self, parity):
+        # mbarrier.try_wait.parity: true once the phase of that parity completed,
+        # i.e. while the current (incomplete) phase has the other parity
+        return (self.phase & 1) != parity
+
+
+class Sim:
+    def __init__(self, nkt, NS, NSB, NH, rng):
+        self.nkt, self.NS, self.NSB, self.NH, self.rng = nkt, NS, NSB, NH, rng
+        self.W = 4 * NH
+        B = Barrier
+        self.bars = {"QFULL": B("QFULL", 1), "XM": B("XM", 8)}
+        for s in range(NS):
+            for n in ("KFULL", "KEMPTY", "VFULL", "VEMPTY"):
+                self.bars[f"{n}{s}"] = B(f"{n}{s}", 1)
+        for s in range(NSB):
+            self.bars[f"SFULL{s}"] = B(f"SFULL{s}", 1)
+            self.bars[f"SEMPTY{s}"] = B(f"SEMPTY{s}", self.W)
+        for s in range(2):
+            self.bars[f"PFULL{s}"] = B(f"PFULL{s}", self.W)
+            self.bars[f"PEMPTY{s}"] = B(f"PEMPTY{s}", 1)
+        # shared state with tags
+        self.s_buf = [None] * NSB          # tile held by each S buffer
+        self.s_readers = [set() for _ in range(NSB)]
+        self.p_buf = [dict() for _ in range(2)]   # warp -> tile written
+        self.k_stage = [None] * NS
+        self.v_stage = [None] * NS
+        self.xm = [dict(), dict()]
+        self.pv_done = -1                  # last PV completed
+        self.pv_started = -1               # last PV begun
+        self.mma_queue = []                # in-order async tensor-core work
+        self.copies = []                   # pending TMA copies
+
+    # -------------------------------------------------------------- waits ---
+    def wait(self, bar, parity, min_phase):
+        """Generator step: block until the parity wait returns, then check that
+        the phase this wait means (min_phase completions) has happened."""
+        b = self.bars[bar]
+        while not b.parity_ready(parity):
+            yield BLOCKED
+        if b.phase < min_phase:
+            raise ProtocolError(f"{bar}: parity wait returned at phase {b.phase}, needs >= {min_phase}")
+
+    # -------------------------------------------------------------- roles ---
+    def tma(self):
+        for j in range(self.nkt):
+            st, ph = j % self.NS, (j // self.NS) & 1
+            yield from self.wait(f"KEMPTY{st}", ph ^ 1, j // self.NS)
+            self.copies.append(("K", st, j))
+            yield from self.wait(f"VEMPTY{st}", ph ^ 1, j // self.NS)
+            self.copies.append(("V", st, j))
+
+    def mma(self):
+        yield from self.wait("QFULL", 0, 1)
+
+        def issue_s(j):
+            st, sb = j % self.NS, j % self.NSB
+            yield from self.wait(f"KFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
+            yield from self.wait(f"SEMPTY{sb}", ((j // self.NSB) & 1) ^ 1, j // self.NSB)
+            self.mma_queue.append(("S", j, [f"SFULL{sb}", f"KEMPTY{st}"]))
+
+        def issue_pv(j):
+            st, pb = j % self.NS, j & 1
+            yield from self.wait(f"PFULL{pb}", (j >> 1) & 1, (j >> 1) + 1)
+            yield from self.wait(f"VFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
+            self.mma_queue.append(("PV", j, [f"VEMPTY{st}", f"PEMPTY{pb}"]))
+
+        if self.nkt > 0:
+            yield from issue_s(0)
+        for j in range(self.nkt):
+            if j + 1 < self.nkt:
+                yield from issue_s(j + 1)
+            yield from issue_pv(j)
+
+    def softmax(self, w):
+        for j in range(self.nkt):
+            sb, pb = j % self.NSB, j & 1
+            yield from self.wait(f"SFULL{sb}", (j // self.NSB) & 1, j // self.NSB + 1)
+            if self.s_buf[sb] != j:
+                raise ProtocolError(f"warp {w} read S buffer {sb} holding tile {self.s_buf[sb]} for tile {j}")
+            self.s_readers[sb].add(w)
+            self.bars[f"SEMPTY{sb}"].arrive()
+            if self.NH == 2:
+                self.xm[j & 1][w] = j
+                self.bars["XM"].arrive()
+                yield from self.wait("XM", j & 1, j + 1)
+                partner = w ^ 4
+                if self.xm[j & 1].get(partner) != j:
+                    raise ProtocolError(f"warp {w} read the row max of tile {self.xm[j & 1].get(partner)} for {j}")
+            if j >= 2:
+                yield from self.wait(f"PEMPTY{pb}", ((j >> 1) & 1) ^ 1, (j >> 1))
+            if self.pv_done < j - 2:
+                raise ProtocolError(f"warp {w} overwrote P-hat buffer {pb} before PV_{j - 2} retired")
+            self.p_buf[pb][w] = j
+            rescale = j > 0 and self.rng.random() < 0.5
+            if rescale:
+                yield from self.wait(f"PEMPTY{(j - 1) & 1}", ((j - 1) >> 1) & 1, ((j - 1) >> 1) + 1)
+                if self.pv_done < j - 1 or self.pv_started >= j:
+                    raise ProtocolError(f"warp {w} rescaled O for tile {j} with PV_{self.pv_done} done, "
+                                        f"PV_{self.pv_started} started")
+            self.bars[f"PFULL{pb}"].arrive()
+        yield from self.epilogue(w)
+
+    def epilogue(self, w):
+        # O is final once the last PV retired
+        if self.nkt > 0:
+            jl = self.nkt - 1
+            yield from self.wait(f"PEMPTY{jl & 1}", (jl >> 1) & 1, (jl >> 1) + 1)
+            self.check_o(w)
+
+    def check_o(self, w):
+        if self.pv_done != self.nkt - 1:
+            raise ProtocolError(f"warp {w} read O with PV_{self.pv_done} of {self.nkt - 1} done")
+
+    # ------------------------------------------------------ async engines ---
+    def step_async(self):
+        """One asynchronous event, if any: a TMA copy lands, or the next MMA in
+        issue order completes and its commits arrive."""
+        events = []
+        if self.copies:
+            events.append("copy")
+        if self.mma_queue:
+            events.append("mma")
+        if not events:
+            return False
+        if self.rng.choice(events) == "copy":
+            kind, st, j = self.copies.pop(self.rng.randrange(len(self.copies)))
+            (self.k_stage if kind == "K" else self.v_stage)[st] = j
+            self.bars[f"{kind}FULL{st}"].arrive()
+            return True
+        kind, j, commits = self.mma_queue.pop(0)
+        if kind == "S":
+            sb = j % self.NSB
+            if self.k_stage[j % self.NS] != j:
+                raise ProtocolError(f"S_{j} read K stage holding tile {self.k_stage[j % self.NS]}")
+            if self.s_buf[sb] is not None and len(self.s_readers[sb]) != self.W:
+                raise ProtocolError(f"S_{j} overwrote buffer {sb} before every warp read tile {self.s_buf[sb]}")
+            self.s_buf[sb], self.s_readers[sb] = j, set()
+        else:
+            pb = j & 1
+            if set(self.p_buf[pb].values()) != {j} or len(self.p_buf[pb]) != self.W:
+                raise ProtocolError(f"PV_{j} read P-hat buffer {pb} holding {self.p_buf[pb]}")
+            if self.v_stage[j % self.NS] != j:
+                raise ProtocolError(f"PV_{j} read V stage holding tile {self.v_stage[j % self.NS]}")
+            self.pv_started = j
+            self.pv_done = j
+        for c in commits:
+            self.bars[c].arrive()
+        return True
+
+    def run(self):
+        self.bars["QFULL"].arrive()        # the Q tile (its copy lands before anything else matters)
+        live = [self.tma(), self.mma()] + [self.softmax(w) for w in range(self.W)]
+        idle = 0
+        while live or self.mma_queue or self.copies:
+            progressed = self.rng.random() < 0.5 and self.step_async()
+            self.rng.shuffle(live)
+            finished = []
+            for p in live[: self.rng.randint(1, len(live))] if live else []:
+                try:
+                    if next(p) != BLOCKED:
+                        progressed = True
+                except StopIteration:
+                    finished.append(p)
+                    progressed = True
+            live = [p for p in live if p not in finished]
+            if progressed or self.step_async():
+                idle = 0
+            else:
+                idle += 1
+                if idle > 500:
+                    raise ProtocolError("deadlock: every role waits and no copy or MMA is in flight")
+        return True
+
+
+@pytest.mark.parametrize("NH,NS,NSB", [(1, 3, 1), (2, 3, 1), (2, 3, 2), (2, 2, 2), (1, 2, 1)])
+@pytest.mark.parametrize("nkt", [1, 2, 3, 5, 9])
+def test_prefill_protocol_random_schedules(NH, NS, NSB, nkt):
+    for seed in range(40):
+        Sim(nkt, NS, NSB, NH, random.Random(1000 * nkt + seed)).run()
+
+
+def test_model_catches_a_one_lap_early_epilogue():
+    """The model must flag the bug class it guards: an epilogue that waits on
+    a barrier only the rescaling tiles await (so it can lag two phases) and
+    parity-waits for the last phase."""
+
+    class Buggy(Sim):
+        def __init__(self, *a):
+            super().__init__(*a)
+            self.bars["ORDY"] = Barrier("ORDY", 1)
+
+        def step_async(self):
+            if self.mma_queue and self.mma_queue[0][0] == "PV":
+                self.mma_queue[0][2].append("ORDY")
+            return super().step_async()
+
+        def epilogue(self, w):
+            # the old epilogue: a parity wait on a barrier that lags when the
+            # last tiles needed no rescale
+            jl = self.nkt - 1
+            b = self.bars["ORDY"]
+            while not b.parity_ready(jl & 1):
+                yield BLOCKED
+            self.check_o(w)
+
+    caught = 0
+    for seed in range(200):
+        sim = Buggy(6, 3, 1, 1, random.Random(seed))
+        sim.rng = random.Random(seed)
+        try:
+            sim.run()
+        except ProtocolError:
+            caught += 1
+    assert caught > 0
