@@ -410,7 +410,14 @@ def run_decode(args):
         tot += e0.elapsed_time(e1)
     ms = tot / n
     kv_bytes = (cache.k_codes.numel() + cache.k_scales.numel() + cache.vt_codes.numel() + cache.vt_scales.numel())
-    return dict(ms=ms, bytes=kv_bytes, gbs=kv_bytes / (ms * 1e-3) / 1e9, splits=splits)
+    # appending one token per sequence to an appendable cache of the same
+    # shape (its cost does not depend on the cache contents)
+    del cache
+    acache, tail = h.alloc_appendable_kv_cache(B, Hq, Hkv, kv + 128, d, h.NVFP4)
+    kn = torch.randn((B, Hkv, 1, d), device=dev).to(torch.bfloat16)
+    vn = torch.randn((B, Hkv, 1, d), device=dev).to(torch.bfloat16)
+    append_ms = time_ms(lambda: h.kv_cache_append(acache, tail, kn, vn, inv, kv), n=20)
+    return dict(ms=ms, bytes=kv_bytes, gbs=kv_bytes / (ms * 1e-3) / 1e9, splits=splits, append_ms=append_ms)
 
 
 # ------------------------------------------------------- reference arm ----
@@ -577,7 +584,8 @@ def main():
         if "gbs" in decode:
             line["decode"] = {"workload": "split_decode", "kv_gbs": decode["gbs"], "ms": decode["ms"],
                               "kv_bytes": decode["bytes"], "hbm_peak_gbs": pk["hbm"],
-                              "frac": decode["gbs"] / pk["hbm"], "splits": decode["splits"]}
+                              "frac": decode["gbs"] / pk["hbm"], "splits": decode["splits"],
+                              "append_one_token_ms": decode["append_ms"]}
         else:
             line["decode"] = decode
     line["tokens_per_s"] = w.B * w.N * world / (res["step_ms"] * 1e-3)

@@ -34,7 +34,7 @@ ABI_FUNCTIONS = (
     "hifa4_quantize_kv",
     "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
-    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_status_string", "hifa4_last_error",
+    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_kv_cache_append", "hifa4_attn_decode_cache", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
 )
 
@@ -71,6 +71,9 @@ def lib():
         L.hifa4_bf16_attn_fwd.argtypes = [vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp]
         L.hifa4_bf16_transpose_v.argtypes = [vp, i, i, i, i, vp, vp]
         L.hifa4_wait_timeout_probe.argtypes = [vp, vp]
+        L.hifa4_kv_cache_append.argtypes = [vp, vp, i, i, i, i, i, vp, i, i, i, vp, vp, vp, vp, vp, vp]
+        L.hifa4_attn_decode_cache.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i,
+                                              ctypes.POINTER(ctypes.c_int), vp, sz, vp, i, vp]
         L.hifa4_status_string.argtypes = [i]; L.hifa4_status_string.restype = ctypes.c_char_p
         L.hifa4_last_error.argtypes = []; L.hifa4_last_error.restype = ctypes.c_char_p
         L.hifa4_device_error.argtypes = []; L.hifa4_device_error.restype = ctypes.c_uint
@@ -191,6 +194,27 @@ def alloc_kv_cache(B, Hq, Hkv, kv_len, d, fmt, device="cuda") -> QuantizedQKV:
                         B, Hq, Hkv, kv_len, d, fmt)
 
 
+def alloc_appendable_kv_cache(B, Hq, Hkv, capacity, d, fmt, dtype=torch.bfloat16, device="cuda"):
+    """An empty 4-bit KV cache for `capacity` tokens (zeroed, as the append
+    contract requires) and its V tail buffer [B, Hkv, beta, d]."""
+    z = alloc_kv_cache(B, Hq, Hkv, capacity, d, fmt, device)
+    for t in (z.k_codes, z.k_scales, z.vt_codes, z.vt_scales):
+        t.zero_()
+    beta = 16 if fmt == NVFP4 else 32
+    return z, torch.zeros((B, Hkv, beta, d), device=device, dtype=dtype)
+
+
+def kv_cache_append(cache: QuantizedQKV, v_tail: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                    inv_s: torch.Tensor | None, pos: int):
+    """Append tokens [pos, pos + T) (k_new, v_new [B, Hkv, T, d]) to an appendable cache."""
+    B, Hkv, T, d = k_new.shape
+    k_new = k_new.contiguous(); v_new = v_new.contiguous()
+    _check(lib().hifa4_kv_cache_append(_ptr(k_new), _ptr(v_new), _dt(k_new), B, Hkv, T, d, _ptr(inv_s), cache.fmt,
+                                       int(pos), cache.N, _ptr(cache.k_codes), _ptr(cache.k_scales),
+                                       _ptr(cache.vt_codes), _ptr(cache.vt_scales), _ptr(v_tail), _stream()),
+           "kv_cache_append")
+
+
 def quantize_kv(k, v, inv_s=None, fmt: int = NVFP4, Hq: int | None = None, out: QuantizedQKV | None = None):
     """Quantize K (scaled by inv_s) and V into a 4-bit KV cache."""
     B, Hkv, N, d = k.shape
@@ -250,11 +274,12 @@ def attn_decode(q: torch.Tensor, s: torch.Tensor | None, cache: QuantizedQKV, kv
     o = out if out is not None else torch.empty((B, Hq, d), device=q.device, dtype=out_dtype)
     used = ctypes.c_int(0)
     q = q.contiguous()
-    _check(lib().hifa4_attn_decode(_ptr(q), _dt(q), _ptr(s), _ptr(cache.k_codes), _ptr(cache.k_scales),
-                                   _ptr(cache.vt_codes), _ptr(cache.vt_scales), B, Hq, cache.Hkv, kv, d,
-                                   cache.fmt, float(softmax_scale), int(mode), 128, int(num_splits),
-                                   ctypes.byref(used), _ptr(workspace), workspace.numel(), _ptr(o), _dt(o),
-                                   _stream()), "attn_decode")
+    # the cache's layout is that of its capacity cache.N; decode reads kv tokens
+    _check(lib().hifa4_attn_decode_cache(_ptr(q), _dt(q), _ptr(s), _ptr(cache.k_codes), _ptr(cache.k_scales),
+                                         _ptr(cache.vt_codes), _ptr(cache.vt_scales), B, Hq, cache.Hkv, kv, cache.N,
+                                         d, cache.fmt, float(softmax_scale), int(mode), 128, int(num_splits),
+                                         ctypes.byref(used), _ptr(workspace), workspace.numel(), _ptr(o), _dt(o),
+                                         _stream()), "attn_decode")
     return o, used.value
 
 

@@ -80,8 +80,10 @@ hifa4_status attn_fwd_launch(const uint8_t*, const uint8_t*, const uint8_t*, con
                              const uint8_t*, int, int, int, int, int, int, float, int, int, int, void*, int, float*,
                              float*, float*, cudaStream_t);
 hifa4_status decode_launch(const void*, int, const float*, const uint8_t*, const uint8_t*, const uint8_t*,
-                           const uint8_t*, int, int, int, int, int, int, float, int, int, int, int*, void*, size_t,
+                           const uint8_t*, int, int, int, int, int, int, int, float, int, int, int, int*, void*, size_t,
                            void*, int, cudaStream_t);
+hifa4_status kv_append_launch(const void*, const void*, int, int, int, int, int, const float*, int, int, int,
+                              uint8_t*, uint8_t*, uint8_t*, uint8_t*, void*, cudaStream_t);
 int decode_default_splits(int B, int Hkv, int kv_len, int block_n);
 hifa4_status fp4_mma_probe_launch(const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*, int, int, int, int,
                                   int, float*, cudaStream_t);
@@ -230,9 +232,55 @@ hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const float* s, 
   HIFA4_REQUIRE(aligned16(q) && aligned16(k_codes) && aligned16(k_scales) && aligned16(vt_codes) &&
                     aligned16(vt_scales) && aligned16(o) && aligned16(workspace) && (!s || aligned16(s)),
                 HIFA4_ERR_INVALID_ARG, "attn_decode: pointers must be 16-byte aligned");
-  return decode_launch(q, q_dt, s, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, kv_len, d, fmt,
+  return decode_launch(q, q_dt, s, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, kv_len, kv_len, d, fmt,
                        softmax_scale, mode, 128, num_splits, num_splits_used, workspace, ws_bytes, o, o_dt,
                        static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_attn_decode_cache(const void* q, hifa4_dtype q_dt, const float* s, const uint8_t* k_codes,
+                                     const uint8_t* k_scales, const uint8_t* vt_codes, const uint8_t* vt_scales,
+                                     int B, int Hq, int Hkv, int kv_len, int kv_capacity, int d, hifa4_format fmt,
+                                     float softmax_scale, hifa4_norm_mode mode, int block_n, int num_splits,
+                                     int* num_splits_used, void* workspace, size_t ws_bytes, void* o,
+                                     hifa4_dtype o_dt, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(kv_capacity >= kv_len, HIFA4_ERR_INVALID_ARG, "attn_decode_cache: kv_len %d > capacity %d", kv_len,
+                kv_capacity);
+  HIFA4_REQUIRE(q && k_codes && k_scales && vt_codes && vt_scales && o && workspace, HIFA4_ERR_INVALID_ARG,
+                "attn_decode_cache: null pointer");
+  HIFA4_REQUIRE(valid_fmt(fmt) && valid_dt(q_dt) && valid_dt(o_dt), HIFA4_ERR_INVALID_ARG,
+                "attn_decode_cache: bad format/dtype");
+  HIFA4_REQUIRE(mode == HIFA4_NORM_PREORDER || mode == HIFA4_NORM_INCONSISTENT, HIFA4_ERR_INVALID_ARG,
+                "attn_decode_cache: bad normalizer mode");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && kv_len > 0, HIFA4_ERR_INVALID_ARG,
+                "attn_decode_cache: bad shape");
+  HIFA4_REQUIRE(d == 128, HIFA4_ERR_UNSUPPORTED, "attn_decode_cache: d=%d (only 128)", d);
+  HIFA4_REQUIRE(Hq / Hkv == 1 || Hq / Hkv == 2 || Hq / Hkv == 4 || Hq / Hkv == 8, HIFA4_ERR_UNSUPPORTED,
+                "attn_decode_cache: GQA group %d not in {1,2,4,8}", Hq / Hkv);
+  HIFA4_REQUIRE(block_n == 0 || block_n == 128, HIFA4_ERR_UNSUPPORTED, "attn_decode_cache: block_n must be 128");
+  HIFA4_REQUIRE(num_splits >= 0 && softmax_scale > 0.0f, HIFA4_ERR_INVALID_ARG, "attn_decode_cache: bad arguments");
+  HIFA4_REQUIRE(aligned16(q) && aligned16(k_codes) && aligned16(k_scales) && aligned16(vt_codes) &&
+                    aligned16(vt_scales) && aligned16(o) && aligned16(workspace) && (!s || aligned16(s)),
+                HIFA4_ERR_INVALID_ARG, "attn_decode_cache: pointers must be 16-byte aligned");
+  return decode_launch(q, q_dt, s, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, kv_len, kv_capacity, d, fmt,
+                       softmax_scale, mode, 128, num_splits, num_splits_used, workspace, ws_bytes, o, o_dt,
+                       static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_kv_cache_append(const void* k_new, const void* v_new, hifa4_dtype dt, int B, int Hkv, int T,
+                                   int d, const float* inv_s, hifa4_format fmt, int pos, int capacity,
+                                   uint8_t* k_codes, uint8_t* k_scales, uint8_t* vt_codes, uint8_t* vt_scales,
+                                   void* v_tail, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(k_new && v_new && k_codes && k_scales && vt_codes && vt_scales && v_tail, HIFA4_ERR_INVALID_ARG,
+                "kv_cache_append: null pointer");
+  HIFA4_REQUIRE(valid_dt(dt) && valid_fmt(fmt), HIFA4_ERR_INVALID_ARG, "kv_cache_append: bad dtype/format");
+  HIFA4_REQUIRE(B > 0 && Hkv > 0 && T > 0 && pos >= 0 && pos + T <= capacity, HIFA4_ERR_INVALID_ARG,
+                "kv_cache_append: bad shape (B=%d Hkv=%d T=%d pos=%d capacity=%d)", B, Hkv, T, pos, capacity);
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "kv_cache_append: d=%d not in {64,128,256}", d);
+  HIFA4_REQUIRE(aligned16(k_codes) && aligned16(k_scales) && aligned16(vt_codes) && aligned16(vt_scales) &&
+                    (!inv_s || aligned16(inv_s)),
+                HIFA4_ERR_INVALID_ARG, "kv_cache_append: cache pointers must be 16-byte aligned");
+  return kv_append_launch(k_new, v_new, dt, B, Hkv, T, d, inv_s, fmt, pos, capacity, k_codes, k_scales, vt_codes,
+                          vt_scales, v_tail, static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_fp4_mma_probe(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,

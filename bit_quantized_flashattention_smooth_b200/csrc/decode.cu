@@ -524,7 +524,8 @@ static hifa4_status launch_decode_t(const uint8_t* kc, const uint8_t* vc, const 
 }
 
 hifa4_status decode_launch(const void* q, int q_dt, const float* s, const uint8_t* kc, const uint8_t* ks,
-                           const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int kv_len, int d, int fmt,
+                           const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int kv_len, int kv_cap,
+                           int d, int fmt,
                            float softmax_scale, int mode, int block_n, int num_splits, int* num_splits_used,
                            void* workspace, size_t ws_bytes, void* o, int o_dt, cudaStream_t st) {
   if (num_splits == 0) num_splits = decode_default_splits(B, Hkv, kv_len, block_n);
@@ -541,8 +542,8 @@ hifa4_status decode_launch(const void* q, int q_dt, const float* s, const uint8_
   p.s = s;
   p.k_sf = ks;
   p.v_sf = vs;
-  p.Np = static_cast<int>(pad128(kv_len));
-  p.sf_k_head = static_cast<int64_t>(hifa4_scale_bytes(kv_len, d, static_cast<hifa4_format>(fmt)));
+  p.Np = static_cast<int>(pad128(kv_cap));          // the cache layout's padded length
+  p.sf_k_head = static_cast<int64_t>(hifa4_scale_bytes(kv_cap, d, static_cast<hifa4_format>(fmt)));
   p.sf_v_head = static_cast<int64_t>(hifa4_scale_bytes(d, p.Np, static_cast<hifa4_format>(fmt)));
   p.B = B;
   p.Hq = Hq;

@@ -185,6 +185,41 @@ HIFA4_API hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const 
                                int* num_splits_used, void* workspace, size_t ws_bytes, void* o,
                                hifa4_dtype o_dt, hifa4_stream_t stream);
 
+/* ------------------------------------------------- appendable cache --- */
+
+/* A KV cache that grows by appends, for decode loops.  Its buffers have the
+ * hifa4_quantize_kv layouts for a fixed `capacity` tokens (Np =
+ * pad128(capacity): k_codes [B][Hkv][Np][d/2], k_scales
+ * hifa4_scale_bytes(capacity, d) per head, vt_codes [B][Hkv][d][Np/2],
+ * vt_scales hifa4_scale_bytes(d, Np) per head), all zero before the first
+ * append, plus v_tail [B][Hkv][beta][d] (dt): the raw V values of the
+ * partially filled last block of beta tokens (beta = 16 NVFP4, 32 MXFP4),
+ * owned by the caller and passed unchanged between appends.
+ *
+ * Appends tokens [pos, pos + T) from k_new, v_new [B][Hkv][T][d] (dt, device):
+ * K rows scaled by inv_s ([Hkv][d] fp32, or NULL for 1) and block-quantized;
+ * every V block the new tokens touch is quantized again from its raw values
+ * (older tokens of the block from v_tail, tokens not yet written as 0); v_tail
+ * is updated.  After appends covering [0, L), the cache equals
+ * hifa4_quantize_kv of the L tokens laid out at this capacity, bit for bit.
+ * Requires 0 <= pos, T >= 1, pos + T <= capacity, d in {64, 128, 256}.  Three
+ * kernel launches on `stream`; no host synchronization. */
+HIFA4_API hifa4_status hifa4_kv_cache_append(const void* k_new, const void* v_new, hifa4_dtype dt, int B, int Hkv,
+                                             int T, int d, const float* inv_s, hifa4_format fmt, int pos,
+                                             int capacity, uint8_t* k_codes, uint8_t* k_scales, uint8_t* vt_codes,
+                                             uint8_t* vt_scales, void* v_tail, hifa4_stream_t stream);
+
+/* hifa4_attn_decode over the first kv_len tokens of an appendable cache laid
+ * out for kv_capacity tokens (kv_len <= kv_capacity); same arguments and
+ * results otherwise.  hifa4_attn_decode is the case kv_capacity = kv_len. */
+HIFA4_API hifa4_status hifa4_attn_decode_cache(const void* q, hifa4_dtype q_dt, const float* s,
+                                               const uint8_t* k_codes, const uint8_t* k_scales,
+                                               const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
+                                               int Hkv, int kv_len, int kv_capacity, int d, hifa4_format fmt,
+                                               float softmax_scale, hifa4_norm_mode mode, int block_n,
+                                               int num_splits, int* num_splits_used, void* workspace,
+                                               size_t ws_bytes, void* o, hifa4_dtype o_dt, hifa4_stream_t stream);
+
 /* Decode for callers that cannot allocate device memory.  (The paper has no
  * counterpart; this is a deployment convenience of this library.)  Callers
  * such as an inference-server plugin or a framework custom operator that is
