@@ -318,6 +318,22 @@ def comparisons(res):
                       "frac_rows_negative": float((eps < 0).float().mean()),
                       "preorder_output_scale_error": 0.0,
                       "inconsistent_output_scale_error_median_over_heads": float(scale_err.median())}
+    # Smooth-QK migration strength and the applicability gate: deviation of
+    # the 4-bit output from exact attention (same 4 heads) and eps per setting
+    sweep = []
+    for label, alpha, enable in (("off", 0.5, 0), ("alpha=0", 0.0, 1), ("alpha=0.25", 0.25, 1),
+                                 ("alpha=0.5", 0.5, 1), ("alpha=0.75", 0.75, 1), ("gate, alpha=0.5", 0.5, h.GATE)):
+        s_a, inv_a = h.calibrate_smooth_qk(qd[:, :, : w.n_cal], kd[:, :, : w.n_cal], w.n_cal, alpha=alpha,
+                                           enable=enable)
+        za = h.quantize_qkv(qd, kd, vd, s_a, inv_a, res["fmt"])
+        oa, lpa, lpp = h.attn_fwd(za, scale, w.causal, h.PREORDER, w.block_n, out_dtype=o_pre.dtype, debug=True)
+        o4a = oa[0, heads].float()
+        ea = (lpa / lpp - 1.0).flatten()
+        sweep.append({"setting": label, "heads_smoothed": int((s_a != 1.0).any(dim=1).sum()),
+                      "max_abs_rel": float((o4a - ex).abs().max() / ex.abs().max()),
+                      "cosine": float(torch.nn.functional.cosine_similarity(o4a.flatten(), ex.flatten(), dim=0)),
+                      "eps_median": float(ea.median())})
+    out["smooth_qk_sweep"] = sweep
     return out
 
 

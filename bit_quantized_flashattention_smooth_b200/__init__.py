@@ -123,16 +123,20 @@ def device_error() -> int:
 
 
 # --------------------------------------------------------------- calibrate ---
+GATE = 2   # calibrate_smooth_qk(enable=GATE): per-head applicability gate
+
+
 def calibrate_smooth_qk(q: torch.Tensor, k: torch.Tensor, n_cal: int, alpha: float = 0.5,
-                        enable: bool = True):
-    """q [B,Hq,T,d], k [B,Hkv,T,d] (cuda, bf16/fp16) -> (s, inv_s) [Hkv,d] float32."""
+                        enable: bool | int = True):
+    """q [B,Hq,T,d], k [B,Hkv,T,d] (cuda, bf16/fp16) -> (s, inv_s) [Hkv,d] float32.
+    enable: False / True, or GATE for the per-head applicability gate."""
     B, Hq, T, d = q.shape
     Hkv = k.shape[1]
     q = q.contiguous(); k = k.contiguous()
     s = torch.empty((Hkv, d), device=q.device, dtype=torch.float32)
     inv = torch.empty_like(s)
     _check(lib().hifa4_calibrate_smooth_qk(_ptr(q), _ptr(k), _dt(q), B, Hq, Hkv, n_cal, T, d, float(alpha),
-                                           int(bool(enable)), _ptr(s), _ptr(inv), _stream()),
+                                           int(enable), _ptr(s), _ptr(inv), _stream()),
            "calibrate_smooth_qk")
     return s, inv
 

@@ -136,6 +136,7 @@ hifa4_status hifa4_calibrate_smooth_qk(const void* q, const void* k, hifa4_dtype
   HIFA4_REQUIRE(n_cal > 0 && n_cal <= ld_tok, HIFA4_ERR_INVALID_ARG, "calibrate: need 0 < n_cal <= ld_tok");
   HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "calibrate: d=%d not in {64,128,256}", d);
   HIFA4_REQUIRE(alpha >= 0.0f && alpha <= 1.0f, HIFA4_ERR_INVALID_ARG, "calibrate: alpha outside [0,1]");
+  HIFA4_REQUIRE(enable >= 0 && enable <= 2, HIFA4_ERR_INVALID_ARG, "calibrate: enable must be 0, 1 or 2");
   return calibrate_launch(q, k, dt, B, Hq, Hkv, n_cal, ld_tok, d, alpha, enable, s_out, inv_s_out,
                           static_cast<cudaStream_t>(stream));
 }

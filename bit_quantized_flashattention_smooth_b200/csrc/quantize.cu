@@ -294,14 +294,42 @@ __global__ void calib_amax_kernel(const T* __restrict__ x, int B, int H, int ld_
 }
 
 // s = clamp(aK^alpha / aQ^(1-alpha), 2^-16, 2^16) in fp64 -> fp32, inv = 1/s.
-// On entry s holds the bits of aQ and inv_s the bits of aK.
-__global__ void calib_finalize_kernel(float* s, float* inv_s, int n, double alpha, int enable) {
-  int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  double aq = static_cast<double>(__uint_as_float(reinterpret_cast<unsigned int*>(s)[i]));
-  double ak = static_cast<double>(__uint_as_float(reinterpret_cast<unsigned int*>(inv_s)[i]));
+// On entry s holds the bits of aQ and inv_s the bits of aK.  One CTA per kv
+// head, one thread per channel.  enable: 0 = off (s = 1), 1 = on, 2 = the
+// applicability gate: on for a head iff max_c aK > kGateTau * median_c aK
+// (median of the d channels: the mean of the two middle order statistics),
+// decided in fp64.
+constexpr double kGateTau = 8.0;
+__global__ void calib_finalize_kernel(float* s, float* inv_s, int d, double alpha, int enable) {
+  __shared__ float ak_sh[256];
+  __shared__ double mid[2];
+  __shared__ int gate_on;
+  const int h = blockIdx.x, c = threadIdx.x;
+  const int i = h * d + c;
+  const double aq = static_cast<double>(__uint_as_float(reinterpret_cast<unsigned int*>(s)[i]));
+  const float akf = __uint_as_float(reinterpret_cast<unsigned int*>(inv_s)[i]);
+  const double ak = static_cast<double>(akf);
+  int on = enable != 0;
+  if (enable == 2) {
+    ak_sh[c] = akf;
+    if (c == 0) gate_on = 0;
+    __syncthreads();
+    // rank of this channel (ties broken by index): the two middle ranks give the median
+    int rank = 0;
+    for (int c2 = 0; c2 < d; ++c2) {
+      const float x = ak_sh[c2];
+      rank += (x < akf || (x == akf && c2 < c)) ? 1 : 0;
+    }
+    if (rank == d / 2 - 1) mid[0] = ak;
+    if (rank == d / 2) mid[1] = ak;
+    __syncthreads();
+    const double median = 0.5 * (mid[0] + mid[1]);
+    if (ak > kGateTau * median) atomicOr(&gate_on, 1);   // some channel exceeds tau * median
+    __syncthreads();
+    on = gate_on;
+  }
   float sv = 1.0f;
-  if (enable && ak > 0.0 && aq > 0.0) {
+  if (on && ak > 0.0 && aq > 0.0) {
     double val = pow(ak, alpha) / pow(aq, 1.0 - alpha);
     val = fmin(fmax(val, 1.52587890625e-05), 65536.0);
     sv = static_cast<float>(val);
@@ -371,8 +399,7 @@ hifa4_status calibrate_launch(const void* q, const void* k, int dt, int B, int H
     launch_calib_amax<__half>(q, B, Hq, ld_tok, n_cal, d, Hq / Hkv, aq, st);
     launch_calib_amax<__half>(k, B, Hkv, ld_tok, n_cal, d, 1, ak, st);
   }
-  const int n = Hkv * d;
-  calib_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(s_out, inv_s_out, n, static_cast<double>(alpha), enable);
+  calib_finalize_kernel<<<Hkv, d, 0, st>>>(s_out, inv_s_out, d, static_cast<double>(alpha), enable);
   return launch_status("calibrate_smooth_qk");
 }
 

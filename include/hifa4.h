@@ -95,6 +95,11 @@ HIFA4_API size_t hifa4_scale_bytes(int64_t rows, int k, hifa4_format fmt);
  * tokens t < n_cal and the G = Hq/Hkv query heads hq of group h;
  *   s = clamp(aK^alpha / aQ^(1-alpha), 2^-16, 2^16) in fp64 -> fp32,
  *   inv_s = fl32(1/s); s = inv_s = 1 where enable == 0 or an amax is 0.
+ * enable == 2 applies an applicability gate per kv head (the paper's Abstract
+ * para 3 names a gate without a rule; this rule is a reading): smoothing is
+ * on for head h iff max_c aK[h][c] > 8 * median_c aK[h][c] (the median of the
+ * d channels is the mean of the two middle order statistics), decided in
+ * fp64; otherwise s = inv_s = 1 for that head.
  * q: device [B][Hq][ld_tok][d], k: device [B][Hkv][ld_tok][d] of `dt`;
  * s_out, inv_s_out: device float [Hkv][d].  Requires 0 < n_cal <= ld_tok,
  * Hq % Hkv == 0, d in {64, 128, 256}.  Issues two small kernels. */

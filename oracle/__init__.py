@@ -202,15 +202,20 @@ def sf_tiled_bytes(rows: int, nb: int) -> int:
 
 
 # ------------------------------------------------------------ calibration ---
-def calibrate(q, k, n_cal: int, alpha: float = 0.5, enable: bool = True):
-    """q [B,Hq,T,d], k [B,Hkv,T,d] (float) -> (s, inv_s) [Hkv, d] float32."""
+GATE = 2   # calibrate(enable=GATE): the per-head applicability gate
+
+
+def calibrate(q, k, n_cal: int, alpha: float = 0.5, enable=True):
+    """q [B,Hq,T,d], k [B,Hkv,T,d] (float) -> (s, inv_s) [Hkv, d] float32.
+    enable: False / True, or GATE (smoothing per kv head only where its
+    largest K channel amax exceeds 8 x the channel median)."""
     q = _f32(q); k = _f32(k)
     B, Hq, T, d = q.shape
     Hkv = k.shape[1]
     s = np.zeros((Hkv, d), np.float32)
     inv = np.zeros((Hkv, d), np.float32)
     lib().or_calibrate(_p(q, ctypes.c_float), _p(k, ctypes.c_float), B, Hq, Hkv, n_cal, T, d,
-                       float(alpha), int(bool(enable)), _p(s, ctypes.c_float), _p(inv, ctypes.c_float))
+                       float(alpha), int(enable), _p(s, ctypes.c_float), _p(inv, ctypes.c_float))
     return s, inv
 
 

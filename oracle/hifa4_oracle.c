@@ -252,11 +252,40 @@ void or_sf_tile(const uint8_t* plain, int64_t rows, int nb, uint8_t* tiled,
  *   in fp64, rounded to fp32; s = 1 when disabled or either amax is 0;
  *   inv_s = fl32(1/s).
  * q, k: [B][H][ld_tok][d] as float (exact copies of the bf16/fp16 inputs). */
+static int or_cmp_double(const void* a, const void* b) {
+  const double x = *(const double*)a, y = *(const double*)b;
+  return (x > y) - (x < y);
+}
+
 void or_calibrate(const float* q, const float* k, int B, int Hq, int Hkv,
                   int n_cal, int ld_tok, int d, double alpha, int enable,
                   float* s, float* inv_s) {
   int G = Hq / Hkv;
+  double* akv = (double*)malloc(sizeof(double) * d);
+  double* sorted = (double*)malloc(sizeof(double) * d);
   for (int h = 0; h < Hkv; ++h) {
+    /* applicability gate [reading of HiFA4, Abstract para 3, which names the
+     * gate but not its rule]: enable == 2 turns smoothing on for head h only
+     * if its largest channel amax of K exceeds 8 times the median over the d
+     * channels (mean of the two middle order statistics). */
+    int on = enable != 0;
+    if (enable == 2) {
+      double mx = 0.0;
+      for (int c = 0; c < d; ++c) {
+        double aK = 0.0;
+        for (int b = 0; b < B; ++b)
+          for (int t = 0; t < n_cal; ++t) {
+            double vk = fabs((double)k[(((int64_t)b * Hkv + h) * ld_tok + t) * d + c]);
+            if (vk > aK) aK = vk;
+          }
+        akv[c] = aK;
+        sorted[c] = aK;
+        if (aK > mx) mx = aK;
+      }
+      qsort(sorted, (size_t)d, sizeof(double), or_cmp_double);
+      const double median = 0.5 * (sorted[d / 2 - 1] + sorted[d / 2]);
+      on = mx > 8.0 * median;
+    }
     for (int c = 0; c < d; ++c) {
       double aK = 0.0, aQ = 0.0;
       for (int b = 0; b < B; ++b) {
@@ -271,7 +300,7 @@ void or_calibrate(const float* q, const float* k, int B, int Hq, int Hkv,
         }
       }
       float sv = 1.0f;
-      if (enable && aK > 0.0 && aQ > 0.0) {
+      if (on && aK > 0.0 && aQ > 0.0) {
         double v = pow(aK, alpha) / pow(aQ, 1.0 - alpha);
         if (v < ldexp(1.0, -16)) v = ldexp(1.0, -16);
         if (v > ldexp(1.0, 16)) v = ldexp(1.0, 16);
@@ -281,6 +310,8 @@ void or_calibrate(const float* q, const float* k, int B, int Hq, int Hkv,
       inv_s[h * d + c] = 1.0f / sv;
     }
   }
+  free(akv);
+  free(sorted);
 }
 
 /* Fused scale + quantize of Q, K, V [HiFA4, Abstract para 2: "only a fusible

@@ -155,6 +155,24 @@ def test_calibrate_and_quantize_bit_exact(B, Hq, Hkv, N, d, fmt, dtype):
         assert np.array_equal(g, tiled[name]), (name, int(np.sum(g != tiled[name])))
 
 
+def test_calibration_gate_matches_oracle():
+    """The per-head applicability gate: the GPU decision and scales equal the
+    oracle's for heads with and without K outliers."""
+    B, Hq, Hkv, N, d = 1, 8, 4, 128, 128
+    q, k, v = U.synthetic(B, Hq, Hkv, N, d, seed=17, dtype=torch.bfloat16, outlier=0.0)
+    k = k.clone()
+    k[:, 1, :, 5] *= 30       # head 1: one strong outlier channel
+    k[:, 3, :, 77] *= 12
+    for alpha in (0.5, 0.25):
+        s_ref, inv_ref = oracle.calibrate(q.float().numpy(), k.float().numpy(), n_cal=64, alpha=alpha,
+                                          enable=oracle.GATE)
+        s, inv = h.calibrate_smooth_qk(q.cuda(), k.cuda(), n_cal=64, alpha=alpha, enable=h.GATE)
+        np.testing.assert_allclose(U.to_np(s), s_ref, rtol=2 ** -22)
+        np.testing.assert_allclose(U.to_np(inv), inv_ref, rtol=2 ** -22)
+        on = [not np.all(s_ref[hh] == 1.0) for hh in range(Hkv)]
+        assert on[1] and on[3] and not on[0] and not on[2], on
+
+
 # -------------------------------------------------------------- attention ---
 ATTN_CASES = [
     # B, Hq, Hkv, N, d, causal, BN, fmt, mode, dtype

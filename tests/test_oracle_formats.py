@@ -205,3 +205,29 @@ def test_calibration_closed_form():
     k[0, 0, 0, 0] = 1e30       # clamp at 2^16
     s4, _ = oracle.calibrate(q, k, n_cal=7, alpha=1.0)
     assert s4[0, 0] == 2.0 ** 16
+
+
+def test_applicability_gate():
+    """The gate (a reading: smoothing on for a kv head only if its largest K
+    channel amax exceeds 8 times the channel median) on hand-built amax
+    patterns: each head's scales are either exactly the ungated ones or all
+    ones, and the decision flips right at the threshold."""
+    B, Hq, Hkv, T, d = 1, 4, 2, 4, 16
+    q = np.full((B, Hq, T, d), 1.0, np.float32)
+    k = np.zeros((B, Hkv, T, d), np.float32)
+    # head 0: channel amax 1..16 except channel 15 = 8 * median + a hair -> on
+    # head 1: channel amax 1..16 with channel 15 = exactly 8 * median -> off
+    base = np.arange(1, d + 1, dtype=np.float32)          # median (8 + 9) / 2 = 8.5
+    for h in range(Hkv):
+        k[0, h, 0, :] = base
+    k[0, 0, 0, 15] = np.nextafter(np.float32(68.0), np.float32(1e9))
+    k[0, 1, 0, 15] = 68.0
+    s_on, inv_on = oracle.calibrate(q, k, n_cal=T, alpha=0.5, enable=True)
+    s_g, inv_g = oracle.calibrate(q, k, n_cal=T, alpha=0.5, enable=oracle.GATE)
+    assert np.array_equal(s_g[0], s_on[0]) and np.array_equal(inv_g[0], inv_on[0])
+    assert np.all(s_g[1] == 1.0) and np.all(inv_g[1] == 1.0)
+    assert not np.all(s_on[1] == 1.0)        # the ungated scales do differ from 1 there
+    # an outlier-free layer keeps every head off
+    k2 = np.ones((B, Hkv, T, d), np.float32)
+    s2, _ = oracle.calibrate(q, k2, n_cal=T, alpha=0.5, enable=oracle.GATE)
+    assert np.all(s2 == 1.0)
