@@ -87,10 +87,10 @@ def lib():
         L.or_quantize_qkv.argtypes = [f32p, f32p, f32p, i, i, i, i, i, f32p, f32p, i,
                                       u8p, u8p, u8p, u8p, u8p, u8p]
         L.or_attention.argtypes = [u8p, u8p, u8p, u8p, u8p, u8p, i, i, i, i, i, i, d, i, i,
-                                   i, i, f64p, f64p, f64p, f64p, u8p, u8p, f64p, i, i, i]
+                                   i, i, f64p, f64p, f64p, f64p, u8p, u8p, f64p, i, i, i, f]
         L.or_split_len.argtypes = [i, i, i]; L.or_split_len.restype = i
         L.or_decode.argtypes = [f32p, f32p, u8p, u8p, u8p, u8p, i, i, i, i, i, i, d, i, i, i,
-                                i, f64p, f64p, i]
+                                i, f64p, f64p, i, f]
         _lib = L
     return _lib
 
@@ -261,12 +261,13 @@ def tile_scales(qz: dict) -> dict:
 def attention(qz: dict, N: int, fmt: int = NVFP4, softmax_scale: float | None = None,
               causal: bool = True, mode: int = PREORDER, BN: int = 128,
               pexp: int = P_PRESCALE_LOG2, rows=None, dump_phat: bool = False,
-              variant: int = 0):
+              variant: int = 0, tau: float = 0.0):
     """Oracle forward over the quantized tensors of quantize_qkv.
 
     Returns dict O [B,Hq,N,d] fp64, lse, l_phat, l_p [B,Hq,N]; optional P-hat
     code dump.  rows=(begin, end) restricts the query rows computed (other
-    rows of the outputs stay NaN).
+    rows of the outputs stay NaN).  tau > 0: the running max moves only when
+    a tile's max exceeds it by more than tau (lazy rescaling).
     """
     qc, qs = qz["q_codes"], qz["q_sc"]
     B, Hq, Np, dh = qc.shape
@@ -281,6 +282,8 @@ def attention(qz: dict, N: int, fmt: int = NVFP4, softmax_scale: float | None = 
     lp = np.full((B, Hq, N), np.nan)
     ntiles = (N + BN - 1) // BN
     beta = beta_of(fmt)
+    if BN % beta:
+        raise ValueError(f"key tile {BN} is not a multiple of the P-hat block {beta}")
     pd = np.zeros((B, Hq, N, ntiles * BN), np.uint8) if dump_phat else None
     psd = np.zeros((B, Hq, N, ntiles * BN // beta), np.uint8) if dump_phat else None
     md = np.full((B, Hq, N, ntiles), np.nan) if dump_phat else None
@@ -289,7 +292,7 @@ def attention(qz: dict, N: int, fmt: int = NVFP4, softmax_scale: float | None = 
                        float(softmax_scale), int(causal), int(mode), int(BN), int(pexp),
                        _p(O, ctypes.c_double), _p(lse, ctypes.c_double), _p(lph, ctypes.c_double),
                        _p(lp, ctypes.c_double), _p(pd, ctypes.c_uint8), _p(psd, ctypes.c_uint8),
-                       _p(md, ctypes.c_double), int(r0), int(r1), int(variant))
+                       _p(md, ctypes.c_double), int(r0), int(r1), int(variant), float(tau))
     res = dict(O=O, lse=lse, l_phat=lph, l_p=lp)
     if dump_phat:
         res["phat_codes"] = pd
@@ -304,11 +307,14 @@ def split_len(kv_len: int, num_splits: int, BN: int) -> int:
 
 def decode(q, s, cache: dict, kv_len: int, fmt: int = NVFP4, softmax_scale: float | None = None,
            mode: int = PREORDER, BN: int = 128, num_splits: int = 1,
-           pexp: int = P_PRESCALE_LOG2, variant: int = 0):
-    """Split-KV decode: q [B,Hq,d] float, cache = quantize_qkv output (N=kv_len)."""
+           pexp: int = P_PRESCALE_LOG2, variant: int = 0, tau: float = 0.0):
+    """Split-KV decode: q [B,Hq,d] float, cache = quantize_qkv output (N=kv_len).
+    tau: lazy running-max threshold of each split, as in attention()."""
     q = _f32(q)
     B, Hq, d = q.shape
     Hkv = cache["k_codes"].shape[1]
+    if BN % beta_of(fmt):
+        raise ValueError(f"key tile {BN} is not a multiple of the P-hat block {beta_of(fmt)}")
     if softmax_scale is None:
         softmax_scale = 1.0 / np.sqrt(d)
     O = np.zeros((B, Hq, d))
@@ -318,5 +324,5 @@ def decode(q, s, cache: dict, kv_len: int, fmt: int = NVFP4, softmax_scale: floa
     lib().or_decode(_p(q, ctypes.c_float), _p(s32, ctypes.c_float) if s32 is not None else None,
                     *[_p(a, ctypes.c_uint8) for a in arrs], B, Hq, Hkv, kv_len, d, fmt,
                     float(softmax_scale), int(mode), int(BN), int(num_splits), int(pexp),
-                    _p(O, ctypes.c_double), _p(lse, ctypes.c_double), int(variant))
+                    _p(O, ctypes.c_double), _p(lse, ctypes.c_double), int(variant), float(tau))
     return dict(O=O, lse=lse)

@@ -403,7 +403,12 @@ static double prob_of(double x, double m, int exact) {
  * [HiFA4, Abstract para 1] with P-hat quantized per beta-block of the tile
  * [HiFA4, Abstract para 2].  x[k] holds fl32(S*c) for the tile's BN keys, with
  * masked keys marked by vis[k] = 0.  State: m, l_phat, l_p, acc[d].
- * vdq: dequantized V̂ of this kv head, [d][Np] (fp64), key offset k0. */
+ * vdq: dequantized V̂ of this kv head, [d][Np] (fp64), key offset k0.
+ * tau: the running max moves to the tile's max x_t only when
+ * x_t > fl32(m + tau) (fp32, as the kernels decide it; fp64 in the exact
+ * variant); tau = 0 is the exact recurrence m' = max(m, x_t).  With a stale
+ * m the probabilities P = 2^(x - m) may exceed 1.  (The lazy rescaling of
+ * FlashAttention-4; the paper states the exact recurrence.) */
 typedef struct {
   double m;        /* running max, in the log2 domain of scaled scores */
   double l_phat;   /* sum of P-hat under the same recurrence */
@@ -413,14 +418,15 @@ typedef struct {
 
 static void tile_update(or_row_state* st, const double* x, const int* vis, int BN,
                         int fmt, float gP, const double* vdq, int64_t Np,
-                        int64_t k0, int d, int variant, uint8_t* phat_dump,
+                        int64_t k0, int d, int variant, float tau, uint8_t* phat_dump,
                         uint8_t* phat_sc_dump) {
   int exact = (variant & OR_VAR_EXACT) != 0;
   double mt = -INFINITY;
   for (int k = 0; k < BN; ++k)
     if (vis[k] && x[k] > mt) mt = x[k];
   double m_old = st->m;
-  double m_new = (m_old > mt) ? m_old : mt;
+  double thr = exact ? m_old + tau : (double)((float)m_old + tau);
+  double m_new = (mt > thr) ? mt : m_old;
   double alpha = (m_old == -INFINITY) ? 0.0 : exp2(m_old - m_new);
   int beta = (fmt == OR_NVFP4) ? 16 : 32;
   double P[256], Phat[256];
@@ -483,7 +489,7 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
                   int causal, int mode, int BN, int pexp, double* O,
                   double* lse, double* l_phat_out, double* l_p_out,
                   uint8_t* phat_dump, uint8_t* phat_sc_dump, double* m_dump,
-                  int row_begin, int row_end, int variant) {
+                  int row_begin, int row_end, int variant, float tau) {
   int G = Hq / Hkv;
   int beta = (fmt == OR_NVFP4) ? 16 : 32;
   int64_t Np = ((int64_t)N + 127) / 128 * 128;
@@ -527,7 +533,7 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
           }
           uint8_t* pd = phat_dump ? phat_dump + row_id * (int64_t)ntiles * BN + (int64_t)j * BN : NULL;
           uint8_t* psd = phat_sc_dump ? phat_sc_dump + row_id * (int64_t)ntiles * (BN / beta) + (int64_t)j * (BN / beta) : NULL;
-          tile_update(&st, x, vis, BN, fmt, gP, vd, Np, (int64_t)j * BN, d, variant, pd, psd);
+          tile_update(&st, x, vis, BN, fmt, gP, vd, Np, (int64_t)j * BN, d, variant, tau, pd, psd);
           if (m_dump) m_dump[row_id * (int64_t)ntiles + j] = st.m;
         }
         double l = (mode == OR_PREORDER) ? st.l_phat : st.l_p;
@@ -561,7 +567,7 @@ void or_decode(const float* q, const float* s, const uint8_t* k_codes,
                const uint8_t* k_sc, const uint8_t* vt_codes,
                const uint8_t* vt_sc, int B, int Hq, int Hkv, int kv_len, int d,
                int fmt, double softmax_scale, int mode, int BN, int num_splits,
-               int pexp, double* O, double* lse, int variant) {
+               int pexp, double* O, double* lse, int variant, float tau) {
   int G = Hq / Hkv;
   int beta = (fmt == OR_NVFP4) ? 16 : 32;
   int64_t Np = ((int64_t)kv_len + 127) / 128 * 128;
@@ -613,7 +619,7 @@ void or_decode(const float* q, const float* s, const uint8_t* k_codes,
               x[kk] = (variant & OR_VAR_EXACT) ? sdot * c_log2 : (double)(float)(sdot * c_log2);
             }
           }
-          tile_update(&st, x, vis, BN, fmt, gP, vd, Np, j0, d, variant, NULL, NULL);
+          tile_update(&st, x, vis, BN, fmt, gP, vd, Np, j0, d, variant, tau, NULL, NULL);
         }
         ms[sp] = st.m;
         ls[sp] = (mode == OR_PREORDER) ? st.l_phat : st.l_p;

@@ -127,8 +127,9 @@ def _deq_row(codes_row, sc_row, fmt):
     return out
 
 
-def attention(qz, N, fmt, softmax_scale, causal, mode, BN, pexp=-8):
-    """Returns O [B,Hq,N,d] (fp64) and (l_phat, l_p)."""
+def attention(qz, N, fmt, softmax_scale, causal, mode, BN, pexp=-8, tau=0.0):
+    """Returns O [B,Hq,N,d] (fp64) and (l_phat, l_p).  tau: the running max
+    moves to the tile max only when that exceeds fl32(m + tau)."""
     qc = qz["q_codes"]
     B, Hq, Np, dh = qc.shape
     d = dh * 2
@@ -161,7 +162,7 @@ def attention(qz, N, fmt, softmax_scale, causal, mode, BN, pexp=-8):
                         else:
                             xs.append(None)
                     mt = max(x for x in xs if x is not None)
-                    m_new = max(m, mt)
+                    m_new = mt if mt > float(np.float32(m) + np.float32(tau)) else m
                     alpha = 0.0 if m == -math.inf else math.exp2(m - m_new)
                     P = []
                     for x in xs:

@@ -225,3 +225,127 @@ def test_decode_split_combine_exact_when_quant_off(splits):
         p = np.exp(sc - sc.max())
         ref = p @ vd[b, h, :N] / p.sum()
         np.testing.assert_allclose(res["O"][b, hq], ref, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------- lazy rescaling ---
+# The running max may be updated lazily (the conditional rescaling of
+# FlashAttention-4): it moves to a tile's max x_t only when x_t exceeds
+# fl32(m + tau).  Pins: a loop-only second implementation bit for bit, exact
+# softmax attention when quantization is off (the stale max cancels), the
+# P-Reordering two-pass identity, and the rule's own invariants on the dumps.
+
+LAZY_CASES = [
+    # (fmt, N, d, BN, causal, G, mode, tau)
+    (oracle.NVFP4, 64, 16, 16, True, 1, oracle.PREORDER, 3.0),
+    (oracle.NVFP4, 48, 32, 16, False, 2, oracle.INCONSISTENT, 1.5),
+    (oracle.MXFP4, 64, 32, 32, True, 2, oracle.PREORDER, 8.0),
+    (oracle.MXFP4, 40, 32, 32, False, 1, oracle.INCONSISTENT, 2.0),
+]
+
+
+@pytest.mark.parametrize("fmt,N,d,BN,causal,G,mode,tau", LAZY_CASES)
+def test_lazy_rescale_equals_bruteforce(fmt, N, d, BN, causal, G, mode, tau):
+    q, k, v = _inputs(1, G, 1, N, d, 80 + N + d)
+    s, inv = oracle.calibrate(q, k, n_cal=8, alpha=0.5)
+    qz = oracle.quantize_qkv(q, k, v, s, inv, fmt)
+    scale = 2.5 / np.sqrt(d)            # wide scores: the max both moves and stays stale
+    ours = oracle.attention(qz, N, fmt, scale, causal, mode, BN, tau=tau)
+    O, lph, lp = bruteforce.attention(qz, N, fmt, scale, causal, mode, BN, tau=tau)
+    np.testing.assert_allclose(ours["O"], O, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(ours["l_phat"], lph, rtol=1e-13)
+    np.testing.assert_allclose(ours["l_p"], lp, rtol=1e-13)
+    # the lazy path changed the result (it is exercised by this input)
+    exact = oracle.attention(qz, N, fmt, scale, causal, mode, BN)
+    assert not np.array_equal(exact["O"], ours["O"])
+
+
+@pytest.mark.parametrize("tau", [0.5, 3.0, 8.0])
+@pytest.mark.parametrize("causal,BN", [(True, 16), (False, 32)])
+def test_lazy_rescale_quant_off_is_textbook_softmax(tau, causal, BN):
+    """Without quantization a stale max cancels between O and l: exact
+    softmax attention for any threshold, both normalizers."""
+    N, d, G = 72, 32, 2
+    q, k, v = _inputs(1, 2 * G, 2, N, d, 90 + BN)
+    qz = oracle.quantize_qkv(q, k, v, None, None, oracle.NVFP4)
+    deq = _dequant_all(qz, oracle.NVFP4)
+    scale = 0.6
+    ref = _textbook(deq["q"], deq["k"], np.swapaxes(deq["vt"], -1, -2), N, scale, causal, G)
+    for mode in (oracle.PREORDER, oracle.INCONSISTENT):
+        res = oracle.attention(qz, N, oracle.NVFP4, scale, causal, mode, BN,
+                               variant=oracle.VAR_NO_PQUANT | oracle.VAR_EXACT, tau=tau)
+        np.testing.assert_allclose(res["O"], ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("fmt,tau", [(oracle.NVFP4, 3.0), (oracle.MXFP4, 6.0)])
+def test_lazy_rescale_rule_and_two_pass_identity(fmt, tau):
+    """On the dumps: m moves only to a tile max above fl32(m + tau) and never
+    down; P-hat reaches above 1 under a stale max (but not past the bound
+    2^tau rounded up to the grid); and O is the P-Reordering two-pass sum
+    over the per-tile P-hat weighted by 2^(m_j - m_final)."""
+    N, d, G = 128, 32, 2
+    BN = 2 * oracle.beta_of(fmt)
+    q, k, v = _inputs(1, G, 1, N, d, 95)
+    s, inv = oracle.calibrate(q, k, n_cal=16)
+    qz = oracle.quantize_qkv(q, k, v, s, inv, fmt)
+    scale = 2.0 / np.sqrt(d)
+    res = oracle.attention(qz, N, fmt, scale, True, oracle.PREORDER, BN, dump_phat=True, tau=tau)
+    beta = oracle.beta_of(fmt)
+    g = 2.0 ** oracle.P_PRESCALE_LOG2 if fmt == oracle.NVFP4 else 1.0
+    vd = np.swapaxes(_dequant_all(qz, fmt)["vt"], -1, -2)[0, 0]
+    stale = above_one = 0
+    for hq in range(G):
+        for i in range(N):
+            ntl = i // BN + 1
+            m = res["m_tiles"][0, hq, i, :ntl]
+            assert np.all(np.diff(m) >= 0)
+            for j in range(1, ntl):
+                if m[j] != m[j - 1]:
+                    assert m[j] > np.float32(np.float32(m[j - 1]) + np.float32(tau))
+            codes = res["phat_codes"][0, hq, i, :ntl * BN]
+            sc = res["phat_sc"][0, hq, i, :ntl * BN // beta]
+            if fmt == oracle.NVFP4:
+                sd = (oracle.ue4m3_decode(sc) * g).astype(np.float32).astype(np.float64)
+            else:
+                sd = 2.0 ** (sc.astype(np.float64) - 127)
+            phat = GRID[codes & 7] * np.repeat(sd, beta)
+            # P <= 2^tau, and P-hat rounds a block's max by at most its scale step
+            assert phat.max() <= 2.0 ** tau * (1.125 if fmt == oracle.NVFP4 else 1.5)
+            above_one += int(phat.max() > 1.0)
+            stale += int(np.any(np.diff(m) == 0))
+            w = np.repeat(2.0 ** (m - m[-1]), BN)
+            num = (w * phat) @ vd[:ntl * BN]
+            den = np.sum(w * phat)
+            np.testing.assert_allclose(res["O"][0, hq, i], num / den, rtol=1e-12, atol=1e-14)
+    assert stale > 0 and above_one > 0
+
+
+@pytest.mark.parametrize("fmt", [oracle.NVFP4, oracle.MXFP4])
+def test_lazy_rescale_zero_threshold_is_exact_recurrence(fmt):
+    """tau = 0 moves the max whenever it rises: the exact recurrence."""
+    N, d = 96, 32
+    q, k, v = _inputs(1, 2, 1, N, d, 97)
+    qz = oracle.quantize_qkv(q, k, v, None, None, fmt)
+    a = oracle.attention(qz, N, fmt, 0.4, True, oracle.PREORDER, 32, dump_phat=True)
+    b = oracle.attention(qz, N, fmt, 0.4, True, oracle.PREORDER, 32, dump_phat=True, tau=0.0)
+    np.testing.assert_array_equal(a["O"], b["O"])
+    # and that recurrence's max is the running maximum of the tile maxima
+    m = a["m_tiles"][0, 0, N - 1]
+    assert np.all(np.diff(m) >= 0) and np.all(np.isfinite(m))
+
+
+@pytest.mark.parametrize("splits", [1, 3])
+def test_lazy_decode_split_combine_exact_when_quant_off(splits):
+    B, Hq, Hkv, N, d = 1, 4, 2, 300, 32
+    q, k, v = _inputs(B, Hq, Hkv, N, d, 71)
+    qz = oracle.quantize_qkv(q, k, v, None, None, oracle.NVFP4)
+    deq = _dequant_all(qz, oracle.NVFP4)
+    qq = oracle.quantize_qkv(q[:, :, N - 1:N], k[:, :, :1], v[:, :, :1], None, None, oracle.NVFP4)
+    qd = _dequant_all(qq, oracle.NVFP4)["q"][:, :, :1]
+    res = oracle.decode(q[:, :, N - 1], None, qz, N, oracle.NVFP4, 0.5, oracle.PREORDER, 32,
+                        num_splits=splits, variant=oracle.VAR_NO_PQUANT | oracle.VAR_EXACT, tau=3.0)
+    vd = np.swapaxes(deq["vt"], -1, -2)
+    for b, hq in itertools.product(range(B), range(Hq)):
+        h = hq // (Hq // Hkv)
+        sc = qd[b, hq, 0] @ deq["k"][b, h, :N].T * 0.5
+        p = np.exp(sc - sc.max())
+        np.testing.assert_allclose(res["O"][b, hq], p @ vd[b, h, :N] / p.sum(), rtol=1e-12, atol=1e-13)
