@@ -318,6 +318,22 @@ def comparisons(res):
                       "frac_rows_negative": float((eps < 0).float().mean()),
                       "preorder_output_scale_error": 0.0,
                       "inconsistent_output_scale_error_median_over_heads": float(scale_err.median())}
+    # Lazy running-max updates (FlashAttention-4's conditional rescaling; the
+    # paper states the exact recurrence, tau = 0): time and deviation from
+    # exact attention against the exact recurrence, same harness and heads
+    lazy = []
+    o_t = torch.empty_like(o_pre)
+    for tau in (0.0, 1.0, 3.0):
+        fn = lambda: h.attn_fwd(z, scale, w.causal, h.PREORDER, w.block_n, out=o_t, rescale_threshold=tau)
+        ms = time_ms(fn)
+        fn()
+        o4t = o_t[0, heads].float()
+        lazy.append({"rescale_threshold": tau, "ms": ms, "tflops": res["flops"] / (ms * 1e-3) / 1e12,
+                     "max_abs_rel": float((o4t - ex).abs().max() / ex.abs().max()),
+                     "cosine": float(torch.nn.functional.cosine_similarity(o4t.flatten(), ex.flatten(), dim=0))})
+    for rec in lazy:
+        rec["speedup_vs_exact_recurrence"] = lazy[0]["ms"] / rec["ms"]
+    out["lazy_rescale"] = lazy
     # Smooth-QK migration strength and the applicability gate: deviation of
     # the 4-bit output from exact attention (same 4 heads) and eps per setting
     sweep = []

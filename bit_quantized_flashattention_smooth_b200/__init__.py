@@ -32,7 +32,7 @@ _lib = None
 ABI_FUNCTIONS = (
     "hifa4_codes_bytes", "hifa4_scale_bytes", "hifa4_calibrate_smooth_qk", "hifa4_quantize_qkv",
     "hifa4_quantize_kv",
-    "hifa4_attn_fwd", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
+    "hifa4_attn_fwd", "hifa4_attn_fwd_ex", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
     "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_kv_cache_append", "hifa4_attn_decode_cache", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
@@ -57,6 +57,8 @@ def lib():
         L.hifa4_quantize_qkv.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, vp, i, vp, vp, vp, vp, vp, vp, vp]
         L.hifa4_quantize_kv.argtypes = [vp, vp, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp]
         L.hifa4_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, vp]
+        L.hifa4_attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, f,
+                                        vp]
         L.hifa4_decode_workspace_size.argtypes = [i, i, i, i]; L.hifa4_decode_workspace_size.restype = sz
         L.hifa4_decode_default_splits.argtypes = [i, i, i, i]; L.hifa4_decode_default_splits.restype = i
         L.hifa4_attn_decode.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
@@ -73,7 +75,7 @@ def lib():
         L.hifa4_wait_timeout_probe.argtypes = [vp, vp]
         L.hifa4_kv_cache_append.argtypes = [vp, vp, i, i, i, i, i, vp, i, i, i, vp, vp, vp, vp, vp, vp]
         L.hifa4_attn_decode_cache.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i,
-                                              ctypes.POINTER(ctypes.c_int), vp, sz, vp, i, vp]
+                                              ctypes.POINTER(ctypes.c_int), vp, sz, vp, i, f, vp]
         L.hifa4_status_string.argtypes = [i]; L.hifa4_status_string.restype = ctypes.c_char_p
         L.hifa4_last_error.argtypes = []; L.hifa4_last_error.restype = ctypes.c_char_p
         L.hifa4_device_error.argtypes = []; L.hifa4_device_error.restype = ctypes.c_uint
@@ -232,8 +234,9 @@ def quantize_kv(k, v, inv_s=None, fmt: int = NVFP4, Hq: int | None = None, out: 
 # --------------------------------------------------------------- attention ---
 def attn_fwd(z: QuantizedQKV, softmax_scale: float | None = None, causal: bool = True, mode: int = PREORDER,
              block_n: int = 128, out_dtype=torch.bfloat16, return_lse: bool = False, debug: bool = False,
-             out: torch.Tensor | None = None):
-    """4-bit attention forward.  Returns O [B,Hq,N,d] (and lse / debug sums)."""
+             out: torch.Tensor | None = None, rescale_threshold: float = 0.0):
+    """4-bit attention forward.  Returns O [B,Hq,N,d] (and lse / debug sums).
+    rescale_threshold > 0 updates the running max lazily (hifa4_attn_fwd_ex)."""
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(z.d)
     dev = z.q_codes.device
@@ -241,10 +244,11 @@ def attn_fwd(z: QuantizedQKV, softmax_scale: float | None = None, causal: bool =
     lse = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if return_lse else None
     lph = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if debug else None
     lp = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if debug else None
-    _check(lib().hifa4_attn_fwd(_ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),
-                                _ptr(z.vt_codes), _ptr(z.vt_scales), z.B, z.Hq, z.Hkv, z.N, z.d, z.fmt,
-                                float(softmax_scale), int(bool(causal)), int(mode), int(block_n), _ptr(o),
-                                _dt(o), _ptr(lse), _ptr(lph), _ptr(lp), _stream()), "attn_fwd")
+    _check(lib().hifa4_attn_fwd_ex(_ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),
+                                   _ptr(z.vt_codes), _ptr(z.vt_scales), z.B, z.Hq, z.Hkv, z.N, z.d, z.fmt,
+                                   float(softmax_scale), int(bool(causal)), int(mode), int(block_n), _ptr(o),
+                                   _dt(o), _ptr(lse), _ptr(lph), _ptr(lp), float(rescale_threshold), _stream()),
+           "attn_fwd")
     res = [o]
     if return_lse:
         res.append(lse)
@@ -264,8 +268,10 @@ def default_splits(B, Hkv, kv_len, block_n=128) -> int:
 
 def attn_decode(q: torch.Tensor, s: torch.Tensor | None, cache: QuantizedQKV, kv_len: int | None = None,
                 softmax_scale: float | None = None, mode: int = PREORDER, num_splits: int = 0,
-                workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, out_dtype=torch.bfloat16):
-    """Split-KV decode of q [B,Hq,d] over the 4-bit cache.  Returns (O, splits_used)."""
+                workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, out_dtype=torch.bfloat16,
+                rescale_threshold: float = 0.0):
+    """Split-KV decode of q [B,Hq,d] over the 4-bit cache.  Returns (O, splits_used).
+    rescale_threshold > 0 updates each split's running max lazily."""
     B, Hq, d = q.shape
     kv = cache.N if kv_len is None else kv_len
     if softmax_scale is None:
@@ -283,7 +289,7 @@ def attn_decode(q: torch.Tensor, s: torch.Tensor | None, cache: QuantizedQKV, kv
                                          _ptr(cache.vt_codes), _ptr(cache.vt_scales), B, Hq, cache.Hkv, kv, cache.N,
                                          d, cache.fmt, float(softmax_scale), int(mode), 128, int(num_splits),
                                          ctypes.byref(used), _ptr(workspace), workspace.numel(), _ptr(o), _dt(o),
-                                         _stream()), "attn_decode")
+                                         float(rescale_threshold), _stream()), "attn_decode")
     return o, used.value
 
 

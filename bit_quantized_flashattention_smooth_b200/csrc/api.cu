@@ -78,10 +78,10 @@ hifa4_status calibrate_launch(const void*, const void*, int, int, int, int, int,
                               cudaStream_t);
 hifa4_status attn_fwd_launch(const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*,
                              const uint8_t*, int, int, int, int, int, int, float, int, int, int, void*, int, float*,
-                             float*, float*, cudaStream_t);
+                             float*, float*, float, cudaStream_t);
 hifa4_status decode_launch(const void*, int, const float*, const uint8_t*, const uint8_t*, const uint8_t*,
                            const uint8_t*, int, int, int, int, int, int, int, float, int, int, int, int*, void*, size_t,
-                           void*, int, cudaStream_t);
+                           void*, int, float, cudaStream_t);
 hifa4_status kv_append_launch(const void*, const void*, int, int, int, int, int, const float*, int, int, int,
                               uint8_t*, uint8_t*, uint8_t*, uint8_t*, void*, cudaStream_t);
 int decode_default_splits(int B, int Hkv, int kv_len, int block_n);
@@ -111,6 +111,10 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 static bool valid_d(int d) { return d == 64 || d == 128 || d == 256; }
 static bool valid_fmt(int f) { return f == HIFA4_NVFP4 || f == HIFA4_MXFP4; }
 static bool valid_dt(int t) { return t == HIFA4_BF16 || t == HIFA4_FP16; }
+// Largest rescale threshold: with a stale running max P reaches 2^tau, and the
+// NVFP4 P-hat scale fl32(amax/6)/2^-8 must stay within UE4M3's 448 (2^tau <= 10.5).
+static float max_tau(int fmt) { return fmt == HIFA4_NVFP4 ? 3.0f : 8.0f; }
+static bool valid_tau(int fmt, float tau) { return tau >= 0.0f && tau <= max_tau(fmt); }
 
 extern "C" {
 
@@ -179,6 +183,17 @@ hifa4_status hifa4_attn_fwd(const uint8_t* q_codes, const uint8_t* q_scales, con
                             int Hq, int Hkv, int N, int d, hifa4_format fmt, float softmax_scale, int causal,
                             hifa4_norm_mode mode, int block_n, void* o, hifa4_dtype o_dt, float* lse,
                             float* dbg_l_phat, float* dbg_l_p, hifa4_stream_t stream) {
+  return hifa4_attn_fwd_ex(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
+                           softmax_scale, causal, mode, block_n, o, o_dt, lse, dbg_l_phat, dbg_l_p, 0.0f, stream);
+}
+
+hifa4_status hifa4_attn_fwd_ex(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                               const uint8_t* k_scales, const uint8_t* vt_codes, const uint8_t* vt_scales, int B,
+                               int Hq, int Hkv, int N, int d, hifa4_format fmt, float softmax_scale, int causal,
+                               hifa4_norm_mode mode, int block_n, void* o, hifa4_dtype o_dt, float* lse,
+                               float* dbg_l_phat, float* dbg_l_p, float rescale_threshold, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(valid_fmt(fmt) && valid_tau(fmt, rescale_threshold), HIFA4_ERR_INVALID_ARG,
+                "attn_fwd: rescale_threshold must be in [0, %g] for this format", max_tau(fmt));
   HIFA4_REQUIRE(q_codes && q_scales && k_codes && k_scales && vt_codes && vt_scales && o, HIFA4_ERR_INVALID_ARG,
                 "attn_fwd: null pointer");
   HIFA4_REQUIRE(valid_fmt(fmt) && valid_dt(o_dt), HIFA4_ERR_INVALID_ARG, "attn_fwd: bad format/dtype");
@@ -197,7 +212,7 @@ hifa4_status hifa4_attn_fwd(const uint8_t* q_codes, const uint8_t* q_scales, con
   HIFA4_REQUIRE(static_cast<int64_t>(B) * Hq * pad128(N) < (int64_t(1) << 31), HIFA4_ERR_UNSUPPORTED,
                 "attn_fwd: problem too large");
   return attn_fwd_launch(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
-                         softmax_scale, causal, mode, block_n, o, o_dt, lse, dbg_l_phat, dbg_l_p,
+                         softmax_scale, causal, mode, block_n, o, o_dt, lse, dbg_l_phat, dbg_l_p, rescale_threshold,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -234,7 +249,7 @@ hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const float* s, 
                     aligned16(vt_scales) && aligned16(o) && aligned16(workspace) && (!s || aligned16(s)),
                 HIFA4_ERR_INVALID_ARG, "attn_decode: pointers must be 16-byte aligned");
   return decode_launch(q, q_dt, s, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, kv_len, kv_len, d, fmt,
-                       softmax_scale, mode, 128, num_splits, num_splits_used, workspace, ws_bytes, o, o_dt,
+                       softmax_scale, mode, 128, num_splits, num_splits_used, workspace, ws_bytes, o, o_dt, 0.0f,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -243,7 +258,9 @@ hifa4_status hifa4_attn_decode_cache(const void* q, hifa4_dtype q_dt, const floa
                                      int B, int Hq, int Hkv, int kv_len, int kv_capacity, int d, hifa4_format fmt,
                                      float softmax_scale, hifa4_norm_mode mode, int block_n, int num_splits,
                                      int* num_splits_used, void* workspace, size_t ws_bytes, void* o,
-                                     hifa4_dtype o_dt, hifa4_stream_t stream) {
+                                     hifa4_dtype o_dt, float rescale_threshold, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(valid_fmt(fmt) && valid_tau(fmt, rescale_threshold), HIFA4_ERR_INVALID_ARG,
+                "attn_decode_cache: rescale_threshold must be in [0, %g] for this format", max_tau(fmt));
   HIFA4_REQUIRE(kv_capacity >= kv_len, HIFA4_ERR_INVALID_ARG, "attn_decode_cache: kv_len %d > capacity %d", kv_len,
                 kv_capacity);
   HIFA4_REQUIRE(q && k_codes && k_scales && vt_codes && vt_scales && o && workspace, HIFA4_ERR_INVALID_ARG,
@@ -264,7 +281,7 @@ hifa4_status hifa4_attn_decode_cache(const void* q, hifa4_dtype q_dt, const floa
                 HIFA4_ERR_INVALID_ARG, "attn_decode_cache: pointers must be 16-byte aligned");
   return decode_launch(q, q_dt, s, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, kv_len, kv_capacity, d, fmt,
                        softmax_scale, mode, 128, num_splits, num_splits_used, workspace, ws_bytes, o, o_dt,
-                       static_cast<cudaStream_t>(stream));
+                       rescale_threshold, static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_kv_cache_append(const void* k_new, const void* v_new, hifa4_dtype dt, int B, int Hkv, int T,

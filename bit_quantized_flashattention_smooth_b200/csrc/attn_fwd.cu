@@ -63,6 +63,7 @@ struct AttnParams {
   int B, Hq, Hkv, N, Np, G;
   int num_qtiles;
   float c_log2;         // softmax_scale * log2(e)
+  float tau;            // rescale threshold (log2 units); 0 = exact running max
   int causal;
   int out_fp16;
   void* o;
@@ -532,10 +533,14 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
           ok = false;
           break;
         }
-        m_new = fmaxf(m, fmaxf(xb[r], xb[128 + r]));
+        m_new = fmaxf(xb[r], xb[128 + r]);
       } else {
-        m_new = fmaxf(m, __fmul_rn(tree_max<NBH>(bms), c));
+        m_new = __fmul_rn(tree_max<NBH>(bms), c);
       }
+      // The running max moves only when the tile's max exceeds it by more
+      // than tau (tau = 0: whenever it rises); otherwise P is taken against
+      // the stale max and may reach 2^tau.  m = -inf always moves.
+      m_new = m_new > m + p.tau ? m_new : m;
       const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);
       if constexpr (C::CORR) {
         if (j > 0) {
@@ -777,7 +782,7 @@ static hifa4_status launch_attn_fm(int fmt, int mode, const uint8_t* qc, const u
 hifa4_status attn_fwd_launch(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
                              const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int N, int d, int fmt,
                              float softmax_scale, int causal, int mode, int block_n, void* o, int o_dt, float* lse,
-                             float* dbg_l_phat, float* dbg_l_p, cudaStream_t st) {
+                             float* dbg_l_phat, float* dbg_l_p, float rescale_threshold, cudaStream_t st) {
   AttnParams p;
   p.q_sf = qs;
   p.k_sf = ks;
@@ -792,6 +797,7 @@ hifa4_status attn_fwd_launch(const uint8_t* qc, const uint8_t* qs, const uint8_t
   p.G = Hq / Hkv;
   p.num_qtiles = p.Np / 128;
   p.c_log2 = softmax_scale * 1.4426950408889634f;
+  p.tau = rescale_threshold;
   p.causal = causal;
   p.out_fp16 = o_dt == HIFA4_FP16;
   p.o = o;

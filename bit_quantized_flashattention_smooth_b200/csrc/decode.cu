@@ -37,6 +37,7 @@ struct DecodeParams {
   int B, Hq, Hkv, G, kv_len, Np, split_len, splits;
   int q_fp16;
   float c_log2;
+  float tau;            // rescale threshold (log2 units); 0 = exact running max
   float* ws;            // [B][Hq][splits][d+2]: acc (true units), m, l
 };
 
@@ -354,7 +355,7 @@ __global__ void __launch_bounds__(192, 4)
 #pragma unroll
       for (int q = 0; q < G; ++q) {
         const float tm = fmaxf(fmaxf(rbuf[q], rbuf[8 + q]), fmaxf(rbuf[16 + q], rbuf[24 + q]));
-        mnew[q] = fmaxf(m[q], tm);
+        mnew[q] = tm > m[q] + p.tau ? tm : m[q];     // lazy: the max moves by more than tau
         alpha[q] = (mnew[q] == m[q]) ? 1.0f : ex2_approx(m[q] - mnew[q]);
       }
       // P-hat buffer pb was last read by PV_{j-2}
@@ -527,7 +528,7 @@ hifa4_status decode_launch(const void* q, int q_dt, const float* s, const uint8_
                            const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int kv_len, int kv_cap,
                            int d, int fmt,
                            float softmax_scale, int mode, int block_n, int num_splits, int* num_splits_used,
-                           void* workspace, size_t ws_bytes, void* o, int o_dt, cudaStream_t st) {
+                           void* workspace, size_t ws_bytes, void* o, int o_dt, float tau, cudaStream_t st) {
   if (num_splits == 0) num_splits = decode_default_splits(B, Hkv, kv_len, block_n);
   const int tiles = (kv_len + block_n - 1) / block_n;
   if (num_splits > tiles) num_splits = tiles;
@@ -554,6 +555,7 @@ hifa4_status decode_launch(const void* q, int q_dt, const float* s, const uint8_
   p.splits = used;
   p.q_fp16 = q_dt == HIFA4_FP16;
   p.c_log2 = softmax_scale * 1.4426950408889634f;
+  p.tau = tau;
   p.ws = static_cast<float*>(workspace);
   hifa4_status r = HIFA4_ERR_UNSUPPORTED;
   const bool pre = mode == HIFA4_NORM_PREORDER;

@@ -486,14 +486,16 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float2 p0, float2 p1, float2 p2, 
       : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
   return w;
 }
-// MXFP4 scale code of a block of probabilities P_i = fl32(2^(y_i)), y_i <= 0,
-// from the block maximum of y alone: floor(log2(fl32(2^y))) equals floor(y),
-// except that y in [log2(1 - 2^-25), 0) rounds to P = 1 (exponent 0).  The
-// code is E + 127 with E = max(floor(log2 amax) - 2, -127); P below 2^-126 is
-// flushed to 0 and gives E = -127 as well.  Exact: no exponential involved.
+// MXFP4 scale code of a block of probabilities P_i = fl32(2^(y_i)) from the
+// block maximum of y alone (y <= 8: with a lazily updated running max P may
+// exceed 1): floor(log2(fl32(2^y))) equals floor(y), except that y in
+// [log2(1 - 2^-25), 0) rounds to P = 1 (exponent 0); below a positive integer
+// no fp32 y lies that close.  The code is E + 127 with
+// E = max(floor(log2 amax) - 2, -127); P below 2^-126 is flushed to 0 and
+// gives E = -127 as well.  Exact: no exponential involved.
 __device__ __forceinline__ uint32_t mx_scale_from_ymax(float ymax) {
-  if (ymax >= -4.2995e-8f) return 125u;
-  const int k = static_cast<int>(floorf(fmaxf(ymax, -200.0f)));   // masked blocks: y = -inf
+  const float y = (ymax >= -4.2995e-8f && ymax < 0.0f) ? 0.0f : ymax;
+  const int k = static_cast<int>(floorf(fmaxf(y, -200.0f)));   // masked blocks: y = -inf
   return k + 125 > 0 ? static_cast<uint32_t>(k + 125) : 0u;
 }
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -162,6 +162,28 @@ HIFA4_API hifa4_status hifa4_attn_fwd(const uint8_t* q_codes, const uint8_t* q_s
                             hifa4_dtype o_dt, float* lse, float* dbg_l_phat, float* dbg_l_p,
                             hifa4_stream_t stream);
 
+/* hifa4_attn_fwd with a lazily updated running max (the conditional rescaling
+ * of FlashAttention-4; the paper states the exact online recurrence, which is
+ * rescale_threshold = 0, i.e. hifa4_attn_fwd).  Per query row and key tile,
+ * with x_t the tile's largest scaled score fl32(S*c):
+ *   if x_t > fl32(m + rescale_threshold):  m_new = x_t, alpha = 2^(m - m_new)
+ *   else:                                   m_new = m,   alpha = 1
+ * (in fp32; m = -inf always moves).  P = 2^(x - m_new) may then reach
+ * 2^rescale_threshold; P-hat is that P block-quantized by the same rules, and
+ * O, l and lse follow the same recurrence, so without quantization the result
+ * is exact attention for any threshold.  Tiles where no row of a warp moves
+ * its max skip the O rescale and its wait for the previous PV product.
+ * rescale_threshold in log2 units: [0, 3] for NVFP4 (P up to 2^3 keeps the
+ * P-hat scale, fl32(amax/6)/2^-8, below UE4M3's 448), [0, 8] for MXFP4;
+ * otherwise HIFA4_ERR_INVALID_ARG (NaN included). */
+HIFA4_API hifa4_status hifa4_attn_fwd_ex(const uint8_t* q_codes, const uint8_t* q_scales,
+                                         const uint8_t* k_codes, const uint8_t* k_scales,
+                                         const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
+                                         int Hkv, int N, int d, hifa4_format fmt, float softmax_scale,
+                                         int causal, hifa4_norm_mode mode, int block_n, void* o,
+                                         hifa4_dtype o_dt, float* lse, float* dbg_l_phat, float* dbg_l_p,
+                                         float rescale_threshold, hifa4_stream_t stream);
+
 /* ----------------------------------------------------- split-KV decode --- */
 
 /* Workspace bytes for hifa4_attn_decode with `num_splits` splits (per split
@@ -215,15 +237,19 @@ HIFA4_API hifa4_status hifa4_kv_cache_append(const void* k_new, const void* v_ne
                                              uint8_t* vt_scales, void* v_tail, hifa4_stream_t stream);
 
 /* hifa4_attn_decode over the first kv_len tokens of an appendable cache laid
- * out for kv_capacity tokens (kv_len <= kv_capacity); same arguments and
- * results otherwise.  hifa4_attn_decode is the case kv_capacity = kv_len. */
+ * out for kv_capacity tokens (kv_len <= kv_capacity), with each split's
+ * running max updated lazily by rescale_threshold under the rule of
+ * hifa4_attn_fwd_ex (0 = the exact recurrence; same bounds); same arguments
+ * and results otherwise.  hifa4_attn_decode is the case kv_capacity = kv_len,
+ * rescale_threshold = 0. */
 HIFA4_API hifa4_status hifa4_attn_decode_cache(const void* q, hifa4_dtype q_dt, const float* s,
                                                const uint8_t* k_codes, const uint8_t* k_scales,
                                                const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
                                                int Hkv, int kv_len, int kv_capacity, int d, hifa4_format fmt,
                                                float softmax_scale, hifa4_norm_mode mode, int block_n,
                                                int num_splits, int* num_splits_used, void* workspace,
-                                               size_t ws_bytes, void* o, hifa4_dtype o_dt, hifa4_stream_t stream);
+                                               size_t ws_bytes, void* o, hifa4_dtype o_dt,
+                                               float rescale_threshold, hifa4_stream_t stream);
 
 /* Decode for callers that cannot allocate device memory.  (The paper has no
  * counterpart; this is a deployment convenience of this library.)  Callers

@@ -66,6 +66,15 @@ def test_host_validation_without_gpu(L):
     st = L.hifa4_attn_fwd(fake, fake, fake, fake, fake, fake, 1, 2, 2, 128, 128, 0, 0.1, 1, 0, 128, nul, 0,
                           nul, nul, nul, nul)
     assert st == 1
+    # lazy rescale threshold: [0, 3] for NVFP4 (P-hat scale range), [0, 8] for MXFP4, NaN refused
+    for fmt, tau in ((0, 3.5), (0, -1.0), (1, 8.5), (0, float("nan"))):
+        st = L.hifa4_attn_fwd_ex(fake, fake, fake, fake, fake, fake, 1, 2, 2, 128, 128, fmt, 0.1, 1, 0, 128, fake,
+                                 0, nul, nul, nul, ctypes.c_float(tau), nul)
+        assert st == 1 and b"rescale_threshold" in L.hifa4_last_error(), (fmt, tau)
+    used0 = ctypes.c_int(0)
+    st = L.hifa4_attn_decode_cache(fake, 0, nul, fake, fake, fake, fake, 1, 8, 2, 1024, 1024, 128, 0, 0.1, 0, 128,
+                                   0, ctypes.byref(used0), fake, 1 << 20, fake, 0, ctypes.c_float(4.0), nul)
+    assert st == 1 and b"rescale_threshold" in L.hifa4_last_error()
     # decode: d must be 128, workspace required
     used = ctypes.c_int(0)
     st = L.hifa4_attn_decode(fake, 0, nul, fake, fake, fake, fake, 1, 8, 2, 1024, 64, 0, 0.1, 0, 128, 0,
