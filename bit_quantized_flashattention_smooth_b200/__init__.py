@@ -34,7 +34,7 @@ ABI_FUNCTIONS = (
     "hifa4_quantize_kv",
     "hifa4_attn_fwd", "hifa4_attn_fwd_ex", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
-    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_kv_cache_append", "hifa4_attn_decode_cache", "hifa4_status_string", "hifa4_last_error",
+    "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_e2m1_map_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_kv_cache_append", "hifa4_attn_decode_cache", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
 )
 
@@ -70,6 +70,7 @@ def lib():
         L.hifa4_convert_probe.argtypes = [vp, i64, vp, vp, vp]
         L.hifa4_div6_probe.argtypes = [ctypes.c_uint32, ctypes.c_uint32, vp, vp, vp]
         L.hifa4_exp2_poly_probe.argtypes = [vp, i64, vp, vp]
+        L.hifa4_e2m1_map_probe.argtypes = [vp, i64, vp, vp, vp]
         L.hifa4_bf16_attn_fwd.argtypes = [vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp]
         L.hifa4_bf16_transpose_v.argtypes = [vp, i, i, i, i, vp, vp]
         L.hifa4_wait_timeout_probe.argtypes = [vp, vp]
@@ -367,6 +368,16 @@ def exp2_poly_probe(y: torch.Tensor) -> torch.Tensor:
     out = torch.empty_like(y)
     _check(lib().hifa4_exp2_poly_probe(_ptr(y), y.numel(), _ptr(out), _stream()), "exp2_poly_probe")
     return out
+
+
+def e2m1_map_probe(y: torch.Tensor):
+    """E2M1 codes of 2^y from the exponential-free code argument and from the
+    MUFU 2^y (one code per byte each)."""
+    y = y.contiguous().float()
+    cm = torch.empty(y.shape, device=y.device, dtype=torch.uint8)
+    ce = torch.empty(y.shape, device=y.device, dtype=torch.uint8)
+    _check(lib().hifa4_e2m1_map_probe(_ptr(y), y.numel(), _ptr(cm), _ptr(ce), _stream()), "e2m1_map_probe")
+    return cm, ce
 
 
 def convert_probe(x: torch.Tensor):

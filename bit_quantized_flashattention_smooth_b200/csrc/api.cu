@@ -90,6 +90,7 @@ hifa4_status fp4_mma_probe_launch(const uint8_t*, const uint8_t*, const uint8_t*
 hifa4_status convert_probe_launch(const float*, int64_t, uint8_t*, uint8_t*, cudaStream_t);
 hifa4_status div6_probe_launch(uint32_t, uint32_t, unsigned long long*, uint32_t*, cudaStream_t);
 hifa4_status exp2_poly_probe_launch(const float*, int64_t, float*, cudaStream_t);
+hifa4_status e2m1_map_probe_launch(const float*, int64_t, uint8_t*, uint8_t*, cudaStream_t);
 hifa4_status wait_timeout_probe_launch(unsigned int*, cudaStream_t);
 hifa4_status bf16_attn_launch(const void*, const void*, const void*, int, int, int, int, int, float, int, void*, float*,
                               cudaStream_t);
@@ -354,6 +355,13 @@ hifa4_status hifa4_wait_timeout_probe(unsigned int* status, hifa4_stream_t strea
 hifa4_status hifa4_exp2_poly_probe(const float* y, int64_t count, float* out, hifa4_stream_t stream) {
   HIFA4_REQUIRE(count >= 0 && (count == 0 || (y && out)), HIFA4_ERR_INVALID_ARG, "exp2_poly_probe: bad args");
   return exp2_poly_probe_launch(y, count, out, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_e2m1_map_probe(const float* y, int64_t count, uint8_t* codes_map, uint8_t* codes_ex2,
+                                   hifa4_stream_t stream) {
+  HIFA4_REQUIRE(count >= 0 && (count == 0 || (y && codes_map && codes_ex2)), HIFA4_ERR_INVALID_ARG,
+                "e2m1_map_probe: bad args");
+  return e2m1_map_probe_launch(y, count, codes_map, codes_ex2, static_cast<cudaStream_t>(stream));
 }
 
 const char* hifa4_status_string(hifa4_status st) {

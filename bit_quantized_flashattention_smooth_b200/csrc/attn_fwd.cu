@@ -38,11 +38,17 @@
 #include "ptx.cuh"
 
 // Tuning knobs (measured on the 32-head, 4096-token causal prefill):
-// element pairs (of every eight pairs) whose 2^y runs on the FMA pipe (-1: 0 for
-// 64-key tiles, 2 for 128-key tiles), and softmax warpgroups per row for
-// 64-key tiles.
+// element pairs (of every eight pairs) whose 2^y (or code argument) runs on
+// the FMA pipe instead of MUFU (-1: 2, the fastest of 0/2/4/8 at both tile
+// widths), and softmax warpgroups per row for 64-key tiles.
 #ifndef HIFA4_POLY_PAIRS
 #define HIFA4_POLY_PAIRS -1
+#endif
+// 1: where only the P-hat codes are needed (P-Reordering without the debug
+// sums), those FMA-pipe pairs take the exponential-free code argument
+// instead of 2^y; 0: 2^y by the polynomial everywhere
+#ifndef HIFA4_CODE_MAP
+#define HIFA4_CODE_MAP 1
 #endif
 #ifndef HIFA4_ATTN_NH_BN64
 #define HIFA4_ATTN_NH_BN64 1
@@ -479,7 +485,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
     constexpr float kInvGP = FMT == HIFA4_NVFP4 ? 256.0f : 1.0f;
     // pairs (of every eight) whose 2^y runs on the FMA pipe instead of MUFU
-    constexpr int kPolyPairs = HIFA4_POLY_PAIRS >= 0 ? HIFA4_POLY_PAIRS : (BN == 128 ? 2 : 0);
+    constexpr int kPolyPairs = HIFA4_POLY_PAIRS >= 0 ? HIFA4_POLY_PAIRS : 2;
     const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
     const float* log_tab = reinterpret_cast<const float*>(smem + C::OFF_LOG);
     float* xm = reinterpret_cast<float*>(smem + C::OFF_XM);  // [2 parities][2 halves][128]
@@ -601,7 +607,9 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
             const int pair16 = (i % 16) / 2;
             float2 pp;
             if (pair16 < kPolyPairs) {
-              pp = exp2_poly2(y);
+              // codes only (no sum of P): the exponential-free code argument
+              if constexpr (!LP && HIFA4_CODE_MAP) pp = e2m1_arg_from_log2(y);
+              else pp = exp2_poly2(y);
             } else {
               pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
             }

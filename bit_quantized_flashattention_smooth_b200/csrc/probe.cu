@@ -198,6 +198,31 @@ hifa4_status exp2_poly_probe_launch(const float* y, int64_t n, float* out, cudaS
   return launch_status("exp2_poly_probe");
 }
 
+// E2M1 codes of 2^y for `n` values y, two ways: from the exponential-free
+// code argument (codes_map) and from the MUFU 2^y (codes_ex2), both through
+// the same RNE, saturating conversion; one code per byte.
+__global__ void e2m1_map_probe_kernel(const float* __restrict__ y, int64_t n, uint8_t* __restrict__ codes_map,
+                                      uint8_t* __restrict__ codes_ex2) {
+  for (int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); i < n;
+       i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float y0 = y[i], y1 = i + 1 < n ? y[i + 1] : -100.0f;
+    const float2 w = e2m1_arg_from_log2(make_float2(y0, y1));
+    const uint32_t a = cvt_e2m1x2(w.y, w.x);
+    const uint32_t b = cvt_e2m1x2(ex2_approx(y1), ex2_approx(y0));
+    codes_map[i] = static_cast<uint8_t>(a & 15u);
+    codes_ex2[i] = static_cast<uint8_t>(b & 15u);
+    if (i + 1 < n) {
+      codes_map[i + 1] = static_cast<uint8_t>((a >> 4) & 15u);
+      codes_ex2[i + 1] = static_cast<uint8_t>((b >> 4) & 15u);
+    }
+  }
+}
+hifa4_status e2m1_map_probe_launch(const float* y, int64_t n, uint8_t* cm, uint8_t* ce, cudaStream_t st) {
+  if (n == 0) return HIFA4_OK;
+  e2m1_map_probe_kernel<<<148 * 4, 256, 0, st>>>(y, n, cm, ce);
+  return launch_status("e2m1_map_probe");
+}
+
 // The failure path of the bounded mbarrier wait, exercised on purpose: one
 // warp waits on a barrier that nothing arrives at.  The wait gives up after
 // its time limit, raises the abort flag and ORs kErrTimeoutOther into the

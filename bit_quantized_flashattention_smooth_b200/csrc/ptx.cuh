@@ -529,4 +529,31 @@ __device__ __forceinline__ float2 exp2_poly2(float2 y) {
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
+// Exponential-free E2M1 code argument for a pair of log2-domain values y
+// (the P-hat element decision of "Hardware-Aware FP4 FlashAttention-4",
+// Abstract: scores map to FP4 probabilities without forming 2^y).  Returns w
+// with enc2m1(w) = enc2m1(2^y) for every y <= 3.5, decided at the same y:
+// with y = n + f, n = round(y), f in [-1/2, 1/2], the E2M1 rounding of
+// 2^n * 2^f only asks on which side of 0.75, 0.875 and 1.25 the factor 2^f
+// lies (0.625 and 1.75 are out of reach; for n = -2 the edge 0.25 is f = 0),
+// so a cubic q(f) with q(0) = 1 that passes through 2^f at f = log2 0.75,
+// log2 0.875 and log2 1.25 (coefficients solved here from those three
+// conditions; increasing on [-1/2, 1/2], within 6e-4 of 2^f) takes every
+// decision where 2^f does; w = 2^n q(f) through the exponent field.
+// y <= -8 gives a w below 2^-7, code 0.  One fewer packed FMA than
+// exp2_poly2, and no MUFU.
+__device__ __forceinline__ float2 e2m1_arg_from_log2(float2 y) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer
+  constexpr float c1 = 0.6933857202529907f, c2 = 0.24133168160915375f, c3 = 0.053009483963251114f;
+  y.x = fmaxf(y.x, -8.0f);
+  y.y = fmaxf(y.y, -8.0f);
+  const float2 t = fadd2(y, make_float2(kShift, kShift));            // kShift + n
+  const float2 f = fsub2(y, fsub2(t, make_float2(kShift, kShift)));  // y - n, exact
+  float2 q = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = ffma2(q, f, make_float2(c1, c1));
+  q = ffma2(q, f, make_float2(1.0f, 1.0f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 }  // namespace hifa4

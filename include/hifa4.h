@@ -330,6 +330,16 @@ HIFA4_API hifa4_status hifa4_bf16_transpose_v(const void* v, int B, int Hkv, int
  * and y = 0 -> 1 edges. */
 HIFA4_API hifa4_status hifa4_exp2_poly_probe(const float* y, int64_t count, float* out, hifa4_stream_t stream);
 
+/* The exponential-free P-hat code decision the prefill kernel uses for its
+ * FMA-pipe share of elements when only codes are needed (a cubic that equals
+ * 2^f at the three E2M1 rounding edges it can meet, see ptx.cuh), applied to
+ * `count` fp32 log2-domain values y <= 3.5: codes_map[i] = E2M1 code (RNE,
+ * saturating) of that argument, codes_ex2[i] = the code of the MUFU 2^y,
+ * one code per byte (device in, device out).  Lets a test compare both with
+ * the written encoder of fl32(2^y). */
+HIFA4_API hifa4_status hifa4_e2m1_map_probe(const float* y, int64_t count, uint8_t* codes_map, uint8_t* codes_ex2,
+                                            hifa4_stream_t stream);
+
 /* The kernels' failure path, exercised: one warp waits on an mbarrier that
  * nothing arrives at.  The bounded wait gives up after its limit (2 s), sets
  * its CTA's abort flag and the timeout bit 8 of the device error word, and the

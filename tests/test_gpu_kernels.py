@@ -89,6 +89,29 @@ def test_exp2_polynomial_error_bound():
     assert np.all(out[yd < -126.0] < 2.0 ** -126) and np.all(out >= 0.0)
 
 
+def test_exponential_free_code_decisions():
+    """The exponential-free P-hat code argument takes every E2M1 decision
+    that the written encoder takes on fl32(2^y): over a dense sweep of
+    log2-domain values, at y = -2 (the 0.25 tie, code 0), for -inf, and
+    near each rounding edge y* = log2(midpoint) it may differ only within
+    1e-6 of y* (the MUFU 2^y has the same kind of window)."""
+    g = torch.Generator().manual_seed(9)
+    mids = np.log2(np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]))
+    near = (mids[:, None] + np.linspace(-2e-5, 2e-5, 4001)[None, :]).ravel()
+    y = torch.cat([torch.rand(1 << 21, generator=g) * 13.5 - 10.0, torch.from_numpy(near).float(),
+                   torch.tensor([-2.0, -1.0, 0.0, 1.0, 2.0, 3.0, 3.5, -8.0, -9.5, -1e30, -float("inf")])])
+    cm, ce = h.e2m1_map_probe(y.cuda())
+    cm, ce = U.to_np(cm).astype(np.uint8), U.to_np(ce).astype(np.uint8)
+    yd = y.double().numpy()
+    ref, _ = oracle.encode_array(np.exp2(yd).astype(np.float32))
+    window = np.min(np.abs(yd[:, None] - mids[None, :]), axis=1) < 1e-6
+    bad = (cm != ref) & ~window
+    assert not bad.any(), f"{bad.sum()} code mismatches, first at y={yd[bad][0]!r}"
+    assert np.all(cm[yd == -2.0] == 0) and np.all(cm[np.isneginf(yd)] == 0)
+    # inside the windows both device paths stay within a few decisions
+    assert np.sum(cm != ref) <= np.sum(ce != ref) + 64, (np.sum(cm != ref), np.sum(ce != ref))
+
+
 def test_bounded_wait_gives_up_and_reports():
     """A wait that nothing completes ends after its limit with the abort flag
     and the timeout bit set, the kernel returns, and the context stays usable
