@@ -151,13 +151,30 @@ def run_prefill(args, rank, world):
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     s, inv = h.calibrate_smooth_qk(qd[:, :, : w.n_cal], kd[:, :, : w.n_cal], w.n_cal)   # offline, untimed
     z = h.alloc_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, fmt, dev)
+    kvz = h.alloc_kv_cache(w.B, w.Hq, w.Hkv, w.N, w.d, fmt, dev)
     o = torch.empty((w.B, w.Hq, w.N, w.d), device=dev, dtype=W.torch_dtype(w.dtype))
     flush = L2Flush(dev)
     scale = 1.0 / math.sqrt(w.d)
+    fused = args.path == "fused"
+
+    # one step = the quantization launch, then the attention launch.  fused:
+    # K, V quantized (hifa4_quantize_kv), Smooth-QK and Q quantization inside
+    # the attention kernel; two-launch: Q, K, V quantized, then attention.
+    def quant_launch():
+        if fused:
+            h.quantize_kv(kd, vd, inv, fmt, Hq=w.Hq, out=kvz)
+        else:
+            h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)
+
+    def attn_launch():
+        if fused:
+            h.attn_fwd_fused(qd, s, kvz, scale, w.causal, mode, w.block_n, out=o)
+        else:
+            h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)
 
     def step():
-        h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)
-        h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)
+        quant_launch()
+        attn_launch()
 
     for _ in range(args.warmup):
         flush()
@@ -174,9 +191,9 @@ def run_prefill(args, rank, world):
         flush()                             # L2 flush between timed steps (outside the step events)
         e0, e1, e2 = ev[i]
         e0.record(stream)
-        h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)
+        quant_launch()
         e1.record(stream)
-        h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)
+        attn_launch()
         e2.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -213,6 +230,7 @@ def run_prefill(args, rank, world):
     e2e_ms = allmax(e_s.elapsed_time(e_e) / n_e2e, world)
     h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
     d2h = o.numel() * o.element_size()
+    h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)      # the comparisons read Q-hat, K-hat, V-hat (untimed)
 
     return dict(w=w, fmt=fmt, mode=mode, step_ms=step_ms_max, attn_ms=attn_ms_max, quant_ms=quant_ms,
                 flops=flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clk, wall=wall,
@@ -353,7 +371,7 @@ def comparisons(res):
     return out
 
 
-def traffic_record(kernel, workload, fmt, block_n):
+def traffic_record(kernel, workload, fmt, block_n, launch_path="fused"):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
     one ncu capture, from profiles/traffic.json, if the kernel source still has
     the hash recorded with it (else None: the counters are stale)."""
@@ -365,7 +383,8 @@ def traffic_record(kernel, workload, fmt, block_n):
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     for rec in json.load(open(path)):
         if (rec.get("kernel") == kernel and rec.get("workload") == workload and rec.get("format") == fmt and
-                rec.get("block_n") == block_n and rec.get("source_sha256_16") == digest):
+                rec.get("block_n") == block_n and rec.get("path", "two-launch") == launch_path and
+                rec.get("source_sha256_16") == digest):
             return rec["bytes_per_launch"]
     return None
 
@@ -512,10 +531,18 @@ def profile_target(args, launches: int = 5):
         z = h.quantize_qkv(qd, kd, vd, s, inv, fmt)
         scale = 1.0 / math.sqrt(w.d)
         if args.profile == "quantize":
-            fn = lambda: h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)  # noqa: E731
+            if args.path == "fused":
+                kvz = h.quantize_kv(kd, vd, inv, fmt, Hq=w.Hq)
+                fn = lambda: h.quantize_kv(kd, vd, inv, fmt, Hq=w.Hq, out=kvz)  # noqa: E731
+            else:
+                fn = lambda: h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)  # noqa: E731
         elif args.profile == "attn":
             o = torch.empty((w.B, w.Hq, w.N, w.d), device=dev, dtype=W.torch_dtype(w.dtype))
-            fn = lambda: h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)  # noqa: E731
+            if args.path == "fused":
+                kvz = h.quantize_kv(kd, vd, inv, fmt, Hq=w.Hq)
+                fn = lambda: h.attn_fwd_fused(qd, s, kvz, scale, w.causal, mode, w.block_n, out=o)  # noqa: E731
+            else:
+                fn = lambda: h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)  # noqa: E731
         else:
             qb, kb = qd.to(torch.bfloat16), kd.to(torch.bfloat16)
             vt = h.bf16_transpose_v(vd.to(torch.bfloat16))
@@ -539,6 +566,9 @@ def main():
     ap.add_argument("--workload", default="qwen3_prefill")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--mode", default="preorder", choices=["preorder", "inconsistent"])
+    ap.add_argument("--path", default="two-launch", choices=["fused", "two-launch"],
+                    help="fused: K/V quantize + attention with Smooth-QK and Q quantization in the kernel; "
+                         "two-launch: Q/K/V quantize + attention")
     ap.add_argument("--block-n", type=int, default=0, help="key tile (0 = the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
@@ -553,7 +583,7 @@ def main():
         W.WORKLOADS[args.workload] = W.Workload(**{**W.WORKLOADS[args.workload].__dict__, "block_n": args.block_n})
     w = W.WORKLOADS[args.workload]
     config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
-              "format": args.fmt, "normalizer": args.mode, "block_n": w.block_n,
+              "format": args.fmt, "normalizer": args.mode, "block_n": w.block_n, "path": args.path,
               "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)", "parallelism": f"replicas x{world}"}
 
     if args.profile:
@@ -630,7 +660,7 @@ def main():
                                 "peak": 16.0 * sms * clk_mhz * 1e6, "exp2_per_launch": n_exp,
                                 "frac": n_exp / (res["attn_ms"] * 1e-3) / (16.0 * sms * clk_mhz * 1e6),
                                 "note": "MUFU ex2 ceiling: 16/clk/SM x SMs x median SM clock"}
-    tr = traffic_record("attn_fwd_fp4", w.name, args.fmt, w.block_n)
+    tr = traffic_record("attn_fwd_fp4", w.name, args.fmt, w.block_n, args.path)
     if tr is not None:
         line["roofline"]["traffic"] = tr
     if rank == 0 and not args.no_compare:

@@ -32,7 +32,7 @@ _lib = None
 ABI_FUNCTIONS = (
     "hifa4_codes_bytes", "hifa4_scale_bytes", "hifa4_calibrate_smooth_qk", "hifa4_quantize_qkv",
     "hifa4_quantize_kv",
-    "hifa4_attn_fwd", "hifa4_attn_fwd_ex", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
+    "hifa4_attn_fwd", "hifa4_attn_fwd_ex", "hifa4_attn_fwd_fused", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
     "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_e2m1_map_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_kv_cache_append", "hifa4_attn_decode_cache", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
@@ -59,6 +59,8 @@ def lib():
         L.hifa4_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, vp]
         L.hifa4_attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, f,
                                         vp]
+        L.hifa4_attn_fwd_fused.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp,
+                                           f, vp]
         L.hifa4_decode_workspace_size.argtypes = [i, i, i, i]; L.hifa4_decode_workspace_size.restype = sz
         L.hifa4_decode_default_splits.argtypes = [i, i, i, i]; L.hifa4_decode_default_splits.restype = i
         L.hifa4_attn_decode.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
@@ -250,6 +252,35 @@ def attn_fwd(z: QuantizedQKV, softmax_scale: float | None = None, causal: bool =
                                    float(softmax_scale), int(bool(causal)), int(mode), int(block_n), _ptr(o),
                                    _dt(o), _ptr(lse), _ptr(lph), _ptr(lp), float(rescale_threshold), _stream()),
            "attn_fwd")
+    res = [o]
+    if return_lse:
+        res.append(lse)
+    if debug:
+        res += [lph, lp]
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def attn_fwd_fused(q: torch.Tensor, s: torch.Tensor | None, kv: QuantizedQKV, softmax_scale: float | None = None,
+                   causal: bool = True, mode: int = PREORDER, block_n: int = 128, out_dtype=torch.bfloat16,
+                   return_lse: bool = False, debug: bool = False, out: torch.Tensor | None = None,
+                   rescale_threshold: float = 0.0):
+    """Prefill forward with Smooth-QK and Q quantization inside the attention
+    kernel: q [B,Hq,N,d] raw (bf16/fp16), s [Hkv,d] or None, kv = quantize_kv(k, v, 1/s).
+    Equals quantize_qkv + attn_fwd bit for bit."""
+    B, Hq, N, d = q.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    q = q.contiguous()
+    dev = q.device
+    o = out if out is not None else torch.empty((B, Hq, N, d), device=dev, dtype=out_dtype)
+    lse = torch.empty((B, Hq, N), device=dev, dtype=torch.float32) if return_lse else None
+    lph = torch.empty((B, Hq, N), device=dev, dtype=torch.float32) if debug else None
+    lp = torch.empty((B, Hq, N), device=dev, dtype=torch.float32) if debug else None
+    _check(lib().hifa4_attn_fwd_fused(_ptr(q), _dt(q), _ptr(s), _ptr(kv.k_codes), _ptr(kv.k_scales),
+                                      _ptr(kv.vt_codes), _ptr(kv.vt_scales), B, Hq, kv.Hkv, N, d, kv.fmt,
+                                      float(softmax_scale), int(bool(causal)), int(mode), int(block_n), _ptr(o),
+                                      _dt(o), _ptr(lse), _ptr(lph), _ptr(lp), float(rescale_threshold), _stream()),
+           "attn_fwd_fused")
     res = [o]
     if return_lse:
         res.append(lse)

@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "quant_rules.cuh"
 
 // Tuning knobs (measured on the 32-head, 4096-token causal prefill):
 // element pairs (of every eight pairs) whose 2^y (or code argument) runs on
@@ -61,6 +62,12 @@
 namespace hifa4 {
 
 struct AttnParams {
+  // Q in its input dtype ([B][Hq][N][d]) and the Smooth-QK scales s ([Hkv][d],
+  // or null): the softmax warps scale and quantize their query tile in the
+  // kernel (the fused path); null: Q-hat comes from q codes / q_sf.
+  const void* q_raw;
+  const float* q_s;
+  int q_fp16;
   const uint8_t* q_sf;
   const uint8_t* k_sf;
   const uint8_t* v_sf;
@@ -257,7 +264,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
 
   // ---- setup ----
   if (threadIdx.x == 0) {
-    mbar_init(BAR(B_QFULL), 1);
+    mbar_init(BAR(B_QFULL), p.q_raw != nullptr ? 4 * C::NH : 1);   // fused: one arrival per softmax warp
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(BAR(B_KFULL + s), 1);
       mbar_init(BAR(B_KEMPTY + s), 1);
@@ -294,6 +301,11 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     reinterpret_cast<float*>(smem + C::OFF_INV)[i] = inv;
     reinterpret_cast<float*>(smem + C::OFF_LOG)[i] = i == 0 ? -INFINITY : log2f(inv);
   }
+  // fused path: the Smooth-QK scales of this head's kv group, staged in the
+  // normalizer-exchange area (free until the epilogue)
+  if (p.q_raw != nullptr && p.q_s != nullptr)
+    for (int i = threadIdx.x; i < D; i += blockDim.x)
+      reinterpret_cast<float*>(smem + C::OFF_LP)[i] = p.q_s[static_cast<int64_t>(hq / p.G) * D + i];
   fence_proxy_async_smem();
   if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_ALLOC);
@@ -312,10 +324,12 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
   if (warp == C::WARP_TMA) {
     // =============================== TMA producer ===============================
     if (lane == 0) {
-      const uint8_t* qsf = p.q_sf + static_cast<int64_t>(bhq) * p.sf_qk_head + static_cast<int64_t>(qtile) * C::NKC_Q * 512;
-      mbar_arrive_expect_tx(BAR(B_QFULL), C::SZ_Q + C::NKC_Q * 512);
-      tma_load_2d(sbase + C::OFF_Q, &tm_q, 0, bhq * p.Np + row0, BAR(B_QFULL));
-      bulk_load(sbase + C::OFF_QSF, qsf, C::NKC_Q * 512, BAR(B_QFULL));
+      if (p.q_raw == nullptr) {
+        const uint8_t* qsf = p.q_sf + static_cast<int64_t>(bhq) * p.sf_qk_head + static_cast<int64_t>(qtile) * C::NKC_Q * 512;
+        mbar_arrive_expect_tx(BAR(B_QFULL), C::SZ_Q + C::NKC_Q * 512);
+        tma_load_2d(sbase + C::OFF_Q, &tm_q, 0, bhq * p.Np + row0, BAR(B_QFULL));
+        bulk_load(sbase + C::OFF_QSF, qsf, C::NKC_Q * 512, BAR(B_QFULL));
+      }
       const int nkc_v_row = p.Np / (4 * C::BETA);  // V^T scale chunks per row group
       for (int j = 0; j < nkt; ++j) {
         const int st = j % C::NS;
@@ -489,6 +503,60 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
     const float* log_tab = reinterpret_cast<const float*>(smem + C::OFF_LOG);
     float* xm = reinterpret_cast<float*>(smem + C::OFF_XM);  // [2 parities][2 halves][128]
+    if (p.q_raw != nullptr) {
+      // Fused Smooth-QK + Q quantization: thread (hw, r) scales and quantizes
+      // its share of row r of the query tile by the rules of the quantize
+      // kernel (shared code), and writes the codes and scale bytes where the
+      // tensor copy would have put them (the swizzled Q tile, the 512-byte
+      // scale chunks).  Rows past N quantize zeros.
+      constexpr int NBQ = D / C::BETA;               // blocks per Q row
+      constexpr int NBQT = NBQ / C::NH;              // this thread's blocks
+      constexpr int NCH = NBQT * C::BETA / 8;        // its 16-byte chunks of the row
+      const float* srow = p.q_s != nullptr ? reinterpret_cast<const float*>(smem + C::OFF_LP) : nullptr;
+      unsigned char* qrow = smem + C::OFF_Q + r * C::QROW;
+      unsigned char* qsfb = smem + C::OFF_QSF + (r & 31) * 16 + (r >> 5) * 4;
+      // all of the thread's loads in flight at once (one memory latency)
+      uint4 raw[NCH];
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.q_raw) +
+                                                          (static_cast<int64_t>(bhq) * p.N + row) * D +
+                                                          hw * NBQT * C::BETA);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) raw[i] = row < p.N ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int bt = 0; bt < NBQT; ++bt) {
+        const int bq = hw * NBQT + bt;
+        float v[C::BETA];
+#pragma unroll
+        for (int k8 = 0; k8 < C::BETA / 8; ++k8) {
+          const uint4 u = raw[bt * (C::BETA / 8) + k8];
+          const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float2 f;
+            if (p.q_fp16) f = __half22float2(*reinterpret_cast<const __half2*>(&wd[e2]));
+            else f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[e2]));
+            const int e = 8 * k8 + 2 * e2;
+            v[e] = srow != nullptr ? __fmul_rn(f.x, srow[bq * C::BETA + e]) : f.x;
+            v[e + 1] = srow != nullptr ? __fmul_rn(f.y, srow[bq * C::BETA + e + 1]) : f.y;
+          }
+        }
+        uint32_t packed[C::BETA / 8];
+        // the shared table holds 1/(scale * g_P) for P-hat: take g_P = 2^-8 back out
+        const uint32_t sc = quant_block<FMT, C::BETA, FMT == HIFA4_NVFP4 ? 8 : 0>(v, packed, inv_tab);
+        const int byte0 = bq * (C::BETA / 2);        // first code byte of the block in the row
+        unsigned char* dst = qrow + swz_chunk(r, byte0 / 16, C::QROW) * 16 + (byte0 % 16);
+        if constexpr (C::BETA == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        qsfb[(bq / 4) * 512 + (bq % 4)] = static_cast<unsigned char>(sc);
+      }
+      if (NBQ < 4 && hw == C::NH - 1)
+        for (int bb = NBQ; bb < 4; ++bb) qsfb[bb] = 0;   // the row's only scale word: unused bytes
+      fence_proxy_async_smem();                          // codes and scales are read by the MMA
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_QFULL));
+    }
     bool ok = true;
     for (int j = 0; j < nkt && ok; ++j) {
       const int sb = j % C::NSB;
@@ -763,7 +831,10 @@ static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const ui
   using C = AttnCfg<D, BN, FMT>;
   CUtensorMap tq, tk, tv;
   const uint64_t Np = static_cast<uint64_t>(p.Np);
-  if (!make_tmap_2d(&tq, qc, D / 2, static_cast<uint64_t>(p.B) * p.Hq * Np, D / 2, 128, D / 2) ||
+  // the fused path quantizes Q in the kernel: its map is never used (built on K)
+  const uint8_t* qmap = p.q_raw != nullptr ? kc : qc;
+  const uint64_t qrows = static_cast<uint64_t>(p.B) * (p.q_raw != nullptr ? p.Hkv : p.Hq) * Np;
+  if (!make_tmap_2d(&tq, qmap, D / 2, qrows, D / 2, 128, D / 2) ||
       !make_tmap_2d(&tk, kc, D / 2, static_cast<uint64_t>(p.B) * p.Hkv * Np, D / 2, BN, D / 2) ||
       !make_tmap_2d(&tv, vc, Np / 2, static_cast<uint64_t>(p.B) * p.Hkv * D, BN / 2, D, BN / 2)) {
     set_last_error("cuTensorMapEncodeTiled failed");
@@ -790,8 +861,12 @@ static hifa4_status launch_attn_fm(int fmt, int mode, const uint8_t* qc, const u
 hifa4_status attn_fwd_launch(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
                              const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int N, int d, int fmt,
                              float softmax_scale, int causal, int mode, int block_n, void* o, int o_dt, float* lse,
-                             float* dbg_l_phat, float* dbg_l_p, float rescale_threshold, cudaStream_t st) {
+                             float* dbg_l_phat, float* dbg_l_p, float rescale_threshold, const void* q_raw,
+                             int q_dt, const float* q_s, cudaStream_t st) {
   AttnParams p;
+  p.q_raw = q_raw;
+  p.q_s = q_s;
+  p.q_fp16 = q_dt == HIFA4_FP16;
   p.q_sf = qs;
   p.k_sf = ks;
   p.v_sf = vs;

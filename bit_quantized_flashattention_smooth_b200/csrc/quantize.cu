@@ -17,88 +17,58 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "quant_rules.cuh"
 
 namespace hifa4 {
 
-template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&f)[8]);
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&f)[8]) {
-  uint4 u = *reinterpret_cast<const uint4*>(p);
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 t = __bfloat1622float2(h[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
-template <>
-__device__ __forceinline__ void load8<__half>(const __half* p, float (&f)[8]) {
-  uint4 u = *reinterpret_cast<const uint4*>(p);
-  const __half2* h = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 t = __half22float2(h[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
+// Rows of Q or K with every load coalesced: lane l of a warp reads the l-th
+// 16-byte chunk (8 values) of the warp's 512 contiguous input bytes (32 / (d/8)
+// whole rows), so one load instruction covers four whole 128-byte lines.  The
+// BETA/8 lanes that share a block combine their maxima by shuffles and each
+// writes its own 4 code bytes (the warp's code writes are one contiguous
+// 128-byte line); the first lane of a block writes the scale byte.  U row
+// groups per lane are loaded before any is quantized.  Rows are flattened
+// (head, token); tokens N..Np-1 are zero padding; head bh uses smoothing row
+// (bh % H) / G of `scale`.
+template <int FMT, int D>
+struct RowTile {
+  static constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
+  static constexpr int U = 4;              // row groups per lane
+  static constexpr int CPR = D / 8;        // 16-byte chunks per row
+  static constexpr int RPI = 32 / CPR;     // rows per warp and row group
+  static constexpr int LPB = BETA / 8;     // lanes per block
+  static constexpr int NB = D / BETA;      // blocks per row
+  static constexpr int ROWS = 8 * U * RPI; // rows per 256-thread CTA; divides 128
+  static_assert(128 % ROWS == 0, "a CTA's rows stay inside one head");
+};
 
-// Quantize one block of BETA fp32 values in place into packed codes
-// (BETA/2 bytes, element 2i in the low nibble) and return the scale code.
-// inv_tab[c] = fl32(1 / UE4M3(c)) (0 for c = 0), in shared memory.
+// One lane's 8 values of a BETA-block spread over LPB = BETA/8 adjacent lanes:
+// the block's scale code (the same in every lane of the block) and this lane's
+// 8 E2M1 codes packed in a word, by exactly the rules of quant_block.
 template <int FMT, int BETA>
-__device__ __forceinline__ uint32_t quant_block(const float (&v)[BETA], uint32_t (&packed)[BETA / 8],
-                                                const float* inv_tab) {
-  float amax = fmaxf(fabsf(v[0]), fabsf(v[1]));
+__device__ __forceinline__ uint32_t quant_part(const float (&v)[8], uint32_t& packed, const float* inv_tab) {
+  float amax = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
+                     fmaxf(fabsf(v[6]), fabsf(v[7])));
 #pragma unroll
-  for (int i = 2; i + 1 < BETA; i += 2) amax = fmax3(amax, fabsf(v[i]), fabsf(v[i + 1]));
+  for (int o = 1; o < BETA / 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   float mult;
   uint32_t sc;
   uint32_t keep = 0xFFFFFFFFu;
   if constexpr (FMT == HIFA4_NVFP4) {
-    // fl32(amax/6): the reciprocal-and-residual form is IEEE-exact on
-    // [2^-122, 2^20] (checked on the GPU); below, both give scale code 0
     const float t = amax <= 1048576.0f ? div6_rn(amax) : __fdiv_rn(amax, 6.0f);
     sc = cvt_e4m3(t);
     mult = inv_tab[sc];
-    if (sc == 0) keep = 0u;                             // scale 0: every code 0 (no -0 codes)
+    if (sc == 0) keep = 0u;
   } else {
     const uint32_t ef = (__float_as_uint(amax) >> 23) & 0xFFu;
-    sc = ef >= 2u ? ef - 2u : 0u;                       // E + 127, E = floor(log2 amax) - 2
-    mult = __uint_as_float((254u - sc) << 23);          // 2^-E
+    sc = ef >= 2u ? ef - 2u : 0u;
+    mult = __uint_as_float((254u - sc) << 23);
   }
   const float2 m2 = make_float2(mult, mult);
-#pragma unroll
-  for (int w = 0; w < BETA / 8; ++w) {
-    const float* e = v + 8 * w;
-    packed[w] = keep & cvt_e2m1x8(fmul2(make_float2(e[0], e[1]), m2), fmul2(make_float2(e[2], e[3]), m2),
-                                  fmul2(make_float2(e[4], e[5]), m2), fmul2(make_float2(e[6], e[7]), m2));
-  }
+  packed = keep & cvt_e2m1x8(fmul2(make_float2(v[0], v[1]), m2), fmul2(make_float2(v[2], v[3]), m2),
+                             fmul2(make_float2(v[4], v[5]), m2), fmul2(make_float2(v[6], v[7]), m2));
   return sc;
 }
-
-// Rows of Q or K, one lane per block: D/BETA lanes cover a row, so each
-// 16-byte load instruction of a warp touches a few whole 128-byte lines
-// instead of one line per lane, and the code bytes of a row are written by
-// consecutive lanes.  kLpbUnroll row groups per lane are loaded before any is
-// quantized.  Rows are flattened (head, token); tokens N..Np-1 are zero
-// padding; head bh uses smoothing row (bh % H) / G of `scale`.
-template <int FMT>
-struct LpbCfg {
-  static constexpr int kUnroll = FMT == HIFA4_NVFP4 ? 2 : 1;
-};
-
-template <int FMT, int D>
-struct RowTile {
-  static constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
-  static constexpr int U = LpbCfg<FMT>::kUnroll;
-  static constexpr int LPR = D / BETA;     // lanes (= blocks) per row
-  static constexpr int RPW = 32 / LPR;     // rows per warp and row group
-  static constexpr int ROWS = 8 * U * RPW; // rows per 256-thread CTA; divides 128
-  static_assert(128 % ROWS == 0, "a CTA's rows stay inside one head");
-};
 
 // CTA `cta` of a tensor with `heads` heads of Np (padded) rows: head
 // cta / (Np / ROWS), rows [chunk * ROWS, +ROWS).  Index arithmetic per CTA,
@@ -109,81 +79,76 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
                                                   uint8_t* __restrict__ sf, int64_t sf_head_bytes, int cta,
                                                   const float* inv_tab) {
   using R = RowTile<FMT, D>;
-  constexpr int BETA = R::BETA, U = R::U, LPR = R::LPR, RPW = R::RPW;
-  constexpr int WPR = (LPR + 3) / 4;       // scale words per row
+  constexpr int BETA = R::BETA, U = R::U, CPR = R::CPR, RPI = R::RPI, LPB = R::LPB, NB = R::NB;
+  constexpr int WPR = (NB + 3) / 4;        // scale words per row
   const int cpt = Np / R::ROWS;
   const int bh = cta / cpt;
   const int chunk = cta - bh * cpt;
   const int kvh = (bh % H) / G;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int lb = lane % LPR;
-  const T* xh = x + static_cast<int64_t>(bh) * N * D + lb * BETA;
-  const float* srow = scale != nullptr ? scale + kvh * D + lb * BETA : nullptr;
-  float v[U][BETA];
+  const int ch = lane % CPR;               // 16-byte chunk of the row
+  const int blk = ch / LPB;                // its block
+  const T* xh = x + static_cast<int64_t>(bh) * N * D + ch * 8;
+  float v[U][8];
   int tok[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    tok[u] = chunk * R::ROWS + (warp * U + u) * RPW + lane / LPR;
+    tok[u] = chunk * R::ROWS + (warp * U + u) * RPI + lane / CPR;
     if (tok[u] < N) {
-      const T* src = xh + static_cast<int64_t>(tok[u]) * D;
-#pragma unroll
-      for (int i = 0; i < BETA / 8; ++i) {
-        float f[8];
-        load8<T>(src + 8 * i, f);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[u][8 * i + j] = f[j];
-      }
+      load8<T>(xh + static_cast<int64_t>(tok[u]) * D, v[u]);
     } else {
 #pragma unroll
-      for (int i = 0; i < BETA; ++i) v[u][i] = 0.0f;
+      for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
     }
   }
-  uint8_t* ch = codes + (static_cast<int64_t>(bh) * Np) * (D / 2) + lb * (BETA / 2);
+  float sv[8];
+  if (scale != nullptr) {
+    const float4* s4 = reinterpret_cast<const float4*>(scale + kvh * D + ch * 8);
+    const float4 a = s4[0], b = s4[1];
+    sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w; sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
+  }
+  uint8_t* cbase = codes + (static_cast<int64_t>(bh) * Np) * (D / 2) + ch * 4;
   uint8_t* sh = sf + static_cast<int64_t>(bh) * sf_head_bytes;
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int t = tok[u];
-    if (srow != nullptr && t < N) {
-      const float4* s4 = reinterpret_cast<const float4*>(srow);
+    if (scale != nullptr && t < N) {
 #pragma unroll
-      for (int i = 0; i < BETA / 4; ++i) {
-        const float4 sv = s4[i];
-        const float2 p0 = fmul2(make_float2(v[u][4 * i + 0], v[u][4 * i + 1]), make_float2(sv.x, sv.y));
-        const float2 p1 = fmul2(make_float2(v[u][4 * i + 2], v[u][4 * i + 3]), make_float2(sv.z, sv.w));
-        v[u][4 * i + 0] = p0.x;
-        v[u][4 * i + 1] = p0.y;
-        v[u][4 * i + 2] = p1.x;
-        v[u][4 * i + 3] = p1.y;
+      for (int i = 0; i < 8; i += 2) {
+        const float2 p2 = fmul2(make_float2(v[u][i], v[u][i + 1]), make_float2(sv[i], sv[i + 1]));
+        v[u][i] = p2.x;
+        v[u][i + 1] = p2.y;
       }
     }
-    uint32_t packed[BETA / 8];
-    const uint32_t sc = quant_block<FMT, BETA>(v[u], packed, inv_tab);
-    uint8_t* dst = ch + static_cast<int64_t>(t) * (D / 2);
-    if constexpr (BETA == 16) {
-      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-    } else {
-      *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    }
-    uint8_t* sfw = sh + sf_word_offset(t, lb / 4, WPR);
-    sfw[lb % 4] = static_cast<uint8_t>(sc);
-    if constexpr (LPR < 4) {
-      // the rest of the row's only scale word holds no block: zero it
-      if (lb == LPR - 1)
+    uint32_t packed;
+    const uint32_t sc = quant_part<FMT, BETA>(v[u], packed, inv_tab);
+    *reinterpret_cast<uint32_t*>(cbase + static_cast<int64_t>(t) * (D / 2)) = packed;
+    if (ch % LPB == 0) {
+      uint8_t* sfw = sh + sf_word_offset(t, blk / 4, WPR);
+      sfw[blk % 4] = static_cast<uint8_t>(sc);
+      if constexpr (NB < 4) {
+        // the rest of the row's only scale word holds no block: zero it
+        if (blk == NB - 1)
 #pragma unroll
-        for (int bb = LPR; bb < 4; ++bb) sfw[bb] = 0;   // lb / 4 == 0: the same word
+          for (int bb = NB; bb < 4; ++bb) sfw[bb] = 0;   // blk / 4 == 0: the same word
+      }
     }
   }
 }
 
 // V: one CTA per (128-token tile, head, 64-channel group).  The tile is staged
 // in shared memory with coalesced 16-byte loads; then one thread per (channel,
-// scale word) quantizes 4 blocks of tokens and writes 4*BETA/2 contiguous code
-// bytes of the channel-major V^T row plus one scale word.
+// token block) quantizes the block (the 32 lanes of a warp read 32 adjacent
+// channels of a token: one shared-memory wavefront) and writes the scale
+// byte, and the codes go through a second staging buffer so that each
+// channel-major V^T row's 64 code bytes of the tile are written by 16-byte
+// stores of consecutive threads.
 constexpr int kVCh = 64;   // channels per V CTA
 template <int FMT, typename T>
 __device__ __forceinline__ void quantize_v_tile(const T* __restrict__ v, int N, int Np, int d,
                                                 uint8_t* __restrict__ vt_codes, uint8_t* __restrict__ vt_sf,
-                                                int64_t sf_head_bytes, int tile, T* tile_smem, const float* inv_tab) {
+                                                int64_t sf_head_bytes, int tile, T* tile_smem,
+                                                unsigned char* code_stage, const float* inv_tab) {
   constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
   const int ncg = d / kVCh;
   const int cg = tile % ncg;
@@ -226,14 +191,30 @@ __device__ __forceinline__ void quantize_v_tile(const T* __restrict__ v, int N, 
     }
     uint32_t packed[BETA / 8];
     const uint32_t sc = quant_block<FMT, BETA>(val, packed, inv_tab);
-    uint8_t* dst = vt_codes + (head * d + c) * static_cast<int64_t>(Np / 2) + (t0 + blk * BETA) / 2;
-    if constexpr (BETA == 16) {
-      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-    } else {
-      *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    }
+    // codes staged per channel row (64 bytes = 128 tokens), pieces swizzled
+    // by the channel so that the 32 channels of a warp spread over the banks
+    unsigned char* srow = code_stage + cl * 64;
+    if constexpr (BETA == 16)
+      *reinterpret_cast<uint2*>(srow + ((blk ^ (cl & 7)) * 8)) = make_uint2(packed[0], packed[1]);
+    else
+      *reinterpret_cast<uint4*>(srow + ((blk ^ (cl & 3)) * 16)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     const int gb = t0 / BETA + blk;                   // block index along the row
     vt_sf[head * sf_head_bytes + sf_word_offset(c, gb / 4, nkc) + (gb % 4)] = static_cast<uint8_t>(sc);
+  }
+  __syncthreads();
+  // each V^T row's 64 code bytes of this tile leave as four 16-byte stores
+  for (int i = threadIdx.x; i < kVCh * 4; i += blockDim.x) {
+    const int cl = i / 4, q = i % 4;
+    const unsigned char* srow = code_stage + cl * 64;
+    uint4 u;
+    if constexpr (BETA == 16) {
+      const uint2 lo = *reinterpret_cast<const uint2*>(srow + (((2 * q) ^ (cl & 7)) * 8));
+      const uint2 hi = *reinterpret_cast<const uint2*>(srow + (((2 * q + 1) ^ (cl & 7)) * 8));
+      u = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    } else {
+      u = *reinterpret_cast<const uint4*>(srow + ((q ^ (cl & 3)) * 16));
+    }
+    *reinterpret_cast<uint4*>(vt_codes + (head * d + c_base + cl) * static_cast<int64_t>(Np / 2) + t0 / 2 + q * 16) = u;
   }
 }
 
@@ -251,6 +232,7 @@ struct QuantArgs {
 template <int FMT, typename T, int D>
 __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a) {
   __shared__ __align__(16) T tile_smem[128 * kVCh];
+  __shared__ __align__(16) unsigned char code_stage[kVCh * 64];
   __shared__ float inv_tab[128];
   if (FMT == HIFA4_NVFP4 && threadIdx.x < 128)
     inv_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __fdiv_rn(1.0f, ue4m3_to_f32(threadIdx.x));
@@ -259,7 +241,7 @@ __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a)
   const int bid = static_cast<int>(blockIdx.x) - a.nv_ctas;
   if (bid < 0) {
     quantize_v_tile<FMT, T>(static_cast<const T*>(a.v), a.N, a.Np, a.d, a.vc, a.vs, a.sf_v_head,
-                            static_cast<int>(blockIdx.x), tile_smem, inv_tab);
+                            static_cast<int>(blockIdx.x), tile_smem, code_stage, inv_tab);
   } else if (bid < a.nq_ctas) {
     quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.s, a.qc, a.qs,
                                  a.sf_qk_head, bid, inv_tab);
@@ -364,10 +346,9 @@ hifa4_status quantize_qkv_launch(const void* q, const void* k, const void* v, in
   a.sf_v_head = static_cast<int64_t>(hifa4_scale_bytes(d, a.Np, static_cast<hifa4_format>(fmt)));
   a.q_rows = q ? static_cast<int64_t>(B) * Hq * a.Np : 0;
   a.k_rows = static_cast<int64_t>(B) * Hkv * a.Np;
-  // 8 warps per CTA, each kUnroll row groups of 32 / (d / BETA) rows
-  const int lpr = d / beta_of(fmt);
-  const int rows_per_cta = 8 * (32 / lpr) * (fmt == HIFA4_NVFP4 ? LpbCfg<HIFA4_NVFP4>::kUnroll
-                                                                 : LpbCfg<HIFA4_MXFP4>::kUnroll);
+  // 8 warps per CTA, each RowTile::U row groups of 32 / (d / 8) rows
+  const int rows_per_cta = d == 64 ? RowTile<HIFA4_NVFP4, 64>::ROWS
+                                   : (d == 128 ? RowTile<HIFA4_NVFP4, 128>::ROWS : RowTile<HIFA4_NVFP4, 256>::ROWS);
   a.nq_ctas = static_cast<int>(a.q_rows / rows_per_cta);    // Np is a multiple of 128, rows_per_cta divides 128
   a.nk_ctas = static_cast<int>(a.k_rows / rows_per_cta);
   a.nv_ctas = (a.Np / 128) * (a.B * a.Hkv) * (a.d / kVCh);

@@ -184,6 +184,24 @@ HIFA4_API hifa4_status hifa4_attn_fwd_ex(const uint8_t* q_codes, const uint8_t* 
                                          hifa4_dtype o_dt, float* lse, float* dbg_l_phat, float* dbg_l_p,
                                          float rescale_threshold, hifa4_stream_t stream);
 
+/* The prefill forward with Smooth-QK and the Q quantization fused into the
+ * attention kernel (the paper's Abstract para 2: Smooth-QK needs "only a
+ * fusible element-wise scaling"): q [B][Hq][N][d] in q_dt, unscaled and
+ * unquantized (device); s the Smooth-QK scales [Hkv][d] fp32 (device) or
+ * NULL for 1.  Each CTA scales and quantizes its 128-row query tile itself,
+ * by exactly the rules of hifa4_quantize_qkv (q' = fl32(q * s[h]), blocks
+ * along d), so the result equals hifa4_quantize_qkv + hifa4_attn_fwd_ex
+ * bit for bit, without the round trip of Q-hat through memory.  K and V come
+ * quantized (hifa4_quantize_kv with inv_s = 1/s).  Other arguments,
+ * requirements and errors as hifa4_attn_fwd_ex. */
+HIFA4_API hifa4_status hifa4_attn_fwd_fused(const void* q, hifa4_dtype q_dt, const float* s,
+                                            const uint8_t* k_codes, const uint8_t* k_scales,
+                                            const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
+                                            int Hkv, int N, int d, hifa4_format fmt, float softmax_scale,
+                                            int causal, hifa4_norm_mode mode, int block_n, void* o,
+                                            hifa4_dtype o_dt, float* lse, float* dbg_l_phat, float* dbg_l_p,
+                                            float rescale_threshold, hifa4_stream_t stream);
+
 /* ----------------------------------------------------- split-KV decode --- */
 
 /* Workspace bytes for hifa4_attn_decode with `num_splits` splits (per split

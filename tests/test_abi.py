@@ -75,6 +75,16 @@ def test_host_validation_without_gpu(L):
     st = L.hifa4_attn_decode_cache(fake, 0, nul, fake, fake, fake, fake, 1, 8, 2, 1024, 1024, 128, 0, 0.1, 0, 128,
                                    0, ctypes.byref(used0), fake, 1 << 20, fake, 0, ctypes.c_float(4.0), nul)
     assert st == 1 and b"rescale_threshold" in L.hifa4_last_error()
+    # fused path: Q dtype, null pointers and tile checks as the unfused entry
+    st = L.hifa4_attn_fwd_fused(fake, 7, nul, fake, fake, fake, fake, 1, 2, 2, 128, 128, 0, 0.1, 1, 0, 128, fake, 0,
+                                nul, nul, nul, ctypes.c_float(0.0), nul)
+    assert st == 1 and b"dtype" in L.hifa4_last_error()
+    st = L.hifa4_attn_fwd_fused(nul, 0, nul, fake, fake, fake, fake, 1, 2, 2, 128, 128, 0, 0.1, 1, 0, 128, fake, 0,
+                                nul, nul, nul, ctypes.c_float(0.0), nul)
+    assert st == 1
+    st = L.hifa4_attn_fwd_fused(fake, 0, nul, fake, fake, fake, fake, 1, 2, 2, 128, 256, 0, 0.1, 1, 0, 64, fake, 0,
+                                nul, nul, nul, ctypes.c_float(0.0), nul)
+    assert st == 2
     # decode: d must be 128, workspace required
     used = ctypes.c_int(0)
     st = L.hifa4_attn_decode(fake, 0, nul, fake, fake, fake, fake, 1, 8, 2, 1024, 64, 0, 0.1, 0, 128, 0,

@@ -155,6 +155,9 @@ QUANT_CASES = [
     (2, 4, 1, 130, 256, oracle.MXFP4, torch.bfloat16),
     (1, 8, 2, 300, 64, oracle.MXFP4, torch.float16),
     (1, 2, 2, 1, 128, oracle.NVFP4, torch.bfloat16),
+    (1, 4, 4, 520, 256, oracle.NVFP4, torch.bfloat16),
+    (2, 4, 2, 333, 128, oracle.MXFP4, torch.float16),
+    (3, 2, 1, 77, 64, oracle.NVFP4, torch.bfloat16),
 ]
 
 
