@@ -70,97 +70,83 @@ struct AppendArgs {
   int64_t sf_k_head, sf_v_head;
 };
 
-// K rows: one thread per (row, block).
+// One launch.  Threads [0, nk) each quantize one (K row, block); threads
+// [nk, nk + nv) each own one (head, channel) of V and walk the touched token
+// blocks in order: every block is quantized again from its raw values (the
+// tokens before pos from v_tail, which only this thread reads or writes for
+// its channel, the new ones from v_new, tokens not yet written 0), and the
+// channel's tail is then rewritten with the raw V of the new partial block.
 template <int FMT, typename T>
-__global__ void __launch_bounds__(256) kv_append_k_kernel(const AppendArgs a) {
+__global__ void __launch_bounds__(256) kv_append_kernel(const AppendArgs a) {
   constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
   const int nb = a.d / BETA;
+  const int64_t nk = static_cast<int64_t>(a.B) * a.Hkv * a.T * nb;
+  const int64_t nv = static_cast<int64_t>(a.B) * a.Hkv * a.d;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * a.T * nb;
-  if (idx >= total) return;
-  const int blk = static_cast<int>(idx % nb);
-  const int64_t r = idx / nb;                  // (bh, t)
-  const int t = static_cast<int>(r % a.T);
-  const int64_t bh = r / a.T;
-  const int kvh = static_cast<int>(bh % a.Hkv);
-  const int p = a.pos + t;
-  const T* src = static_cast<const T*>(a.k_new) + r * a.d + blk * BETA;
-  float v[BETA];
+  if (idx < nk) {
+    // ---- K: one (row, block) ----
+    const int blk = static_cast<int>(idx % nb);
+    const int64_t r = idx / nb;                  // (bh, t)
+    const int t = static_cast<int>(r % a.T);
+    const int64_t bh = r / a.T;
+    const int kvh = static_cast<int>(bh % a.Hkv);
+    const int p = a.pos + t;
+    const T* src = static_cast<const T*>(a.k_new) + r * a.d + blk * BETA;
+    float v[BETA];
 #pragma unroll
-  for (int i = 0; i < BETA; ++i) {
-    v[i] = to_f32(src[i]);
-    if (a.inv_s != nullptr) v[i] = __fmul_rn(v[i], a.inv_s[kvh * a.d + blk * BETA + i]);
+    for (int i = 0; i < BETA; ++i) {
+      v[i] = to_f32(src[i]);
+      if (a.inv_s != nullptr) v[i] = __fmul_rn(v[i], a.inv_s[kvh * a.d + blk * BETA + i]);
+    }
+    uint32_t packed[BETA / 8];
+    const uint32_t sc = append_quant_block<FMT, BETA>(v, packed);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(a.kc + (bh * a.Np + p) * static_cast<int64_t>(a.d / 2) + blk * (BETA / 2));
+#pragma unroll
+    for (int w = 0; w < BETA / 8; ++w) dst[w] = packed[w];
+    const int wpr = (nb + 3) / 4;
+    a.ks[bh * a.sf_k_head + sf_word_offset(p, blk / 4, wpr) + (blk % 4)] = static_cast<uint8_t>(sc);
+    return;
   }
-  uint32_t packed[BETA / 8];
-  const uint32_t sc = append_quant_block<FMT, BETA>(v, packed);
-  uint32_t* dst = reinterpret_cast<uint32_t*>(a.kc + (bh * a.Np + p) * static_cast<int64_t>(a.d / 2) + blk * (BETA / 2));
-#pragma unroll
-  for (int w = 0; w < BETA / 8; ++w) dst[w] = packed[w];
-  const int wpr = (nb + 3) / 4;
-  a.ks[bh * a.sf_k_head + sf_word_offset(p, blk / 4, wpr) + (blk % 4)] = static_cast<uint8_t>(sc);
-}
-
-// V^T blocks: one thread per (head, touched token block, channel).
-template <int FMT, typename T>
-__global__ void __launch_bounds__(256) kv_append_v_kernel(const AppendArgs a) {
-  constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * a.nblk * a.d;
-  if (idx >= total) return;
-  const int c = static_cast<int>(idx % a.d);
-  const int gi = static_cast<int>((idx / a.d) % a.nblk);
-  const int64_t bh = idx / (static_cast<int64_t>(a.d) * a.nblk);
-  const int g = a.g0 + gi;
-  const int tok0 = g * BETA;
-  const T* tail = static_cast<const T*>(a.v_tail) + bh * BETA * a.d;
+  if (idx >= nk + nv) return;
+  // ---- V: one (head, channel), all touched blocks, then the tail ----
+  const int64_t vi = idx - nk;
+  const int c = static_cast<int>(vi % a.d);
+  const int64_t bh = vi / a.d;
+  T* tail = static_cast<T*>(a.v_tail) + bh * BETA * a.d;
   const T* vn = static_cast<const T*>(a.v_new) + bh * static_cast<int64_t>(a.T) * a.d;
-  float val[BETA];
-#pragma unroll
-  for (int i = 0; i < BETA; ++i) {
-    const int tok = tok0 + i;
-    float x = 0.0f;
-    if (tok < a.pos) x = to_f32(tail[(tok - a.g0 * BETA) * a.d + c]);          // only in block g0
-    else if (tok < a.pos + a.T) x = to_f32(vn[static_cast<int64_t>(tok - a.pos) * a.d + c]);
-    val[i] = x;
-  }
-  uint32_t packed[BETA / 8];
-  const uint32_t sc = append_quant_block<FMT, BETA>(val, packed);
-  uint32_t* dst = reinterpret_cast<uint32_t*>(a.vc + (bh * a.d + c) * static_cast<int64_t>(a.Np / 2) + tok0 / 2);
-#pragma unroll
-  for (int w = 0; w < BETA / 8; ++w) dst[w] = packed[w];
   const int nkc = a.Np / (4 * BETA);
-  a.vs[bh * a.sf_v_head + sf_word_offset(c, g / 4, nkc) + (g % 4)] = static_cast<uint8_t>(sc);
-}
-
-// v_tail <- raw V of the new partially filled block (its tokens from v_new;
-// tokens before pos in the same block are already in place).
-template <typename T>
-__global__ void __launch_bounds__(256) kv_append_tail_kernel(const AppendArgs a, int beta) {
+  for (int gi = 0; gi < a.nblk; ++gi) {
+    const int g = a.g0 + gi;
+    const int tok0 = g * BETA;
+    float val[BETA];
+#pragma unroll
+    for (int i = 0; i < BETA; ++i) {
+      const int tok = tok0 + i;
+      float x = 0.0f;
+      if (tok < a.pos) x = to_f32(tail[(tok - a.g0 * BETA) * a.d + c]);          // only in block g0
+      else if (tok < a.pos + a.T) x = to_f32(vn[static_cast<int64_t>(tok - a.pos) * a.d + c]);
+      val[i] = x;
+    }
+    uint32_t packed[BETA / 8];
+    const uint32_t sc = append_quant_block<FMT, BETA>(val, packed);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(a.vc + (bh * a.d + c) * static_cast<int64_t>(a.Np / 2) + tok0 / 2);
+#pragma unroll
+    for (int w = 0; w < BETA / 8; ++w) dst[w] = packed[w];
+    a.vs[bh * a.sf_v_head + sf_word_offset(c, g / 4, nkc) + (g % 4)] = static_cast<uint8_t>(sc);
+  }
+  // tail <- raw V of the new partially filled block (tokens before pos in
+  // the same block are already in place)
   const int end = a.pos + a.T;
-  const int start = end / beta * beta;
-  const int first = start > a.pos ? start : a.pos;     // first new token of the block
-  const int n = end - first;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * n * a.d;
-  if (n <= 0 || idx >= total) return;
-  const int c = static_cast<int>(idx % a.d);
-  const int i = static_cast<int>((idx / a.d) % n);
-  const int64_t bh = idx / (static_cast<int64_t>(a.d) * n);
-  const int tok = first + i;
-  const T* vn = static_cast<const T*>(a.v_new) + bh * static_cast<int64_t>(a.T) * a.d;
-  T* tail = static_cast<T*>(a.v_tail) + bh * beta * a.d;
-  tail[(tok - start) * a.d + c] = vn[static_cast<int64_t>(tok - a.pos) * a.d + c];
+  const int start = end / BETA * BETA;
+  for (int tok = start > a.pos ? start : a.pos; tok < end; ++tok)
+    tail[(tok - start) * a.d + c] = vn[static_cast<int64_t>(tok - a.pos) * a.d + c];
 }
 
 template <int FMT, typename T>
 static hifa4_status append_t(const AppendArgs& a, cudaStream_t st) {
   constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
-  const int64_t nk = static_cast<int64_t>(a.B) * a.Hkv * a.T * (a.d / BETA);
-  const int64_t nv = static_cast<int64_t>(a.B) * a.Hkv * a.nblk * a.d;
-  const int64_t nt = static_cast<int64_t>(a.B) * a.Hkv * BETA * a.d;
-  kv_append_k_kernel<FMT, T><<<static_cast<unsigned>((nk + 255) / 256), 256, 0, st>>>(a);
-  kv_append_v_kernel<FMT, T><<<static_cast<unsigned>((nv + 255) / 256), 256, 0, st>>>(a);
-  kv_append_tail_kernel<T><<<static_cast<unsigned>((nt + 255) / 256), 256, 0, st>>>(a, BETA);
+  const int64_t n = static_cast<int64_t>(a.B) * a.Hkv * a.T * (a.d / BETA) + static_cast<int64_t>(a.B) * a.Hkv * a.d;
+  kv_append_kernel<FMT, T><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(a);
   return launch_status("kv_cache_append");
 }
 

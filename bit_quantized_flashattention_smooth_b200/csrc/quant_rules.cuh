@@ -14,7 +14,21 @@
 #include "common.cuh"
 #include "ptx.cuh"
 
+// 1: element multiplies as packed fp32 pairs (FMUL2); 0: scalar multiplies.
+// Both round each product to nearest: the results are identical.
+#ifndef HIFA4_QUANT_PACKED_MUL
+#define HIFA4_QUANT_PACKED_MUL 1
+#endif
+
 namespace hifa4 {
+
+__device__ __forceinline__ float2 qmul2(float2 a, float2 b) {
+#if HIFA4_QUANT_PACKED_MUL
+  return fmul2(a, b);
+#else
+  return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
+#endif
+}
 
 template <typename T>
 __device__ __forceinline__ void load8(const T* p, float (&f)[8]);
@@ -70,8 +84,8 @@ __device__ __forceinline__ uint32_t quant_block(const float (&v)[BETA], uint32_t
 #pragma unroll
   for (int w = 0; w < BETA / 8; ++w) {
     const float* e = v + 8 * w;
-    packed[w] = keep & cvt_e2m1x8(fmul2(make_float2(e[0], e[1]), m2), fmul2(make_float2(e[2], e[3]), m2),
-                                  fmul2(make_float2(e[4], e[5]), m2), fmul2(make_float2(e[6], e[7]), m2));
+    packed[w] = keep & cvt_e2m1x8(qmul2(make_float2(e[0], e[1]), m2), qmul2(make_float2(e[2], e[3]), m2),
+                                  qmul2(make_float2(e[4], e[5]), m2), qmul2(make_float2(e[6], e[7]), m2));
   }
   return sc;
 }

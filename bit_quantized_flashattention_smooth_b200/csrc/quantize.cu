@@ -65,8 +65,8 @@ __device__ __forceinline__ uint32_t quant_part(const float (&v)[8], uint32_t& pa
     mult = __uint_as_float((254u - sc) << 23);
   }
   const float2 m2 = make_float2(mult, mult);
-  packed = keep & cvt_e2m1x8(fmul2(make_float2(v[0], v[1]), m2), fmul2(make_float2(v[2], v[3]), m2),
-                             fmul2(make_float2(v[4], v[5]), m2), fmul2(make_float2(v[6], v[7]), m2));
+  packed = keep & cvt_e2m1x8(qmul2(make_float2(v[0], v[1]), m2), qmul2(make_float2(v[2], v[3]), m2),
+                             qmul2(make_float2(v[4], v[5]), m2), qmul2(make_float2(v[6], v[7]), m2));
   return sc;
 }
 
@@ -115,7 +115,7 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
     if (scale != nullptr && t < N) {
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
-        const float2 p2 = fmul2(make_float2(v[u][i], v[u][i + 1]), make_float2(sv[i], sv[i + 1]));
+        const float2 p2 = qmul2(make_float2(v[u][i], v[u][i + 1]), make_float2(sv[i], sv[i + 1]));
         v[u][i] = p2.x;
         v[u][i + 1] = p2.y;
       }

@@ -247,8 +247,8 @@ HIFA4_API hifa4_status hifa4_attn_decode(const void* q, hifa4_dtype q_dt, const 
  * (older tokens of the block from v_tail, tokens not yet written as 0); v_tail
  * is updated.  After appends covering [0, L), the cache equals
  * hifa4_quantize_kv of the L tokens laid out at this capacity, bit for bit.
- * Requires 0 <= pos, T >= 1, pos + T <= capacity, d in {64, 128, 256}.  Three
- * kernel launches on `stream`; no host synchronization. */
+ * Requires 0 <= pos, T >= 1, pos + T <= capacity, d in {64, 128, 256}.  One
+ * kernel launch on `stream`; no host synchronization. */
 HIFA4_API hifa4_status hifa4_kv_cache_append(const void* k_new, const void* v_new, hifa4_dtype dt, int B, int Hkv,
                                              int T, int d, const float* inv_s, hifa4_format fmt, int pos,
                                              int capacity, uint8_t* k_codes, uint8_t* k_scales, uint8_t* vt_codes,
