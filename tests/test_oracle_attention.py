@@ -349,3 +349,26 @@ def test_lazy_decode_split_combine_exact_when_quant_off(splits):
         sc = qd[b, hq, 0] @ deq["k"][b, h, :N].T * 0.5
         p = np.exp(sc - sc.max())
         np.testing.assert_allclose(res["O"][b, hq], p @ vd[b, h, :N] / p.sum(), rtol=1e-12, atol=1e-13)
+
+
+def test_lazy_rescale_threshold_is_strict_and_fp32():
+    """The rule on crafted scores: with NVFP4-exact Q and K (a single 6 in
+    each Q row, a single 3 or 6 in a key row) and c = 1, tile 0's max is 18
+    and tile 1's is 36.  tau = 18 keeps the max (36 > fl32(18 + 18) is
+    false: the comparison is strict); tau = 17.9995 moves it (fl32(18 +
+    17.9995) < 36); tau = 0 moves it."""
+    N, d, BN = 32, 16, 16
+    q = np.zeros((1, 1, N, d), np.float32)
+    q[..., 0] = 6.0
+    k = np.zeros((1, 1, N, d), np.float32)
+    k[0, 0, 0, 0] = 3.0          # tile 0: score 18
+    k[0, 0, 16, 0] = 6.0         # tile 1: score 36
+    v = np.random.default_rng(3).standard_normal((1, 1, N, d)).astype(np.float32)
+    qz = oracle.quantize_qkv(q, k, v, None, None, oracle.NVFP4)
+    deq = _dequant_all(qz, oracle.NVFP4)
+    assert deq["q"][0, 0, 0, 0] == 6.0 and deq["k"][0, 0, 0, 0] == 3.0 and deq["k"][0, 0, 16, 0] == 6.0
+    scale = 1.0 / 1.4426950408889634          # c = scale * log2(e) = 1 up to fp64 rounding
+    for tau, moved in ((18.0, False), (17.9995, True), (0.0, True)):
+        res = oracle.attention(qz, N, oracle.NVFP4, scale, False, oracle.PREORDER, BN, dump_phat=True, tau=tau)
+        m = res["m_tiles"][0, 0, 5]
+        assert m[0] == 18.0 and m[1] == (36.0 if moved else 18.0), (tau, m)
