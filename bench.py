@@ -166,11 +166,13 @@ def run_prefill(args, rank, world):
         else:
             h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)
 
+    tau = args.rescale_threshold
+
     def attn_launch():
         if fused:
-            h.attn_fwd_fused(qd, s, kvz, scale, w.causal, mode, w.block_n, out=o)
+            h.attn_fwd_fused(qd, s, kvz, scale, w.causal, mode, w.block_n, out=o, rescale_threshold=tau)
         else:
-            h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o)
+            h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o, rescale_threshold=tau)
 
     def step():
         quant_launch()
@@ -566,6 +568,8 @@ def main():
     ap.add_argument("--workload", default="qwen3_prefill")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--mode", default="preorder", choices=["preorder", "inconsistent"])
+    ap.add_argument("--rescale-threshold", type=float, default=0.0,
+                    help="lazy running-max threshold tau (0 = the exact online recurrence)")
     ap.add_argument("--path", default="two-launch", choices=["fused", "two-launch"],
                     help="fused: K/V quantize + attention with Smooth-QK and Q quantization in the kernel; "
                          "two-launch: Q/K/V quantize + attention")
@@ -584,6 +588,7 @@ def main():
     w = W.WORKLOADS[args.workload]
     config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
               "format": args.fmt, "normalizer": args.mode, "block_n": w.block_n, "path": args.path,
+              "rescale_threshold": args.rescale_threshold,
               "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)", "parallelism": f"replicas x{world}"}
 
     if args.profile:
