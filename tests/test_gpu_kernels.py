@@ -57,6 +57,31 @@ def test_hw_conversions_match_written_rounding():
     assert bad.size == 0, f"E4M3: {bad.size} mismatches e.g. x={x[bad[:8]]} gpu={e4_gpu[bad[:8]]} ref={e4_ref[bad[:8]]}"
 
 
+def test_hw_conversions_exhaustive():
+    """Every finite fp32 bit pattern, in 16 chunks of 2^28: the E2M1
+    conversion the kernels use equals the oracle's written encoder, and the
+    UE4M3 scale conversion equals it on every non-negative finite value (NaN
+    and infinities are outside the encoders' domain)."""
+    chunk = 1 << 28
+    for start in range(0, 1 << 32, chunk):
+        s0 = start if start < (1 << 31) else start - (1 << 32)     # the same bits as int32
+        x = torch.arange(s0, s0 + chunk, dtype=torch.int32, device="cuda").view(torch.float32)
+        e2_gpu, e4_gpu = h.convert_probe(x)
+        e2_gpu = e2_gpu.cpu().numpy()
+        e4_gpu = e4_gpu.cpu().numpy()
+        del x
+        xn = np.arange(start, start + chunk, dtype=np.uint64).astype(np.uint32).view(np.float32)
+        e2_ref, e4_ref = oracle.encode_array(xn)
+        fin = np.isfinite(xn)
+        bad = np.nonzero((e2_gpu != e2_ref) & fin)[0]
+        assert bad.size == 0, (f"E2M1: {bad.size} mismatches in chunk {start:#x}, e.g. bits "
+                               f"{xn[bad[:4]].view(np.uint32)} gpu={e2_gpu[bad[:4]]} ref={e2_ref[bad[:4]]}")
+        pos = fin & ~np.signbit(xn)
+        bad = np.nonzero((e4_gpu != e4_ref) & pos)[0]
+        assert bad.size == 0, (f"UE4M3: {bad.size} mismatches in chunk {start:#x}, e.g. bits "
+                               f"{xn[bad[:4]].view(np.uint32)} gpu={e4_gpu[bad[:4]]} ref={e4_ref[bad[:4]]}")
+
+
 def test_fast_div6_is_ieee_division():
     """The P-hat scale path computes fl32(amax/6) without a division; it must
     equal IEEE division for zero and every float in [2^-122, 2^20] (quotients
