@@ -372,3 +372,16 @@ def test_lazy_rescale_threshold_is_strict_and_fp32():
         res = oracle.attention(qz, N, oracle.NVFP4, scale, False, oracle.PREORDER, BN, dump_phat=True, tau=tau)
         m = res["m_tiles"][0, 0, 5]
         assert m[0] == 18.0 and m[1] == (36.0 if moved else 18.0), (tau, m)
+
+
+def test_lazy_decode_single_split_equals_last_causal_row():
+    """With one split, decode under the lazy rule is the last causal prefill
+    row under the same rule, exactly (the rule is per row and per tile)."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 200, 64
+    q, k, v = _inputs(B, Hq, Hkv, N, d, 61)
+    s, inv = oracle.calibrate(q, k, n_cal=32)
+    qz = oracle.quantize_qkv(q, k, v, s, inv, oracle.NVFP4)
+    for tau in (1.0, 3.0):
+        pre = oracle.attention(qz, N, oracle.NVFP4, 0.5, True, oracle.PREORDER, 64, rows=(N - 1, N), tau=tau)
+        dec = oracle.decode(q[:, :, N - 1], s, qz, N, oracle.NVFP4, 0.5, oracle.PREORDER, 64, num_splits=1, tau=tau)
+        np.testing.assert_array_equal(dec["O"], pre["O"][:, :, N - 1])
