@@ -20,7 +20,10 @@
  *
  * The pages never define HIF4, the Smooth-QK scale formula, the P-hat scale,
  * or epsilon; the reading taken for each is stated in the comment of the
- * function that implements it.
+ * function that implements it.  Attention and decode also take an optional
+ * lazy running-max threshold tau (the conditional rescaling of
+ * FlashAttention-4, which the pages do not describe); tau = 0 is the pages'
+ * exact online recurrence.
  *
  * Arithmetic: everything that is not a 4-bit/8-bit format decision is done in
  * double precision.  Format decisions (block amax, scale, element rounding)
