@@ -48,11 +48,15 @@ class Barrier:
 
 
 class Sim:
-    def __init__(self, nkt, NS, NSB, NH, rng):
+    def __init__(self, nkt, NS, NSB, NH, rng, fused_q=False):
         self.nkt, self.NS, self.NSB, self.NH, self.rng = nkt, NS, NSB, NH, rng
         self.W = 4 * NH
+        self.fused_q = fused_q
         B = Barrier
-        self.bars = {"QFULL": B("QFULL", 1), "XM": B("XM", 8)}
+        # the Q tile comes from one tensor copy, or (fused path) from every
+        # softmax warp quantizing its rows, one arrival each
+        self.bars = {"QFULL": B("QFULL", self.W if fused_q else 1), "XM": B("XM", 8)}
+        self.q_rows_written = set()
         for s in range(NS):
             for n in ("KFULL", "KEMPTY", "VFULL", "VEMPTY"):
                 self.bars[f"{n}{s}"] = B(f"{n}{s}", 1)
@@ -95,6 +99,8 @@ class Sim:
 
     def mma(self):
         yield from self.wait("QFULL", 0, 1)
+        if self.fused_q and len(self.q_rows_written) != self.W:
+            raise ProtocolError(f"QK^T issued with Q-hat rows of {sorted(self.q_rows_written)} written")
 
         def issue_s(j):
             st, sb = j % self.NS, j % self.NSB
@@ -116,6 +122,11 @@ class Sim:
             yield from issue_pv(j)
 
     def softmax(self, w):
+        if self.fused_q:
+            # quantize this warp's share of the Q tile, then arrive
+            yield "work"
+            self.q_rows_written.add(w)
+            self.bars["QFULL"].arrive()
         for j in range(self.nkt):
             sb, pb = j % self.NSB, j & 1
             yield from self.wait(f"SFULL{sb}", (j // self.NSB) & 1, j // self.NSB + 1)
@@ -192,7 +203,8 @@ class Sim:
         return True
 
     def run(self):
-        self.bars["QFULL"].arrive()        # the Q tile (its copy lands before anything else matters)
+        if not self.fused_q:
+            self.bars["QFULL"].arrive()    # the Q tile (its copy lands before anything else matters)
         live = [self.tma(), self.mma()] + [self.softmax(w) for w in range(self.W)]
         idle = 0
         while live or self.mma_queue or self.copies:
@@ -221,6 +233,29 @@ class Sim:
 def test_prefill_protocol_random_schedules(NH, NS, NSB, nkt):
     for seed in range(40):
         Sim(nkt, NS, NSB, NH, random.Random(1000 * nkt + seed)).run()
+
+
+@pytest.mark.parametrize("NH,NS,NSB", [(1, 3, 1), (2, 3, 2), (2, 2, 2)])
+@pytest.mark.parametrize("nkt", [1, 2, 5])
+def test_fused_q_protocol_random_schedules(NH, NS, NSB, nkt):
+    """The fused path: the softmax warps write Q-hat before their first wait;
+    QK^T must not start before every warp's rows are written."""
+    for seed in range(40):
+        Sim(nkt, NS, NSB, NH, random.Random(7000 * nkt + seed), fused_q=True).run()
+
+
+def test_model_catches_a_short_q_barrier():
+    """A Q barrier that completes after one arrival lets QK^T start before
+    the other warps have written their rows: the model must flag it."""
+    caught = 0
+    for seed in range(100):
+        sim = Sim(3, 3, 1, 1, random.Random(seed), fused_q=True)
+        sim.bars["QFULL"] = Barrier("QFULL", 1)
+        try:
+            sim.run()
+        except ProtocolError:
+            caught += 1
+    assert caught > 0
 
 
 def test_model_catches_a_one_lap_early_epilogue():
