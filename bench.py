@@ -582,7 +582,8 @@ def main():
                     help="run only this kernel a few times (for an ncu capture) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
-    rank, world, local = dist_setup(args.gpus)
+    # the reference arm is the CPU oracle: its ranks need no GPU (gloo plumbing)
+    rank, world, local = dist_setup(args.gpus, "gloo" if args.impl == "reference" else "nccl")
     if args.block_n:
         W.WORKLOADS[args.workload] = W.Workload(**{**W.WORKLOADS[args.workload].__dict__, "block_n": args.block_n})
     w = W.WORKLOADS[args.workload]
