@@ -140,103 +140,191 @@ def rank_seed(seed: int, rank: int) -> int:
 
 
 # ------------------------------------------------------------ our arm -----
-def run_prefill(args, rank, world):
+class PrefillSetup:
+    """Device-resident inputs of one prefill workload (this rank's batch):
+    raw Q, K, V, the Smooth-QK scales (offline, untimed) and the quantized
+    buffers the timed step writes."""
+
+    def __init__(self, w, fmt, rank=0, alpha=0.5, inputs=None):
+        import bit_quantized_flashattention_smooth_b200 as h
+        self.w, self.fmt = w, fmt
+        wr = W.Workload(**{**w.__dict__, "seed": rank_seed(w.seed, rank)})   # each rank its own batch
+        self.host = inputs if inputs is not None else W.make_prefill(wr)
+        dev = torch.device("cuda")
+        self.qd, self.kd, self.vd = (t.to(dev) for t in self.host)
+        self.s, self.inv = h.calibrate_smooth_qk(self.qd[:, :, : w.n_cal], self.kd[:, :, : w.n_cal], w.n_cal,
+                                                 alpha=alpha)
+        self.z = h.alloc_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, fmt, dev)
+        self.o = torch.empty((w.B, w.Hq, w.N, w.d), device=dev, dtype=W.torch_dtype(w.dtype))
+        self.scale = 1.0 / math.sqrt(w.d)
+
+    def quantize(self):
+        import bit_quantized_flashattention_smooth_b200 as h
+        h.quantize_qkv(self.qd, self.kd, self.vd, self.s, self.inv, self.fmt, out=self.z)
+
+    def attention(self, mode, tau=0.0):
+        import bit_quantized_flashattention_smooth_b200 as h
+        h.attn_fwd(self.z, self.scale, self.w.causal, mode, self.w.block_n, out=self.o, rescale_threshold=tau)
+
+
+def time_step(setup, mode, steps, warmup, tau=0.0, world=1, clocks=False):
+    """One step = the quantize launch, then the attention launch; L2 flushed
+    between timed steps (outside the step's events).  Returns per-step device
+    ms of the step, the attention and the quantize (means over `steps`)."""
     import bit_quantized_flashattention_smooth_b200 as h
-    w = W.WORKLOADS[args.workload]
-    fmt = h.NVFP4 if args.fmt == "nvfp4" else h.MXFP4
-    mode = h.PREORDER if args.mode == "preorder" else h.INCONSISTENT
-    wr = W.Workload(**{**w.__dict__, "seed": rank_seed(w.seed, rank)})   # each rank its own batch
-    q, k, v = W.make_prefill(wr)
-    dev = torch.device("cuda")
-    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    s, inv = h.calibrate_smooth_qk(qd[:, :, : w.n_cal], kd[:, :, : w.n_cal], w.n_cal)   # offline, untimed
-    z = h.alloc_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, fmt, dev)
-    kvz = h.alloc_kv_cache(w.B, w.Hq, w.Hkv, w.N, w.d, fmt, dev)
-    o = torch.empty((w.B, w.Hq, w.N, w.d), device=dev, dtype=W.torch_dtype(w.dtype))
-    flush = L2Flush(dev)
-    scale = 1.0 / math.sqrt(w.d)
-    fused = args.path == "fused"
-
-    # one step = the quantization launch, then the attention launch.  fused:
-    # K, V quantized (hifa4_quantize_kv), Smooth-QK and Q quantization inside
-    # the attention kernel; two-launch: Q, K, V quantized, then attention.
-    def quant_launch():
-        if fused:
-            h.quantize_kv(kd, vd, inv, fmt, Hq=w.Hq, out=kvz)
-        else:
-            h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)
-
-    tau = args.rescale_threshold
-
-    def attn_launch():
-        if fused:
-            h.attn_fwd_fused(qd, s, kvz, scale, w.causal, mode, w.block_n, out=o, rescale_threshold=tau)
-        else:
-            h.attn_fwd(z, scale, w.causal, mode, w.block_n, out=o, rescale_threshold=tau)
-
-    def step():
-        quant_launch()
-        attn_launch()
-
-    for _ in range(args.warmup):
+    flush = L2Flush()
+    for _ in range(warmup):
         flush()
-        step()
+        setup.quantize()
+        setup.attention(mode, tau)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    clocks = ClockSampler(torch.cuda.current_device())
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
     barrier(world)
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    for i in range(args.steps):
-        flush()                             # L2 flush between timed steps (outside the step events)
+    for i in range(steps):
+        flush()
         e0, e1, e2 = ev[i]
         e0.record(stream)
-        quant_launch()
+        setup.quantize()
         e1.record(stream)
-        attn_launch()
+        setup.attention(mode, tau)
         e2.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     wall = time.perf_counter() - t_wall
-    clk = clocks.stop() if clocks else None
-    step_ms = sum(a.elapsed_time(c) for a, b, c in ev) / args.steps
-    attn_ms = sum(b.elapsed_time(c) for a, b, c in ev) / args.steps
-    quant_ms = sum(a.elapsed_time(b) for a, b, c in ev) / args.steps
+    clk = sampler.stop() if sampler else None
     dev_err = h.device_error()
     if dev_err:
         raise RuntimeError(f"device error word {dev_err:#x}")
-    step_ms_max = allmax(step_ms, world)
-    attn_ms_max = allmax(attn_ms, world)
+    return dict(step_ms=sum(a.elapsed_time(c) for a, b, c in ev) / steps,
+                attn_ms=sum(b.elapsed_time(c) for a, b, c in ev) / steps,
+                quant_ms=sum(a.elapsed_time(b) for a, b, c in ev) / steps, clocks=clk, wall=wall)
+
+
+def run_prefill(args, rank, world):
+    """The headline: the workload's step timed over args.steps, then the same
+    step end to end through the C ABI with host buffers."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    w = W.WORKLOADS[args.workload]
+    fmt = h.NVFP4 if args.fmt == "nvfp4" else h.MXFP4
+    mode = h.PREORDER if args.mode == "preorder" else h.INCONSISTENT
+    st = PrefillSetup(w, fmt, rank)
+    t = time_step(st, mode, args.steps, args.warmup, args.rescale_threshold, world, clocks=True)
+    step_ms_max = allmax(t["step_ms"], world)
+    attn_ms_max = allmax(t["attn_ms"], world)
     flops = W.prefill_flops(w)
 
     # ---- end to end through the C ABI with host buffers (pinned) ----
-    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    n_e2e = max(3, min(args.steps, 200))
+    qh, kh, vh = (x.pin_memory() for x in st.host)
+    oh = torch.empty(st.o.shape, dtype=st.o.dtype).pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def e2e_step():
+        st.qd.copy_(qh, non_blocking=True); st.kd.copy_(kh, non_blocking=True); st.vd.copy_(vh, non_blocking=True)
+        st.quantize()
+        st.attention(mode, args.rescale_threshold)
+        oh.copy_(st.o, non_blocking=True)
+
+    n_e2e = max(3, min(args.steps, args.e2e_steps))
     for _ in range(3):
-        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
-        step()
-        oh.copy_(o, non_blocking=True)
+        e2e_step()
     torch.cuda.synchronize()
     barrier(world)
     e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_s.record(stream)
     for _ in range(n_e2e):
-        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
-        step()
-        oh.copy_(o, non_blocking=True)
+        e2e_step()
     e_e.record(stream)
     torch.cuda.synchronize()
     e2e_ms = allmax(e_s.elapsed_time(e_e) / n_e2e, world)
-    h2d = (q.numel() + k.numel() + v.numel()) * q.element_size()
-    d2h = o.numel() * o.element_size()
-    h.quantize_qkv(qd, kd, vd, s, inv, fmt, out=z)      # the comparisons read Q-hat, K-hat, V-hat (untimed)
+    h2d = sum(x.numel() * x.element_size() for x in st.host)
+    d2h = st.o.numel() * st.o.element_size()
+    st.quantize()      # the comparisons read Q-hat, K-hat, V-hat (untimed)
+    return dict(w=w, fmt=fmt, mode=mode, step_ms=step_ms_max, attn_ms=attn_ms_max, quant_ms=t["quant_ms"],
+                flops=flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=t["clocks"], wall=t["wall"],
+                launches=2 * args.steps, setup=st, n_e2e=n_e2e)
 
-    return dict(w=w, fmt=fmt, mode=mode, step_ms=step_ms_max, attn_ms=attn_ms_max, quant_ms=quant_ms,
-                flops=flops, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clk, wall=wall,
-                launches=2 * args.steps, qd=qd, kd=kd, vd=vd, z=z, o=o, s=s, inv=inv)
+
+def _phat_grid(device):
+    return torch.tensor([0, .5, 1, 1.5, 2, 3, 4, 6], dtype=torch.float64, device=device)
+
+
+def tile_epsilon_gpu(setup, mode):
+    """Per-tile normalizer error of the kernel (the pages measure it per
+    attention tile): sum(P-hat) / sum(P) - 1 over the 128 rows x BN keys of
+    every visited tile, from the kernel's own P-hat dump and sums of P.
+    Also returns the per-row error l_P-hat / l_P - 1."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    w, z = setup.w, setup.z
+    _, dump = h.attn_fwd_dump(z, setup.scale, w.causal, mode, w.block_n, sum_p=True)
+    beta = h.beta_of(z.fmt)
+    dev = dump.codes.device
+    grid = _phat_grid(dev)
+    if z.fmt == h.NVFP4:
+        e = torch.arange(128, device=dev)
+        ex, mant = (e >> 3) & 15, (e & 7).double()
+        ue4m3 = torch.where(ex == 0, mant * 2.0 ** -9, (1 + mant / 8) * torch.pow(2.0, ex.double() - 7))
+        sd_tab = (ue4m3 * 2.0 ** h.P_PRESCALE_LOG2).float().double()
+        sd = sd_tab[dump.scales.long().clamp(max=127)]
+    else:
+        sd = torch.pow(2.0, dump.scales.double() - 127)
+    sph = torch.zeros(dump.m.shape, dtype=torch.float64, device=dev)
+    for half in (0, 1):                                  # low / high nibbles: even / odd keys
+        c = (dump.codes >> (4 * half)) & 15
+        vals = grid[(c & 7).long()]                      # [B,H,N,nkt,BN/2], key 2i+half
+        idx = torch.arange(half, w.block_n, 2, device=dev) // beta
+        sph += (vals * sd[..., idx]).sum(-1)
+    visited = torch.isfinite(dump.m)
+    sp = dump.sum_p.double()
+    B, H, N, nkt = sp.shape
+    nq = (N + 127) // 128
+    pad = nq * 128 - N
+    num = torch.nn.functional.pad(torch.where(visited, sph, 0.0), (0, 0, 0, pad)).view(B, H, nq, 128, nkt).sum(3)
+    den = torch.nn.functional.pad(torch.where(visited, sp, 0.0), (0, 0, 0, pad)).view(B, H, nq, 128, nkt).sum(3)
+    eps = (num / den - 1.0)[den > 0]
+    return dict(tiles=int(eps.numel()), median=float(eps.median()), frac_negative=float((eps < 0).double().mean()),
+                p10=float(eps.quantile(0.1)) if eps.numel() < (1 << 24) else None,
+                p90=float(eps.quantile(0.9)) if eps.numel() < (1 << 24) else None)
+
+
+def measure_config(name, fmt_name, mode_name, steps, warmup, alpha=0.5, want_eps=False):
+    """One config of the path timed alone (quantize + attention, L2 flushed),
+    with its throughput against the FP4 peak and the softmax ceiling."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    w = W.WORKLOADS[name]
+    fmt = h.NVFP4 if fmt_name == "nvfp4" else h.MXFP4
+    mode = h.PREORDER if mode_name == "preorder" else h.INCONSISTENT
+    st = PrefillSetup(w, fmt, alpha=alpha)
+    t = time_step(st, mode, steps, warmup)
+    flops = W.prefill_flops(w)
+    rec = {"workload": name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+           "format": fmt_name, "normalizer": mode_name, "alpha": alpha, "block_n": w.block_n, "steps": steps,
+           "step_ms": t["step_ms"], "attn_ms": t["attn_ms"], "quantize_ms": t["quant_ms"],
+           "step_tflops": flops / (t["step_ms"] * 1e-3) / 1e12, "attn_tflops": flops / (t["attn_ms"] * 1e-3) / 1e12,
+           "tokens_per_s": w.B * w.N / (t["step_ms"] * 1e-3)}
+    if want_eps:
+        rec["epsilon_tile"] = tile_epsilon_gpu(st, mode)
+        o, lph, lp = h.attn_fwd(st.z, st.scale, w.causal, mode, w.block_n, out_dtype=W.torch_dtype(w.dtype),
+                                debug=True)
+        e = (lph / lp - 1.0).flatten()
+        rec["epsilon_row"] = {"median": float(e.median()), "frac_negative": float((e < 0).float().mean())}
+    return rec, st
+
+
+def deviation_by_rows(o4, ex, N):
+    """Deviation of the 4-bit output from exact attention on the first,
+    middle and last 128-row query tile and overall."""
+    out = {}
+    for label, (r0, r1) in (("first_tile", (0, min(128, N))), ("middle_tile", (N // 2, min(N, N // 2 + 128))),
+                            ("last_tile", (max(0, N - 128), N)), ("all", (0, N))):
+        a, b = o4[:, r0:r1].float(), ex[:, r0:r1]
+        out[label] = {"rows": [r0, r1], "max_abs_rel": float((a - b).abs().max() / b.abs().max()),
+                      "cosine": float(torch.nn.functional.cosine_similarity(a.flatten(), b.flatten(), dim=0))}
+    return out
 
 
 class L2Flush:
@@ -288,64 +376,70 @@ def exact_attention_rows(q, k, v, causal, scale, heads):
 
 
 def comparisons(res):
-    """Outside the timed region: the in-house BF16 kernel and the cuDNN BF16
-    attention on the same (unsmoothed, unquantized) inputs, the deviation of
-    the 4-bit output from exact attention, and the normalizer error eps of
-    both modes (Theorem 1)."""
+    """Outside the timed region, on the headline workload: the in-house BF16
+    kernel and the cuDNN BF16 attention on the same (unsmoothed,
+    unquantized) inputs, the deviation of the 4-bit output from exact
+    attention by query-tile range, the normalizer error of both modes per row
+    and per tile (Theorem 1), lazy rescaling and the Smooth-QK sweep."""
     import bit_quantized_flashattention_smooth_b200 as h
-    w, z = res["w"], res["z"]
-    qd, kd, vd = res["qd"], res["kd"], res["vd"]
-    scale = 1.0 / math.sqrt(w.d)
-    out = {}
+    st = res["setup"]
+    w, z = st.w, st.z
+    qd, kd, vd = st.qd, st.kd, st.vd
+    scale = st.scale
+    out = {"workload": w.name}
     qb, kb, vb = qd.to(torch.bfloat16), kd.to(torch.bfloat16), vd.to(torch.bfloat16)
     attn_ms = res["attn_ms"]
+    ob = None
     if w.d in (64, 128, 256) and w.N % 8 == 0:
         vt = h.bf16_transpose_v(vb)
         ob = h.bf16_attn_fwd(qb, kb, vt, scale, w.causal)
-        ms = time_ms(lambda: h.bf16_attn_fwd(qb, kb, vt, scale, w.causal, out=ob))
+        ms = time_ms(lambda: h.bf16_attn_fwd(qb, kb, vt, scale, w.causal, out=ob), n=10)
         out["bf16_inhouse"] = {"ms": ms, "tflops": res["flops"] / (ms * 1e-3) / 1e12,
                                "fp4_speedup": ms / attn_ms, "kernel": "attn_fwd_bf16 (tcgen05 kind::f16)"}
+        del vt
     try:
         import torch.nn.functional as F
         from torch.nn.attention import SDPBackend, sdpa_kernel
         G = w.Hq // w.Hkv
         kk, vv = kb.repeat_interleave(G, dim=1), vb.repeat_interleave(G, dim=1)
         with sdpa_kernel(SDPBackend.CUDNN_ATTENTION):
-            ms = time_ms(lambda: F.scaled_dot_product_attention(qb, kk, vv, is_causal=w.causal, scale=scale))
+            ms = time_ms(lambda: F.scaled_dot_product_attention(qb, kk, vv, is_causal=w.causal, scale=scale), n=10)
         out["bf16_cudnn_sdpa"] = {"ms": ms, "tflops": res["flops"] / (ms * 1e-3) / 1e12,
                                   "fp4_speedup": ms / attn_ms, "note": "library kernel, context only"}
         del kk, vv
     except Exception as e:  # context only
         out["bf16_cudnn_sdpa"] = {"error": str(e)[:120]}
-    # deviation from exact attention (4 heads of batch 0)
+    # deviation from exact attention (4 heads of batch 0), by query-tile range
     heads = list(range(min(4, w.Hq)))
     ex = exact_attention_rows(qd, kd, vd, w.causal, scale, heads)
-    o4 = res["o"][0, heads].float()
-    out["deviation_from_exact"] = {"heads": heads, "max_abs_rel": float((o4 - ex).abs().max() / ex.abs().max()),
-                                   "cosine": float(torch.nn.functional.cosine_similarity(o4.flatten(), ex.flatten(), dim=0))}
-    if "bf16_inhouse" in out:
-        obf = ob[0, heads].float()
-        out["deviation_from_exact"]["bf16_inhouse_max_abs_rel"] = float((obf - ex).abs().max() / ex.abs().max())
-    # normalizer error: eps_row = l_Phat / l_P - 1; under P-Reordering the
-    # output divides by l_Phat itself, under the inconsistent mode by l_P, so
-    # O_incons / O_preorder - 1 equals eps row by row (coherent scaling)
-    o_pre, lph, lp = h.attn_fwd(z, scale, w.causal, h.PREORDER, w.block_n, out_dtype=torch.float16 if w.dtype == "fp16" else torch.bfloat16, debug=True)
-    o_inc = h.attn_fwd(z, scale, w.causal, h.INCONSISTENT, w.block_n, out_dtype=o_pre.dtype)
+    dev = {"heads": heads, "fp4": deviation_by_rows(st.o[0, heads], ex, w.N)}
+    if ob is not None:
+        dev["bf16_inhouse"] = deviation_by_rows(ob[0, heads], ex, w.N)
+    out["deviation_from_exact"] = dev
+    # normalizer error: eps_row = l_Phat / l_P - 1 per row; per tile, sum(P-hat)
+    # / sum(P) - 1 over each 128-row x BN tile (the pages' unit of measurement)
+    odt = W.torch_dtype(w.dtype)
+    o_pre, lph, lp = h.attn_fwd(z, scale, w.causal, h.PREORDER, w.block_n, out_dtype=odt, debug=True)
+    o_inc = h.attn_fwd(z, scale, w.causal, h.INCONSISTENT, w.block_n, out_dtype=odt)
     eps = (lph / lp - 1.0).flatten()
     a, b = o_inc[0, heads].float().flatten(1), o_pre[0, heads].float().flatten(1)
     scale_err = ((a * b).sum(1) / (b * b).sum(1) - 1.0)
-    out["epsilon"] = {"median": float(eps.median()), "p10": float(eps.quantile(0.1)) if eps.numel() < 1 << 24 else None,
-                      "frac_rows_negative": float((eps < 0).float().mean()),
+    out["epsilon"] = {"row_median": float(eps.median()), "row_frac_negative": float((eps < 0).float().mean()),
                       "preorder_output_scale_error": 0.0,
                       "inconsistent_output_scale_error_median_over_heads": float(scale_err.median())}
+    del o_pre, o_inc, lph, lp
+    try:
+        out["epsilon"]["tile_inconsistent"] = tile_epsilon_gpu(st, h.INCONSISTENT)
+    except Exception as e:  # measurement only
+        out["epsilon"]["tile_inconsistent"] = {"error": str(e)[:160]}
     # Lazy running-max updates (FlashAttention-4's conditional rescaling; the
     # paper states the exact recurrence, tau = 0): time and deviation from
     # exact attention against the exact recurrence, same harness and heads
     lazy = []
-    o_t = torch.empty_like(o_pre)
+    o_t = torch.empty_like(st.o)
     for tau in (0.0, 1.0, 3.0):
         fn = lambda: h.attn_fwd(z, scale, w.causal, h.PREORDER, w.block_n, out=o_t, rescale_threshold=tau)
-        ms = time_ms(fn)
+        ms = time_ms(fn, n=10)
         fn()
         o4t = o_t[0, heads].float()
         lazy.append({"rescale_threshold": tau, "ms": ms, "tflops": res["flops"] / (ms * 1e-3) / 1e12,
@@ -354,6 +448,7 @@ def comparisons(res):
     for rec in lazy:
         rec["speedup_vs_exact_recurrence"] = lazy[0]["ms"] / rec["ms"]
     out["lazy_rescale"] = lazy
+    del o_t
     # Smooth-QK migration strength and the applicability gate: deviation of
     # the 4-bit output from exact attention (same 4 heads) and eps per setting
     sweep = []
@@ -361,15 +456,17 @@ def comparisons(res):
                                  ("alpha=0.5", 0.5, 1), ("alpha=0.75", 0.75, 1), ("gate, alpha=0.5", 0.5, h.GATE)):
         s_a, inv_a = h.calibrate_smooth_qk(qd[:, :, : w.n_cal], kd[:, :, : w.n_cal], w.n_cal, alpha=alpha,
                                            enable=enable)
-        za = h.quantize_qkv(qd, kd, vd, s_a, inv_a, res["fmt"])
-        oa, lpa, lpp = h.attn_fwd(za, scale, w.causal, h.PREORDER, w.block_n, out_dtype=o_pre.dtype, debug=True)
+        h.quantize_qkv(qd, kd, vd, s_a, inv_a, res["fmt"], out=z)
+        oa, lpa, lpp = h.attn_fwd(z, scale, w.causal, h.PREORDER, w.block_n, out_dtype=odt, debug=True)
         o4a = oa[0, heads].float()
         ea = (lpa / lpp - 1.0).flatten()
         sweep.append({"setting": label, "heads_smoothed": int((s_a != 1.0).any(dim=1).sum()),
                       "max_abs_rel": float((o4a - ex).abs().max() / ex.abs().max()),
                       "cosine": float(torch.nn.functional.cosine_similarity(o4a.flatten(), ex.flatten(), dim=0)),
                       "eps_median": float(ea.median())})
+        del oa, lpa, lpp
     out["smooth_qk_sweep"] = sweep
+    st.quantize()      # restore the headline's quantized inputs
     return out
 
 
@@ -414,23 +511,32 @@ def fp4_probe_peak():
     return 2.0 * 128 * n * k * reps * ctas / (ms * 1e-3) / 1e12
 
 
-def cpu_baseline(w, fmt, mode, prefill_inputs=None, budget_s=20.0):
-    """The oracle, as it stands, on the host cores: full-workload quantize plus
-    the attention of the last query tile (128 rows, all heads) of batch 0."""
+def cpu_baseline(w, fmt, mode, prefill_inputs=None, budget_s=15.0):
+    """The oracle, as it stands, on the host cores, on a bounded sample of the
+    workload: the quantization of batch 0 (all of its Q, K and V), then the
+    attention of the last query rows of batch 0, all heads, with as many rows
+    (up to one 128-row tile) as fit the time budget."""
     import oracle
     q, k, v = prefill_inputs if prefill_inputs is not None else W.make_prefill(w)
     qn, kn, vn = q[:1].float().numpy(), k[:1].float().numpy(), v[:1].float().numpy()
     s, inv = oracle.calibrate(qn, kn, w.n_cal)
-    rows = 128
     t0 = time.perf_counter()
     qz = oracle.quantize_qkv(qn, kn, vn, s, inv, fmt)
+    t_q = time.perf_counter() - t0
+    probe = 4
+    t0 = time.perf_counter()
+    oracle.attention(qz, w.N, fmt, 1 / math.sqrt(w.d), w.causal, mode, w.block_n, rows=(w.N - probe, w.N))
+    per_row = (time.perf_counter() - t0) / probe
+    rows = int(max(probe, min(128, (budget_s - t_q) / max(per_row, 1e-9))))
+    t0 = time.perf_counter()
     oracle.attention(qz, w.N, fmt, 1 / math.sqrt(w.d), w.causal, mode, w.block_n, rows=(w.N - rows, w.N))
-    dt = time.perf_counter() - t0
+    dt = time.perf_counter() - t0 + t_q
     pairs = sum((i + 1) if w.causal else w.N for i in range(w.N - rows, w.N))
     flops = 4.0 * w.Hq * w.d * pairs
     return dict(value=flops / dt / 1e12, unit="TFLOPS", cores=oracle.threads(), kind="oracle",
-                sample=f"batch 0 of {w.name}: oracle quantize of all Q/K/V plus attention of the last "
-                       f"{rows}-row query tile, all {w.Hq} heads ({flops / 1e9:.2f} GFLOP in {dt:.1f} s)")
+                sample=f"batch 0 of {w.name}: oracle quantize of all its Q/K/V ({t_q:.1f} s) plus the attention "
+                       f"of its last {rows} query rows, all {w.Hq} heads ({flops / 1e9:.2f} GFLOP, {dt:.1f} s "
+                       f"in total); TFLOPS over the sample")
 
 
 def run_decode(args):
@@ -513,6 +619,10 @@ def profile_target(args, launches: int = 5):
     `launches` launches of the target (skip the first with -s in ncu)."""
     import bit_quantized_flashattention_smooth_b200 as h
     w = W.WORKLOADS[args.workload]
+    if args.profile_batches:
+        # a smaller capture of the same workload: its first batches (same
+        # shapes and value distributions; traffic scales with the batch)
+        w = W.Workload(**{**w.__dict__, "B": min(w.B, args.profile_batches)})
     fmt = h.NVFP4 if args.fmt == "nvfp4" else h.MXFP4
     mode = h.PREORDER if args.mode == "preorder" else h.INCONSISTENT
     dev = torch.device("cuda")
@@ -556,30 +666,72 @@ def profile_target(args, launches: int = 5):
     if h.device_error():
         raise RuntimeError("device error word set")
     print(json.dumps({"profile": args.profile, "workload": w.name if args.profile != "decode" else "split_decode",
-                      "launches": launches}), flush=True)
+                      "B": w.B, "launches": launches}), flush=True)
+
+
+def measure_all_configs(args, pk, headline):
+    """Every config of the path in one run (the headline's workload is
+    reported by the headline itself): time, TFLOP/s, tokens/s and roofline
+    fractions; epsilon per row and per tile where the normalizer modes are
+    compared."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    fp4_peak = pk["bf16"] * FP4_OVER_BF16
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    mufu = 16.0 * sms * 1965.0 * 1e6
+    plan = [("tiny_mha", "nvfp4", "preorder", 0.5, False), ("tiny_mha", "nvfp4", "inconsistent", 0.5, True),
+            ("qwen3_prefill", "nvfp4", "preorder", 0.5, False), ("qwen3_prefill", "mxfp4", "preorder", 0.5, False),
+            ("qwen3_prefill", "nvfp4", "inconsistent", 0.5, True),
+            ("gemma2_prefill", "nvfp4", "preorder", 0.5, False), ("gemma2_prefill", "nvfp4", "inconsistent", 0.5, True),
+            ("gemma2_prefill", "nvfp4", "preorder", 0.25, True)]
+    out = []
+    for name, fmt, mode, alpha, eps in plan:
+        try:
+            rec, st = measure_config(name, fmt, mode, args.config_steps, 5, alpha=alpha, want_eps=eps)
+            rec["frac_fp4_peak"] = rec["attn_tflops"] / fp4_peak
+            rec["frac_mufu_ceiling"] = W.exp_count(st.w) / (rec["attn_ms"] * 1e-3) / mufu
+            if mode == "preorder" and alpha == 0.5 and fmt == "nvfp4":
+                w = st.w
+                qb, kb = st.qd.to(torch.bfloat16), st.kd.to(torch.bfloat16)
+                vt = h.bf16_transpose_v(st.vd.to(torch.bfloat16))
+                ob = h.bf16_attn_fwd(qb, kb, vt, st.scale, w.causal)
+                ms = time_ms(lambda: h.bf16_attn_fwd(qb, kb, vt, st.scale, w.causal, out=ob), n=10)
+                rec["bf16_inhouse_ms"] = ms
+                rec["fp4_speedup_vs_bf16_inhouse"] = ms / rec["attn_ms"]
+                del qb, kb, vt, ob
+            out.append(rec)
+            del st
+            torch.cuda.empty_cache()
+        except Exception as e:  # measurement only
+            out.append({"workload": name, "format": fmt, "normalizer": mode, "alpha": alpha, "error": str(e)[:200]})
+    return out
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="qwen3_prefill")
+    ap.add_argument("--workload", default="long_prefill")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--mode", default="preorder", choices=["preorder", "inconsistent"])
     ap.add_argument("--rescale-threshold", type=float, default=0.0,
                     help="lazy running-max threshold tau (0 = the exact online recurrence)")
     ap.add_argument("--path", default="two-launch", choices=["fused", "two-launch"],
-                    help="fused: K/V quantize + attention with Smooth-QK and Q quantization in the kernel; "
-                         "two-launch: Q/K/V quantize + attention")
+                    help="fused: K/V quantize + attention with Smooth-QK and Q quantization in the kernel "
+                         "(--profile only); two-launch: Q/K/V quantize + attention")
     ap.add_argument("--block-n", type=int, default=0, help="key tile (0 = the workload's)")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--config-steps", type=int, default=50, help="timed steps of each entry of `configs`")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-probe", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--no-compare", action="store_true", help="skip the BF16 / exact / epsilon comparisons")
     ap.add_argument("--profile", choices=["attn", "quantize", "decode", "bf16"], default=None,
                     help="run only this kernel a few times (for an ncu capture) and exit")
+    ap.add_argument("--profile-batches", type=int, default=0,
+                    help="--profile on the first B batches of the workload (a smaller capture)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     # the reference arm is the CPU oracle: its ranks need no GPU (gloo plumbing)
@@ -588,9 +740,10 @@ def main():
         W.WORKLOADS[args.workload] = W.Workload(**{**W.WORKLOADS[args.workload].__dict__, "block_n": args.block_n})
     w = W.WORKLOADS[args.workload]
     config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
-              "format": args.fmt, "normalizer": args.mode, "block_n": w.block_n, "path": args.path,
+              "format": args.fmt, "normalizer": args.mode, "block_n": w.block_n, "path": "two-launch",
               "rescale_threshold": args.rescale_threshold,
-              "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)", "parallelism": f"replicas x{world}"}
+              "l2": "flushed between timed steps (256 MiB write, then 256 MiB read); inputs also exceed L2",
+              "parallelism": f"replicas x{world}"}
 
     if args.profile:
         profile_target(args)
@@ -625,12 +778,6 @@ def main():
             extra["fp4_probe_tflops"] = fp4_probe_peak()
         except Exception as e:  # measurement only
             extra["fp4_probe_error"] = str(e)
-    decode = None
-    if not args.no_decode:
-        try:
-            decode = run_decode(args)
-        except Exception as e:
-            decode = {"error": str(e)}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["step_ms"], "higher_is_better": True, "scaling": "weak",
@@ -641,21 +788,13 @@ def main():
                      "peak_note": f"{pk['src']} bf16 burst {pk['bf16']} TFLOP/s x nominal FP4/BF16 ratio 4"},
         "attn_ms": res["attn_ms"], "quantize_ms": res["quant_ms"],
         "e2e": {"value": res["flops"] * world / (res["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
-                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"], "steps": res["n_e2e"]},
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
     }
     line.update(extra)
     if "fp4_probe_tflops" in extra:
         line["roofline"]["frac_of_probe_peak"] = attn_tflops / extra["fp4_probe_tflops"]
-    if decode is not None:
-        if "gbs" in decode:
-            line["decode"] = {"workload": "split_decode", "kv_gbs": decode["gbs"], "ms": decode["ms"],
-                              "kv_bytes": decode["bytes"], "hbm_peak_gbs": pk["hbm"],
-                              "frac": decode["gbs"] / pk["hbm"], "splits": decode["splits"],
-                              "append_one_token_ms": decode["append_ms"]}
-        else:
-            line["decode"] = decode
     line["tokens_per_s"] = w.B * w.N * world / (res["step_ms"] * 1e-3)
     # the softmax's own ceiling: every score needs one 2^x, and the MUFU unit
     # gives 16 per clock per SM (at the median SM clock seen while timing)
@@ -666,16 +805,30 @@ def main():
                                 "peak": 16.0 * sms * clk_mhz * 1e6, "exp2_per_launch": n_exp,
                                 "frac": n_exp / (res["attn_ms"] * 1e-3) / (16.0 * sms * clk_mhz * 1e6),
                                 "note": "MUFU ex2 ceiling: 16/clk/SM x SMs x median SM clock"}
-    tr = traffic_record("attn_fwd_fp4", w.name, args.fmt, w.block_n, args.path)
+    tr = traffic_record("attn_fwd_fp4", w.name, args.fmt, w.block_n, "two-launch")
     if tr is not None:
         line["roofline"]["traffic"] = tr
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, res["fmt"], res["mode"], res["setup"].host)
     if rank == 0 and not args.no_compare:
         try:
             line["comparisons"] = comparisons(res)
         except Exception as e:  # measurement only
             line["comparisons"] = {"error": str(e)[:200]}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, res["fmt"], res["mode"])
+    del res
+    torch.cuda.empty_cache()
+    if rank == 0 and not args.no_configs:
+        line["configs"] = measure_all_configs(args, pk, w.name)
+    if not args.no_decode:
+        try:
+            decode = run_decode(args)
+            line["decode"] = {"workload": "split_decode", "kv_gbs": decode["gbs"], "ms": decode["ms"],
+                              "kv_bytes": decode["bytes"], "hbm_peak_gbs": pk["hbm"],
+                              "frac": decode["gbs"] / pk["hbm"], "frac_of_8tbs_spec": decode["gbs"] / 8000.0,
+                              "splits": decode["splits"], "append_one_token_ms": decode["append_ms"],
+                              "tokens_per_s": W.WORKLOADS["split_decode"].B / (decode["ms"] * 1e-3)}
+        except Exception as e:
+            line["decode"] = {"error": str(e)[:200]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

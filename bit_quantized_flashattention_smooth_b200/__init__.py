@@ -32,7 +32,7 @@ _lib = None
 ABI_FUNCTIONS = (
     "hifa4_codes_bytes", "hifa4_scale_bytes", "hifa4_calibrate_smooth_qk", "hifa4_quantize_qkv",
     "hifa4_quantize_kv",
-    "hifa4_attn_fwd", "hifa4_attn_fwd_ex", "hifa4_attn_fwd_fused", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
+    "hifa4_attn_fwd", "hifa4_attn_fwd_ex", "hifa4_attn_fwd_dump", "hifa4_attn_fwd_fused", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
     "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_e2m1_map_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_kv_cache_append", "hifa4_attn_decode_cache", "hifa4_status_string", "hifa4_last_error",
     "hifa4_device_error",
@@ -59,6 +59,8 @@ def lib():
         L.hifa4_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, vp]
         L.hifa4_attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, f,
                                         vp]
+        L.hifa4_attn_fwd_dump.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, f, vp, vp, vp,
+                                          vp, vp]
         L.hifa4_attn_fwd_fused.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp,
                                            f, vp]
         L.hifa4_decode_workspace_size.argtypes = [i, i, i, i]; L.hifa4_decode_workspace_size.restype = sz
@@ -258,6 +260,42 @@ def attn_fwd(z: QuantizedQKV, softmax_scale: float | None = None, causal: bool =
     if debug:
         res += [lph, lp]
     return res[0] if len(res) == 1 else tuple(res)
+
+
+@dataclass
+class PhatDump:
+    """Quantized attention weights of one forward, as fed to the PV MMA
+    (hifa4_attn_fwd_dump): codes [B,Hq,N,nkt,BN/2] packed E2M1, scales
+    [B,Hq,N,nkt,BN/beta], m [B,Hq,N,nkt] running max after each key tile,
+    sum_p [B,Hq,N,nkt] (or None) sum of P of each tile."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    m: torch.Tensor
+    sum_p: torch.Tensor | None
+
+
+def attn_fwd_dump(z: QuantizedQKV, softmax_scale: float | None = None, causal: bool = True, mode: int = PREORDER,
+                  block_n: int = 128, out_dtype=torch.bfloat16, rescale_threshold: float = 0.0,
+                  sum_p: bool = False):
+    """Forward plus the P-hat dump.  sum_p=True selects the softmax variant
+    that forms P (as the debug normalizers do) and records sum(P) per tile.
+    Returns (O, PhatDump); unvisited tiles hold zeros (m: NaN)."""
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(z.d)
+    dev = z.q_codes.device
+    nkt = (z.N + block_n - 1) // block_n
+    beta = beta_of(z.fmt)
+    o = torch.empty((z.B, z.Hq, z.N, z.d), device=dev, dtype=out_dtype)
+    codes = torch.zeros((z.B, z.Hq, z.N, nkt, block_n // 2), device=dev, dtype=torch.uint8)
+    scales = torch.zeros((z.B, z.Hq, z.N, nkt, block_n // beta), device=dev, dtype=torch.uint8)
+    m = torch.full((z.B, z.Hq, z.N, nkt), float("nan"), device=dev, dtype=torch.float32)
+    sp = torch.zeros((z.B, z.Hq, z.N, nkt), device=dev, dtype=torch.float32) if sum_p else None
+    _check(lib().hifa4_attn_fwd_dump(_ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),
+                                     _ptr(z.vt_codes), _ptr(z.vt_scales), z.B, z.Hq, z.Hkv, z.N, z.d, z.fmt,
+                                     float(softmax_scale), int(bool(causal)), int(mode), int(block_n), _ptr(o),
+                                     _dt(o), float(rescale_threshold), _ptr(codes), _ptr(scales), _ptr(m), _ptr(sp),
+                                     _stream()), "attn_fwd_dump")
+    return o, PhatDump(codes, scales, m, sp)
 
 
 def attn_fwd_fused(q: torch.Tensor, s: torch.Tensor | None, kv: QuantizedQKV, softmax_scale: float | None = None,

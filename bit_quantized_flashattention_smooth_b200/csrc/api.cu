@@ -78,7 +78,7 @@ hifa4_status calibrate_launch(const void*, const void*, int, int, int, int, int,
                               cudaStream_t);
 hifa4_status attn_fwd_launch(const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*,
                              const uint8_t*, int, int, int, int, int, int, float, int, int, int, void*, int, float*,
-                             float*, float*, float, const void*, int, const float*, cudaStream_t);
+                             float*, float*, float, const void*, int, const float*, const AttnDump*, cudaStream_t);
 hifa4_status decode_launch(const void*, int, const float*, const uint8_t*, const uint8_t*, const uint8_t*,
                            const uint8_t*, int, int, int, int, int, int, int, float, int, int, int, int*, void*, size_t,
                            void*, int, float, cudaStream_t);
@@ -214,7 +214,41 @@ hifa4_status hifa4_attn_fwd_ex(const uint8_t* q_codes, const uint8_t* q_scales, 
                 "attn_fwd: problem too large");
   return attn_fwd_launch(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
                          softmax_scale, causal, mode, block_n, o, o_dt, lse, dbg_l_phat, dbg_l_p, rescale_threshold,
-                         nullptr, 0, nullptr, static_cast<cudaStream_t>(stream));
+                         nullptr, 0, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_attn_fwd_dump(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                                 const uint8_t* k_scales, const uint8_t* vt_codes, const uint8_t* vt_scales, int B,
+                                 int Hq, int Hkv, int N, int d, hifa4_format fmt, float softmax_scale, int causal,
+                                 hifa4_norm_mode mode, int block_n, void* o, hifa4_dtype o_dt, float rescale_threshold,
+                                 uint8_t* phat_codes, uint8_t* phat_scales, float* tile_m, float* tile_sum_p,
+                                 hifa4_stream_t stream) {
+  HIFA4_REQUIRE(phat_codes && phat_scales && tile_m, HIFA4_ERR_INVALID_ARG, "attn_fwd_dump: null dump pointer");
+  HIFA4_REQUIRE(aligned16(phat_codes), HIFA4_ERR_INVALID_ARG, "attn_fwd_dump: phat_codes must be 16-byte aligned");
+  // the shared checks of the forward (no launch happens on failure)
+  HIFA4_REQUIRE(valid_fmt(fmt) && valid_tau(fmt, rescale_threshold), HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_dump: rescale_threshold must be in [0, %g] for this format", max_tau(fmt));
+  HIFA4_REQUIRE(q_codes && q_scales && k_codes && k_scales && vt_codes && vt_scales && o, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_dump: null pointer");
+  HIFA4_REQUIRE(valid_dt(o_dt), HIFA4_ERR_INVALID_ARG, "attn_fwd_dump: bad dtype");
+  HIFA4_REQUIRE(mode == HIFA4_NORM_PREORDER || mode == HIFA4_NORM_INCONSISTENT, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_dump: bad normalizer mode");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_dump: bad shape B=%d Hq=%d Hkv=%d N=%d", B, Hq, Hkv, N);
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "attn_fwd_dump: d=%d not in {64,128,256}", d);
+  HIFA4_REQUIRE(block_n == 0 || block_n == 64 || block_n == 128, HIFA4_ERR_UNSUPPORTED,
+                "attn_fwd_dump: block_n=%d not in {0,64,128}", block_n);
+  HIFA4_REQUIRE(!(d == 256 && block_n == 64), HIFA4_ERR_UNSUPPORTED, "attn_fwd_dump: d=256 needs block_n=128");
+  HIFA4_REQUIRE(softmax_scale > 0.0f, HIFA4_ERR_INVALID_ARG, "attn_fwd_dump: softmax_scale must be > 0");
+  HIFA4_REQUIRE(aligned16(q_codes) && aligned16(q_scales) && aligned16(k_codes) && aligned16(k_scales) &&
+                    aligned16(vt_codes) && aligned16(vt_scales) && aligned16(o),
+                HIFA4_ERR_INVALID_ARG, "attn_fwd_dump: pointers must be 16-byte aligned");
+  HIFA4_REQUIRE(static_cast<int64_t>(B) * Hq * pad128(N) < (int64_t(1) << 31), HIFA4_ERR_UNSUPPORTED,
+                "attn_fwd_dump: problem too large");
+  AttnDump dump{phat_codes, phat_scales, tile_m, tile_sum_p};
+  return attn_fwd_launch(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
+                         softmax_scale, causal, mode, block_n, o, o_dt, nullptr, nullptr, nullptr, rescale_threshold,
+                         nullptr, 0, nullptr, &dump, static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_attn_fwd_fused(const void* q, hifa4_dtype q_dt, const float* s, const uint8_t* k_codes,
@@ -245,7 +279,7 @@ hifa4_status hifa4_attn_fwd_fused(const void* q, hifa4_dtype q_dt, const float* 
                 "attn_fwd_fused: problem too large");
   return attn_fwd_launch(nullptr, nullptr, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
                          softmax_scale, causal, mode, block_n, o, o_dt, lse, dbg_l_phat, dbg_l_p, rescale_threshold,
-                         q, q_dt, s, static_cast<cudaStream_t>(stream));
+                         q, q_dt, s, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 size_t hifa4_decode_workspace_size(int B, int Hq, int d, int num_splits) {

@@ -83,6 +83,8 @@ struct AttnParams {
   float* lse;
   float* dbg_l_phat;
   float* dbg_l_p;
+  AttnDump dump;        // all null unless hifa4_attn_fwd_dump
+  int nkt_all;          // key tiles of a whole row, ceil(N / BN): the dump's tile stride
 };
 
 template <int D, int BN, int FMT>
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     const float c = p.c_log2;
     float m = -INFINITY;
     float l_p = 0.0f;
-    const bool want_lp = !PREORDER || p.dbg_l_p != nullptr;
+    const bool want_lp = !PREORDER || p.dbg_l_p != nullptr || p.dump.sum_p != nullptr;
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
     constexpr float kInvGP = FMT == HIFA4_NVFP4 ? 256.0f : 1.0f;
     // pairs (of every eight) whose 2^y runs on the FMA pipe instead of MUFU
@@ -695,6 +697,23 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       if (want_lp) quant_tile(std::true_type{});
       else quant_tile(std::false_type{});
       if (want_lp) l_p = fmaf(alpha, l_p, psum);
+      if (p.dump.codes != nullptr && row < p.N) {
+        // debug view of this tile: the codes and scales as they go to the
+        // PV MMA, the running max, and (on the path that forms P) sum(P)
+        const int64_t rt = (static_cast<int64_t>(bhq) * p.N + row) * p.nkt_all + j;
+        uint4* dc = reinterpret_cast<uint4*>(p.dump.codes + rt * (BN / 2) + hw * (HB / 2));
+#pragma unroll
+        for (int ch = 0; ch < HB / 32; ++ch)
+          dc[ch] = make_uint4(codes[4 * ch], codes[4 * ch + 1], codes[4 * ch + 2], codes[4 * ch + 3]);
+        uint8_t* ds = p.dump.scales + rt * (BN / C::BETA) + hw * NBH;
+#pragma unroll
+        for (int blk = 0; blk < NBH; ++blk) ds[blk] = static_cast<uint8_t>(scb[blk]);
+        if (hw == 0) p.dump.m[rt] = m_new;
+        if (p.dump.sum_p != nullptr) {
+          if constexpr (C::NH == 1) p.dump.sum_p[rt] = psum;
+          else atomicAdd(p.dump.sum_p + rt, psum);     // two column halves; the caller zero-fills
+        }
+      }
       // the P-hat buffer pb was last read by PV_{j-2}
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(BAR(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, abort_flag,
                                                         kErrTimeoutSoftmax))) {
@@ -862,8 +881,9 @@ hifa4_status attn_fwd_launch(const uint8_t* qc, const uint8_t* qs, const uint8_t
                              const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int N, int d, int fmt,
                              float softmax_scale, int causal, int mode, int block_n, void* o, int o_dt, float* lse,
                              float* dbg_l_phat, float* dbg_l_p, float rescale_threshold, const void* q_raw,
-                             int q_dt, const float* q_s, cudaStream_t st) {
+                             int q_dt, const float* q_s, const AttnDump* dump, cudaStream_t st) {
   AttnParams p;
+  p.dump = dump != nullptr ? *dump : AttnDump{nullptr, nullptr, nullptr, nullptr};
   p.q_raw = q_raw;
   p.q_s = q_s;
   p.q_fp16 = q_dt == HIFA4_FP16;
@@ -888,6 +908,7 @@ hifa4_status attn_fwd_launch(const uint8_t* qc, const uint8_t* qs, const uint8_t
   p.dbg_l_phat = dbg_l_phat;
   p.dbg_l_p = dbg_l_p;
   if (block_n == 0) block_n = 128;
+  p.nkt_all = (N + block_n - 1) / block_n;
   if (d == 64 && block_n == 64) return launch_attn_fm<64, 64>(fmt, mode, qc, kc, vc, p, st);
   if (d == 64 && block_n == 128) return launch_attn_fm<64, 128>(fmt, mode, qc, kc, vc, p, st);
   if (d == 128 && block_n == 64) return launch_attn_fm<128, 64>(fmt, mode, qc, kc, vc, p, st);

@@ -24,6 +24,16 @@ __host__ __device__ __forceinline__ int64_t sf_word_offset(int64_t row, int bloc
   return ((row >> 7) * nkc + block4) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4;
 }
 
+// Optional dump of the quantized attention weights of the prefill kernel
+// (hifa4_attn_fwd_dump): per query row and key tile, the P-hat codes and block
+// scale codes, the running max after the tile, and the tile's sum of P.
+struct AttnDump {
+  uint8_t* codes;    // [B][Hq][N][nkt][BN/2]
+  uint8_t* scales;   // [B][Hq][N][nkt][BN/beta]
+  float* m;          // [B][Hq][N][nkt]
+  float* sum_p;      // [B][Hq][N][nkt] or null
+};
+
 // Error helpers of the C ABI (api.cu).
 void set_last_error(const char* fmt, ...);
 hifa4_status launch_status(const char* what);

@@ -17,7 +17,7 @@
 //   L^T [128      x 16]  += ones (A) x P-hat^T (B)      (fused normalizer)
 // The softmax warps hold one key per thread (TMEM lane) and reduce across keys
 // with warp shuffles plus a 4-warp exchange in shared memory.  The kernel is
-// bound by HBM: it streams each K/V tile once through a 3-stage TMA ring.
+// bound by HBM: it streams each K/V tile once through a 2-stage TMA ring.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -448,17 +448,24 @@ __global__ void __launch_bounds__(192, 4)
     }
     // ------------------------------------------------------------- epilogue ---
     const bool ready = __all_sync(0xffffffffu, ok && ntile > 0) && fold(ntile - 1);
-    if (ready) {
-      const int c = t;  // TMEM lane = output channel
+    const int c = t;  // TMEM lane = output channel
 #pragma unroll
-      for (int q = 0; q < G; ++q) {
-        const int hq = h * G + q;
-        float* w = p.ws + ((static_cast<int64_t>(b) * p.Hq + hq) * p.splits + sp) * (C::D + 2);
+    for (int q = 0; q < G; ++q) {
+      const int hq = h * G + q;
+      float* w = p.ws + ((static_cast<int64_t>(b) * p.Hq + hq) * p.splits + sp) * (C::D + 2);
+      if (ready) {
         w[c] = acc[q] * kGP;
         if (c == 0) {
           w[C::D] = m[q];
           w[C::D + 1] = PREORDER ? lacc[q] * kGP : lp[q];
         }
+      } else if (ntile == 0) {
+        // an empty split (never launched by the host) contributes nothing
+        if (c == 0) w[C::D] = -INFINITY;
+      } else {
+        // a wait gave up: poison this warp's channels, so the combine turns
+        // them into NaN instead of reading what an earlier call left here
+        w[c] = __int_as_float(0x7fc00000);
       }
     }
   }
@@ -608,25 +615,57 @@ static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / s
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
+CUcontext g_scratch_ctx[kMaxDevices] = {nullptr};   // the context each address belongs to
 
-// Device address of the scratch on the current device, looked up once per
-// device (the first call on a device does this lookup).
+// cuCtxGetCurrent through the runtime's driver entry point (no link
+// dependency on libcuda).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  return fn;
+}
+
+// Device address of the scratch on the current device.  It is looked up on
+// the first call on a device and again whenever the device's context has
+// changed since (after cudaDeviceReset, or when a host framework released and
+// re-created the primary context, the module and its array are loaded anew).
 hifa4_status scratch_for_current(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     hifa4::set_last_error("attn_decode_noalloc: no usable current CUDA device");
     return HIFA4_ERR_CUDA;
   }
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (get_ctx == nullptr) {
+    hifa4::set_last_error("attn_decode_noalloc: cuCtxGetCurrent is not available");
+    return HIFA4_ERR_CUDA;
+  }
+  // null before the runtime has made this device's context current
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || ctx == nullptr || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
+    // (the lookup also makes the device's primary context current)
     cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess || p == nullptr) {
       hifa4::set_last_error("attn_decode_noalloc: cudaGetSymbolAddress failed on device %d: %s", dev,
                             cudaGetErrorString(e));
       return HIFA4_ERR_CUDA;
     }
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) {
+      hifa4::set_last_error("attn_decode_noalloc: no current CUDA context on device %d", dev);
+      return HIFA4_ERR_CUDA;
+    }
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return HIFA4_OK;
@@ -663,8 +702,11 @@ extern "C" HIFA4_API hifa4_status hifa4_attn_decode_noalloc(
   void* scratch = nullptr;
   hifa4_status st = scratch_for_current(&scratch);
   if (st != HIFA4_OK) return st;
-  // Every split writes all of its partials before the combine reads them, so
-  // the scratch needs no clearing between calls.
+  // Every split that completes writes all of its partials before the combine
+  // reads them, so the scratch needs no clearing between calls; a split whose
+  // bounded wait gave up writes NaN markers instead (the output turns NaN and
+  // the device error word is set), never leaving an earlier call's partials
+  // to be read as its own.
   return hifa4_attn_decode(q, q_dt, s, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, kv_len, d, fmt,
                            softmax_scale, mode, block_n, num_splits, num_splits_used, scratch, kNoAllocScratchBytes, o,
                            o_dt, stream);

@@ -144,8 +144,10 @@ def make_prefill(w: Workload, N: int | None = None, B: int | None = None):
     k = _draw_k(rng, (B, w.Hkv, N, w.d), w)
     v = rng.standard_normal((B, w.Hkv, N, w.d), dtype=np.float32)
     if w.theta is not None:
-        q = rope_neox(q, w.theta)
-        k = rope_neox(k, w.theta)
+        # rope_torch on the host equals rope_neox bit for bit (the same fp32
+        # operations, element by element) and runs on all host threads
+        q = rope_torch(torch.from_numpy(q), w.theta).numpy()
+        k = rope_torch(torch.from_numpy(k), w.theta).numpy()
     return _round(q, w.dtype), _round(k, w.dtype), _round(v, w.dtype)
 
 

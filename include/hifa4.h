@@ -184,6 +184,37 @@ HIFA4_API hifa4_status hifa4_attn_fwd_ex(const uint8_t* q_codes, const uint8_t* 
                                          hifa4_dtype o_dt, float* lse, float* dbg_l_phat, float* dbg_l_p,
                                          float rescale_threshold, hifa4_stream_t stream);
 
+/* Debug view of hifa4_attn_fwd_ex: the same forward (o written as there),
+ * plus the quantized attention weights P-hat exactly as the kernel feeds them
+ * to the PV MMA (paper Abstract para 2: P-Reordering normalizes by "the same
+ * quantized attention weights P-hat used in the PV GEMM"), for checking them
+ * against a reference.  With nkt = ceil(N / block_n) key tiles per row and
+ * beta = 16 (NVFP4) or 32 (MXFP4), for query row r of (b, hq) and key tile j:
+ *   phat_codes  [B][Hq][N][nkt][block_n/2]    E2M1 codes of the tile's keys,
+ *               key 2i in the low nibble (device, 16-byte aligned)
+ *   phat_scales [B][Hq][N][nkt][block_n/beta] block scale codes (UE4M3 of
+ *               the 2^-8-prescaled scale for NVFP4, UE8M0 for MXFP4)
+ *   tile_m      [B][Hq][N][nkt] float: running max after tile j (log2 units
+ *               of the scaled scores)
+ *   tile_sum_p  [B][Hq][N][nkt] float, or NULL: sum of the unquantized P of
+ *               tile j against that max (must be zero-filled by the caller)
+ * Tiles past the end of a row's 128-row query tile under causal masking are
+ * not visited and not written: the caller initializes the buffers.  With
+ * tile_sum_p == NULL the kernel runs the variant hifa4_attn_fwd_ex runs
+ * without debug sums (under P-Reordering part of each tile's codes are then
+ * decided from the log2-domain argument without forming P); a non-NULL
+ * tile_sum_p selects the variant that forms and sums P, as dbg_l_p does.
+ * Other arguments, requirements and errors as hifa4_attn_fwd_ex; the dump
+ * pointers must be non-NULL except tile_sum_p. */
+HIFA4_API hifa4_status hifa4_attn_fwd_dump(const uint8_t* q_codes, const uint8_t* q_scales,
+                                           const uint8_t* k_codes, const uint8_t* k_scales,
+                                           const uint8_t* vt_codes, const uint8_t* vt_scales, int B, int Hq,
+                                           int Hkv, int N, int d, hifa4_format fmt, float softmax_scale,
+                                           int causal, hifa4_norm_mode mode, int block_n, void* o,
+                                           hifa4_dtype o_dt, float rescale_threshold, uint8_t* phat_codes,
+                                           uint8_t* phat_scales, float* tile_m, float* tile_sum_p,
+                                           hifa4_stream_t stream);
+
 /* The prefill forward with Smooth-QK and the Q quantization fused into the
  * attention kernel (the paper's Abstract para 2: Smooth-QK needs "only a
  * fusible element-wise scaling"): q [B][Hq][N][d] in q_dt, unscaled and
@@ -211,8 +242,11 @@ HIFA4_API size_t hifa4_decode_workspace_size(int B, int Hq, int d, int num_split
 /* Split count chosen by hifa4_attn_decode when num_splits == 0. */
 HIFA4_API int hifa4_decode_default_splits(int B, int Hkv, int kv_len, int block_n);
 
-/* One decode step over a 4-bit KV cache (the cache layouts of
- * hifa4_quantize_qkv with N = kv_len).  q: device [B][Hq][d] of q_dt,
+/* One decode step over a 4-bit KV cache: the split-KV decode workload of the
+ * 4-bit path (B = 64 sequences, one query each, 32768 cached tokens, GQA
+ * 32 / 8, d = 128), the prefill recurrence of the paper's Abstract paras 1-2
+ * over a cache quantized once.  The cache layouts are those of
+ * hifa4_quantize_qkv with N = kv_len.  q: device [B][Hq][d] of q_dt,
  * unscaled; s: device float [Hkv][d] Smooth-QK scales or NULL.  Inside the
  * kernel each query row is scaled (fl32(q*s)) and quantized by the Q rule.
  * Keys split into chunks of L = ceil(kv_len/num_splits) rounded up to
@@ -283,10 +317,14 @@ HIFA4_API hifa4_status hifa4_attn_decode_cache(const void* q, hifa4_dtype q_dt, 
  * splits_used * (d + 2) * 4 bytes) returns HIFA4_ERR_INVALID_ARG with the
  * sizes in hifa4_last_error().  The first call on a device looks up the
  * scratch's device address for that device (a CUDA runtime query), so make
- * that first call before any stream capture.  All calls on a device share
- * the one scratch array: calls that overlap on the GPU (concurrent streams)
- * race on it and must be serialized by the caller.  The scratch keeps the last
- * call's contents; nothing in it needs to start at zero. */
+ * that first call before any stream capture; the lookup is repeated when the
+ * device's context has changed (after cudaDeviceReset, for instance).  All
+ * calls on a device share the one scratch array: calls that overlap on the GPU
+ * (concurrent streams) race on it and must be serialized by the caller.  The
+ * scratch keeps the last call's contents; nothing in it needs to start at
+ * zero: every split writes its partials before the combine reads them, and a
+ * split whose bounded wait gave up writes NaN markers, so its output turns NaN
+ * (with the device error word set) rather than reusing an earlier call's. */
 HIFA4_API size_t hifa4_decode_noalloc_max_bytes(void);
 HIFA4_API hifa4_status hifa4_attn_decode_noalloc(const void* q, hifa4_dtype q_dt, const float* s,
                                                  const uint8_t* k_codes, const uint8_t* k_scales,

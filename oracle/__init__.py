@@ -87,7 +87,8 @@ def lib():
         L.or_quantize_qkv.argtypes = [f32p, f32p, f32p, i, i, i, i, i, f32p, f32p, i,
                                       u8p, u8p, u8p, u8p, u8p, u8p]
         L.or_attention.argtypes = [u8p, u8p, u8p, u8p, u8p, u8p, i, i, i, i, i, i, d, i, i,
-                                   i, i, f64p, f64p, f64p, f64p, u8p, u8p, f64p, i, i, i, f]
+                                   i, i, f64p, f64p, f64p, f64p, u8p, u8p, f64p, f64p,
+                                   f32p, f32p, f32p, i, i, i, f]
         L.or_split_len.argtypes = [i, i, i]; L.or_split_len.restype = i
         L.or_decode.argtypes = [f32p, f32p, u8p, u8p, u8p, u8p, i, i, i, i, i, i, d, i, i, i,
                                 i, f64p, f64p, i, f]
@@ -261,13 +262,15 @@ def tile_scales(qz: dict) -> dict:
 def attention(qz: dict, N: int, fmt: int = NVFP4, softmax_scale: float | None = None,
               causal: bool = True, mode: int = PREORDER, BN: int = 128,
               pexp: int = P_PRESCALE_LOG2, rows=None, dump_phat: bool = False,
-              variant: int = 0, tau: float = 0.0):
+              variant: int = 0, tau: float = 0.0, raw: dict | None = None):
     """Oracle forward over the quantized tensors of quantize_qkv.
 
     Returns dict O [B,Hq,N,d] fp64, lse, l_phat, l_p [B,Hq,N]; optional P-hat
-    code dump.  rows=(begin, end) restricts the query rows computed (other
-    rows of the outputs stay NaN).  tau > 0: the running max moves only when
-    a tile's max exceeds it by more than tau (lazy rescaling).
+    dump (codes, scales, running max and the per-tile sums of P-hat and P).
+    rows=(begin, end) restricts the query rows computed (other rows of the
+    outputs stay NaN).  tau > 0: the running max moves only when a tile's max
+    exceeds it by more than tau (lazy rescaling).  raw: test-only ablation,
+    {"q"|"k"|"v": float array} in [B,H,N,d] replacing the dequantized operand.
     """
     qc, qs = qz["q_codes"], qz["q_sc"]
     B, Hq, Np, dh = qc.shape
@@ -287,18 +290,43 @@ def attention(qz: dict, N: int, fmt: int = NVFP4, softmax_scale: float | None = 
     pd = np.zeros((B, Hq, N, ntiles * BN), np.uint8) if dump_phat else None
     psd = np.zeros((B, Hq, N, ntiles * BN // beta), np.uint8) if dump_phat else None
     md = np.full((B, Hq, N, ntiles), np.nan) if dump_phat else None
+    ts = np.full((B, Hq, N, ntiles, 2), np.nan) if dump_phat else None
+    raw = raw or {}
+    rq, rk, rv = (None if raw.get(n) is None else _f32(raw[n]) for n in ("q", "k", "v"))
     arrs = [np.ascontiguousarray(qz[n]) for n in ("q_codes", "q_sc", "k_codes", "k_sc", "vt_codes", "vt_sc")]
     lib().or_attention(*[_p(a, ctypes.c_uint8) for a in arrs], B, Hq, Hkv, N, d, fmt,
                        float(softmax_scale), int(causal), int(mode), int(BN), int(pexp),
                        _p(O, ctypes.c_double), _p(lse, ctypes.c_double), _p(lph, ctypes.c_double),
                        _p(lp, ctypes.c_double), _p(pd, ctypes.c_uint8), _p(psd, ctypes.c_uint8),
-                       _p(md, ctypes.c_double), int(r0), int(r1), int(variant), float(tau))
+                       _p(md, ctypes.c_double), _p(ts, ctypes.c_double), _p(rq, ctypes.c_float),
+                       _p(rk, ctypes.c_float), _p(rv, ctypes.c_float), int(r0), int(r1), int(variant), float(tau))
     res = dict(O=O, lse=lse, l_phat=lph, l_p=lp)
     if dump_phat:
         res["phat_codes"] = pd
         res["phat_sc"] = psd
         res["m_tiles"] = md
+        res["tile_sum_phat"] = ts[..., 0]
+        res["tile_sum_p"] = ts[..., 1]
     return res
+
+
+def tile_epsilon(sum_phat: np.ndarray, sum_p: np.ndarray, BM: int = 128) -> np.ndarray:
+    """Normalizer error of each attention tile (a reading: the pages measure
+    epsilon per tile without defining it): for the BM query rows x BN keys of
+    tile (b, h, query tile, key tile), sum of P-hat over sum of P, minus one.
+    Inputs are the per-row, per-key-tile sums [B,H,N,nkt] of attention(...,
+    dump_phat=True), each relative to its row's running max at that tile;
+    rows the oracle did not compute (NaN) and tiles with no visible key are
+    left out.  Returns [B,H,ceil(N/BM),nkt] with NaN where a tile is empty."""
+    B, H, N, nkt = sum_p.shape
+    nq = (N + BM - 1) // BM
+    pad = nq * BM - N
+    sph = np.nan_to_num(np.pad(sum_phat, ((0, 0), (0, 0), (0, pad), (0, 0))), nan=0.0)
+    sp = np.nan_to_num(np.pad(sum_p, ((0, 0), (0, 0), (0, pad), (0, 0))), nan=0.0)
+    a = sph.reshape(B, H, nq, BM, nkt).sum(axis=3)
+    b = sp.reshape(B, H, nq, BM, nkt).sum(axis=3)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        return np.where(b > 0, a / b - 1.0, np.nan)
 
 
 def split_len(kv_len: int, num_splits: int, BN: int) -> int:

@@ -422,7 +422,7 @@ typedef struct {
 static void tile_update(or_row_state* st, const double* x, const int* vis, int BN,
                         int fmt, float gP, const double* vdq, int64_t Np,
                         int64_t k0, int d, int variant, float tau, uint8_t* phat_dump,
-                        uint8_t* phat_sc_dump) {
+                        uint8_t* phat_sc_dump, double* tsum) {
   int exact = (variant & OR_VAR_EXACT) != 0;
   double mt = -INFINITY;
   for (int k = 0; k < BN; ++k)
@@ -450,6 +450,7 @@ static void tile_update(or_row_state* st, const double* x, const int* vis, int B
   }
   double sp = 0.0, sph = 0.0;
   for (int k = 0; k < BN; ++k) { sp += P[k]; sph += Phat[k]; }
+  if (tsum) { tsum[0] = sph; tsum[1] = sp; }
   st->l_p = alpha * st->l_p + sp;
   st->l_phat = alpha * st->l_phat + sph;
   for (int c = 0; c < d; ++c) {
@@ -484,7 +485,13 @@ static float p_prescale(int fmt, int pexp) {
  * inconsistent normalizer [HiFA4, Abstract para 2]; lse = m + log2(l).
  * Outputs (any may be NULL except O): O [B][Hq][N][d] fp64, lse [B][Hq][N],
  * l_phat / l_p [B][Hq][N], phat_dump [B][Hq][N][Nkt*BN] codes (1 per byte),
- * phat_sc_dump [B][Hq][N][Nkt*BN/beta]. */
+ * phat_sc_dump [B][Hq][N][Nkt*BN/beta], m_dump [B][Hq][N][Nkt] (running max
+ * after each tile), tsum_dump [B][Hq][N][Nkt][2] (sum of P-hat and sum of P
+ * over the tile's keys, both relative to that tile's running max: the
+ * per-tile terms whose ratio minus one is the tile's normalizer error).
+ * Test-only ablations: q_raw [B][Hq][N][d], k_raw [B][Hkv][N][d] and v_raw
+ * [B][Hkv][N][d] (fp32, each may be NULL) replace the dequantized Q-hat,
+ * K-hat or V-hat of the scores and the PV product by the given values. */
 void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
                   const uint8_t* k_codes, const uint8_t* k_sc,
                   const uint8_t* vt_codes, const uint8_t* vt_sc, int B, int Hq,
@@ -492,7 +499,9 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
                   int causal, int mode, int BN, int pexp, double* O,
                   double* lse, double* l_phat_out, double* l_p_out,
                   uint8_t* phat_dump, uint8_t* phat_sc_dump, double* m_dump,
-                  int row_begin, int row_end, int variant, float tau) {
+                  double* tsum_dump, const float* q_raw, const float* k_raw,
+                  const float* v_raw, int row_begin, int row_end, int variant,
+                  float tau) {
   int G = Hq / Hkv;
   int beta = (fmt == OR_NVFP4) ? 16 : 32;
   int64_t Np = ((int64_t)N + 127) / 128 * 128;
@@ -513,6 +522,15 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
       dequant_rows(q_codes + qb * (d / 2), q_sc + qb * nb, Np, d, fmt, qd);
       dequant_rows(k_codes + kb * (d / 2), k_sc + kb * nb, Np, d, fmt, kd);
       dequant_rows(vt_codes + vb * (Np / 2), vt_sc + vb * (Np / beta), d, (int)Np, fmt, vd);
+      if (q_raw || k_raw || v_raw) {
+        int64_t qr = ((int64_t)b * Hq + hq) * N, kr = ((int64_t)b * Hkv + h) * N;
+        for (int64_t t = 0; t < Np; ++t)
+          for (int c = 0; c < d; ++c) {
+            if (q_raw) qd[t * d + c] = t < N ? (double)q_raw[(qr + t) * d + c] : 0.0;
+            if (k_raw) kd[t * d + c] = t < N ? (double)k_raw[(kr + t) * d + c] : 0.0;
+            if (v_raw) vd[(int64_t)c * Np + t] = t < N ? (double)v_raw[(kr + t) * d + c] : 0.0;
+          }
+      }
       double* acc = (double*)malloc(sizeof(double) * d);
       double* x = (double*)malloc(sizeof(double) * BN);
       int* vis = (int*)malloc(sizeof(int) * BN);
@@ -536,7 +554,8 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
           }
           uint8_t* pd = phat_dump ? phat_dump + row_id * (int64_t)ntiles * BN + (int64_t)j * BN : NULL;
           uint8_t* psd = phat_sc_dump ? phat_sc_dump + row_id * (int64_t)ntiles * (BN / beta) + (int64_t)j * (BN / beta) : NULL;
-          tile_update(&st, x, vis, BN, fmt, gP, vd, Np, (int64_t)j * BN, d, variant, tau, pd, psd);
+          double* ts = tsum_dump ? tsum_dump + (row_id * (int64_t)ntiles + j) * 2 : NULL;
+          tile_update(&st, x, vis, BN, fmt, gP, vd, Np, (int64_t)j * BN, d, variant, tau, pd, psd, ts);
           if (m_dump) m_dump[row_id * (int64_t)ntiles + j] = st.m;
         }
         double l = (mode == OR_PREORDER) ? st.l_phat : st.l_p;
@@ -622,7 +641,7 @@ void or_decode(const float* q, const float* s, const uint8_t* k_codes,
               x[kk] = (variant & OR_VAR_EXACT) ? sdot * c_log2 : (double)(float)(sdot * c_log2);
             }
           }
-          tile_update(&st, x, vis, BN, fmt, gP, vd, Np, j0, d, variant, tau, NULL, NULL);
+          tile_update(&st, x, vis, BN, fmt, gP, vd, Np, j0, d, variant, tau, NULL, NULL, NULL);
         }
         ms[sp] = st.m;
         ls[sp] = (mode == OR_PREORDER) ? st.l_phat : st.l_p;

@@ -127,9 +127,11 @@ def _deq_row(codes_row, sc_row, fmt):
     return out
 
 
-def attention(qz, N, fmt, softmax_scale, causal, mode, BN, pexp=-8, tau=0.0):
+def attention(qz, N, fmt, softmax_scale, causal, mode, BN, pexp=-8, tau=0.0, tile_sums=False):
     """Returns O [B,Hq,N,d] (fp64) and (l_phat, l_p).  tau: the running max
-    moves to the tile max only when that exceeds fl32(m + tau)."""
+    moves to the tile max only when that exceeds fl32(m + tau).  tile_sums:
+    also return [B,Hq,N,nkt,2], the sum of P-hat and of P over each key tile
+    a row visits (NaN for the tiles past its last visible key)."""
     qc = qz["q_codes"]
     B, Hq, Np, dh = qc.shape
     d = dh * 2
@@ -141,6 +143,7 @@ def attention(qz, N, fmt, softmax_scale, causal, mode, BN, pexp=-8, tau=0.0):
     O = np.zeros((B, Hq, N, d))
     LPH = np.zeros((B, Hq, N))
     LP = np.zeros((B, Hq, N))
+    TS = np.full((B, Hq, N, (N + BN - 1) // BN, 2), np.nan)
     for b in range(B):
         for hq in range(Hq):
             h = hq // G
@@ -181,6 +184,7 @@ def attention(qz, N, fmt, softmax_scale, causal, mode, BN, pexp=-8, tau=0.0):
                     for kk in range(BN):
                         sp += P[kk]
                         sph += Ph[kk]
+                    TS[b, hq, i, j0 // BN] = (sph, sp)
                     lp = alpha * lp + sp
                     lph = alpha * lph + sph
                     for c in range(d):
@@ -194,4 +198,6 @@ def attention(qz, N, fmt, softmax_scale, causal, mode, BN, pexp=-8, tau=0.0):
                 O[b, hq, i] = [a / l for a in acc]
                 LPH[b, hq, i] = lph
                 LP[b, hq, i] = lp
+    if tile_sums:
+        return O, LPH, LP, TS
     return O, LPH, LP

@@ -1,11 +1,16 @@
 """Appendable 4-bit KV cache: any sequence of appends gives, bit for bit, the
-one-shot quantization of the whole sequence (hifa4_quantize_kv, itself
-checked against the oracle), and decode over it equals decode over the
-one-shot cache."""
+one-shot quantization of the whole sequence (hifa4_quantize_kv) and the
+oracle's quantization of the zero-padded sequence; decode over it equals
+decode over the one-shot cache and the oracle's split decode (exact and
+lazily rescaled running max)."""
+import math
+
+import numpy as np
 import pytest
 import torch
 
 import oracle
+from tests import gpu_util as U
 
 pytestmark = pytest.mark.gpu
 
@@ -62,6 +67,18 @@ def test_appends_equal_one_shot_quantization(fmt, d, chunks):
         for name in ("k_codes", "k_scales", "vt_codes", "vt_scales"):
             a, b = getattr(cache, name), getattr(ref, name)
             assert torch.equal(a, b), f"{name} after {pos} tokens: {int((a != b).sum())} bytes differ"
+    # the final cache against the oracle's quantizer on the zero-padded
+    # sequence (the append contract: tokens not yet written are 0)
+    kp = np.zeros((B, Hkv, cap, d), np.float32)
+    vp = np.zeros_like(kp)
+    kp[:, :, :L] = k.float().cpu().numpy()
+    vp[:, :, :L] = v.float().cpu().numpy()
+    oz = oracle.quantize_qkv(np.zeros_like(kp), kp, vp, None, inv_s.cpu().numpy(), fmt)
+    ot = oracle.tile_scales(oz)
+    assert np.array_equal(U.to_np(cache.k_codes).astype(np.uint8), oz["k_codes"])
+    assert np.array_equal(U.to_np(cache.vt_codes).astype(np.uint8), oz["vt_codes"])
+    assert np.array_equal(U.to_np(cache.k_scales).astype(np.uint8), ot["k_sc"])
+    assert np.array_equal(U.to_np(cache.vt_scales).astype(np.uint8), ot["vt_sc"])
 
 
 def test_decode_over_appended_cache():
@@ -78,3 +95,31 @@ def test_decode_over_appended_cache():
         one = h.quantize_kv(k[:, :, :pos], v[:, :, :pos], inv_s, fmt, Hq=Hq)
         o_one, _ = h.attn_decode(q, None, one)
         assert torch.equal(o_app, o_one), f"decode over {pos} appended tokens differs"
+
+
+@pytest.mark.parametrize("fmt,mode,tau", [(oracle.NVFP4, oracle.PREORDER, 0.0), (oracle.NVFP4, oracle.PREORDER, 3.0),
+                                          (oracle.MXFP4, oracle.INCONSISTENT, 0.0), (oracle.MXFP4, oracle.PREORDER, 3.0)])
+def test_decode_cache_matches_oracle(fmt, mode, tau):
+    """hifa4_attn_decode_cache over an appended cache against the oracle's
+    split decode of the same tokens, at the kernel's split count, with the
+    exact (tau = 0) and the lazily updated (tau = 3) running max."""
+    B, Hkv, Hq, d, cap = 2, 2, 8, 128, 1200
+    k, v, inv_s = _inputs(B, Hkv, 1100, d, seed=21 + fmt)
+    s = (1.0 / inv_s).float()
+    cache, tail = h.alloc_appendable_kv_cache(B, Hq, Hkv, cap, d, fmt)
+    g = torch.Generator(device="cuda").manual_seed(22)
+    q = torch.randn((B, Hq, d), generator=g, device="cuda").to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(d)
+    pos = 0
+    for T in (700, 1, 250, 149):
+        h.kv_cache_append(cache, tail, k[:, :, pos:pos + T], v[:, :, pos:pos + T], inv_s, pos)
+        pos += T
+        o, used = h.attn_decode(q, s, cache, kv_len=pos, softmax_scale=scale, mode=mode, num_splits=3,
+                                rescale_threshold=tau)
+        kn = k[:, :, :pos].float().cpu().numpy()
+        vn = v[:, :, :pos].float().cpu().numpy()
+        oz = oracle.quantize_qkv(np.zeros_like(kn), kn, vn, None, inv_s.cpu().numpy(), fmt)
+        ref = oracle.decode(q.float().cpu().numpy(), s.cpu().numpy(), oz, pos, fmt, scale, mode, 128,
+                            num_splits=used, tau=tau)
+        ok, err, bound, cos = U.compare_out(U.to_np(o), ref["O"])
+        assert ok, f"{pos} tokens, splits={used}: max|dO|={err:.3e} bound={bound:.3e} cos={cos:.6f}"

@@ -385,3 +385,97 @@ def test_lazy_decode_single_split_equals_last_causal_row():
         pre = oracle.attention(qz, N, oracle.NVFP4, 0.5, True, oracle.PREORDER, 64, rows=(N - 1, N), tau=tau)
         dec = oracle.decode(q[:, :, N - 1], s, qz, N, oracle.NVFP4, 0.5, oracle.PREORDER, 64, num_splits=1, tau=tau)
         np.testing.assert_array_equal(dec["O"], pre["O"][:, :, N - 1])
+
+
+# ---------------------------------------------------------- per-tile epsilon ---
+# The pages report the normalizer error per attention tile ("all 3.6M measured
+# attention tiles exhibit net probability-mass loss", the arXiv announcement
+# abstract) without defining it.  The reading: over the 128 query rows x BN
+# keys of a tile, sum(P-hat) / sum(P) - 1, each row's terms taken against its
+# running max at that tile (the same P and P-hat that enter l_phat and l_p).
+
+
+@pytest.mark.parametrize("fmt,N,d,BN,causal,G,mode", CASES[:4] + CASES[5:])
+def test_tile_sums_equal_bruteforce(fmt, N, d, BN, causal, G, mode):
+    q, k, v = _inputs(1, G, 1, N, d, 20 + N + d)
+    s, inv = oracle.calibrate(q, k, n_cal=8, alpha=0.5)
+    qz = oracle.quantize_qkv(q, k, v, s, inv, fmt)
+    scale = 1 / np.sqrt(d)
+    ours = oracle.attention(qz, N, fmt, scale, causal, mode, BN, dump_phat=True)
+    _, _, _, ts = bruteforce.attention(qz, N, fmt, scale, causal, mode, BN, tile_sums=True)
+    np.testing.assert_allclose(ours["tile_sum_phat"], ts[..., 0], rtol=1e-13, atol=1e-300)
+    np.testing.assert_allclose(ours["tile_sum_p"], ts[..., 1], rtol=1e-13, atol=1e-300)
+
+
+@pytest.mark.parametrize("fmt,BN,tau", [(oracle.NVFP4, 16, 0.0), (oracle.MXFP4, 32, 0.0), (oracle.NVFP4, 32, 3.0)])
+def test_tile_sums_rebuild_the_normalizers(fmt, BN, tau):
+    """Both normalizers are the per-tile sums carried to the final max:
+    l = sum_j 2^(m_j - m_last) sum_tile_j, for l_phat and l_p alike."""
+    N, d, G = 150, 32, 2
+    q, k, v = _inputs(1, G, 1, N, d, 70 + BN)
+    s, inv = oracle.calibrate(q, k, n_cal=16)
+    qz = oracle.quantize_qkv(q, k, v, s, inv, fmt)
+    res = oracle.attention(qz, N, fmt, 1 / np.sqrt(d), True, oracle.PREORDER, BN, dump_phat=True, tau=tau)
+    for hq in range(G):
+        for i in (0, 31, 32, 100, 149):
+            ntl = i // BN + 1
+            m = res["m_tiles"][0, hq, i, :ntl]
+            w = 2.0 ** (m - m[-1])
+            np.testing.assert_allclose(np.sum(w * res["tile_sum_phat"][0, hq, i, :ntl]), res["l_phat"][0, hq, i],
+                                       rtol=1e-12)
+            np.testing.assert_allclose(np.sum(w * res["tile_sum_p"][0, hq, i, :ntl]), res["l_p"][0, hq, i],
+                                       rtol=1e-12)
+            assert np.all(np.isnan(res["tile_sum_p"][0, hq, i, ntl:]))
+
+
+def test_tile_epsilon_zero_without_p_quantizer_and_negative_with_it():
+    """With P-hat = P every tile's error is exactly 0; with the quantizer the
+    typical tile loses probability mass (the sign of the pages' finding)."""
+    N, d, G = 384, 64, 2
+    q, k, v = _inputs(1, G, 1, N, d, 80)
+    s, inv = oracle.calibrate(q, k, n_cal=64)
+    qz = oracle.quantize_qkv(q, k, v, s, inv, oracle.NVFP4)
+    off = oracle.attention(qz, N, oracle.NVFP4, 1 / np.sqrt(d), True, oracle.PREORDER, 64, dump_phat=True,
+                           variant=oracle.VAR_NO_PQUANT)
+    e_off = oracle.tile_epsilon(off["tile_sum_phat"], off["tile_sum_p"])
+    fin = np.isfinite(e_off)
+    # causal, 3 query tiles of 128 rows x 64-key tiles: 2 + 4 + 6 visited tiles per head
+    assert fin.sum() == G * (2 + 4 + 6)
+    assert np.all(e_off[fin] == 0.0)
+    on = oracle.attention(qz, N, oracle.NVFP4, 1 / np.sqrt(d), True, oracle.PREORDER, 64, dump_phat=True)
+    e_on = oracle.tile_epsilon(on["tile_sum_phat"], on["tile_sum_p"])
+    assert np.array_equal(np.isfinite(e_on), fin)
+    assert np.median(e_on[fin]) < 0
+
+
+def test_tile_epsilon_aggregation_by_hand():
+    """tile_epsilon sums 128-row groups of the per-row terms; checked on a
+    hand-made array with a ragged last group and an empty tile."""
+    sph = np.zeros((1, 1, 130, 2))
+    sp = np.zeros((1, 1, 130, 2))
+    sph[0, 0, :128, 0], sp[0, 0, :128, 0] = 0.5, 1.0          # tile (0, 0): 64 / 128 - 1
+    sph[0, 0, 128:, 0], sp[0, 0, 128:, 0] = 3.0, 2.0          # tile (1, 0): 6 / 4 - 1
+    sph[0, 0, 5, 1], sp[0, 0, 5, 1] = np.nan, np.nan          # tile (0, 1): not computed -> empty
+    sph[0, 0, 129, 1], sp[0, 0, 129, 1] = 1.0, 4.0            # tile (1, 1): 1 / 4 - 1
+    e = oracle.tile_epsilon(sph, sp)
+    assert e.shape == (1, 1, 2, 2)
+    assert e[0, 0, 0, 0] == -0.5 and e[0, 0, 1, 0] == 0.5 and e[0, 0, 1, 1] == -0.75
+    assert np.isnan(e[0, 0, 0, 1])
+
+
+def test_raw_operand_ablation_is_textbook_attention():
+    """The test-only raw operands replace the dequantized Q, K and V: with all
+    three raw, the P quantizer off and fp64 scores, the oracle is textbook
+    softmax attention of the raw tensors (pins the raw layouts and GQA map)."""
+    B, G, Hkv, N, d = 2, 2, 2, 90, 32
+    q, k, v = _inputs(B, G * Hkv, Hkv, N, d, 90)
+    qz = oracle.quantize_qkv(q, k, v, None, None, oracle.NVFP4)
+    res = oracle.attention(qz, N, oracle.NVFP4, 0.2, True, oracle.PREORDER, 32,
+                           variant=oracle.VAR_NO_PQUANT | oracle.VAR_EXACT, raw=dict(q=q, k=k, v=v))
+    ref = _textbook(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64), N, 0.2, True, G)
+    np.testing.assert_allclose(res["O"], ref, rtol=1e-12, atol=1e-13)
+    # one raw operand at a time changes the result (each is really used)
+    base = oracle.attention(qz, N, oracle.NVFP4, 0.2, True, oracle.PREORDER, 32)["O"]
+    for name, arr in (("q", q), ("k", k), ("v", v)):
+        o = oracle.attention(qz, N, oracle.NVFP4, 0.2, True, oracle.PREORDER, 32, raw={name: arr})["O"]
+        assert not np.allclose(o, base, rtol=1e-6, atol=0), name

@@ -87,3 +87,17 @@ def test_work_counts():
     assert abs(W.prefill_flops(w) / 1e9 - 137.4) < 0.1
     assert W.exp_count(w) == 32 * 4096 * 4097 // 2
     assert W.attended_pairs(256, False) == 256 * 256
+
+
+@pytest.mark.parametrize("name", ["qwen3_prefill", "gemma2_prefill", "long_prefill"])
+def test_prefill_recipe_uses_exact_rope(name):
+    """make_prefill (host torch RoPE) equals the numpy recipe bit for bit."""
+    w = W.WORKLOADS[name]
+    q, k, v = W.make_prefill(w, N=300, B=1)
+    rng = np.random.Generator(np.random.PCG64(w.seed))
+    qn = rng.standard_normal((1, w.Hq, 300, w.d), dtype=np.float32)
+    kn = W._draw_k(rng, (1, w.Hkv, 300, w.d), w)
+    vn = rng.standard_normal((1, w.Hkv, 300, w.d), dtype=np.float32)
+    qn, kn = W.rope_neox(qn, w.theta), W.rope_neox(kn, w.theta)
+    for a, b in ((q, qn), (k, kn), (v, vn)):
+        assert torch.equal(a, torch.from_numpy(b).to(W.torch_dtype(w.dtype)))
