@@ -234,7 +234,7 @@ __device__ __forceinline__ void rescale_o_rows(uint32_t a0, uint32_t al, bool wi
   }
 }
 
-template <int D, int BN, int FMT, bool PREORDER>
+template <int D, int BN, int FMT, bool PREORDER, bool DUMP>
 __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     const float c = p.c_log2;
     float m = -INFINITY;
     float l_p = 0.0f;
-    const bool want_lp = !PREORDER || p.dbg_l_p != nullptr || p.dump.sum_p != nullptr;
+    const bool want_lp = !PREORDER || p.dbg_l_p != nullptr || (DUMP && p.dump.sum_p != nullptr);
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
     constexpr float kInvGP = FMT == HIFA4_NVFP4 ? 256.0f : 1.0f;
     // pairs (of every eight) whose 2^y runs on the FMA pipe instead of MUFU
@@ -697,7 +697,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       if (want_lp) quant_tile(std::true_type{});
       else quant_tile(std::false_type{});
       if (want_lp) l_p = fmaf(alpha, l_p, psum);
-      if (p.dump.codes != nullptr && row < p.N) {
+      if (DUMP && row < p.N) {
         // debug view of this tile: the codes and scales as they go to the
         // PV MMA, the running max, and (on the path that forms P) sum(P)
         const int64_t rt = (static_cast<int64_t>(bhq) * p.N + row) * p.nkt_all + j;
@@ -847,6 +847,9 @@ bool make_tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner_bytes, uint6
 template <int D, int BN, int FMT, bool PRE>
 static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const uint8_t* vc, const AttnParams& p,
                                   cudaStream_t st) {
+  // the P-hat dump (a debug view) is its own instantiation: the production
+  // kernel carries none of its code
+  const bool dump = p.dump.codes != nullptr;
   using C = AttnCfg<D, BN, FMT>;
   CUtensorMap tq, tk, tv;
   const uint64_t Np = static_cast<uint64_t>(p.Np);
@@ -859,7 +862,7 @@ static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const ui
     set_last_error("cuTensorMapEncodeTiled failed");
     return HIFA4_ERR_CUDA;
   }
-  auto kern = attn_fwd_fp4_kernel<D, BN, FMT, PRE>;
+  auto kern = dump ? attn_fwd_fp4_kernel<D, BN, FMT, PRE, true> : attn_fwd_fp4_kernel<D, BN, FMT, PRE, false>;
   const int smem = C::SMEM_REQ;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * p.num_qtiles;
