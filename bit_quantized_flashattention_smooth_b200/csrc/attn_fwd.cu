@@ -58,6 +58,11 @@
 #ifndef HIFA4_ATTN_CORR
 #define HIFA4_ATTN_CORR 0
 #endif
+// 1: two MMA-issuing warps, one for S = Q K^T and one for O += P V, so that
+// the next tile's S never queues behind the previous tile's PV issue
+#ifndef HIFA4_TWO_ISSUERS
+#define HIFA4_TWO_ISSUERS 0
+#endif
 
 namespace hifa4 {
 
@@ -97,9 +102,6 @@ struct AttnCfg {
   // correction warps (4, one per TMEM lane quadrant) rescale the O rows
   // when the running max rises, off the softmax warps' path
   static constexpr int CORR = (NH == 1 && HIFA4_ATTN_CORR) ? 1 : 0;
-  static constexpr int WARP_TMA = 4 * NH + 4 * CORR;
-  static constexpr int WARP_MMA = WARP_TMA + 1;
-  static constexpr int NTHREADS = 32 * (WARP_MMA + 1);
   static constexpr int NS = D == 256 ? 2 : 3;               // K/V pipeline stages
   static constexpr int QROW = D / 2;                        // bytes per Q/K row
   static constexpr int PROW = BN / 2;                       // bytes per P-hat / V^T row
@@ -107,27 +109,42 @@ struct AttnCfg {
   static constexpr int KSTEPS_P = BN / 64;
   static constexpr int NKC_Q = (D / BETA + 3) / 4;          // scale chunks per Q/K row group
   static constexpr int NRG_V = (D + 127) / 128;             // 128-row groups of V^T
+  // The fused normalizer's 16 all-ones rows follow the V^T rows of every V
+  // stage, so one MMA of N = D + 16 writes O and L; otherwise a second
+  // N = 16 MMA reads a separate ones tile.
+  // (D a multiple of 128 keeps the ones rows in a scale row group of their
+  // own; with D = 64 they would fall among V's zero-padded scale rows)
+  static constexpr bool FUSE_L = D == 128;
+  static constexpr int NRG_B = NRG_V + (FUSE_L ? 1 : 0);    // B-operand row groups of the PV MMA
   static constexpr int NCH_V = (BN / BETA + 3) / 4;         // V^T scale chunks per tile per row group
   static constexpr int NKC_P = (BN / BETA + 3) / 4;         // P-hat scale chunks per tile
   // TMEM columns with `nsb` S buffers: S, O, L (16), scale regions.
   static constexpr int cols(int nsb) {
-    return nsb * BN + D + 16 + 8 * NKC_Q + 4 * NKC_P + 4 * NCH_V * NRG_V + 4;
+    return nsb * BN + D + 16 + 8 * NKC_Q + 4 * NKC_P + 4 * NCH_V * NRG_B + (FUSE_L ? 0 : 4);
   }
   // Prefer a footprint of 256 columns so that two CTAs share an SM (twice the
   // softmax warps per scheduler); otherwise own all 512 columns.
   static constexpr int NSB = cols(2) <= 256 ? 2 : (cols(1) <= 256 ? 1 : (cols(2) <= 512 ? 2 : 1));
   static constexpr int TMEM_ALLOC = cols(NSB) <= 256 ? 256 : 512;
   static constexpr int CTAS_PER_SM = TMEM_ALLOC == 256 ? 2 : 1;
+  // a second MMA-issuing warp where the register file allows it (two CTAs of
+  // two softmax warpgroups each would leave too few registers per thread)
+  static constexpr int TWO_ISSUERS = (HIFA4_TWO_ISSUERS && (NH == 1 || CTAS_PER_SM == 1)) ? 1 : 0;
+  static constexpr int WARP_TMA = 4 * NH + 4 * CORR;
+  static constexpr int WARP_MMA = WARP_TMA + 1;             // issues S (and PV with one issuer)
+  static constexpr int WARP_PV = WARP_MMA + TWO_ISSUERS;     // issues PV
+  static constexpr int NTHREADS = 32 * (WARP_PV + 1);
   // shared memory layout (byte offsets; operand tiles 1024-aligned)
   static constexpr int SZ_Q = BM * QROW;
   static constexpr int SZ_K = BN * QROW;
   static constexpr int SZ_V = D * PROW;
   static constexpr int SZ_P = BM * PROW;
   static constexpr int SZ_ONES = 16 * PROW;
+  static constexpr int SZ_VX = SZ_V + (FUSE_L ? SZ_ONES : 0);   // a V stage: the V^T tile, then the ones rows
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + SZ_Q;
   static constexpr int OFF_V = OFF_K + NS * SZ_K;
-  static constexpr int OFF_P = OFF_V + NS * SZ_V;
+  static constexpr int OFF_P = OFF_V + NS * SZ_VX;
   static constexpr int OFF_ONES = OFF_P + 2 * SZ_P;
   static constexpr int OFF_QSF = (OFF_ONES + SZ_ONES + 1023) / 1024 * 1024;
   static constexpr int OFF_KSF = OFF_QSF + NKC_Q * 512;
@@ -153,8 +170,10 @@ struct AttnCfg {
   static constexpr int TM_SFB_K = TM_SFA_Q + 4 * NKC_Q;
   static constexpr int TM_SFA_P = TM_SFB_K + 4 * NKC_Q;
   static constexpr int TM_SFB_V = TM_SFA_P + 4 * NKC_P;
-  static constexpr int TM_SFB_1 = TM_SFB_V + 4 * NCH_V * NRG_V;
-  static constexpr int TM_COLS_USED = TM_SFB_1 + 4;
+  // V^T scale chunk (lc, row group rg) at TM_SFB_V + 4 * (lc * NRG_B + rg);
+  // with FUSE_L, group NRG_V of every chunk holds the ones rows' scales
+  static constexpr int TM_SFB_1 = TM_SFB_V + 4 * NCH_V * NRG_B;
+  static constexpr int TM_COLS_USED = TM_SFB_1 + (FUSE_L ? 0 : 4);
   static_assert(TM_COLS_USED <= TMEM_ALLOC, "TMEM budget");
   // Dynamic shared memory requested: enough that at most CTAS_PER_SM CTAs are
   // resident (a further CTA would stall in tcgen05.alloc).
@@ -290,8 +309,12 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
   }
   // constant operands of the fused normalizer: 16 rows of E2M1 1.0 (code 2)
   // and their scale chunk (scale 1.0 for rows 0..15 in every block byte).
-  for (int i = threadIdx.x; i < C::SZ_ONES / 4; i += blockDim.x)
+  for (int i = threadIdx.x; i < C::SZ_ONES / 4; i += blockDim.x) {
     reinterpret_cast<uint32_t*>(smem + C::OFF_ONES)[i] = 0x22222222u;
+    if constexpr (C::FUSE_L)
+      for (int st = 0; st < C::NS; ++st)
+        reinterpret_cast<uint32_t*>(smem + C::OFF_V + st * C::SZ_VX + C::SZ_V)[i] = 0x22222222u;
+  }
   for (int i = threadIdx.x; i < 128; i += blockDim.x) {
     const uint32_t one = FMT == HIFA4_NVFP4 ? 0x38u : 0x7Fu;
     // word i of the chunk sits at byte 4*i: line (i/4) = row%32, word (i%4) = row/32
@@ -344,7 +367,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
                   C::NKC_Q * 512, BAR(B_KFULL + st));
         if (!mbar_wait(BAR(B_VEMPTY + st), ph ^ 1, abort_flag, kErrTimeoutTma)) break;
         mbar_arrive_expect_tx(BAR(B_VFULL + st), C::SZ_V + C::NRG_V * C::NCH_V * 512);
-        tma_load_2d(sbase + C::OFF_V + st * C::SZ_V, &tm_v, j * C::PROW, kvbh * D, BAR(B_VFULL + st));
+        tma_load_2d(sbase + C::OFF_V + st * C::SZ_VX, &tm_v, j * C::PROW, kvbh * D, BAR(B_VFULL + st));
         const int chunk0 = (j * BN) / (4 * C::BETA);
         for (int rg = 0; rg < C::NRG_V; ++rg)
           bulk_load(sbase + C::OFF_VSF + (st * C::NRG_V + rg) * C::NCH_V * 512,
@@ -352,20 +375,38 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
                     C::NCH_V * 512, BAR(B_VFULL + st));
       }
     }
-  } else if (warp == C::WARP_MMA) {
-    // ================================ MMA issuer ================================
+  } else if (warp == C::WARP_MMA || warp == C::WARP_PV) {
+    // ================================ MMA issuers ================================
+    // With two issuers, warp WARP_MMA issues every S = Q K_j^T as soon as its
+    // K tile has landed and the S buffer is free, and warp WARP_PV every
+    // O += P-hat V_j as soon as P-hat_j is written; they touch disjoint TMEM
+    // columns and shared memory.  With one, WARP_MMA interleaves both.
+    const bool s_role = warp == C::WARP_MMA;
+    const bool pv_role = warp == C::WARP_PV;
     if (lane == 0) {
       constexpr bool MX = FMT == HIFA4_MXFP4;
       auto mma = [&](uint32_t d_t, uint64_t a, uint64_t bdesc, uint32_t idesc, uint32_t sfa, uint32_t sfb, uint32_t acc) {
         if constexpr (MX) mma_mxfp4(d_t, a, bdesc, idesc, sfa, sfb, acc);
         else mma_nvfp4(d_t, a, bdesc, idesc, sfa, sfb, acc);
       };
-      bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, kErrTimeoutMma);
-      if (ok) {
-        tc_fence_after();
-        for (int kc = 0; kc < C::NKC_Q; ++kc)
-          tc_cp_32x128b_warpx4(tmem + C::TM_SFA_Q + 4 * kc, make_sf_desc(sbase + C::OFF_QSF + kc * 512));
-        tc_cp_32x128b_warpx4(tmem + C::TM_SFB_1, make_sf_desc(sbase + C::OFF_ONESF));
+      bool ok = true;
+      if (s_role) {
+        ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, kErrTimeoutMma);
+        if (ok) {
+          tc_fence_after();
+          for (int kc = 0; kc < C::NKC_Q; ++kc)
+            tc_cp_32x128b_warpx4(tmem + C::TM_SFA_Q + 4 * kc, make_sf_desc(sbase + C::OFF_QSF + kc * 512));
+        }
+      }
+      if (pv_role) {
+        // scales of the fused normalizer's ones rows (constant, written at setup)
+        if constexpr (C::FUSE_L) {
+          for (int lc = 0; lc < C::NCH_V; ++lc)
+            tc_cp_32x128b_warpx4(tmem + C::TM_SFB_V + 4 * (lc * C::NRG_B + C::NRG_V),
+                                 make_sf_desc(sbase + C::OFF_ONESF));
+        } else {
+          tc_cp_32x128b_warpx4(tmem + C::TM_SFB_1, make_sf_desc(sbase + C::OFF_ONESF));
+        }
       }
       // S_j = Q K_j^T into S buffer j % NSB
       auto issue_s = [&](int j) -> bool {
@@ -375,9 +416,13 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         if (!mbar_wait(BAR(B_KFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
         if (!mbar_wait(BAR(B_SEMPTY + sb), ((j / C::NSB) & 1) ^ 1, abort_flag, kErrTimeoutMma)) return false;
         tc_fence_after();
-        for (int kc = 0; kc < C::NKC_Q; ++kc)
-          tc_cp_32x128b_warpx4(tmem + C::TM_SFB_K + 4 * kc,
-                               make_sf_desc(sbase + C::OFF_KSF + st * C::NKC_Q * 512 + kc * 512));
+        // 64-key tiles: a 128-row chunk of K scales serves tiles 2i and 2i+1,
+        // so it is copied on even tiles only (the copy of tile 2i+2 is issued
+        // after, and so executes after, the MMAs of tile 2i+1)
+        if (!(BN == 64 && (j & 1)))
+          for (int kc = 0; kc < C::NKC_Q; ++kc)
+            tc_cp_32x128b_warpx4(tmem + C::TM_SFB_K + 4 * kc,
+                                 make_sf_desc(sbase + C::OFF_KSF + st * C::NKC_Q * 512 + kc * 512));
         const uint32_t half_off = (BN == 64 && (j & 1)) ? 2u : 0u;  // rows 64..127 of the K row group
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS_S; ++ks) {
@@ -393,7 +438,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         tc_commit(BAR(B_KEMPTY + st));
         return true;
       };
-      // O += P-hat V-hat_j ; L += P-hat ones
+      // O += P-hat V-hat_j ; L += P-hat ones (the same MMA when FUSE_L)
       auto issue_pv = [&](int j) -> bool {
         const int st = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
@@ -415,7 +460,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
                                make_sf_desc(sbase + C::OFF_PSF + pb * C::NKC_P * 512 + pc * 512));
         for (int lc = 0; lc < C::NCH_V; ++lc)
           for (int rg = 0; rg < C::NRG_V; ++rg)
-            tc_cp_32x128b_warpx4(tmem + C::TM_SFB_V + 4 * (lc * C::NRG_V + rg),
+            tc_cp_32x128b_warpx4(tmem + C::TM_SFB_V + 4 * (lc * C::NRG_B + rg),
                                  make_sf_desc(sbase + C::OFF_VSF + ((st * C::NRG_V + rg) * C::NCH_V + lc) * 512));
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS_P; ++ks) {
@@ -425,23 +470,37 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
           const uint32_t vchunk = kk / (4 * C::BETA) - (j * BN) / (4 * C::BETA);
           const uint32_t vbyte = (kk / C::BETA) % 4;
           const uint64_t a = make_kmajor_desc(sbase + C::OFF_P + pb * C::SZ_P + ks * 32, C::PROW);
-          const uint64_t bv = make_kmajor_desc(sbase + C::OFF_V + st * C::SZ_V + ks * 32, C::PROW);
+          const uint64_t bv = make_kmajor_desc(sbase + C::OFF_V + st * C::SZ_VX + ks * 32, C::PROW);
           const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
           const uint32_t sfa = (tmem + C::TM_SFA_P + 4 * pchunk) | (pbyte << 30);
-          mma(tmem + C::TM_O, a, bv, idesc_fp4(128, D, MX, pbyte, vbyte), sfa,
-              (tmem + C::TM_SFB_V + 4 * vchunk * C::NRG_V) | (vbyte << 30), acc);
-          const uint64_t b1 = make_kmajor_desc(sbase + C::OFF_ONES + ks * 32, C::PROW);
-          mma(tmem + C::TM_L, a, b1, idesc_fp4(128, 16, MX, pbyte, pbyte), sfa,
-              (tmem + C::TM_SFB_1) | (pbyte << 30), acc);
+          if constexpr (C::FUSE_L) {
+            // B = [V^T tile; 16 ones rows]: columns D..D+15 of the result, L,
+            // follow O in TMEM
+            mma(tmem + C::TM_O, a, bv, idesc_fp4(128, D + 16, MX, pbyte, vbyte), sfa,
+                (tmem + C::TM_SFB_V + 4 * vchunk * C::NRG_B) | (vbyte << 30), acc);
+          } else {
+            mma(tmem + C::TM_O, a, bv, idesc_fp4(128, D, MX, pbyte, vbyte), sfa,
+                (tmem + C::TM_SFB_V + 4 * vchunk * C::NRG_B) | (vbyte << 30), acc);
+            const uint64_t b1 = make_kmajor_desc(sbase + C::OFF_ONES + ks * 32, C::PROW);
+            mma(tmem + C::TM_L, a, b1, idesc_fp4(128, 16, MX, pbyte, pbyte), sfa,
+                (tmem + C::TM_SFB_1) | (pbyte << 30), acc);
+          }
         }
         tc_commit(BAR(B_VEMPTY + st));
         tc_commit(BAR(B_PEMPTY + pb));
         return true;
       };
-      if (ok && nkt > 0) ok = issue_s(0);
-      for (int j = 0; ok && j < nkt; ++j) {
-        if (j + 1 < nkt) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
+      if constexpr (C::TWO_ISSUERS) {
+        if (s_role)
+          for (int j = 0; ok && j < nkt; ++j) ok = issue_s(j);
+        else
+          for (int j = 0; ok && j < nkt; ++j) ok = issue_pv(j);
+      } else {
+        if (ok && nkt > 0) ok = issue_s(0);
+        for (int j = 0; ok && j < nkt; ++j) {
+          if (j + 1 < nkt) ok = issue_s(j + 1);
+          if (ok) ok = issue_pv(j);
+        }
       }
       if (!ok) drain_after_abort();
     }
