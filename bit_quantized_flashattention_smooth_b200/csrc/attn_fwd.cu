@@ -773,11 +773,20 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
           else atomicAdd(p.dump.sum_p + rt, psum);     // two column halves; the caller zero-fills
         }
       }
-      // the P-hat buffer pb was last read by PV_{j-2}
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(BAR(B_PEMPTY + pb), ((j >> 1) & 1) ^ 1, abort_flag,
-                                                        kErrTimeoutSoftmax))) {
-        ok = false;
-        break;
+      // One wait covers both uses of the previous product: PV_{j-1} done
+      // means the P-hat buffer pb's last reader PV_{j-2} is done too (a
+      // commit completes only after all earlier MMAs of its thread), and the
+      // O rescale below may then touch O.  (PV_{j-1}'s barrier is phase
+      // (j-1)/2 of buffer (j-1)%2, whose earlier phase PV_{j-3} completed
+      // before tile j-1 passed this point.)  With the correction warps the
+      // rescale is theirs, and only the buffer's reuse is awaited here.
+      if (j >= (C::CORR ? 2 : 1)) {
+        const int jw = C::CORR ? j - 2 : j - 1;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(BAR(B_PEMPTY + (jw & 1)), (jw >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
+          ok = false;
+          break;
+        }
       }
       {
         unsigned char* prow = smem + C::OFF_P + pb * C::SZ_P + r * C::PROW;
@@ -794,15 +803,9 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
           psf[(gb / 4) * 512 + (gb % 4)] = static_cast<unsigned char>(scb[blk]);
         }
       }
-      // rescale this slice of the O row (and L) when the max rose, after
-      // PV_{j-1} retired (awaited on its P-hat buffer's barrier, whose earlier
-      // phase, PV_{j-3}, completed before this tile's P-hat stores)
+      // rescale this slice of the O row (and L) when the max rose (PV_{j-1}
+      // retired: awaited above)
       if (!C::CORR && j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PEMPTY + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag,
-                                               kErrTimeoutSoftmax))) {
-          ok = false;
-          break;
-        }
         tc_fence_after();
         rescale_o_rows<HD>(tmem + lane_base + C::TM_O + hw * HD, tmem + lane_base + C::TM_L, hw == 0, alpha);
         tmem_wait_st();
