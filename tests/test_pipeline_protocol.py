@@ -120,6 +120,8 @@ class Sim:
             if j + 1 < self.nkt:
                 yield from issue_s(j + 1)
             yield from issue_pv(j)
+        # (the kernel's K-scale copy on even tiles only and the normalizer
+        # fused into the PV MMA change no barrier)
 
     def softmax(self, w):
         if self.fused_q:
@@ -141,14 +143,15 @@ class Sim:
                 partner = w ^ 4
                 if self.xm[j & 1].get(partner) != j:
                     raise ProtocolError(f"warp {w} read the row max of tile {self.xm[j & 1].get(partner)} for {j}")
-            if j >= 2:
-                yield from self.wait(f"PEMPTY{pb}", ((j >> 1) & 1) ^ 1, (j >> 1))
+            # one wait for the previous product PV_{j-1}: it also covers the
+            # P-hat buffer's last reader PV_{j-2} (commits complete in order)
+            if j >= 1:
+                yield from self.wait(f"PEMPTY{(j - 1) & 1}", ((j - 1) >> 1) & 1, ((j - 1) >> 1) + 1)
             if self.pv_done < j - 2:
                 raise ProtocolError(f"warp {w} overwrote P-hat buffer {pb} before PV_{j - 2} retired")
             self.p_buf[pb][w] = j
             rescale = j > 0 and self.rng.random() < 0.5
             if rescale:
-                yield from self.wait(f"PEMPTY{(j - 1) & 1}", ((j - 1) >> 1) & 1, ((j - 1) >> 1) + 1)
                 if self.pv_done < j - 1 or self.pv_started >= j:
                     raise ProtocolError(f"warp {w} rescaled O for tile {j} with PV_{self.pv_done} done, "
                                         f"PV_{self.pv_started} started")
