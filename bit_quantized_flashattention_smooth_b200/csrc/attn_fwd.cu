@@ -51,6 +51,14 @@
 #ifndef HIFA4_CODE_MAP
 #define HIFA4_CODE_MAP 1
 #endif
+// 1: where only the P-hat codes are needed, P = 2^(S*c - m) is formed first
+// and multiplied by the block multiplier afterwards (the exponentials then
+// need only the row max, not the block scales); 0: the multiplier is folded
+// into the exponent; -1: per shape (measured: first at d = 256, 1.024 times
+// faster; folded at d = 128, 1.03 times faster)
+#ifndef HIFA4_EXP_FIRST
+#define HIFA4_EXP_FIRST -1
+#endif
 #ifndef HIFA4_ATTN_NH_BN64
 #define HIFA4_ATTN_NH_BN64 1
 #endif
@@ -677,6 +685,9 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       // the stale max and may reach 2^tau.  m = -inf always moves.
       m_new = m_new > m + p.tau ? m_new : m;
       const float alpha = (m_new == m) ? 1.0f : ex2_approx(m - m_new);
+      // whether any row of this warp rescales O (voted early: its latency
+      // hides behind the block scales and the exponentials)
+      const bool warp_rescale = __any_sync(0xffffffffu, m_new != m);
       if constexpr (C::CORR) {
         if (j > 0) {
           reinterpret_cast<float*>(smem + C::OFF_XM)[(j % 3) * 128 + r] = alpha;
@@ -712,11 +723,13 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       // per element would split the block the compiler schedules)
       auto quant_tile = [&](auto lp_tag) {
         constexpr bool LP = decltype(lp_tag)::value;
+        // codes only, exponentials first: P, then P * mult (LP without the sum)
+        constexpr bool MULT = !LP && (HIFA4_EXP_FIRST < 0 ? D == 256 : HIFA4_EXP_FIRST != 0);
         float2 acc = make_float2(0.0f, 0.0f);
         // Without the sum of P, the multiplier folds into the exponent:
         // P * mult = 2^(S*c - m + log2 mult), one packed FMA per pair.
         float lnb[NBH];
-        if constexpr (!LP) {
+        if constexpr (!LP && !MULT) {
 #pragma unroll
           for (int blk = 0; blk < NBH; ++blk) {
             const float lm = FMT == HIFA4_NVFP4 ? log_tab[scb[blk]] : static_cast<float>(127 - static_cast<int>(scb[blk]));
@@ -727,7 +740,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         for (int w = 0; w < HB / 8; ++w) {
           const int blk = (8 * w) / C::BETA;
           const float2 m2 = make_float2(mult[blk], mult[blk]);
-          const float2 nb2 = LP ? nm2 : make_float2(lnb[blk], lnb[blk]);
+          const float2 nb2 = (LP || MULT) ? nm2 : make_float2(lnb[blk], lnb[blk]);
           float2 e[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -737,13 +750,15 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
             float2 pp;
             if (pair16 < kPolyPairs) {
               // codes only (no sum of P): the exponential-free code argument
-              if constexpr (!LP && HIFA4_CODE_MAP) pp = e2m1_arg_from_log2(y);
+              if constexpr (!LP && !MULT && HIFA4_CODE_MAP) pp = e2m1_arg_from_log2(y);
               else pp = exp2_poly2(y);
             } else {
               pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
             }
             if constexpr (LP) {
               acc = fadd2(acc, pp);
+              e[q] = fmul2(pp, m2);
+            } else if constexpr (MULT) {
               e[q] = fmul2(pp, m2);
             } else {
               e[q] = pp;
@@ -797,15 +812,27 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
               make_uint4(codes[4 * ch], codes[4 * ch + 1], codes[4 * ch + 2], codes[4 * ch + 3]);
         }
         unsigned char* psf = smem + C::OFF_PSF + pb * C::NKC_P * 512 + (r & 31) * 16 + (r >> 5) * 4;
+        if constexpr (NBH % 4 == 0) {
+          // whole scale words: this thread's blocks 4i..4i+3 are the 4 bytes of
+          // one word of chunk (hw * NBH) / 4 + i
 #pragma unroll
-        for (int blk = 0; blk < NBH; ++blk) {
-          const int gb = hw * NBH + blk;                       // block index within the tile
-          psf[(gb / 4) * 512 + (gb % 4)] = static_cast<unsigned char>(scb[blk]);
+          for (int wd = 0; wd < NBH / 4; ++wd)
+            *reinterpret_cast<uint32_t*>(psf + ((hw * NBH) / 4 + wd) * 512) =
+                scb[4 * wd] | (scb[4 * wd + 1] << 8) | (scb[4 * wd + 2] << 16) | (scb[4 * wd + 3] << 24);
+        } else if constexpr (NBH == 2) {
+          // two blocks: bytes 2hw, 2hw+1 of the row's word (one chunk per tile)
+          *reinterpret_cast<uint16_t*>(psf + 2 * hw) = static_cast<uint16_t>(scb[0] | (scb[1] << 8));
+        } else {
+#pragma unroll
+          for (int blk = 0; blk < NBH; ++blk) {
+            const int gb = hw * NBH + blk;                     // block index within the tile
+            psf[(gb / 4) * 512 + (gb % 4)] = static_cast<unsigned char>(scb[blk]);
+          }
         }
       }
       // rescale this slice of the O row (and L) when the max rose (PV_{j-1}
       // retired: awaited above)
-      if (!C::CORR && j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+      if (!C::CORR && j > 0 && warp_rescale) {
         tc_fence_after();
         rescale_o_rows<HD>(tmem + lane_base + C::TM_O + hw * HD, tmem + lane_base + C::TM_L, hw == 0, alpha);
         tmem_wait_st();
