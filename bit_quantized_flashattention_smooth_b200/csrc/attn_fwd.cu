@@ -167,7 +167,7 @@ struct AttnCfg {
   static constexpr int OFF_BAR = OFF_LP + 1024;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
   // s_full[NSB], s_empty[NSB], p_full[2], p_empty[2], o_ready
-  static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1 + 3 + 24;
+  static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1 + 3 + 24 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   // TMEM columns
@@ -278,7 +278,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
             B_SFULL = 1 + 4 * C::NS, B_SEMPTY = B_SFULL + C::NSB, B_PFULL = B_SEMPTY + C::NSB,
             B_PEMPTY = B_PFULL + 2, B_ORDY = B_PEMPTY + 2, B_XM = B_ORDY + 1, B_EP1 = B_XM + 1, B_EP2 = B_EP1 + 1,
             B_AF = B_EP2 + 1,   // [quadrant][4]: softmax warp -> correction warp, alpha of tile j ready
-            B_OC = B_AF + 16;   // [quadrant][2]: correction warp -> MMA, O rescaled for PV_j
+            B_OC = B_AF + 16,   // [quadrant][2]: correction warp -> MMA, O rescaled for PV_j
+            B_XQ = B_OC + 8;    // [quadrant]: row-max exchange of the two warps sharing a lane quadrant
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -308,7 +309,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       mbar_init(BAR(B_PFULL + s), 4 * C::NH);
       mbar_init(BAR(B_PEMPTY + s), 1);
     }
-    mbar_init(BAR(B_XM), 8);      // row-max exchange between two column halves (one arrival per warp)
+    mbar_init(BAR(B_XM), 8);      // (unused: the exchange is per lane quadrant, below)
+    for (int q = 0; q < 4; ++q) mbar_init(BAR(B_XQ + q), 2);   // the two warps of quadrant q
     mbar_init(BAR(B_EP1), 4);     // epilogue: half 1 -> half 0
     mbar_init(BAR(B_EP2), 4);     // epilogue: half 0 -> half 1
     for (int i = 0; i < 24; ++i) mbar_init(BAR(B_AF + i), 1);
@@ -671,8 +673,11 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         float* xb = xm + (j & 1) * 256;
         xb[hw * 128 + r] = __fmul_rn(tree_max<NBH>(bms), c);
         __syncwarp();             // the warp's stores are ordered before lane 0's release
-        if (lane == 0) mbar_arrive(BAR(B_XM));
-        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_XM), j & 1, abort_flag, kErrTimeoutSoftmax))) {
+        // only the two warps that share these rows synchronize (phase j of
+        // their quadrant's barrier; neither can arrive for tile j+1 before
+        // both passed tile j, so a parity wait is exact)
+        if (lane == 0) mbar_arrive(BAR(B_XQ + (warp & 3)));
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_XQ + (warp & 3)), j & 1, abort_flag, kErrTimeoutSoftmax))) {
           ok = false;
           break;
         }

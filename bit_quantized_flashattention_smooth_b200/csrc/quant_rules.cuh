@@ -55,19 +55,15 @@ __device__ __forceinline__ void load8<__half>(const __half* p, float (&f)[8]) {
   }
 }
 
-// Quantize one block of BETA fp32 values in place into packed codes
-// (BETA/2 bytes, element 2i in the low nibble) and return the scale code.
-// inv_tab[c] = fl32(1 / UE4M3(c)) * 2^TAB_LOG2 (0 for c = 0), in shared
-// memory; the power of two is taken out exactly.
-template <int FMT, int BETA, int TAB_LOG2 = 0>
-__device__ __forceinline__ uint32_t quant_block(const float (&v)[BETA], uint32_t (&packed)[BETA / 8],
-                                                const float* inv_tab) {
-  float amax = fmaxf(fabsf(v[0]), fabsf(v[1]));
-#pragma unroll
-  for (int i = 2; i + 1 < BETA; i += 2) amax = fmax3(amax, fabsf(v[i]), fabsf(v[i + 1]));
-  float mult;
+// The scale decision of one block from its amax: returns the scale code and
+// sets the element multiplier fl32(1/scale) and the code mask (0 when the
+// scale is 0, so that no -0 codes appear).  inv_tab[c] = fl32(1 / UE4M3(c)) *
+// 2^TAB_LOG2 (0 for c = 0), in shared memory; the power of two is taken out
+// exactly.
+template <int FMT, int TAB_LOG2 = 0>
+__device__ __forceinline__ uint32_t block_scale(float amax, const float* inv_tab, float& mult, uint32_t& keep) {
   uint32_t sc;
-  uint32_t keep = 0xFFFFFFFFu;
+  keep = 0xFFFFFFFFu;
   if constexpr (FMT == HIFA4_NVFP4) {
     // fl32(amax/6): the reciprocal-and-residual form is IEEE-exact on
     // [2^-122, 2^20] (checked on the GPU); below, both give scale code 0
@@ -80,6 +76,20 @@ __device__ __forceinline__ uint32_t quant_block(const float (&v)[BETA], uint32_t
     sc = ef >= 2u ? ef - 2u : 0u;                       // E + 127, E = floor(log2 amax) - 2
     mult = __uint_as_float((254u - sc) << 23);          // 2^-E
   }
+  return sc;
+}
+
+// Quantize one block of BETA fp32 values in place into packed codes
+// (BETA/2 bytes, element 2i in the low nibble) and return the scale code.
+template <int FMT, int BETA, int TAB_LOG2 = 0>
+__device__ __forceinline__ uint32_t quant_block(const float (&v)[BETA], uint32_t (&packed)[BETA / 8],
+                                                const float* inv_tab) {
+  float amax = fmaxf(fabsf(v[0]), fabsf(v[1]));
+#pragma unroll
+  for (int i = 2; i + 1 < BETA; i += 2) amax = fmax3(amax, fabsf(v[i]), fabsf(v[i + 1]));
+  float mult;
+  uint32_t keep;
+  const uint32_t sc = block_scale<FMT, TAB_LOG2>(amax, inv_tab, mult, keep);
   const float2 m2 = make_float2(mult, mult);
 #pragma unroll
   for (int w = 0; w < BETA / 8; ++w) {

@@ -42,6 +42,18 @@ struct RowTile {
   static_assert(128 % ROWS == 0, "a CTA's rows stay inside one head");
 };
 
+// Element ch (0: low half, 1: high half) of a packed pair of 16-bit floats,
+// exactly in fp32.
+template <typename T>
+__device__ __forceinline__ float chan_of(uint32_t w, int ch);
+template <>
+__device__ __forceinline__ float chan_of<__nv_bfloat16>(uint32_t w, int ch) {
+  return __uint_as_float(ch == 0 ? (w << 16) : (w & 0xFFFF0000u));
+}
+template <>
+__device__ __forceinline__ float chan_of<__half>(uint32_t w, int ch) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(ch == 0 ? (w & 0xFFFFu) : (w >> 16))));
+}
 // One lane's 8 values of a BETA-block spread over LPB = BETA/8 adjacent lanes:
 // the block's scale code (the same in every lane of the block) and this lane's
 // 8 E2M1 codes packed in a word, by exactly the rules of quant_block.
@@ -89,17 +101,15 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
   const int ch = lane % CPR;               // 16-byte chunk of the row
   const int blk = ch / LPB;                // its block
   const T* xh = x + static_cast<int64_t>(bh) * N * D + ch * 8;
-  float v[U][8];
+  // all U loads in flight at once, kept packed (4 registers each) until their
+  // row group is quantized
+  uint4 raw[U];
   int tok[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     tok[u] = chunk * R::ROWS + (warp * U + u) * RPI + lane / CPR;
-    if (tok[u] < N) {
-      load8<T>(xh + static_cast<int64_t>(tok[u]) * D, v[u]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
-    }
+    raw[u] = tok[u] < N ? *reinterpret_cast<const uint4*>(xh + static_cast<int64_t>(tok[u]) * D)
+                        : make_uint4(0u, 0u, 0u, 0u);
   }
   float sv[8];
   if (scale != nullptr) {
@@ -112,16 +122,25 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const int t = tok[u];
+    float v[8];
+    {
+      const uint32_t wd[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = chan_of<T>(wd[i], 0);
+        v[2 * i + 1] = chan_of<T>(wd[i], 1);
+      }
+    }
     if (scale != nullptr && t < N) {
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
-        const float2 p2 = qmul2(make_float2(v[u][i], v[u][i + 1]), make_float2(sv[i], sv[i + 1]));
-        v[u][i] = p2.x;
-        v[u][i + 1] = p2.y;
+        const float2 p2 = qmul2(make_float2(v[i], v[i + 1]), make_float2(sv[i], sv[i + 1]));
+        v[i] = p2.x;
+        v[i + 1] = p2.y;
       }
     }
     uint32_t packed;
-    const uint32_t sc = quant_part<FMT, BETA>(v[u], packed, inv_tab);
+    const uint32_t sc = quant_part<FMT, BETA>(v, packed, inv_tab);
     *reinterpret_cast<uint32_t*>(cbase + static_cast<int64_t>(t) * (D / 2)) = packed;
     if (ch % LPB == 0) {
       uint8_t* sfw = sh + sf_word_offset(t, blk / 4, WPR);
@@ -136,103 +155,124 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
   }
 }
 
-// V: one CTA per (128-token tile, head, 64-channel group).  The tile is staged
-// in shared memory with coalesced 16-byte loads; then one thread per (channel,
-// token block) quantizes the block (the 32 lanes of a warp read 32 adjacent
-// channels of a token: one shared-memory wavefront) and writes the scale
-// byte, and the codes go through a second staging buffer so that each
-// channel-major V^T row's 64 code bytes of the tile are written by 16-byte
-// stores of consecutive threads.
-constexpr int kVCh = 64;   // channels per V CTA
+// V: one warp per (head, 32-token chunk, 64-channel group), quantized along
+// tokens in registers.  Lane l owns channels c = 64g + 2l and c + 1: for each
+// of the chunk's 32 tokens it loads the two channels' values as one 32-bit
+// word (the warp's 32 words of a token are one contiguous 128-byte line), then
+// quantizes each channel's blocks of BETA tokens by the rules of quant_block
+// and writes the channel's 16 code bytes of the chunk (one V^T row segment)
+// and its block scale bytes directly.  Tokens N..Np-1 are zero padding.
+constexpr int kVCh = 64;   // channels per V warp task
+constexpr int kVTok = 32;  // tokens per V warp task
+template <typename T>
+__device__ __forceinline__ float2 unpack_pair(uint32_t w);
+template <>
+__device__ __forceinline__ float2 unpack_pair<__nv_bfloat16>(uint32_t w) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+}
+template <>
+__device__ __forceinline__ float2 unpack_pair<__half>(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+// Element-wise max of |x| over two packed 16-bit values: an exact selection,
+// so the block amax of each channel can be taken before any conversion.
+template <typename T>
+__device__ __forceinline__ uint32_t absmax_pair(uint32_t a, uint32_t b);
+template <>
+__device__ __forceinline__ uint32_t absmax_pair<__nv_bfloat16>(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmax2(__habs2(*reinterpret_cast<const __nv_bfloat162*>(&a)),
+                             __habs2(*reinterpret_cast<const __nv_bfloat162*>(&b)));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+template <>
+__device__ __forceinline__ uint32_t absmax_pair<__half>(uint32_t a, uint32_t b) {
+  __half2 r = __hmax2(__habs2(*reinterpret_cast<const __half2*>(&a)), __habs2(*reinterpret_cast<const __half2*>(&b)));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
 template <int FMT, typename T>
-__device__ __forceinline__ void quantize_v_tile(const T* __restrict__ v, int N, int Np, int d,
+__device__ __forceinline__ void quantize_v_cols(const T* __restrict__ v, int N, int Np, int d,
                                                 uint8_t* __restrict__ vt_codes, uint8_t* __restrict__ vt_sf,
-                                                int64_t sf_head_bytes, int tile, T* tile_smem,
-                                                unsigned char* code_stage, const float* inv_tab) {
+                                                int64_t sf_head_bytes, int64_t task, const float* inv_tab) {
   constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
+  constexpr int NBLK = kVTok / BETA;             // blocks of the chunk per channel
+  const int lane = threadIdx.x & 31;
   const int ncg = d / kVCh;
-  const int cg = tile % ncg;
-  const int64_t bhx = tile / ncg;          // head * (Np / 128) + token tile
-  const int ntt = Np / 128;
-  const int t0 = static_cast<int>(bhx % ntt) * 128;
-  const int64_t head = bhx / ntt;
-  const int c_base = cg * kVCh;
-  constexpr int VEC = kVCh / 8;   // 16-byte vectors per token row
-  for (int i = threadIdx.x; i < 128 * VEC; i += blockDim.x) {
-    const int r = i / VEC, cv = i % VEC;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (t0 + r < N)
-      u = *reinterpret_cast<const uint4*>(v + (head * N + t0 + r) * static_cast<int64_t>(d) + c_base + cv * 8);
-    *reinterpret_cast<uint4*>(tile_smem + r * kVCh + cv * 8) = u;
+  const int nchunk = Np / kVTok;
+  const int cg = static_cast<int>(task % ncg);
+  const int64_t rest = task / ncg;
+  const int t0 = static_cast<int>(rest % nchunk) * kVTok;
+  const int64_t head = rest / nchunk;
+  const int c = cg * kVCh + 2 * lane;
+  const int nkc = Np / (4 * BETA);               // scale chunks per 128-row group of V^T
+  uint32_t w[kVTok];
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(v + (head * N + t0) * static_cast<int64_t>(d) + c);
+#pragma unroll
+  for (int i = 0; i < kVTok; ++i) w[i] = (t0 + i < N) ? src[static_cast<int64_t>(i) * (d / 2)] : 0u;
+  uint32_t codes0[kVTok / 8], codes1[kVTok / 8];
+  uint32_t scw0 = 0, scw1 = 0;
+#pragma unroll
+  for (int b = 0; b < NBLK; ++b) {
+    // both channels' block amax at once (exact), then each channel's scale
+    uint32_t am = absmax_pair<T>(w[b * BETA], w[b * BETA + 1]);
+#pragma unroll
+    for (int i = 2; i < BETA; ++i) am = absmax_pair<T>(am, w[b * BETA + i]);
+    const float2 amf = unpack_pair<T>(am);
+    float mult0, mult1;
+    uint32_t keep0, keep1;
+    scw0 |= block_scale<FMT>(amf.x, inv_tab, mult0, keep0) << (8 * b);
+    scw1 |= block_scale<FMT>(amf.y, inv_tab, mult1, keep1) << (8 * b);
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+      const float2 m2 = ch == 0 ? make_float2(mult0, mult0) : make_float2(mult1, mult1);
+      const uint32_t keep = ch == 0 ? keep0 : keep1;
+#pragma unroll
+      for (int q = 0; q < BETA / 8; ++q) {
+        const uint32_t* e = w + b * BETA + 8 * q;
+        const uint32_t cw = keep & cvt_e2m1x8(qmul2(make_float2(chan_of<T>(e[0], ch), chan_of<T>(e[1], ch)), m2),
+                                              qmul2(make_float2(chan_of<T>(e[2], ch), chan_of<T>(e[3], ch)), m2),
+                                              qmul2(make_float2(chan_of<T>(e[4], ch), chan_of<T>(e[5], ch)), m2),
+                                              qmul2(make_float2(chan_of<T>(e[6], ch), chan_of<T>(e[7], ch)), m2));
+        if (ch == 0) codes0[b * (BETA / 8) + q] = cw;
+        else codes1[b * (BETA / 8) + q] = cw;
+      }
+    }
   }
-  __syncthreads();
-  const int words_per_ch = 128 / (4 * BETA);
-  const int nkc = Np / (4 * BETA);
+  const int gb = t0 / BETA;                      // the chunk's NBLK blocks: consecutive bytes of one word
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    const int cc = c + ch;
+    const uint32_t* cw = ch == 0 ? codes0 : codes1;
+    *reinterpret_cast<uint4*>(vt_codes + (head * d + cc) * static_cast<int64_t>(Np / 2) + t0 / 2) =
+        make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    uint8_t* sfw = vt_sf + head * sf_head_bytes + sf_word_offset(cc, gb / 4, nkc) + (gb % 4);
+    const uint32_t scw = ch == 0 ? scw0 : scw1;
+    if constexpr (NBLK == 2) *reinterpret_cast<uint16_t*>(sfw) = static_cast<uint16_t>(scw);
+    else *sfw = static_cast<uint8_t>(scw);
+  }
   if (cg == 0 && d < 128) {
     // rows d..127 of the 128-row scale group are padding (d = 64): zero them
-    for (int task = threadIdx.x; task < (128 - d) * words_per_ch; task += blockDim.x) {
-      const int c = d + task % (128 - d), w = task / (128 - d);
-      *reinterpret_cast<uint32_t*>(vt_sf + head * sf_head_bytes + sf_word_offset(c, t0 / (4 * BETA) + w, nkc)) = 0u;
+    for (int r = d + lane; r < 128; r += 32) {
+      uint8_t* sfw = vt_sf + head * sf_head_bytes + sf_word_offset(r, gb / 4, nkc) + (gb % 4);
+      if constexpr (NBLK == 2) *reinterpret_cast<uint16_t*>(sfw) = 0;
+      else *sfw = 0;
     }
-  }
-  // one task per (channel, token block): all threads busy, codes and the
-  // scale byte written per block
-  for (int task = threadIdx.x; task < kVCh * (128 / BETA); task += blockDim.x) {
-    const int cl = task % kVCh, blk = task / kVCh;
-    const int c = c_base + cl;
-    float val[BETA];
-#pragma unroll
-    for (int i = 0; i < BETA; ++i) {
-      const int tt = blk * BETA + i;
-      if constexpr (std::is_same<T, __nv_bfloat16>::value)
-        val[i] = __bfloat162float(tile_smem[tt * kVCh + cl]);
-      else
-        val[i] = __half2float(tile_smem[tt * kVCh + cl]);
-    }
-    uint32_t packed[BETA / 8];
-    const uint32_t sc = quant_block<FMT, BETA>(val, packed, inv_tab);
-    // codes staged per channel row (64 bytes = 128 tokens), pieces swizzled
-    // by the channel so that the 32 channels of a warp spread over the banks
-    unsigned char* srow = code_stage + cl * 64;
-    if constexpr (BETA == 16)
-      *reinterpret_cast<uint2*>(srow + ((blk ^ (cl & 7)) * 8)) = make_uint2(packed[0], packed[1]);
-    else
-      *reinterpret_cast<uint4*>(srow + ((blk ^ (cl & 3)) * 16)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    const int gb = t0 / BETA + blk;                   // block index along the row
-    vt_sf[head * sf_head_bytes + sf_word_offset(c, gb / 4, nkc) + (gb % 4)] = static_cast<uint8_t>(sc);
-  }
-  __syncthreads();
-  // each V^T row's 64 code bytes of this tile leave as four 16-byte stores
-  for (int i = threadIdx.x; i < kVCh * 4; i += blockDim.x) {
-    const int cl = i / 4, q = i % 4;
-    const unsigned char* srow = code_stage + cl * 64;
-    uint4 u;
-    if constexpr (BETA == 16) {
-      const uint2 lo = *reinterpret_cast<const uint2*>(srow + (((2 * q) ^ (cl & 7)) * 8));
-      const uint2 hi = *reinterpret_cast<const uint2*>(srow + (((2 * q + 1) ^ (cl & 7)) * 8));
-      u = make_uint4(lo.x, lo.y, hi.x, hi.y);
-    } else {
-      u = *reinterpret_cast<const uint4*>(srow + ((q ^ (cl & 3)) * 16));
-    }
-    *reinterpret_cast<uint4*>(vt_codes + (head * d + c_base + cl) * static_cast<int64_t>(Np / 2) + t0 / 2 + q * 16) = u;
   }
 }
 
-// One launch for the whole step: CTAs [0, nv) quantize V tiles, the next nq
-// Q rows, the rest K rows.
+// One launch for the whole step: CTAs [0, nv) quantize V (8 warp tasks each),
+// the next nq Q rows, the rest K rows.
 struct QuantArgs {
   const void *q, *k, *v;
   const float *s, *inv_s;
   uint8_t *qc, *qs, *kc, *ks, *vc, *vs;
   int B, Hq, Hkv, N, Np, d;
-  int64_t sf_qk_head, sf_v_head, q_rows, k_rows;
+  int64_t sf_qk_head, sf_v_head, q_rows, k_rows, v_tasks;
   int nq_ctas, nk_ctas, nv_ctas;
 };
 
 template <int FMT, typename T, int D>
 __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a) {
-  __shared__ __align__(16) T tile_smem[128 * kVCh];
-  __shared__ __align__(16) unsigned char code_stage[kVCh * 64];
   __shared__ float inv_tab[128];
   if (FMT == HIFA4_NVFP4 && threadIdx.x < 128)
     inv_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __fdiv_rn(1.0f, ue4m3_to_f32(threadIdx.x));
@@ -240,8 +280,9 @@ __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a)
   // V tiles first (the longest CTAs start early), then Q rows, then K rows
   const int bid = static_cast<int>(blockIdx.x) - a.nv_ctas;
   if (bid < 0) {
-    quantize_v_tile<FMT, T>(static_cast<const T*>(a.v), a.N, a.Np, a.d, a.vc, a.vs, a.sf_v_head,
-                            static_cast<int>(blockIdx.x), tile_smem, code_stage, inv_tab);
+    const int64_t task = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (task < a.v_tasks)
+      quantize_v_cols<FMT, T>(static_cast<const T*>(a.v), a.N, a.Np, a.d, a.vc, a.vs, a.sf_v_head, task, inv_tab);
   } else if (bid < a.nq_ctas) {
     quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.s, a.qc, a.qs,
                                  a.sf_qk_head, bid, inv_tab);
@@ -351,7 +392,8 @@ hifa4_status quantize_qkv_launch(const void* q, const void* k, const void* v, in
                                    : (d == 128 ? RowTile<HIFA4_NVFP4, 128>::ROWS : RowTile<HIFA4_NVFP4, 256>::ROWS);
   a.nq_ctas = static_cast<int>(a.q_rows / rows_per_cta);    // Np is a multiple of 128, rows_per_cta divides 128
   a.nk_ctas = static_cast<int>(a.k_rows / rows_per_cta);
-  a.nv_ctas = (a.Np / 128) * (a.B * a.Hkv) * (a.d / kVCh);
+  a.v_tasks = static_cast<int64_t>(a.Np / kVTok) * (a.B * a.Hkv) * (a.d / kVCh);   // one warp each
+  a.nv_ctas = static_cast<int>((a.v_tasks + 7) / 8);
   if (dt == HIFA4_BF16) launch_quant<__nv_bfloat16>(a, fmt, st);
   else launch_quant<__half>(a, fmt, st);
   return launch_status(q ? "quantize_qkv" : "quantize_kv");

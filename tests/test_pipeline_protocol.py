@@ -55,7 +55,11 @@ class Sim:
         B = Barrier
         # the Q tile comes from one tensor copy, or (fused path) from every
         # softmax warp quantizing its rows, one arrival each
-        self.bars = {"QFULL": B("QFULL", self.W if fused_q else 1), "XM": B("XM", 8)}
+        self.bars = {"QFULL": B("QFULL", self.W if fused_q else 1)}
+        # row-max exchange: one barrier per TMEM lane quadrant, the two warps
+        # that share its rows arrive once per tile
+        for q in range(4):
+            self.bars[f"XM{q}"] = B(f"XM{q}", 2)
         self.q_rows_written = set()
         for s in range(NS):
             for n in ("KFULL", "KEMPTY", "VFULL", "VEMPTY"):
@@ -138,8 +142,8 @@ class Sim:
             self.bars[f"SEMPTY{sb}"].arrive()
             if self.NH == 2:
                 self.xm[j & 1][w] = j
-                self.bars["XM"].arrive()
-                yield from self.wait("XM", j & 1, j + 1)
+                self.bars[f"XM{w & 3}"].arrive()
+                yield from self.wait(f"XM{w & 3}", j & 1, j + 1)
                 partner = w ^ 4
                 if self.xm[j & 1].get(partner) != j:
                     raise ProtocolError(f"warp {w} read the row max of tile {self.xm[j & 1].get(partner)} for {j}")
