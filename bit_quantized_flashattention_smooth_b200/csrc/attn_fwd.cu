@@ -63,6 +63,13 @@
 #define HIFA4_ATTN_NH_BN64 1
 #endif
 // with one softmax warpgroup per row: a correction warpgroup rescales O
+// 1: a softmax warp that does not rescale O in tile j waits for no PV
+// product (the S_j wait already covers PV_{j-2}, the last reader of the P-hat
+// buffer it is about to overwrite); one that rescales waits for PV_{j-1}.
+// 0: every tile waits for PV_{j-1}.
+#ifndef HIFA4_RELAX_PV
+#define HIFA4_RELAX_PV 1
+#endif
 #ifndef HIFA4_ATTN_CORR
 #define HIFA4_ATTN_CORR 0
 #endif
@@ -568,7 +575,6 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     float l_p = 0.0f;
     const bool want_lp = !PREORDER || p.dbg_l_p != nullptr || (DUMP && p.dump.sum_p != nullptr);
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
-    constexpr float kInvGP = FMT == HIFA4_NVFP4 ? 256.0f : 1.0f;
     // pairs (of every eight) whose 2^y runs on the FMA pipe instead of MUFU
     constexpr int kPolyPairs = HIFA4_POLY_PAIRS >= 0 ? HIFA4_POLY_PAIRS : 2;
     const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
@@ -709,7 +715,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       for (int blk = 0; blk < NBH; ++blk) {
         const float ym = __fadd_rn(__fmul_rn(bms[blk], c), -m_new);
         if constexpr (FMT == HIFA4_NVFP4) {
-          const float t = __fmul_rn(div6_rn(ex2_approx(ym)), kInvGP);   // fl32(amax/6) / g_P
+          const float t = div6_rn_x256(ex2_approx(ym));                  // fl32(amax/6) / g_P, g_P = 2^-8
           scb[blk] = cvt_e4m3(t);
           mult[blk] = inv_tab[scb[blk]];                                  // fl32(1/(scale*g_P)), 0 for scale 0
         } else {
@@ -793,15 +799,22 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
           else atomicAdd(p.dump.sum_p + rt, psum);     // two column halves; the caller zero-fills
         }
       }
-      // One wait covers both uses of the previous product: PV_{j-1} done
-      // means the P-hat buffer pb's last reader PV_{j-2} is done too (a
-      // commit completes only after all earlier MMAs of its thread), and the
-      // O rescale below may then touch O.  (PV_{j-1}'s barrier is phase
-      // (j-1)/2 of buffer (j-1)%2, whose earlier phase PV_{j-3} completed
-      // before tile j-1 passed this point.)  With the correction warps the
-      // rescale is theirs, and only the buffer's reuse is awaited here.
-      if (j >= (C::CORR ? 2 : 1)) {
-        const int jw = C::CORR ? j - 2 : j - 1;
+      // Two uses of earlier PV products before the P-hat store and the O
+      // rescale below:
+      // - the P-hat buffer pb was last read by PV_{j-2}.  With one
+      //   MMA-issuing thread, S_j was issued after PV_{j-2}, and a commit
+      //   completes only after every earlier MMA of its thread, so the S_j
+      //   wait above already covered that product.  (With a second issuer
+      //   nothing orders the two, and PV_{j-2} is awaited here.)
+      // - a warp that rescales O (a warp-uniform vote) needs PV_{j-1} retired.
+      //   Its barrier is phase (j-1)/2 of buffer (j-1)%2, whose next phase
+      //   PV_{j+1} cannot complete before this tile's P-hat exists, and whose
+      //   earlier phase PV_{j-3} completed before S_j: the parity wait is exact.
+      // With the correction warps the rescale is theirs.
+      int jw = -1;
+      if (!C::CORR && (!HIFA4_RELAX_PV || warp_rescale)) jw = j - 1;
+      else if (C::TWO_ISSUERS) jw = j - 2;
+      if (jw >= 0) {
         if (!__all_sync(0xffffffffu,
                         mbar_wait(BAR(B_PEMPTY + (jw & 1)), (jw >> 1) & 1, abort_flag, kErrTimeoutSoftmax))) {
           ok = false;

@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(192, 4)
           float bm = pr;
 #pragma unroll
           for (int o = C::BETA / 2; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-          sc = cvt_e4m3(__fmul_rn(div6_rn(bm), 256.0f));
+          sc = cvt_e4m3(div6_rn_x256(bm));
           mult = inv_tab[sc];
         } else {
           // shared exponent from the block maximum of y (exact, see ptx.cuh)

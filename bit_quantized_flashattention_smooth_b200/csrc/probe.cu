@@ -160,12 +160,15 @@ __global__ void convert_probe_kernel(const float* __restrict__ x, int64_t n, uin
 }
 
 // Every float bit pattern in [lo, hi): count where div6_rn differs from the
-// IEEE quotient; record the smallest failing pattern.
+// IEEE quotient, or div6_rn_x256 from 2^8 times it; record the smallest
+// failing pattern.
 __global__ void div6_probe_kernel(uint32_t lo, uint32_t hi, unsigned long long* count, uint32_t* first_bad) {
   for (uint64_t b = lo + static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < hi;
        b += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
     const float a = __uint_as_float(static_cast<uint32_t>(b));
-    if (__float_as_uint(div6_rn(a)) != __float_as_uint(__fdiv_rn(a, 6.0f))) {
+    const float q = __fdiv_rn(a, 6.0f);
+    if (__float_as_uint(div6_rn(a)) != __float_as_uint(q) ||
+        __float_as_uint(div6_rn_x256(a)) != __float_as_uint(__fmul_rn(q, 256.0f))) {
       atomicAdd(count, 1ull);
       atomicMin(first_bad, static_cast<uint32_t>(b));
     }

@@ -434,6 +434,18 @@ __device__ __forceinline__ float div6_rn(float a) {
   const float rem = __fmaf_rn(-q0, 6.0f, a);
   return __fmaf_rn(rem, r6, q0);
 }
+// fl32(a / 6) * 2^8 for the same a, with the power of two folded into the
+// constants: every step is div6_rn's scaled by 2^8 (the residual is the same
+// number), and scaling by a power of two commutes with each rounding while the
+// quotient stays normal.  Only for a whose quotient feeds an E4M3 scale code:
+// below 6 * 2^-126 the two can differ, and both round to code 0.
+__device__ __forceinline__ float div6_rn_x256(float a) {
+  const float r6s = 42.666667938232421875f;        // fl32(1/6) * 2^8
+  const float six_s = 0.0234375f;                  // 6 * 2^-8
+  const float q0 = __fmul_rn(a, r6s);
+  const float rem = __fmaf_rn(-q0, six_s, a);
+  return __fmaf_rn(rem, r6s, q0);
+}
 // Packed fp32 pair arithmetic (sm_100 FFMA2 / FMUL2 / FADD2), each lane RN.
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   float2 r;

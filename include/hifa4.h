@@ -354,8 +354,9 @@ HIFA4_API hifa4_status hifa4_convert_probe(const float* x, int64_t count, uint8_
                                  uint8_t* e4m3_out, hifa4_stream_t stream);
 
 /* Conformance of the kernels' fast fl32(a/6) (reciprocal plus one exact
- * residual correction) with IEEE division, for every float bit pattern in
- * [lo_bits, hi_bits): adds the number of differing patterns to *mismatches
+ * residual correction) with IEEE division, and of its variant with 2^8 folded
+ * into the constants with 2^8 * fl32(a/6), for every float bit pattern in
+ * [lo_bits, hi_bits): adds the number of patterns where either differs to *mismatches
  * and lowers *first_bad (both device; caller initializes 0 / 0xFFFFFFFF). */
 HIFA4_API hifa4_status hifa4_div6_probe(uint32_t lo_bits, uint32_t hi_bits, unsigned long long* mismatches,
                                         uint32_t* first_bad, hifa4_stream_t stream);

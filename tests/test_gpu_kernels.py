@@ -85,7 +85,9 @@ def test_hw_conversions_exhaustive():
 def test_fast_div6_is_ieee_division():
     """The P-hat scale path computes fl32(amax/6) without a division; it must
     equal IEEE division for zero and every float in [2^-122, 2^20] (quotients
-    that are normal).  Below 2^-122 the scale code is 0 either way: the
+    that are normal), and the variant with g_P = 2^-8 folded into its
+    constants must equal 2^8 times that quotient over the same range.  Below
+    2^-122 the scale code is 0 either way: the
     quotient times 2^8 is under 2^-116, far below half the smallest UE4M3
     subnormal."""
     n, first = h.div6_probe(0x02800000, 0x49800000)

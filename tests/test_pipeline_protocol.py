@@ -48,8 +48,16 @@ class Barrier:
 
 
 class Sim:
-    def __init__(self, nkt, NS, NSB, NH, rng, fused_q=False):
+    def __init__(self, nkt, NS, NSB, NH, rng, fused_q=False, relax_lag=None, two_issuers=False):
         self.nkt, self.NS, self.NSB, self.NH, self.rng = nkt, NS, NSB, NH, rng
+        # a warp that does not rescale O in tile j waits for PV_{j - relax_lag},
+        # or for no product at all (None: the kernel with one MMA-issuing
+        # thread, where the S_j wait covers PV_{j-2}); 1 waits for the
+        # previous product on every tile
+        self.relax_lag = relax_lag
+        # two MMA-issuing threads: S and PV products complete in two
+        # independent orders
+        self.two_issuers = two_issuers
         self.W = 4 * NH
         self.fused_q = fused_q
         B = Barrier
@@ -79,7 +87,8 @@ class Sim:
         self.xm = [dict(), dict()]
         self.pv_done = -1                  # last PV completed
         self.pv_started = -1               # last PV begun
-        self.mma_queue = []                # in-order async tensor-core work
+        self.mma_queue = []                # in-order async tensor-core work (one issuer)
+        self.pv_queue = []                 # PV products of a second issuer
         self.copies = []                   # pending TMA copies
 
     # -------------------------------------------------------------- waits ---
@@ -116,7 +125,7 @@ class Sim:
             st, pb = j % self.NS, j & 1
             yield from self.wait(f"PFULL{pb}", (j >> 1) & 1, (j >> 1) + 1)
             yield from self.wait(f"VFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
-            self.mma_queue.append(("PV", j, [f"VEMPTY{st}", f"PEMPTY{pb}"]))
+            (self.pv_queue if self.two_issuers else self.mma_queue).append(("PV", j, [f"VEMPTY{st}", f"PEMPTY{pb}"]))
 
         if self.nkt > 0:
             yield from issue_s(0)
@@ -147,14 +156,17 @@ class Sim:
                 partner = w ^ 4
                 if self.xm[j & 1].get(partner) != j:
                     raise ProtocolError(f"warp {w} read the row max of tile {self.xm[j & 1].get(partner)} for {j}")
-            # one wait for the previous product PV_{j-1}: it also covers the
-            # P-hat buffer's last reader PV_{j-2} (commits complete in order)
-            if j >= 1:
-                yield from self.wait(f"PEMPTY{(j - 1) & 1}", ((j - 1) >> 1) & 1, ((j - 1) >> 1) + 1)
+            # the warp's rescale vote comes first; a rescaling warp waits for
+            # the previous product PV_{j-1} (which also covers the P-hat
+            # buffer's last reader PV_{j-2}: commits complete in order), any
+            # other warp for PV_{j-relax_lag} only
+            rescale = j > 0 and self.rng.random() < 0.5
+            jw = j - 1 if rescale else (j - self.relax_lag if self.relax_lag is not None else -1)
+            if jw >= 0:
+                yield from self.wait(f"PEMPTY{jw & 1}", (jw >> 1) & 1, (jw >> 1) + 1)
             if self.pv_done < j - 2:
                 raise ProtocolError(f"warp {w} overwrote P-hat buffer {pb} before PV_{j - 2} retired")
             self.p_buf[pb][w] = j
-            rescale = j > 0 and self.rng.random() < 0.5
             if rescale:
                 if self.pv_done < j - 1 or self.pv_started >= j:
                     raise ProtocolError(f"warp {w} rescaled O for tile {j} with PV_{self.pv_done} done, "
@@ -182,14 +194,17 @@ class Sim:
             events.append("copy")
         if self.mma_queue:
             events.append("mma")
+        if self.pv_queue:
+            events.append("pv")
         if not events:
             return False
-        if self.rng.choice(events) == "copy":
+        ev = self.rng.choice(events)
+        if ev == "copy":
             kind, st, j = self.copies.pop(self.rng.randrange(len(self.copies)))
             (self.k_stage if kind == "K" else self.v_stage)[st] = j
             self.bars[f"{kind}FULL{st}"].arrive()
             return True
-        kind, j, commits = self.mma_queue.pop(0)
+        kind, j, commits = (self.mma_queue if ev == "mma" else self.pv_queue).pop(0)
         if kind == "S":
             sb = j % self.NSB
             if self.k_stage[j % self.NS] != j:
@@ -214,7 +229,7 @@ class Sim:
             self.bars["QFULL"].arrive()    # the Q tile (its copy lands before anything else matters)
         live = [self.tma(), self.mma()] + [self.softmax(w) for w in range(self.W)]
         idle = 0
-        while live or self.mma_queue or self.copies:
+        while live or self.mma_queue or self.pv_queue or self.copies:
             progressed = self.rng.random() < 0.5 and self.step_async()
             self.rng.shuffle(live)
             finished = []
@@ -237,9 +252,33 @@ class Sim:
 
 @pytest.mark.parametrize("NH,NS,NSB", [(1, 3, 1), (2, 3, 1), (2, 3, 2), (2, 2, 2), (1, 2, 1)])
 @pytest.mark.parametrize("nkt", [1, 2, 3, 5, 9])
-def test_prefill_protocol_random_schedules(NH, NS, NSB, nkt):
+@pytest.mark.parametrize("relax_lag", [None, 1])
+def test_prefill_protocol_random_schedules(NH, NS, NSB, nkt, relax_lag):
     for seed in range(40):
-        Sim(nkt, NS, NSB, NH, random.Random(1000 * nkt + seed)).run()
+        Sim(nkt, NS, NSB, NH, random.Random(1000 * nkt + seed), relax_lag=relax_lag).run()
+
+
+@pytest.mark.parametrize("nkt", [2, 5, 9])
+def test_two_issuers_wait_for_the_buffer_reader(nkt):
+    """With S and PV issued by two threads, nothing orders S_j after
+    PV_{j-2}: the kernel then waits for PV_{j-2} in tiles without a rescale."""
+    for seed in range(40):
+        Sim(nkt, 3, 1, 1, random.Random(3000 * nkt + seed), relax_lag=2, two_issuers=True).run()
+
+
+@pytest.mark.parametrize("kw", [dict(relax_lag=3), dict(relax_lag=None, two_issuers=True)])
+def test_model_catches_a_missing_buffer_wait(kw):
+    """Waiting for PV_{j-3} in tiles without a rescale, or for nothing when
+    two threads issue the products, lets a warp overwrite the P-hat buffer
+    that PV_{j-2} may still read (or parity-wait on a phase two laps back):
+    the model must flag it."""
+    caught = 0
+    for seed in range(200):
+        try:
+            Sim(7, 3, 1, 1, random.Random(seed), **kw).run()
+        except ProtocolError:
+            caught += 1
+    assert caught > 0
 
 
 @pytest.mark.parametrize("NH,NS,NSB", [(1, 3, 1), (2, 3, 2), (2, 2, 2)])
