@@ -434,6 +434,15 @@ __device__ __forceinline__ float div6_rn(float a) {
   const float rem = __fmaf_rn(-q0, 6.0f, a);
   return __fmaf_rn(rem, r6, q0);
 }
+// fl32(a / 6) for any a: div6_rn where it was checked (a <= 2^20, every
+// float), IEEE division above and for inf / NaN.  The division sits behind a
+// branch in a function of its own, so its instructions run only for such a.
+static __device__ __noinline__ float div6_ieee(float a) { return __fdiv_rn(a, 6.0f); }
+__device__ __forceinline__ float div6_any(float a) {
+  float t = div6_rn(a);
+  if (!(a <= 1048576.0f)) t = div6_ieee(a);
+  return t;
+}
 // fl32(a / 6) * 2^8 for the same a, with the power of two folded into the
 // constants: every step is div6_rn's scaled by 2^8 (the residual is the same
 // number), and scaling by a power of two commutes with each rounding while the

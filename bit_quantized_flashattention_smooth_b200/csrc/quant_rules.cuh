@@ -67,8 +67,7 @@ __device__ __forceinline__ uint32_t block_scale(float amax, const float* inv_tab
   if constexpr (FMT == HIFA4_NVFP4) {
     // fl32(amax/6): the reciprocal-and-residual form is IEEE-exact on
     // [2^-122, 2^20] (checked on the GPU); below, both give scale code 0
-    const float t = amax <= 1048576.0f ? div6_rn(amax) : __fdiv_rn(amax, 6.0f);
-    sc = cvt_e4m3(t);
+    sc = cvt_e4m3(div6_any(amax));
     mult = TAB_LOG2 == 0 ? inv_tab[sc] : __fmul_rn(inv_tab[sc], __uint_as_float(static_cast<uint32_t>(127 - TAB_LOG2) << 23));
     if (sc == 0) keep = 0u;                             // scale 0: every code 0 (no -0 codes)
   } else {

@@ -64,18 +64,8 @@ __device__ __forceinline__ uint32_t quant_part(const float (&v)[8], uint32_t& pa
 #pragma unroll
   for (int o = 1; o < BETA / 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   float mult;
-  uint32_t sc;
-  uint32_t keep = 0xFFFFFFFFu;
-  if constexpr (FMT == HIFA4_NVFP4) {
-    const float t = amax <= 1048576.0f ? div6_rn(amax) : __fdiv_rn(amax, 6.0f);
-    sc = cvt_e4m3(t);
-    mult = inv_tab[sc];
-    if (sc == 0) keep = 0u;
-  } else {
-    const uint32_t ef = (__float_as_uint(amax) >> 23) & 0xFFu;
-    sc = ef >= 2u ? ef - 2u : 0u;
-    mult = __uint_as_float((254u - sc) << 23);
-  }
+  uint32_t keep;
+  const uint32_t sc = block_scale<FMT>(amax, inv_tab, mult, keep);
   const float2 m2 = make_float2(mult, mult);
   packed = keep & cvt_e2m1x8(qmul2(make_float2(v[0], v[1]), m2), qmul2(make_float2(v[2], v[3]), m2),
                              qmul2(make_float2(v[4], v[5]), m2), qmul2(make_float2(v[6], v[7]), m2));
@@ -83,8 +73,12 @@ __device__ __forceinline__ uint32_t quant_part(const float (&v)[8], uint32_t& pa
 }
 
 // CTA `cta` of a tensor with `heads` heads of Np (padded) rows: head
-// cta / (Np / ROWS), rows [chunk * ROWS, +ROWS).  Index arithmetic per CTA,
-// none per lane beyond shifts.
+// cta / (Np / ROWS), rows [chunk * ROWS, +ROWS).  A lane's U row groups are
+// RPI rows apart and all fall inside one 32-row band of one 128-row scale
+// group (a warp's U * RPI rows start on a multiple of U * RPI, which divides
+// 32, and a CTA's rows on a multiple of ROWS), so every per-group address is
+// the lane's first one plus a constant: the scale byte moves by RPI * 16
+// bytes per group, the codes by RPI * D/2, the input by RPI * D values.
 template <int FMT, typename T, int D>
 __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H, int G, int N, int Np,
                                                   const float* __restrict__ scale, uint8_t* __restrict__ codes,
@@ -93,6 +87,7 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
   using R = RowTile<FMT, D>;
   constexpr int BETA = R::BETA, U = R::U, CPR = R::CPR, RPI = R::RPI, LPB = R::LPB, NB = R::NB;
   constexpr int WPR = (NB + 3) / 4;        // scale words per row
+  static_assert(32 % (U * RPI) == 0, "a warp's rows stay inside one 32-row band");
   const int cpt = Np / R::ROWS;
   const int bh = cta / cpt;
   const int chunk = cta - bh * cpt;
@@ -100,28 +95,25 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ch = lane % CPR;               // 16-byte chunk of the row
   const int blk = ch / LPB;                // its block
-  const T* xh = x + static_cast<int64_t>(bh) * N * D + ch * 8;
+  const int t0 = chunk * R::ROWS + warp * U * RPI + lane / CPR;   // the lane's first row
+  const int nvalid = N - t0;               // groups u with u * RPI < nvalid hold real rows
+  const T* src = x + (static_cast<int64_t>(bh) * N + t0) * D + ch * 8;
   // all U loads in flight at once, kept packed (4 registers each) until their
-  // row group is quantized
+  // row group is quantized; rows past N are zeros
   uint4 raw[U];
-  int tok[U];
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    tok[u] = chunk * R::ROWS + (warp * U + u) * RPI + lane / CPR;
-    raw[u] = tok[u] < N ? *reinterpret_cast<const uint4*>(xh + static_cast<int64_t>(tok[u]) * D)
-                        : make_uint4(0u, 0u, 0u, 0u);
-  }
+  for (int u = 0; u < U; ++u)
+    raw[u] = u * RPI < nvalid ? *reinterpret_cast<const uint4*>(src + u * RPI * D) : make_uint4(0u, 0u, 0u, 0u);
   float sv[8];
   if (scale != nullptr) {
     const float4* s4 = reinterpret_cast<const float4*>(scale + kvh * D + ch * 8);
     const float4 a = s4[0], b = s4[1];
     sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w; sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
   }
-  uint8_t* cbase = codes + (static_cast<int64_t>(bh) * Np) * (D / 2) + ch * 4;
-  uint8_t* sh = sf + static_cast<int64_t>(bh) * sf_head_bytes;
+  uint8_t* cdst = codes + (static_cast<int64_t>(bh) * Np + t0) * (D / 2) + ch * 4;
+  uint8_t* sdst = sf + static_cast<int64_t>(bh) * sf_head_bytes + sf_word_offset(t0, blk / 4, WPR) + blk % 4;
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    const int t = tok[u];
     float v[8];
     {
       const uint32_t wd[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
@@ -131,7 +123,8 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
         v[2 * i + 1] = chan_of<T>(wd[i], 1);
       }
     }
-    if (scale != nullptr && t < N) {
+    if (scale != nullptr) {
+      // padding rows are +0 and stay +0 (s is finite and positive)
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
         const float2 p2 = qmul2(make_float2(v[i], v[i + 1]), make_float2(sv[i], sv[i + 1]));
@@ -141,15 +134,15 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
     }
     uint32_t packed;
     const uint32_t sc = quant_part<FMT, BETA>(v, packed, inv_tab);
-    *reinterpret_cast<uint32_t*>(cbase + static_cast<int64_t>(t) * (D / 2)) = packed;
+    *reinterpret_cast<uint32_t*>(cdst + u * RPI * (D / 2)) = packed;
     if (ch % LPB == 0) {
-      uint8_t* sfw = sh + sf_word_offset(t, blk / 4, WPR);
-      sfw[blk % 4] = static_cast<uint8_t>(sc);
+      uint8_t* sb = sdst + u * RPI * 16;
+      *sb = static_cast<uint8_t>(sc);
       if constexpr (NB < 4) {
         // the rest of the row's only scale word holds no block: zero it
         if (blk == NB - 1)
 #pragma unroll
-          for (int bb = NB; bb < 4; ++bb) sfw[bb] = 0;   // blk / 4 == 0: the same word
+          for (int bb = NB; bb < 4; ++bb) sb[bb - blk] = 0;   // blk / 4 == 0: the same word
       }
     }
   }
