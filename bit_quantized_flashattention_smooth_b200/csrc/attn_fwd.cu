@@ -70,6 +70,14 @@
 #ifndef HIFA4_RELAX_PV
 #define HIFA4_RELAX_PV 1
 #endif
+// 1: with three or more K/V stages, a key tile's K-hat and V-hat^T copies
+// (with their scales) complete on one barrier per stage, awaited once by the
+// MMA issuer before S_j (measured 1.2 % faster at d = 128; with two stages,
+// d = 256, S_j would wait for V_j's stage and it is 10 % slower); 0: one
+// barrier each, V's awaited before PV_j.
+#ifndef HIFA4_KV_ONE_BAR
+#define HIFA4_KV_ONE_BAR 1
+#endif
 #ifndef HIFA4_ATTN_CORR
 #define HIFA4_ATTN_CORR 0
 #endif
@@ -118,6 +126,7 @@ struct AttnCfg {
   // when the running max rises, off the softmax warps' path
   static constexpr int CORR = (NH == 1 && HIFA4_ATTN_CORR) ? 1 : 0;
   static constexpr int NS = D == 256 ? 2 : 3;               // K/V pipeline stages
+  static constexpr bool KV_ONE = HIFA4_KV_ONE_BAR && NS >= 3;  // one full barrier per K/V stage
   static constexpr int QROW = D / 2;                        // bytes per Q/K row
   static constexpr int PROW = BN / 2;                       // bytes per P-hat / V^T row
   static constexpr int KSTEPS_S = D / 64;
@@ -377,19 +386,22 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         const int st = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
         if (!mbar_wait(BAR(B_KEMPTY + st), ph ^ 1, abort_flag, kErrTimeoutTma)) break;
-        mbar_arrive_expect_tx(BAR(B_KFULL + st), C::SZ_K + C::NKC_Q * 512);
+        // with one barrier per stage it expects the V copies' bytes too
+        mbar_arrive_expect_tx(BAR(B_KFULL + st), C::SZ_K + C::NKC_Q * 512 +
+                                                     (C::KV_ONE ? C::SZ_V + C::NRG_V * C::NCH_V * 512 : 0));
         tma_load_2d(sbase + C::OFF_K + st * C::SZ_K, &tm_k, 0, kvbh * p.Np + j * BN, BAR(B_KFULL + st));
         bulk_load(sbase + C::OFF_KSF + st * C::NKC_Q * 512,
                   p.k_sf + static_cast<int64_t>(kvbh) * p.sf_qk_head + static_cast<int64_t>((j * BN) >> 7) * C::NKC_Q * 512,
                   C::NKC_Q * 512, BAR(B_KFULL + st));
         if (!mbar_wait(BAR(B_VEMPTY + st), ph ^ 1, abort_flag, kErrTimeoutTma)) break;
-        mbar_arrive_expect_tx(BAR(B_VFULL + st), C::SZ_V + C::NRG_V * C::NCH_V * 512);
-        tma_load_2d(sbase + C::OFF_V + st * C::SZ_VX, &tm_v, j * C::PROW, kvbh * D, BAR(B_VFULL + st));
+        const uint32_t vbar = BAR((C::KV_ONE ? B_KFULL : B_VFULL) + st);
+        if (!C::KV_ONE) mbar_arrive_expect_tx(vbar, C::SZ_V + C::NRG_V * C::NCH_V * 512);
+        tma_load_2d(sbase + C::OFF_V + st * C::SZ_VX, &tm_v, j * C::PROW, kvbh * D, vbar);
         const int chunk0 = (j * BN) / (4 * C::BETA);
         for (int rg = 0; rg < C::NRG_V; ++rg)
           bulk_load(sbase + C::OFF_VSF + (st * C::NRG_V + rg) * C::NCH_V * 512,
                     p.v_sf + static_cast<int64_t>(kvbh) * p.sf_v_head + static_cast<int64_t>(rg * nkc_v_row + chunk0) * 512,
-                    C::NCH_V * 512, BAR(B_VFULL + st));
+                    C::NCH_V * 512, vbar);
       }
     }
   } else if (warp == C::WARP_MMA || warp == C::WARP_PV) {
@@ -470,7 +482,10 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
               if (!mbar_wait(BAR(B_OC + 2 * q + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, kErrTimeoutMma))
                 return false;
         }
-        if (!mbar_wait(BAR(B_VFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
+        // V_j landed: with one barrier per stage the S_j wait covered it (S_j
+        // is issued first by the same thread), unless a second thread issues PV
+        if (!C::KV_ONE || C::TWO_ISSUERS)
+          if (!mbar_wait(BAR((C::KV_ONE ? B_KFULL : B_VFULL) + st), ph, abort_flag, kErrTimeoutMma)) return false;
         tc_fence_after();
         for (int pc = 0; pc < C::NKC_P; ++pc)
           tc_cp_32x128b_warpx4(tmem + C::TM_SFA_P + 4 * pc,

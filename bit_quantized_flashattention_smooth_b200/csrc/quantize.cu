@@ -59,8 +59,10 @@ __device__ __forceinline__ float chan_of<__half>(uint32_t w, int ch) {
 // 8 E2M1 codes packed in a word, by exactly the rules of quant_block.
 template <int FMT, int BETA>
 __device__ __forceinline__ uint32_t quant_part(const float (&v)[8], uint32_t& packed, const float* inv_tab) {
-  float amax = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
-                     fmaxf(fabsf(v[6]), fabsf(v[7])));
+  // two-input maxima with |x| as operand modifiers (measured faster here than
+  // the three-input form)
+  float amax = fmaxf(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))),
+                     fmaxf(fmaxf(fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7]))));
 #pragma unroll
   for (int o = 1; o < BETA / 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   float mult;

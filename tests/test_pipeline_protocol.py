@@ -48,7 +48,7 @@ class Barrier:
 
 
 class Sim:
-    def __init__(self, nkt, NS, NSB, NH, rng, fused_q=False, relax_lag=None, two_issuers=False):
+    def __init__(self, nkt, NS, NSB, NH, rng, fused_q=False, relax_lag=None, two_issuers=False, kv_one=True):
         self.nkt, self.NS, self.NSB, self.NH, self.rng = nkt, NS, NSB, NH, rng
         # a warp that does not rescale O in tile j waits for PV_{j - relax_lag},
         # or for no product at all (None: the kernel with one MMA-issuing
@@ -58,6 +58,9 @@ class Sim:
         # two MMA-issuing threads: S and PV products complete in two
         # independent orders
         self.two_issuers = two_issuers
+        # one barrier per K/V stage that completes when both copies landed
+        # (the kernel's default), or one barrier per copy
+        self.kv_one = kv_one
         self.W = 4 * NH
         self.fused_q = fused_q
         B = Barrier
@@ -72,6 +75,7 @@ class Sim:
         for s in range(NS):
             for n in ("KFULL", "KEMPTY", "VFULL", "VEMPTY"):
                 self.bars[f"{n}{s}"] = B(f"{n}{s}", 1)
+            self.bars[f"KVFULL{s}"] = B(f"KVFULL{s}", 2)
         for s in range(NSB):
             self.bars[f"SFULL{s}"] = B(f"SFULL{s}", 1)
             self.bars[f"SEMPTY{s}"] = B(f"SEMPTY{s}", self.W)
@@ -117,14 +121,18 @@ class Sim:
 
         def issue_s(j):
             st, sb = j % self.NS, j % self.NSB
-            yield from self.wait(f"KFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
+            full = "KVFULL" if self.kv_one else "KFULL"
+            yield from self.wait(f"{full}{st}", (j // self.NS) & 1, j // self.NS + 1)
             yield from self.wait(f"SEMPTY{sb}", ((j // self.NSB) & 1) ^ 1, j // self.NSB)
             self.mma_queue.append(("S", j, [f"SFULL{sb}", f"KEMPTY{st}"]))
 
         def issue_pv(j):
             st, pb = j % self.NS, j & 1
             yield from self.wait(f"PFULL{pb}", (j >> 1) & 1, (j >> 1) + 1)
-            yield from self.wait(f"VFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
+            if not self.kv_one:
+                yield from self.wait(f"VFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
+            elif self.two_issuers:
+                yield from self.wait(f"KVFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
             (self.pv_queue if self.two_issuers else self.mma_queue).append(("PV", j, [f"VEMPTY{st}", f"PEMPTY{pb}"]))
 
         if self.nkt > 0:
@@ -202,7 +210,7 @@ class Sim:
         if ev == "copy":
             kind, st, j = self.copies.pop(self.rng.randrange(len(self.copies)))
             (self.k_stage if kind == "K" else self.v_stage)[st] = j
-            self.bars[f"{kind}FULL{st}"].arrive()
+            self.bars[f"KVFULL{st}" if self.kv_one else f"{kind}FULL{st}"].arrive()
             return True
         kind, j, commits = (self.mma_queue if ev == "mma" else self.pv_queue).pop(0)
         if kind == "S":
@@ -252,10 +260,10 @@ class Sim:
 
 @pytest.mark.parametrize("NH,NS,NSB", [(1, 3, 1), (2, 3, 1), (2, 3, 2), (2, 2, 2), (1, 2, 1)])
 @pytest.mark.parametrize("nkt", [1, 2, 3, 5, 9])
-@pytest.mark.parametrize("relax_lag", [None, 1])
-def test_prefill_protocol_random_schedules(NH, NS, NSB, nkt, relax_lag):
+@pytest.mark.parametrize("relax_lag,kv_one", [(None, True), (1, True), (None, False)])
+def test_prefill_protocol_random_schedules(NH, NS, NSB, nkt, relax_lag, kv_one):
     for seed in range(40):
-        Sim(nkt, NS, NSB, NH, random.Random(1000 * nkt + seed), relax_lag=relax_lag).run()
+        Sim(nkt, NS, NSB, NH, random.Random(1000 * nkt + seed), relax_lag=relax_lag, kv_one=kv_one).run()
 
 
 @pytest.mark.parametrize("nkt", [2, 5, 9])
@@ -268,6 +276,7 @@ def test_two_issuers_wait_for_the_buffer_reader(nkt):
 
 @pytest.mark.parametrize("kw", [dict(relax_lag=3), dict(relax_lag=None, two_issuers=True)])
 def test_model_catches_a_missing_buffer_wait(kw):
+    # (the K/V barrier layout does not matter here)
     """Waiting for PV_{j-3} in tiles without a rescale, or for nothing when
     two threads issue the products, lets a warp overwrite the P-hat buffer
     that PV_{j-2} may still read (or parity-wait on a phase two laps back):
