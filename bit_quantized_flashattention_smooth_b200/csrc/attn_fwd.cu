@@ -40,8 +40,8 @@
 
 // Tuning knobs (measured on the 32-head, 4096-token causal prefill):
 // element pairs (of every eight pairs) whose 2^y (or code argument) runs on
-// the FMA pipe instead of MUFU (-1: 2, the fastest of 0/2/4/8 at both tile
-// widths), and softmax warpgroups per row for 64-key tiles.
+// the FMA pipe instead of MUFU (-1: 2 at d <= 128 and 1 at d = 256, the
+// fastest of 0..3 for each), and softmax warpgroups per row for 64-key tiles.
 #ifndef HIFA4_POLY_PAIRS
 #define HIFA4_POLY_PAIRS -1
 #endif
@@ -277,7 +277,7 @@ __device__ __forceinline__ void rescale_o_rows(uint32_t a0, uint32_t al, bool wi
   }
 }
 
-template <int D, int BN, int FMT, bool PREORDER, bool DUMP>
+template <int D, int BN, int FMT, bool PREORDER, bool DBG>
 __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -588,10 +588,15 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     const float c = p.c_log2;
     float m = -INFINITY;
     float l_p = 0.0f;
-    const bool want_lp = !PREORDER || p.dbg_l_p != nullptr || (DUMP && p.dump.sum_p != nullptr);
+    // the running sum of P: the normalizer of the inconsistent mode, else a
+    // debug output only (its pointers reach the DBG instantiation alone).  At
+    // d = 256 the production kernel knows at compile time that it forms no
+    // sum (measured 1.7 % faster); at d <= 128 the runtime test schedules
+    // better (1.3 % faster), although the pointer is always null there.
+    const bool want_lp = !PREORDER || ((DBG || D != 256) && (p.dbg_l_p != nullptr || (DBG && p.dump.sum_p != nullptr)));
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
     // pairs (of every eight) whose 2^y runs on the FMA pipe instead of MUFU
-    constexpr int kPolyPairs = HIFA4_POLY_PAIRS >= 0 ? HIFA4_POLY_PAIRS : 2;
+    constexpr int kPolyPairs = HIFA4_POLY_PAIRS >= 0 ? HIFA4_POLY_PAIRS : (D == 256 ? 1 : 2);
     const float* inv_tab = reinterpret_cast<const float*>(smem + C::OFF_INV);
     const float* log_tab = reinterpret_cast<const float*>(smem + C::OFF_LOG);
     float* xm = reinterpret_cast<float*>(smem + C::OFF_XM);  // [2 parities][2 halves][128]
@@ -797,7 +802,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       if (want_lp) quant_tile(std::true_type{});
       else quant_tile(std::false_type{});
       if (want_lp) l_p = fmaf(alpha, l_p, psum);
-      if (DUMP && row < p.N) {
+      if (DBG && p.dump.codes != nullptr && row < p.N) {
         // debug view of this tile: the codes and scales as they go to the
         // PV MMA, the running max, and (on the path that forms P) sum(P)
         const int64_t rt = (static_cast<int64_t>(bhq) * p.N + row) * p.nkt_all + j;
@@ -948,8 +953,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       if (store && hw == 0) {
         const int64_t ri = static_cast<int64_t>(bhq) * p.N + row;
         if (p.lse) p.lse[ri] = m + log2f(l_used);
-        if (p.dbg_l_phat) p.dbg_l_phat[ri] = l_phat;
-        if (p.dbg_l_p) p.dbg_l_p[ri] = l_p;
+        if (DBG && p.dbg_l_phat) p.dbg_l_phat[ri] = l_phat;
+        if (DBG && p.dbg_l_p) p.dbg_l_p[ri] = l_p;
       }
     }
   }
@@ -969,9 +974,9 @@ bool make_tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner_bytes, uint6
 template <int D, int BN, int FMT, bool PRE>
 static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const uint8_t* vc, const AttnParams& p,
                                   cudaStream_t st) {
-  // the P-hat dump (a debug view) is its own instantiation: the production
-  // kernel carries none of its code
-  const bool dump = p.dump.codes != nullptr;
+  // the debug views (the P-hat dump, the sums of P and P-hat) are their own
+  // instantiation: the production kernel carries none of their code
+  const bool dbg = p.dump.codes != nullptr || p.dbg_l_p != nullptr || p.dbg_l_phat != nullptr;
   using C = AttnCfg<D, BN, FMT>;
   CUtensorMap tq, tk, tv;
   const uint64_t Np = static_cast<uint64_t>(p.Np);
@@ -984,7 +989,7 @@ static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const ui
     set_last_error("cuTensorMapEncodeTiled failed");
     return HIFA4_ERR_CUDA;
   }
-  auto kern = dump ? attn_fwd_fp4_kernel<D, BN, FMT, PRE, true> : attn_fwd_fp4_kernel<D, BN, FMT, PRE, false>;
+  auto kern = dbg ? attn_fwd_fp4_kernel<D, BN, FMT, PRE, true> : attn_fwd_fp4_kernel<D, BN, FMT, PRE, false>;
   const int smem = C::SMEM_REQ;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * p.num_qtiles;
