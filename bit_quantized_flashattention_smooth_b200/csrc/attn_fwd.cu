@@ -443,15 +443,17 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         const uint32_t ph = (j / C::NS) & 1;
         const int sb = j % C::NSB;
         if (!mbar_wait(BAR(B_KFULL + st), ph, abort_flag, kErrTimeoutMma)) return false;
-        if (!mbar_wait(BAR(B_SEMPTY + sb), ((j / C::NSB) & 1) ^ 1, abort_flag, kErrTimeoutMma)) return false;
         tc_fence_after();
         // 64-key tiles: a 128-row chunk of K scales serves tiles 2i and 2i+1,
         // so it is copied on even tiles only (the copy of tile 2i+2 is issued
-        // after, and so executes after, the MMAs of tile 2i+1)
+        // after, and so executes after, the MMAs of tile 2i+1).  It needs only
+        // the K tile, so it goes before the wait for the S buffer.
         if (!(BN == 64 && (j & 1)))
           for (int kc = 0; kc < C::NKC_Q; ++kc)
             tc_cp_32x128b_warpx4(tmem + C::TM_SFB_K + 4 * kc,
                                  make_sf_desc(sbase + C::OFF_KSF + st * C::NKC_Q * 512 + kc * 512));
+        if (!mbar_wait(BAR(B_SEMPTY + sb), ((j / C::NSB) & 1) ^ 1, abort_flag, kErrTimeoutMma)) return false;
+        tc_fence_after();
         const uint32_t half_off = (BN == 64 && (j & 1)) ? 2u : 0u;  // rows 64..127 of the K row group
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS_S; ++ks) {
@@ -472,6 +474,17 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         const int st = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
         const int pb = j & 1;
+        // V_j landed: with one barrier per stage the S_j wait covered it (S_j
+        // is issued first by the same thread), unless a second thread issues PV
+        if (!C::KV_ONE || C::TWO_ISSUERS)
+          if (!mbar_wait(BAR((C::KV_ONE ? B_KFULL : B_VFULL) + st), ph, abort_flag, kErrTimeoutMma)) return false;
+        tc_fence_after();
+        // V_j's scales need only V_j: copied before the wait for P-hat_j (the
+        // copy executes after PV_{j-1}, issued earlier by this thread)
+        for (int lc = 0; lc < C::NCH_V; ++lc)
+          for (int rg = 0; rg < C::NRG_V; ++rg)
+            tc_cp_32x128b_warpx4(tmem + C::TM_SFB_V + 4 * (lc * C::NRG_B + rg),
+                                 make_sf_desc(sbase + C::OFF_VSF + ((st * C::NRG_V + rg) * C::NCH_V + lc) * 512));
         if (!mbar_wait(BAR(B_PFULL + pb), (j >> 1) & 1, abort_flag, kErrTimeoutMma)) return false;
         if constexpr (C::CORR) {
           // O (and L) rescaled for this tile's max by every lane quadrant
@@ -482,18 +495,10 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
               if (!mbar_wait(BAR(B_OC + 2 * q + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, kErrTimeoutMma))
                 return false;
         }
-        // V_j landed: with one barrier per stage the S_j wait covered it (S_j
-        // is issued first by the same thread), unless a second thread issues PV
-        if (!C::KV_ONE || C::TWO_ISSUERS)
-          if (!mbar_wait(BAR((C::KV_ONE ? B_KFULL : B_VFULL) + st), ph, abort_flag, kErrTimeoutMma)) return false;
         tc_fence_after();
         for (int pc = 0; pc < C::NKC_P; ++pc)
           tc_cp_32x128b_warpx4(tmem + C::TM_SFA_P + 4 * pc,
                                make_sf_desc(sbase + C::OFF_PSF + pb * C::NKC_P * 512 + pc * 512));
-        for (int lc = 0; lc < C::NCH_V; ++lc)
-          for (int rg = 0; rg < C::NRG_V; ++rg)
-            tc_cp_32x128b_warpx4(tmem + C::TM_SFB_V + 4 * (lc * C::NRG_B + rg),
-                                 make_sf_desc(sbase + C::OFF_VSF + ((st * C::NRG_V + rg) * C::NCH_V + lc) * 512));
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS_P; ++ks) {
           const int kk = j * BN + ks * 64;                        // first key of this K-step

@@ -128,11 +128,12 @@ class Sim:
 
         def issue_pv(j):
             st, pb = j % self.NS, j & 1
-            yield from self.wait(f"PFULL{pb}", (j >> 1) & 1, (j >> 1) + 1)
+            # V_j first (its scale copy goes ahead of the wait for P-hat_j)
             if not self.kv_one:
                 yield from self.wait(f"VFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
             elif self.two_issuers:
                 yield from self.wait(f"KVFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
+            yield from self.wait(f"PFULL{pb}", (j >> 1) & 1, (j >> 1) + 1)
             (self.pv_queue if self.two_issuers else self.mma_queue).append(("PV", j, [f"VEMPTY{st}", f"PEMPTY{pb}"]))
 
         if self.nkt > 0:
