@@ -84,11 +84,12 @@ def lib():
         L.or_sf_tiled_offset.argtypes = [i64, i, i]; L.or_sf_tiled_offset.restype = i64
         L.or_sf_tile.argtypes = [u8p, i64, i, u8p, i64]
         L.or_calibrate.argtypes = [f32p, f32p, i, i, i, i, i, i, d, i, f32p, f32p]
+        L.or_calibrate_q_mean.argtypes = [f32p, i, i, i, i, i, i, f32p, f32p]
         L.or_quantize_qkv.argtypes = [f32p, f32p, f32p, i, i, i, i, i, f32p, f32p, i,
-                                      u8p, u8p, u8p, u8p, u8p, u8p]
+                                      u8p, u8p, u8p, u8p, u8p, u8p, f32p]
         L.or_attention.argtypes = [u8p, u8p, u8p, u8p, u8p, u8p, i, i, i, i, i, i, d, i, i,
                                    i, i, f64p, f64p, f64p, f64p, u8p, u8p, f64p, f64p,
-                                   f32p, f32p, f32p, i, i, i, f]
+                                   f32p, f32p, f32p, i, i, i, f, f32p]
         L.or_split_len.argtypes = [i, i, i]; L.or_split_len.restype = i
         L.or_decode.argtypes = [f32p, f32p, u8p, u8p, u8p, u8p, i, i, i, i, i, i, d, i, i, i,
                                 i, f64p, f64p, i, f]
@@ -220,9 +221,24 @@ def calibrate(q, k, n_cal: int, alpha: float = 0.5, enable=True):
     return s, inv
 
 
+def calibrate_q_mean(q, s, n_cal: int):
+    """Q-Mean auxiliary (a reading; the pages name it only): the per-channel
+    mean of the smoothed query over the calibration tokens, q [B,Hq,T,d],
+    s [Hkv,d] or None -> mu [Hq,d] float32."""
+    q = _f32(q)
+    B, Hq, T, d = q.shape
+    s32 = _f32(s) if s is not None else None
+    Hkv = s32.shape[0] if s32 is not None else Hq
+    mu = np.zeros((Hq, d), np.float32)
+    lib().or_calibrate_q_mean(_p(q, ctypes.c_float), B, Hq, Hkv, n_cal, T, d,
+                              _p(s32, ctypes.c_float) if s32 is not None else None, _p(mu, ctypes.c_float))
+    return mu
+
+
 # ------------------------------------------------------------- quantize ---
-def quantize_qkv(q, k, v, s=None, inv_s=None, fmt: int = NVFP4):
+def quantize_qkv(q, k, v, s=None, inv_s=None, fmt: int = NVFP4, q_mu=None):
     """Fused Smooth-QK scale + block quantization; plain scale layouts.
+    q_mu [Hq,d]: the Q-Mean auxiliary, subtracted from the smoothed query.
 
     Returns dict with q_codes [B,Hq,Np,d/2], q_sc [B,Hq,Np,d/beta],
     k_codes, k_sc (Hkv), vt_codes [B,Hkv,d,Np/2], vt_sc [B,Hkv,d,Np/beta].
@@ -239,10 +255,12 @@ def quantize_qkv(q, k, v, s=None, inv_s=None, fmt: int = NVFP4):
     s_keep = (_f32(s) if s is not None else None, _f32(inv_s) if inv_s is not None else None)
     sp = _p(s_keep[0], ctypes.c_float) if s_keep[0] is not None else None
     ip = _p(s_keep[1], ctypes.c_float) if s_keep[1] is not None else None
+    mu = _f32(q_mu) if q_mu is not None else None
     lib().or_quantize_qkv(_p(q, ctypes.c_float), _p(k, ctypes.c_float), _p(v, ctypes.c_float),
                           B, Hq, Hkv, N, d, sp, ip, fmt,
                           *[_p(out[n], ctypes.c_uint8) for n in
-                            ("q_codes", "q_sc", "k_codes", "k_sc", "vt_codes", "vt_sc")])
+                            ("q_codes", "q_sc", "k_codes", "k_sc", "vt_codes", "vt_sc")],
+                          _p(mu, ctypes.c_float) if mu is not None else None)
     return out
 
 
@@ -262,7 +280,7 @@ def tile_scales(qz: dict) -> dict:
 def attention(qz: dict, N: int, fmt: int = NVFP4, softmax_scale: float | None = None,
               causal: bool = True, mode: int = PREORDER, BN: int = 128,
               pexp: int = P_PRESCALE_LOG2, rows=None, dump_phat: bool = False,
-              variant: int = 0, tau: float = 0.0, raw: dict | None = None):
+              variant: int = 0, tau: float = 0.0, raw: dict | None = None, q_mu=None):
     """Oracle forward over the quantized tensors of quantize_qkv.
 
     Returns dict O [B,Hq,N,d] fp64, lse, l_phat, l_p [B,Hq,N]; optional P-hat
@@ -271,6 +289,7 @@ def attention(qz: dict, N: int, fmt: int = NVFP4, softmax_scale: float | None = 
     outputs stay NaN).  tau > 0: the running max moves only when a tile's max
     exceeds it by more than tau (lazy rescaling).  raw: test-only ablation,
     {"q"|"k"|"v": float array} in [B,H,N,d] replacing the dequantized operand.
+    q_mu [Hq,d]: the Q-Mean auxiliary; every score gets back mu . k of its key.
     """
     qc, qs = qz["q_codes"], qz["q_sc"]
     B, Hq, Np, dh = qc.shape
@@ -294,12 +313,14 @@ def attention(qz: dict, N: int, fmt: int = NVFP4, softmax_scale: float | None = 
     raw = raw or {}
     rq, rk, rv = (None if raw.get(n) is None else _f32(raw[n]) for n in ("q", "k", "v"))
     arrs = [np.ascontiguousarray(qz[n]) for n in ("q_codes", "q_sc", "k_codes", "k_sc", "vt_codes", "vt_sc")]
+    mu = _f32(q_mu) if q_mu is not None else None
     lib().or_attention(*[_p(a, ctypes.c_uint8) for a in arrs], B, Hq, Hkv, N, d, fmt,
                        float(softmax_scale), int(causal), int(mode), int(BN), int(pexp),
                        _p(O, ctypes.c_double), _p(lse, ctypes.c_double), _p(lph, ctypes.c_double),
                        _p(lp, ctypes.c_double), _p(pd, ctypes.c_uint8), _p(psd, ctypes.c_uint8),
                        _p(md, ctypes.c_double), _p(ts, ctypes.c_double), _p(rq, ctypes.c_float),
-                       _p(rk, ctypes.c_float), _p(rv, ctypes.c_float), int(r0), int(r1), int(variant), float(tau))
+                       _p(rk, ctypes.c_float), _p(rv, ctypes.c_float), int(r0), int(r1), int(variant), float(tau),
+                       _p(mu, ctypes.c_float) if mu is not None else None)
     res = dict(O=O, lse=lse, l_phat=lph, l_p=lp)
     if dump_phat:
         res["phat_codes"] = pd

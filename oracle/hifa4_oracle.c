@@ -317,12 +317,40 @@ void or_calibrate(const float* q, const float* k, int B, int Hq, int Hkv,
   free(sorted);
 }
 
+/* Q-Mean auxiliary [a reading of HiFA4, Abstract para 3, which names "the
+ * adopted Q-Mean auxiliary" and nothing more]: the per-channel mean of the
+ * smoothed query over the calibration tokens,
+ *   mu[hq][c] = fl32( sum_{b, t < n_cal} fl32(q * s[h(hq)][c]) / (B * n_cal) ),
+ * the sum in fp64 in the order b, then t.  The quantized query is then
+ * q' - mu (or_quantize_qkv), and each score gets back the rank-one term
+ * mu . K-hat of its key (or_attention), so that without quantization the
+ * scores are unchanged: (q' - mu) . k + mu . k = q' . k.
+ * q [B][Hq][ld_tok][d]; s [Hkv][d] or NULL (= 1); mu out [Hq][d]. */
+void or_calibrate_q_mean(const float* q, int B, int Hq, int Hkv, int n_cal,
+                         int ld_tok, int d, const float* s, float* mu) {
+  int G = Hq / Hkv;
+  for (int hq = 0; hq < Hq; ++hq) {
+    int h = hq / G;
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int b = 0; b < B; ++b)
+        for (int t = 0; t < n_cal; ++t) {
+          float x = q[(((int64_t)b * Hq + hq) * ld_tok + t) * d + c];
+          float xs = s ? x * s[h * d + c] : x;
+          acc += (double)xs;
+        }
+      mu[hq * d + c] = (float)(acc / (double)((int64_t)B * n_cal));
+    }
+  }
+}
+
 /* Fused scale + quantize of Q, K, V [HiFA4, Abstract para 2: "only a fusible
  * element-wise scaling"].  q' = fl32(q*s[c]), k' = fl32(k*inv_s[c]) on the
  * kv-head of the row, then blocks along d.  V is not scaled; it is blocked
  * along tokens and written transposed ([d][Np] codes, tokens contiguous).
  * Rows/tokens from N up to Np (N rounded up to 128) are zero padding.
- * s/inv_s may be NULL (treated as 1).
+ * s/inv_s may be NULL (treated as 1).  q_mu [Hq][d] (the Q-Mean auxiliary,
+ * or NULL): rows t < N of Q quantize fl32(fl32(q*s) - mu) instead.
  * Outputs: q_codes [B][Hq][Np][d/2], q_sc plain [B][Hq][Np][d/beta];
  *          k likewise with Hkv; vt_codes [B][Hkv][d][Np/2],
  *          vt_sc plain [B][Hkv][d][Np/beta]. */
@@ -330,7 +358,7 @@ void or_quantize_qkv(const float* q, const float* k, const float* v, int B,
                      int Hq, int Hkv, int N, int d, const float* s,
                      const float* inv_s, int fmt, uint8_t* q_codes,
                      uint8_t* q_sc, uint8_t* k_codes, uint8_t* k_sc,
-                     uint8_t* vt_codes, uint8_t* vt_sc) {
+                     uint8_t* vt_codes, uint8_t* vt_sc, const float* q_mu) {
   int G = Hq / Hkv;
   int beta = (fmt == OR_NVFP4) ? 16 : 32;
   int64_t Np = ((int64_t)N + 127) / 128 * 128;
@@ -343,7 +371,9 @@ void or_quantize_qkv(const float* q, const float* k, const float* v, int B,
       for (int t = 0; t < N; ++t)
         for (int c = 0; c < d; ++c) {
           float x = q[(((int64_t)b * Hq + hq) * N + t) * d + c];
-          buf[(int64_t)t * d + c] = s ? x * s[h * d + c] : x;
+          float xs = s ? x * s[h * d + c] : x;
+          if (q_mu) xs = xs - q_mu[hq * d + c];
+          buf[(int64_t)t * d + c] = xs;
         }
       int64_t base = ((int64_t)b * Hq + hq) * Np;
       or_quantize_rows(buf, Np, d, fmt, 1.0f, q_codes + base * (d / 2), q_sc + base * nb);
@@ -491,7 +521,10 @@ static float p_prescale(int fmt, int pexp) {
  * per-tile terms whose ratio minus one is the tile's normalizer error).
  * Test-only ablations: q_raw [B][Hq][N][d], k_raw [B][Hkv][N][d] and v_raw
  * [B][Hkv][N][d] (fp32, each may be NULL) replace the dequantized Q-hat,
- * K-hat or V-hat of the scores and the PV product by the given values. */
+ * K-hat or V-hat of the scores and the PV product by the given values.
+ * q_mu [Hq][d] (the Q-Mean auxiliary of or_calibrate_q_mean, or NULL): every
+ * score gets back mu . K-hat of its key, computed in fp64 from the
+ * dequantized K-hat (or k_raw), before the scaling: x = fl32((q.k + mu.k) * c). */
 void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
                   const uint8_t* k_codes, const uint8_t* k_sc,
                   const uint8_t* vt_codes, const uint8_t* vt_sc, int B, int Hq,
@@ -501,7 +534,7 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
                   uint8_t* phat_dump, uint8_t* phat_sc_dump, double* m_dump,
                   double* tsum_dump, const float* q_raw, const float* k_raw,
                   const float* v_raw, int row_begin, int row_end, int variant,
-                  float tau) {
+                  float tau, const float* q_mu) {
   int G = Hq / Hkv;
   int beta = (fmt == OR_NVFP4) ? 16 : 32;
   int64_t Np = ((int64_t)N + 127) / 128 * 128;
@@ -531,6 +564,14 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
             if (v_raw) vd[(int64_t)c * Np + t] = t < N ? (double)v_raw[(kr + t) * d + c] : 0.0;
           }
       }
+      /* the Q-Mean term of every key: bias[key] = mu . k */
+      double* bias = (double*)calloc((size_t)Np, sizeof(double));
+      if (q_mu)
+        for (int64_t key = 0; key < Np; ++key) {
+          double sb = 0.0;
+          for (int c = 0; c < d; ++c) sb += (double)q_mu[hq * d + c] * kd[key * d + c];
+          bias[key] = sb;
+        }
       double* acc = (double*)malloc(sizeof(double) * d);
       double* x = (double*)malloc(sizeof(double) * BN);
       int* vis = (int*)malloc(sizeof(int) * BN);
@@ -549,6 +590,7 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
               double sdot = 0.0;
               for (int c = 0; c < d; ++c)
                 sdot += qd[(int64_t)i * d + c] * kd[(int64_t)key * d + c];
+              sdot += bias[key];
               x[kk] = (variant & OR_VAR_EXACT) ? sdot * c_log2 : (double)(float)(sdot * c_log2);
             }
           }
@@ -564,7 +606,7 @@ void or_attention(const uint8_t* q_codes, const uint8_t* q_sc,
         if (l_phat_out) l_phat_out[row_id] = st.l_phat;
         if (l_p_out) l_p_out[row_id] = st.l_p;
       }
-      free(qd); free(kd); free(vd); free(acc); free(x); free(vis);
+      free(qd); free(kd); free(vd); free(bias); free(acc); free(x); free(vis);
     }
 }
 
