@@ -31,7 +31,8 @@ _lib = None
 
 ABI_FUNCTIONS = (
     "hifa4_codes_bytes", "hifa4_scale_bytes", "hifa4_calibrate_smooth_qk", "hifa4_quantize_qkv",
-    "hifa4_quantize_kv",
+    "hifa4_quantize_kv", "hifa4_calibrate_q_mean", "hifa4_quantize_qkv_qmean", "hifa4_q_mean_bias",
+    "hifa4_attn_fwd_qmean",
     "hifa4_attn_fwd", "hifa4_attn_fwd_ex", "hifa4_attn_fwd_dump", "hifa4_attn_fwd_fused", "hifa4_decode_workspace_size", "hifa4_decode_default_splits", "hifa4_attn_decode",
     "hifa4_decode_noalloc_max_bytes", "hifa4_attn_decode_noalloc",
     "hifa4_fp4_mma_probe", "hifa4_convert_probe", "hifa4_div6_probe", "hifa4_exp2_poly_probe", "hifa4_e2m1_map_probe", "hifa4_bf16_attn_fwd", "hifa4_bf16_transpose_v", "hifa4_wait_timeout_probe", "hifa4_kv_cache_append", "hifa4_attn_decode_cache", "hifa4_status_string", "hifa4_last_error",
@@ -56,6 +57,12 @@ def lib():
         L.hifa4_calibrate_smooth_qk.argtypes = [vp, vp, i, i, i, i, i, i, i, f, i, vp, vp, vp]
         L.hifa4_quantize_qkv.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, vp, i, vp, vp, vp, vp, vp, vp, vp]
         L.hifa4_quantize_kv.argtypes = [vp, vp, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp]
+        L.hifa4_calibrate_q_mean.argtypes = [vp, i, i, i, i, i, i, i, vp, vp, vp]
+        L.hifa4_quantize_qkv_qmean.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, vp, vp, i, vp, vp, vp, vp, vp, vp,
+                                               vp]
+        L.hifa4_q_mean_bias.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, vp]
+        L.hifa4_attn_fwd_qmean.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, f,
+                                           vp]
         L.hifa4_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, vp]
         L.hifa4_attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, i, vp, vp, vp, f,
                                         vp]
@@ -182,16 +189,45 @@ def alloc_qkv(B, Hq, Hkv, N, d, fmt, device="cuda") -> QuantizedQKV:
         B, Hq, Hkv, N, d, fmt)
 
 
-def quantize_qkv(q, k, v, s=None, inv_s=None, fmt: int = NVFP4, out: QuantizedQKV | None = None):
-    """Fused Smooth-QK scale + block quantization.  q [B,Hq,N,d], k/v [B,Hkv,N,d]."""
+def quantize_qkv(q, k, v, s=None, inv_s=None, fmt: int = NVFP4, out: QuantizedQKV | None = None,
+                 q_mu: torch.Tensor | None = None):
+    """Fused Smooth-QK scale + block quantization.  q [B,Hq,N,d], k/v [B,Hkv,N,d].
+    q_mu [Hq,d] (calibrate_q_mean): the Q-Mean auxiliary, subtracted from the
+    smoothed query (hifa4_quantize_qkv_qmean)."""
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
     q = q.contiguous(); k = k.contiguous(); v = v.contiguous()
     z = out if out is not None else alloc_qkv(B, Hq, Hkv, N, d, fmt, q.device)
+    if q_mu is not None:
+        _check(lib().hifa4_quantize_qkv_qmean(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hq, Hkv, N, d, _ptr(s),
+                                              _ptr(inv_s), _ptr(q_mu), fmt, _ptr(z.q_codes), _ptr(z.q_scales),
+                                              _ptr(z.k_codes), _ptr(z.k_scales), _ptr(z.vt_codes),
+                                              _ptr(z.vt_scales), _stream()), "quantize_qkv_qmean")
+        return z
     _check(lib().hifa4_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hq, Hkv, N, d, _ptr(s), _ptr(inv_s),
                                     fmt, _ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),
                                     _ptr(z.vt_codes), _ptr(z.vt_scales), _stream()), "quantize_qkv")
     return z
+
+
+def calibrate_q_mean(q: torch.Tensor, s: torch.Tensor | None, n_cal: int, Hkv: int | None = None) -> torch.Tensor:
+    """Q-Mean auxiliary: the per-channel mean of the smoothed query over the
+    calibration tokens.  q [B,Hq,T,d] (cuda), s [Hkv,d] or None -> mu [Hq,d]."""
+    B, Hq, T, d = q.shape
+    Hkv = s.shape[0] if s is not None else (Hkv or Hq)
+    q = q.contiguous()
+    mu = torch.empty((Hq, d), device=q.device, dtype=torch.float32)
+    _check(lib().hifa4_calibrate_q_mean(_ptr(q), _dt(q), B, Hq, Hkv, n_cal, T, d, _ptr(s), _ptr(mu), _stream()),
+           "calibrate_q_mean")
+    return mu
+
+
+def q_mean_bias(z: QuantizedQKV, q_mu: torch.Tensor) -> torch.Tensor:
+    """The Q-Mean score term mu . K-hat per key: [B,Hq,Np] float32."""
+    bias = torch.empty((z.B, z.Hq, z.Np), device=z.k_codes.device, dtype=torch.float32)
+    _check(lib().hifa4_q_mean_bias(_ptr(z.k_codes), _ptr(z.k_scales), _ptr(q_mu), z.B, z.Hq, z.Hkv, z.N, z.d, z.fmt,
+                                   _ptr(bias), _stream()), "q_mean_bias")
+    return bias
 
 
 def alloc_kv_cache(B, Hq, Hkv, kv_len, d, fmt, device="cuda") -> QuantizedQKV:
@@ -239,14 +275,24 @@ def quantize_kv(k, v, inv_s=None, fmt: int = NVFP4, Hq: int | None = None, out: 
 # --------------------------------------------------------------- attention ---
 def attn_fwd(z: QuantizedQKV, softmax_scale: float | None = None, causal: bool = True, mode: int = PREORDER,
              block_n: int = 128, out_dtype=torch.bfloat16, return_lse: bool = False, debug: bool = False,
-             out: torch.Tensor | None = None, rescale_threshold: float = 0.0):
+             out: torch.Tensor | None = None, rescale_threshold: float = 0.0, qk_bias: torch.Tensor | None = None):
     """4-bit attention forward.  Returns O [B,Hq,N,d] (and lse / debug sums).
-    rescale_threshold > 0 updates the running max lazily (hifa4_attn_fwd_ex)."""
+    rescale_threshold > 0 updates the running max lazily (hifa4_attn_fwd_ex).
+    qk_bias [B,Hq,Np] (q_mean_bias): the Q-Mean score term (hifa4_attn_fwd_qmean)."""
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(z.d)
     dev = z.q_codes.device
     o = out if out is not None else torch.empty((z.B, z.Hq, z.N, z.d), device=dev, dtype=out_dtype)
     lse = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if return_lse else None
+    if qk_bias is not None:
+        if debug:
+            raise HiFA4Error("attn_fwd: the Q-Mean forward has no debug sums")
+        _check(lib().hifa4_attn_fwd_qmean(_ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),
+                                          _ptr(z.vt_codes), _ptr(z.vt_scales), _ptr(qk_bias), z.B, z.Hq, z.Hkv, z.N,
+                                          z.d, z.fmt, float(softmax_scale), int(bool(causal)), int(mode),
+                                          int(block_n), _ptr(o), _dt(o), _ptr(lse), float(rescale_threshold),
+                                          _stream()), "attn_fwd_qmean")
+        return (o, lse) if return_lse else o
     lph = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if debug else None
     lp = torch.empty((z.B, z.Hq, z.N), device=dev, dtype=torch.float32) if debug else None
     _check(lib().hifa4_attn_fwd_ex(_ptr(z.q_codes), _ptr(z.q_scales), _ptr(z.k_codes), _ptr(z.k_scales),

@@ -73,12 +73,16 @@ bool make_tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner_bytes, uint6
 
 hifa4_status quantize_qkv_launch(const void*, const void*, const void*, int, int, int, int, int, int, const float*,
                                  const float*, int, uint8_t*, uint8_t*, uint8_t*, uint8_t*, uint8_t*, uint8_t*,
-                                 cudaStream_t);
+                                 const float*, cudaStream_t);
+hifa4_status calib_q_mean_launch(const void*, int, int, int, int, int, int, int, const float*, float*, cudaStream_t);
+hifa4_status q_mean_bias_launch(const uint8_t*, const uint8_t*, const float*, int, int, int, int, int, int, float*,
+                                cudaStream_t);
 hifa4_status calibrate_launch(const void*, const void*, int, int, int, int, int, int, int, float, int, float*, float*,
                               cudaStream_t);
 hifa4_status attn_fwd_launch(const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*, const uint8_t*,
                              const uint8_t*, int, int, int, int, int, int, float, int, int, int, void*, int, float*,
-                             float*, float*, float, const void*, int, const float*, const AttnDump*, cudaStream_t);
+                             float*, float*, float, const void*, int, const float*, const AttnDump*, const float*,
+                             cudaStream_t);
 hifa4_status decode_launch(const void*, int, const float*, const uint8_t*, const uint8_t*, const uint8_t*,
                            const uint8_t*, int, int, int, int, int, int, int, float, int, int, int, int*, void*, size_t,
                            void*, int, float, cudaStream_t);
@@ -161,7 +165,7 @@ hifa4_status hifa4_quantize_qkv(const void* q, const void* k, const void* v, hif
                     (!s || aligned16(s)) && (!inv_s || aligned16(inv_s)),
                 HIFA4_ERR_INVALID_ARG, "quantize_qkv: pointers must be 16-byte aligned");
   return quantize_qkv_launch(q, k, v, dt, B, Hq, Hkv, N, d, s, inv_s, fmt, q_codes, q_scales, k_codes, k_scales,
-                             vt_codes, vt_scales, static_cast<cudaStream_t>(stream));
+                             vt_codes, vt_scales, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dt, int B, int Hkv, int N, int d,
@@ -176,7 +180,51 @@ hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dtype dt, int
                     aligned16(vt_scales) && (!inv_s || aligned16(inv_s)),
                 HIFA4_ERR_INVALID_ARG, "quantize_kv: pointers must be 16-byte aligned");
   return quantize_qkv_launch(nullptr, k, v, dt, B, Hkv, Hkv, N, d, nullptr, inv_s, fmt, nullptr, nullptr, k_codes,
-                             k_scales, vt_codes, vt_scales, static_cast<cudaStream_t>(stream));
+                             k_scales, vt_codes, vt_scales, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_calibrate_q_mean(const void* q, hifa4_dtype dt, int B, int Hq, int Hkv, int n_cal, int ld_tok,
+                                   int d, const float* s, float* mu_out, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(q && mu_out, HIFA4_ERR_INVALID_ARG, "calibrate_q_mean: null pointer");
+  HIFA4_REQUIRE(valid_dt(dt), HIFA4_ERR_INVALID_ARG, "calibrate_q_mean: bad dtype %d", (int)dt);
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0, HIFA4_ERR_INVALID_ARG,
+                "calibrate_q_mean: bad heads B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
+  HIFA4_REQUIRE(n_cal > 0 && n_cal <= ld_tok, HIFA4_ERR_INVALID_ARG, "calibrate_q_mean: need 0 < n_cal <= ld_tok");
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "calibrate_q_mean: d=%d not in {64,128,256}", d);
+  return calib_q_mean_launch(q, dt, B, Hq, Hkv, n_cal, ld_tok, d, s, mu_out, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_quantize_qkv_qmean(const void* q, const void* k, const void* v, hifa4_dtype dt, int B, int Hq,
+                                      int Hkv, int N, int d, const float* s, const float* inv_s, const float* q_mu,
+                                      hifa4_format fmt, uint8_t* q_codes, uint8_t* q_scales, uint8_t* k_codes,
+                                      uint8_t* k_scales, uint8_t* vt_codes, uint8_t* vt_scales,
+                                      hifa4_stream_t stream) {
+  HIFA4_REQUIRE(q_mu && aligned16(q_mu), HIFA4_ERR_INVALID_ARG,
+                "quantize_qkv_qmean: q_mu must be a 16-byte aligned device pointer");
+  HIFA4_REQUIRE(q && k && v && q_codes && q_scales && k_codes && k_scales && vt_codes && vt_scales,
+                HIFA4_ERR_INVALID_ARG, "quantize_qkv_qmean: null pointer");
+  HIFA4_REQUIRE(valid_dt(dt) && valid_fmt(fmt), HIFA4_ERR_INVALID_ARG, "quantize_qkv_qmean: bad dtype/format");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0, HIFA4_ERR_INVALID_ARG,
+                "quantize_qkv_qmean: bad shape B=%d Hq=%d Hkv=%d N=%d", B, Hq, Hkv, N);
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "quantize_qkv_qmean: d=%d not in {64,128,256}", d);
+  HIFA4_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(q_codes) && aligned16(q_scales) &&
+                    aligned16(k_codes) && aligned16(k_scales) && aligned16(vt_codes) && aligned16(vt_scales) &&
+                    (!s || aligned16(s)) && (!inv_s || aligned16(inv_s)),
+                HIFA4_ERR_INVALID_ARG, "quantize_qkv_qmean: pointers must be 16-byte aligned");
+  return quantize_qkv_launch(q, k, v, dt, B, Hq, Hkv, N, d, s, inv_s, fmt, q_codes, q_scales, k_codes, k_scales,
+                             vt_codes, vt_scales, q_mu, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_q_mean_bias(const uint8_t* k_codes, const uint8_t* k_scales, const float* q_mu, int B, int Hq,
+                               int Hkv, int N, int d, hifa4_format fmt, float* bias_out, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(k_codes && k_scales && q_mu && bias_out, HIFA4_ERR_INVALID_ARG, "q_mean_bias: null pointer");
+  HIFA4_REQUIRE(valid_fmt(fmt), HIFA4_ERR_INVALID_ARG, "q_mean_bias: bad format");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0, HIFA4_ERR_INVALID_ARG,
+                "q_mean_bias: bad shape B=%d Hq=%d Hkv=%d N=%d", B, Hq, Hkv, N);
+  HIFA4_REQUIRE(Hq / Hkv <= 8, HIFA4_ERR_UNSUPPORTED, "q_mean_bias: at most 8 query heads per kv head");
+  HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "q_mean_bias: d=%d not in {64,128,256}", d);
+  return q_mean_bias_launch(k_codes, k_scales, q_mu, B, Hq, Hkv, N, d, fmt, bias_out,
+                            static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_attn_fwd(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
@@ -214,7 +262,37 @@ hifa4_status hifa4_attn_fwd_ex(const uint8_t* q_codes, const uint8_t* q_scales, 
                 "attn_fwd: problem too large");
   return attn_fwd_launch(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
                          softmax_scale, causal, mode, block_n, o, o_dt, lse, dbg_l_phat, dbg_l_p, rescale_threshold,
-                         nullptr, 0, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+                         nullptr, 0, nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+hifa4_status hifa4_attn_fwd_qmean(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                                  const uint8_t* k_scales, const uint8_t* vt_codes, const uint8_t* vt_scales,
+                                  const float* qk_bias, int B, int Hq, int Hkv, int N, int d, hifa4_format fmt,
+                                  float softmax_scale, int causal, hifa4_norm_mode mode, int block_n, void* o,
+                                  hifa4_dtype o_dt, float* lse, float rescale_threshold, hifa4_stream_t stream) {
+  HIFA4_REQUIRE(qk_bias && aligned16(qk_bias), HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_qmean: qk_bias must be a 16-byte aligned device pointer");
+  HIFA4_REQUIRE(d == 64 || d == 128, HIFA4_ERR_UNSUPPORTED, "attn_fwd_qmean: d=%d not in {64,128}", d);
+  HIFA4_REQUIRE(valid_fmt(fmt) && valid_tau(fmt, rescale_threshold), HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_qmean: rescale_threshold must be in [0, %g] for this format", max_tau(fmt));
+  HIFA4_REQUIRE(q_codes && q_scales && k_codes && k_scales && vt_codes && vt_scales && o, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_qmean: null pointer");
+  HIFA4_REQUIRE(valid_dt(o_dt), HIFA4_ERR_INVALID_ARG, "attn_fwd_qmean: bad dtype");
+  HIFA4_REQUIRE(mode == HIFA4_NORM_PREORDER || mode == HIFA4_NORM_INCONSISTENT, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_qmean: bad normalizer mode");
+  HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0, HIFA4_ERR_INVALID_ARG,
+                "attn_fwd_qmean: bad shape B=%d Hq=%d Hkv=%d N=%d", B, Hq, Hkv, N);
+  HIFA4_REQUIRE(block_n == 0 || block_n == 64 || block_n == 128, HIFA4_ERR_UNSUPPORTED,
+                "attn_fwd_qmean: block_n=%d not in {0,64,128}", block_n);
+  HIFA4_REQUIRE(softmax_scale > 0.0f, HIFA4_ERR_INVALID_ARG, "attn_fwd_qmean: softmax_scale must be > 0");
+  HIFA4_REQUIRE(aligned16(q_codes) && aligned16(q_scales) && aligned16(k_codes) && aligned16(k_scales) &&
+                    aligned16(vt_codes) && aligned16(vt_scales) && aligned16(o),
+                HIFA4_ERR_INVALID_ARG, "attn_fwd_qmean: pointers must be 16-byte aligned");
+  HIFA4_REQUIRE(static_cast<int64_t>(B) * Hq * pad128(N) < (int64_t(1) << 31), HIFA4_ERR_UNSUPPORTED,
+                "attn_fwd_qmean: problem too large");
+  return attn_fwd_launch(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
+                         softmax_scale, causal, mode, block_n, o, o_dt, lse, nullptr, nullptr, rescale_threshold,
+                         nullptr, 0, nullptr, nullptr, qk_bias, static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_attn_fwd_dump(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
@@ -248,7 +326,7 @@ hifa4_status hifa4_attn_fwd_dump(const uint8_t* q_codes, const uint8_t* q_scales
   AttnDump dump{phat_codes, phat_scales, tile_m, tile_sum_p};
   return attn_fwd_launch(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
                          softmax_scale, causal, mode, block_n, o, o_dt, nullptr, nullptr, nullptr, rescale_threshold,
-                         nullptr, 0, nullptr, &dump, static_cast<cudaStream_t>(stream));
+                         nullptr, 0, nullptr, &dump, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 hifa4_status hifa4_attn_fwd_fused(const void* q, hifa4_dtype q_dt, const float* s, const uint8_t* k_codes,
@@ -279,7 +357,7 @@ hifa4_status hifa4_attn_fwd_fused(const void* q, hifa4_dtype q_dt, const float* 
                 "attn_fwd_fused: problem too large");
   return attn_fwd_launch(nullptr, nullptr, k_codes, k_scales, vt_codes, vt_scales, B, Hq, Hkv, N, d, fmt,
                          softmax_scale, causal, mode, block_n, o, o_dt, lse, dbg_l_phat, dbg_l_p, rescale_threshold,
-                         q, q_dt, s, nullptr, static_cast<cudaStream_t>(stream));
+                         q, q_dt, s, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 size_t hifa4_decode_workspace_size(int B, int Hq, int d, int num_splits) {

@@ -112,6 +112,7 @@ struct AttnParams {
   float* dbg_l_phat;
   float* dbg_l_p;
   AttnDump dump;        // all null unless hifa4_attn_fwd_dump
+  const float* qk_bias; // [B*Hq][Np]: the Q-Mean term mu . K-hat per key, or null
   int nkt_all;          // key tiles of a whole row, ceil(N / BN): the dump's tile stride
 };
 
@@ -180,7 +181,8 @@ struct AttnCfg {
   static constexpr int OFF_XM = OFF_LOG + 512;              // row-max exchange [2][2][128] floats, or
                                                             // the correction warps' alpha [3][128]
   static constexpr int OFF_LP = OFF_XM + 2048;              // normalizer exchange [2][128] floats
-  static constexpr int OFF_BAR = OFF_LP + 1024;
+  static constexpr int OFF_BIAS = OFF_LP + 1024;            // Q-Mean score term per key: [NS][BN] floats
+  static constexpr int OFF_BAR = OFF_BIAS + NS * BN * 4;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
   // s_full[NSB], s_empty[NSB], p_full[2], p_empty[2], o_ready
   static constexpr int NBAR = 1 + 4 * NS + 2 * NSB + 4 + 1 + 3 + 24 + 4;
@@ -277,7 +279,7 @@ __device__ __forceinline__ void rescale_o_rows(uint32_t a0, uint32_t al, bool wi
   }
 }
 
-template <int D, int BN, int FMT, bool PREORDER, bool DBG>
+template <int D, int BN, int FMT, bool PREORDER, bool EXT>
 __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, FMT>::CTAS_PER_SM)
     attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -307,6 +309,9 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
   const int row0 = qtile * C::BM;
   const int kv_end = p.causal ? min(p.N, row0 + C::BM) : p.N;
   const int nkt = (kv_end + BN - 1) / BN;
+  // Q-Mean auxiliary: add the score term mu . K-hat of each key (EXT only;
+  // needs the single K/V barrier per stage, d <= 128)
+  const bool qbias = EXT && C::KV_ONE && p.qk_bias != nullptr;
 
   // ---- setup ----
   if (threadIdx.x == 0) {
@@ -386,9 +391,11 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         const int st = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
         if (!mbar_wait(BAR(B_KEMPTY + st), ph ^ 1, abort_flag, kErrTimeoutTma)) break;
-        // with one barrier per stage it expects the V copies' bytes too
+        // with one barrier per stage it expects the V copies' bytes too (and
+        // the Q-Mean score terms of the tile's keys)
         mbar_arrive_expect_tx(BAR(B_KFULL + st), C::SZ_K + C::NKC_Q * 512 +
-                                                     (C::KV_ONE ? C::SZ_V + C::NRG_V * C::NCH_V * 512 : 0));
+                                                     (C::KV_ONE ? C::SZ_V + C::NRG_V * C::NCH_V * 512 : 0) +
+                                                     (C::KV_ONE && qbias ? BN * 4 : 0));
         tma_load_2d(sbase + C::OFF_K + st * C::SZ_K, &tm_k, 0, kvbh * p.Np + j * BN, BAR(B_KFULL + st));
         bulk_load(sbase + C::OFF_KSF + st * C::NKC_Q * 512,
                   p.k_sf + static_cast<int64_t>(kvbh) * p.sf_qk_head + static_cast<int64_t>((j * BN) >> 7) * C::NKC_Q * 512,
@@ -397,6 +404,11 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
         const uint32_t vbar = BAR((C::KV_ONE ? B_KFULL : B_VFULL) + st);
         if (!C::KV_ONE) mbar_arrive_expect_tx(vbar, C::SZ_V + C::NRG_V * C::NCH_V * 512);
         tma_load_2d(sbase + C::OFF_V + st * C::SZ_VX, &tm_v, j * C::PROW, kvbh * D, vbar);
+        // the tile's Q-Mean score terms go with V: stage st is free once PV of
+        // its previous tile retired, which the softmax warps' use precedes
+        if (C::KV_ONE && qbias)
+          bulk_load(sbase + C::OFF_BIAS + st * BN * 4, p.qk_bias + static_cast<int64_t>(bhq) * p.Np + j * BN, BN * 4,
+                    vbar);
         const int chunk0 = (j * BN) / (4 * C::BETA);
         for (int rg = 0; rg < C::NRG_V; ++rg)
           bulk_load(sbase + C::OFF_VSF + (st * C::NRG_V + rg) * C::NCH_V * 512,
@@ -594,11 +606,11 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
     float m = -INFINITY;
     float l_p = 0.0f;
     // the running sum of P: the normalizer of the inconsistent mode, else a
-    // debug output only (its pointers reach the DBG instantiation alone).  At
+    // debug output only (its pointers reach the EXT instantiation alone).  At
     // d = 256 the production kernel knows at compile time that it forms no
     // sum (measured 1.7 % faster); at d <= 128 the runtime test schedules
     // better (1.3 % faster), although the pointer is always null there.
-    const bool want_lp = !PREORDER || ((DBG || D != 256) && (p.dbg_l_p != nullptr || (DBG && p.dump.sum_p != nullptr)));
+    const bool want_lp = !PREORDER || ((EXT || D != 256) && (p.dbg_l_p != nullptr || (EXT && p.dump.sum_p != nullptr)));
     constexpr float kGP = FMT == HIFA4_NVFP4 ? 0.00390625f : 1.0f;   // g_P = 2^-8 (NVFP4)
     // pairs (of every eight) whose 2^y runs on the FMA pipe instead of MUFU
     constexpr int kPolyPairs = HIFA4_POLY_PAIRS >= 0 ? HIFA4_POLY_PAIRS : (D == 256 ? 1 : 2);
@@ -686,6 +698,26 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_SEMPTY + sb));
+      if (qbias) {
+        // the score terms of this tile's keys landed with its K/V copies (the
+        // stage's barrier: its next phase, tile j + NS, needs PV_j, which
+        // needs this warp's P-hat_j, so the parity wait is exact)
+        const int st = j % C::NS;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(BAR(B_KFULL + st), (j / C::NS) & 1, abort_flag, kErrTimeoutSoftmax))) {
+          ok = false;
+          break;
+        }
+        const float4* b4 = reinterpret_cast<const float4*>(smem + C::OFF_BIAS + st * BN * 4 + hw * HB * 4);
+#pragma unroll
+        for (int i = 0; i < HB / 4; ++i) {
+          const float4 bb = b4[i];
+          s[4 * i] = __fadd_rn(s[4 * i], bb.x);
+          s[4 * i + 1] = __fadd_rn(s[4 * i + 1], bb.y);
+          s[4 * i + 2] = __fadd_rn(s[4 * i + 2], bb.z);
+          s[4 * i + 3] = __fadd_rn(s[4 * i + 3], bb.w);
+        }
+      }
       // mask (only tiles that reach past the diagonal or past N need it)
       const int kbase = j * BN + hw * HB;
       const bool need_mask = (j * BN + BN > p.N) || (p.causal && j * BN + BN - 1 > row0);
@@ -807,7 +839,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       if (want_lp) quant_tile(std::true_type{});
       else quant_tile(std::false_type{});
       if (want_lp) l_p = fmaf(alpha, l_p, psum);
-      if (DBG && p.dump.codes != nullptr && row < p.N) {
+      if (EXT && p.dump.codes != nullptr && row < p.N) {
         // debug view of this tile: the codes and scales as they go to the
         // PV MMA, the running max, and (on the path that forms P) sum(P)
         const int64_t rt = (static_cast<int64_t>(bhq) * p.N + row) * p.nkt_all + j;
@@ -958,8 +990,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BN, FMT>::NTHREADS, AttnCfg<D, BN, 
       if (store && hw == 0) {
         const int64_t ri = static_cast<int64_t>(bhq) * p.N + row;
         if (p.lse) p.lse[ri] = m + log2f(l_used);
-        if (DBG && p.dbg_l_phat) p.dbg_l_phat[ri] = l_phat;
-        if (DBG && p.dbg_l_p) p.dbg_l_p[ri] = l_p;
+        if (EXT && p.dbg_l_phat) p.dbg_l_phat[ri] = l_phat;
+        if (EXT && p.dbg_l_p) p.dbg_l_p[ri] = l_p;
       }
     }
   }
@@ -979,9 +1011,10 @@ bool make_tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner_bytes, uint6
 template <int D, int BN, int FMT, bool PRE>
 static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const uint8_t* vc, const AttnParams& p,
                                   cudaStream_t st) {
-  // the debug views (the P-hat dump, the sums of P and P-hat) are their own
-  // instantiation: the production kernel carries none of their code
-  const bool dbg = p.dump.codes != nullptr || p.dbg_l_p != nullptr || p.dbg_l_phat != nullptr;
+  // the optional extras (the debug views -- the P-hat dump, the sums of P
+  // and P-hat -- and the Q-Mean score term) are their own instantiation: the
+  // production kernel carries none of their code
+  const bool ext = p.dump.codes != nullptr || p.dbg_l_p != nullptr || p.dbg_l_phat != nullptr || p.qk_bias != nullptr;
   using C = AttnCfg<D, BN, FMT>;
   CUtensorMap tq, tk, tv;
   const uint64_t Np = static_cast<uint64_t>(p.Np);
@@ -994,7 +1027,7 @@ static hifa4_status launch_attn_t(const uint8_t* qc, const uint8_t* kc, const ui
     set_last_error("cuTensorMapEncodeTiled failed");
     return HIFA4_ERR_CUDA;
   }
-  auto kern = dbg ? attn_fwd_fp4_kernel<D, BN, FMT, PRE, true> : attn_fwd_fp4_kernel<D, BN, FMT, PRE, false>;
+  auto kern = ext ? attn_fwd_fp4_kernel<D, BN, FMT, PRE, true> : attn_fwd_fp4_kernel<D, BN, FMT, PRE, false>;
   const int smem = C::SMEM_REQ;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * p.num_qtiles;
@@ -1016,8 +1049,10 @@ hifa4_status attn_fwd_launch(const uint8_t* qc, const uint8_t* qs, const uint8_t
                              const uint8_t* vc, const uint8_t* vs, int B, int Hq, int Hkv, int N, int d, int fmt,
                              float softmax_scale, int causal, int mode, int block_n, void* o, int o_dt, float* lse,
                              float* dbg_l_phat, float* dbg_l_p, float rescale_threshold, const void* q_raw,
-                             int q_dt, const float* q_s, const AttnDump* dump, cudaStream_t st) {
+                             int q_dt, const float* q_s, const AttnDump* dump, const float* qk_bias,
+                             cudaStream_t st) {
   AttnParams p;
+  p.qk_bias = qk_bias;
   p.dump = dump != nullptr ? *dump : AttnDump{nullptr, nullptr, nullptr, nullptr};
   p.q_raw = q_raw;
   p.q_s = q_s;

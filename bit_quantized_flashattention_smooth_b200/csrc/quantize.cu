@@ -83,9 +83,9 @@ __device__ __forceinline__ uint32_t quant_part(const float (&v)[8], uint32_t& pa
 // bytes per group, the codes by RPI * D/2, the input by RPI * D values.
 template <int FMT, typename T, int D>
 __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H, int G, int N, int Np,
-                                                  const float* __restrict__ scale, uint8_t* __restrict__ codes,
-                                                  uint8_t* __restrict__ sf, int64_t sf_head_bytes, int cta,
-                                                  const float* inv_tab) {
+                                                  const float* __restrict__ scale, const float* __restrict__ mu,
+                                                  uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                  int64_t sf_head_bytes, int cta, const float* inv_tab) {
   using R = RowTile<FMT, D>;
   constexpr int BETA = R::BETA, U = R::U, CPR = R::CPR, RPI = R::RPI, LPB = R::LPB, NB = R::NB;
   constexpr int WPR = (NB + 3) / 4;        // scale words per row
@@ -112,6 +112,15 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
     const float4 a = s4[0], b = s4[1];
     sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w; sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
   }
+  // Q-Mean auxiliary: the head's calibration mean, subtracted after the
+  // smoothing multiply from real rows (negated here: x - mu = x + (-mu) exactly)
+  float nmu[8];
+  if (mu != nullptr) {
+    const float4* m4 = reinterpret_cast<const float4*>(mu + static_cast<int64_t>(bh % H) * D + ch * 8);
+    const float4 a = m4[0], b = m4[1];
+    nmu[0] = -a.x; nmu[1] = -a.y; nmu[2] = -a.z; nmu[3] = -a.w; nmu[4] = -b.x; nmu[5] = -b.y; nmu[6] = -b.z;
+    nmu[7] = -b.w;
+  }
   uint8_t* cdst = codes + (static_cast<int64_t>(bh) * Np + t0) * (D / 2) + ch * 4;
   uint8_t* sdst = sf + static_cast<int64_t>(bh) * sf_head_bytes + sf_word_offset(t0, blk / 4, WPR) + blk % 4;
 #pragma unroll
@@ -132,6 +141,14 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
         const float2 p2 = qmul2(make_float2(v[i], v[i + 1]), make_float2(sv[i], sv[i + 1]));
         v[i] = p2.x;
         v[i + 1] = p2.y;
+      }
+    }
+    if (mu != nullptr && u * RPI < nvalid) {
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const float2 d2 = fadd2(make_float2(v[i], v[i + 1]), make_float2(nmu[i], nmu[i + 1]));
+        v[i] = d2.x;
+        v[i + 1] = d2.y;
       }
     }
     uint32_t packed;
@@ -259,7 +276,7 @@ __device__ __forceinline__ void quantize_v_cols(const T* __restrict__ v, int N, 
 // the next nq Q rows, the rest K rows.
 struct QuantArgs {
   const void *q, *k, *v;
-  const float *s, *inv_s;
+  const float *s, *inv_s, *q_mu;
   uint8_t *qc, *qs, *kc, *ks, *vc, *vs;
   int B, Hq, Hkv, N, Np, d;
   int64_t sf_qk_head, sf_v_head, q_rows, k_rows, v_tasks;
@@ -279,10 +296,10 @@ __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a)
     if (task < a.v_tasks)
       quantize_v_cols<FMT, T>(static_cast<const T*>(a.v), a.N, a.Np, a.d, a.vc, a.vs, a.sf_v_head, task, inv_tab);
   } else if (bid < a.nq_ctas) {
-    quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.s, a.qc, a.qs,
-                                 a.sf_qk_head, bid, inv_tab);
+    quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.s, a.q_mu, a.qc,
+                                 a.qs, a.sf_qk_head, bid, inv_tab);
   } else if (bid < a.nq_ctas + a.nk_ctas) {
-    quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.k), a.Hkv, 1, a.N, a.Np, a.inv_s, a.kc, a.ks,
+    quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.k), a.Hkv, 1, a.N, a.Np, a.inv_s, nullptr, a.kc, a.ks,
                                  a.sf_qk_head, bid - a.nq_ctas, inv_tab);
   }
 }
@@ -356,6 +373,74 @@ __global__ void calib_finalize_kernel(float* s, float* inv_s, int d, double alph
   inv_s[i] = __fdiv_rn(1.0f, sv);
 }
 
+// Q-Mean auxiliary (a reading: the pages name "the adopted Q-Mean auxiliary"
+// and nothing more): mu[hq][c] = fl32(sum_{b, t < n_cal} fl32(q * s[h][c]) /
+// (B * n_cal)), the sum in fp64 in the order b, then t -- one thread per
+// (q head, channel), so the result is reproducible bit for bit.
+template <typename T>
+__global__ void calib_q_mean_kernel(const T* __restrict__ q, int B, int Hq, int G, int ld_tok, int n_cal, int d,
+                                    const float* __restrict__ s, float* __restrict__ mu) {
+  const int hq = blockIdx.x, c = threadIdx.x;
+  if (c >= d) return;
+  const float sc = s != nullptr ? s[(hq / G) * d + c] : 1.0f;
+  double acc = 0.0;
+  for (int b = 0; b < B; ++b) {
+    const T* p = q + ((static_cast<int64_t>(b) * Hq + hq) * ld_tok) * d + c;
+    for (int t = 0; t < n_cal; ++t) {
+      float x;
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) x = __bfloat162float(p[static_cast<int64_t>(t) * d]);
+      else x = __half2float(p[static_cast<int64_t>(t) * d]);
+      acc += static_cast<double>(s != nullptr ? __fmul_rn(x, sc) : x);
+    }
+  }
+  mu[hq * d + c] = static_cast<float>(acc / static_cast<double>(static_cast<int64_t>(B) * n_cal));
+}
+
+// The rank-one score term of the Q-Mean auxiliary: bias[b][hq][key] =
+// mu[hq] . K-hat[b][h(hq)][key] for every key of the padded rows (padding
+// keys have zero codes: bias 0), accumulated in fp64 (each product of an fp32
+// mu and an exact K-hat element is exact there) and rounded once to fp32.  One
+// thread per (b, kv head, key) decodes its K-hat row once (E2M1 x block
+// scale, exact in fp32) and serves the G query heads of the group.
+template <int FMT>
+__global__ void q_mean_bias_kernel(const uint8_t* __restrict__ kc, const uint8_t* __restrict__ ks,
+                                   const float* __restrict__ mu, int Hq, int Hkv, int Np, int d,
+                                   int64_t sf_head_bytes, float* __restrict__ bias) {
+  constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
+  extern __shared__ float mu_sh[];                 // [G][d] of this kv head
+  const int G = Hq / Hkv;
+  const int bh = blockIdx.y;                       // b * Hkv + kv head
+  const int kvh = bh % Hkv, b = bh / Hkv;
+  for (int i = threadIdx.x; i < G * d; i += blockDim.x) mu_sh[i] = mu[(kvh * G) * d + i];
+  __syncthreads();
+  const int key = blockIdx.x * blockDim.x + threadIdx.x;
+  if (key >= Np) return;
+  const uint8_t* row = kc + (static_cast<int64_t>(bh) * Np + key) * (d / 2);
+  const uint8_t* sfh = ks + static_cast<int64_t>(bh) * sf_head_bytes;
+  const int nkc = (d / BETA + 3) / 4;
+  double acc[8];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) acc[g] = 0.0;
+  for (int c0 = 0; c0 < d; c0 += BETA) {
+    const int blk = c0 / BETA;
+    const uint32_t sc = sfh[sf_word_offset(key, blk / 4, nkc) + blk % 4];
+    // UE4M3 value, or 2^(sc - 127) (code 0 is 2^-127, a subnormal)
+    const float scale = FMT == HIFA4_NVFP4 ? ue4m3_to_f32(sc) : __uint_as_float(sc == 0 ? 0x00400000u : sc << 23);
+    for (int c = c0; c < c0 + BETA; ++c) {
+      const uint32_t code = (row[c / 2] >> (4 * (c & 1))) & 15u;
+      // E2M1 magnitude: exponent field e, mantissa bit m: 0.5 m for e = 0,
+      // else 2^(e-1) (1 + m/2)
+      const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+      const float mag = e == 0 ? 0.5f * static_cast<float>(m) : __uint_as_float(((e + 126u) << 23) | (m << 22));
+      const float kv = __fmul_rn((code & 8u) ? -mag : mag, scale);
+      for (int g = 0; g < G && g < 8; ++g)
+        acc[g] = __fma_rn(static_cast<double>(mu_sh[g * d + c]), static_cast<double>(kv), acc[g]);
+    }
+  }
+  for (int g = 0; g < G && g < 8; ++g)
+    bias[(static_cast<int64_t>(b) * Hq + kvh * G + g) * Np + key] = static_cast<float>(acc[g]);
+}
+
 // ---------------------------------------------------------- host launchers ---
 template <typename T, int D>
 static void launch_quant_d(const QuantArgs& a, int fmt, cudaStream_t st) {
@@ -373,9 +458,10 @@ static void launch_quant(const QuantArgs& a, int fmt, cudaStream_t st) {
 // q == nullptr quantizes only K and V (a KV cache).
 hifa4_status quantize_qkv_launch(const void* q, const void* k, const void* v, int dt, int B, int Hq, int Hkv, int N,
                                  int d, const float* s, const float* inv_s, int fmt, uint8_t* qc, uint8_t* qs,
-                                 uint8_t* kc, uint8_t* ks, uint8_t* vc, uint8_t* vs, cudaStream_t st) {
+                                 uint8_t* kc, uint8_t* ks, uint8_t* vc, uint8_t* vs, const float* q_mu,
+                                 cudaStream_t st) {
   QuantArgs a;
-  a.q = q; a.k = k; a.v = v; a.s = s; a.inv_s = inv_s;
+  a.q = q; a.k = k; a.v = v; a.s = s; a.inv_s = inv_s; a.q_mu = q_mu;
   a.qc = qc; a.qs = qs; a.kc = kc; a.ks = ks; a.vc = vc; a.vs = vs;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.N = N; a.Np = static_cast<int>(pad128(N)); a.d = d;
   a.sf_qk_head = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
@@ -401,6 +487,30 @@ static void launch_calib_amax(const void* x, int B, int H, int ld_tok, int n_cal
   const int rows_per_cta = 64;
   dim3 grid(static_cast<unsigned>((rows + rows_per_cta - 1) / rows_per_cta), H);
   calib_amax_kernel<T><<<grid, d, 0, st>>>(static_cast<const T*>(x), B, H, ld_tok, n_cal, d, hpg, rows_per_cta, out);
+}
+
+hifa4_status calib_q_mean_launch(const void* q, int dt, int B, int Hq, int Hkv, int n_cal, int ld_tok, int d,
+                                 const float* s, float* mu, cudaStream_t st) {
+  if (dt == HIFA4_BF16)
+    calib_q_mean_kernel<__nv_bfloat16><<<Hq, d, 0, st>>>(static_cast<const __nv_bfloat16*>(q), B, Hq, Hq / Hkv,
+                                                         ld_tok, n_cal, d, s, mu);
+  else
+    calib_q_mean_kernel<__half><<<Hq, d, 0, st>>>(static_cast<const __half*>(q), B, Hq, Hq / Hkv, ld_tok, n_cal,
+                                                  d, s, mu);
+  return launch_status("calibrate_q_mean");
+}
+
+hifa4_status q_mean_bias_launch(const uint8_t* kc, const uint8_t* ks, const float* mu, int B, int Hq, int Hkv, int N,
+                                int d, int fmt, float* bias, cudaStream_t st) {
+  const int Np = static_cast<int>(pad128(N));
+  const int64_t sf_head = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
+  const dim3 grid(static_cast<unsigned>(Np / 128), static_cast<unsigned>(B * Hkv));
+  const size_t smem = static_cast<size_t>(Hq / Hkv) * d * sizeof(float);
+  if (fmt == HIFA4_NVFP4)
+    q_mean_bias_kernel<HIFA4_NVFP4><<<grid, 128, smem, st>>>(kc, ks, mu, Hq, Hkv, Np, d, sf_head, bias);
+  else
+    q_mean_bias_kernel<HIFA4_MXFP4><<<grid, 128, smem, st>>>(kc, ks, mu, Hq, Hkv, Np, d, sf_head, bias);
+  return launch_status("q_mean_bias");
 }
 
 hifa4_status calibrate_launch(const void* q, const void* k, int dt, int B, int Hq, int Hkv, int n_cal, int ld_tok,

@@ -18,6 +18,12 @@ Recipes (one per workload):
   long_prefill   B8 Hq32 Hkv8 d128 N16384 causal bf16; Q ~ N(0,1); K i.i.d.
                  Student-t (nu=3) in every channel; RoPE theta 1e6; V ~ N(0,1);
                  calibration tokens 0..255.
+  qwen3_qmean    qwen3_prefill's shapes and K, with seed 5 and a per-channel
+                 offset in Q: channels 58-60 (the first halves of the next
+                 three lowest-frequency RoPE pairs, beside K's outliers) get +8
+                 before RoPE, so after the slow rotation they carry a
+                 near-constant channel mean (the case the Q-Mean auxiliary
+                 addresses).
   split_decode   B64 Hq32 Hkv8 d128, KV length 32768, one query; K,V ~ N(0,1)
                  with qwen3_prefill's outlier pattern and RoPE; the calibration
                  set is a 256-token slice of K plus an independent 256-token Q
@@ -49,6 +55,8 @@ class Workload:
     outlier_scale: float = 0.0
     k_dist: str = "normal"   # "normal" | "student_t3"
     decode: bool = False
+    q_offset_channels: tuple = field(default_factory=tuple)
+    q_offset: float = 0.0
 
     @property
     def G(self) -> int:
@@ -70,6 +78,8 @@ WORKLOADS = {
                                _lowfreq_pairs(256, 4), 10.0),
     "long_prefill": Workload("long_prefill", 8, 32, 8, 16384, 128, True, "bf16", 3, 256, 64, 1e6,
                              (), 0.0, "student_t3"),
+    "qwen3_qmean": Workload("qwen3_qmean", 1, 32, 8, 4096, 128, True, "bf16", 5, 256, 64, 1e6,
+                            _lowfreq_pairs(128, 3), 15.0, q_offset_channels=(58, 59, 60), q_offset=8.0),
     "split_decode": Workload("split_decode", 64, 32, 8, 32768, 128, False, "bf16", 4, 256, 128, 1e6,
                              _lowfreq_pairs(128, 3), 15.0, decode=True),
 }
@@ -141,6 +151,8 @@ def make_prefill(w: Workload, N: int | None = None, B: int | None = None):
     B = w.B if B is None else B
     rng = np.random.Generator(np.random.PCG64(w.seed))
     q = rng.standard_normal((B, w.Hq, N, w.d), dtype=np.float32)
+    for c in w.q_offset_channels:
+        q[..., c] += np.float32(w.q_offset)
     k = _draw_k(rng, (B, w.Hkv, N, w.d), w)
     v = rng.standard_normal((B, w.Hkv, N, w.d), dtype=np.float32)
     if w.theta is not None:

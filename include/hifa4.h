@@ -138,6 +138,47 @@ HIFA4_API hifa4_status hifa4_quantize_kv(const void* k, const void* v, hifa4_dty
                                          uint8_t* k_scales, uint8_t* vt_codes, uint8_t* vt_scales,
                                          hifa4_stream_t stream);
 
+/* ------------------------------------------------- Q-Mean auxiliary --- */
+
+/* The pages name "the adopted Q-Mean auxiliary" (paper Abstract para 3) and
+ * nothing more; the reading built here (off unless these entry points are
+ * used): the per-channel calibration mean mu of the smoothed query is
+ * subtracted before Q is quantized, and every score gets back the rank-one
+ * term mu . K-hat of its key, so that without quantization the scores are
+ * unchanged ((q - mu) . k + mu . k = q . k).  Use: hifa4_calibrate_q_mean ->
+ * hifa4_quantize_qkv_qmean -> hifa4_q_mean_bias -> hifa4_attn_fwd_qmean. */
+
+/* mu[hq][c] = fl32( sum_{b, t < n_cal} fl32(q[b][hq][t][c] * s[hq/G][c]) /
+ * (B * n_cal) ), the sum in fp64 in the order b, then t (reproducible bit for
+ * bit).  q: device [B][Hq][ld_tok][d] of `dt`; s: device float [Hkv][d] (the
+ * Smooth-QK scales of hifa4_calibrate_smooth_qk) or NULL for 1; mu_out:
+ * device float [Hq][d], caller-owned.  Requires 0 < n_cal <= ld_tok,
+ * Hq % Hkv == 0, d in {64, 128, 256}. */
+HIFA4_API hifa4_status hifa4_calibrate_q_mean(const void* q, hifa4_dtype dt, int B, int Hq, int Hkv, int n_cal,
+                                              int ld_tok, int d, const float* s, float* mu_out,
+                                              hifa4_stream_t stream);
+
+/* hifa4_quantize_qkv with the Q-Mean auxiliary: rows t < N of Q quantize
+ * fl32(fl32(q*s) - mu[hq]) (padding rows stay zero); K and V exactly as in
+ * hifa4_quantize_qkv.  q_mu: device float [Hq][d], 16-byte aligned.  Other
+ * arguments, layouts and requirements as hifa4_quantize_qkv. */
+HIFA4_API hifa4_status hifa4_quantize_qkv_qmean(const void* q, const void* k, const void* v, hifa4_dtype dt,
+                                                int B, int Hq, int Hkv, int N, int d, const float* s,
+                                                const float* inv_s, const float* q_mu, hifa4_format fmt,
+                                                uint8_t* q_codes, uint8_t* q_scales, uint8_t* k_codes,
+                                                uint8_t* k_scales, uint8_t* vt_codes, uint8_t* vt_scales,
+                                                hifa4_stream_t stream);
+
+/* The rank-one score term of the Q-Mean auxiliary: bias_out[b][hq][key] =
+ * mu[hq] . K-hat[b][hq/G][key] (fp32) for every key of the padded rows
+ * (Np = N rounded up to 128; padding keys give 0).  k_codes / k_scales: the
+ * K-hat layouts of hifa4_quantize_qkv(_qmean) with the same fmt; q_mu:
+ * device float [Hq][d]; bias_out: device float [B][Hq][Np], caller-owned.
+ * Requires Hq / Hkv <= 8. */
+HIFA4_API hifa4_status hifa4_q_mean_bias(const uint8_t* k_codes, const uint8_t* k_scales, const float* q_mu,
+                                         int B, int Hq, int Hkv, int N, int d, hifa4_format fmt,
+                                         float* bias_out, hifa4_stream_t stream);
+
 /* ------------------------------------------------ attention forward --- */
 
 /* 4-bit FlashAttention forward (paper Abstract paras 1-2).  For each (b, hq)
@@ -214,6 +255,22 @@ HIFA4_API hifa4_status hifa4_attn_fwd_dump(const uint8_t* q_codes, const uint8_t
                                            hifa4_dtype o_dt, float rescale_threshold, uint8_t* phat_codes,
                                            uint8_t* phat_scales, float* tile_m, float* tile_sum_p,
                                            hifa4_stream_t stream);
+
+/* hifa4_attn_fwd_ex with the Q-Mean auxiliary: every score S of key k gets
+ * qk_bias[b][hq][k] added before the softmax scaling (fl32(S + bias), then
+ * as in hifa4_attn_fwd_ex).  Inputs: Q-hat from hifa4_quantize_qkv_qmean,
+ * qk_bias from hifa4_q_mean_bias (device float [B][Hq][Np], 16-byte
+ * aligned).  Runs in the kernel instantiation that carries the optional
+ * extras.  Requires d in {64, 128} (the score terms ride on the key tile's
+ * single K/V barrier, which the two-stage d = 256 pipeline does not use);
+ * other arguments and requirements as hifa4_attn_fwd_ex (no debug sums). */
+HIFA4_API hifa4_status hifa4_attn_fwd_qmean(const uint8_t* q_codes, const uint8_t* q_scales,
+                                            const uint8_t* k_codes, const uint8_t* k_scales,
+                                            const uint8_t* vt_codes, const uint8_t* vt_scales,
+                                            const float* qk_bias, int B, int Hq, int Hkv, int N, int d,
+                                            hifa4_format fmt, float softmax_scale, int causal,
+                                            hifa4_norm_mode mode, int block_n, void* o, hifa4_dtype o_dt,
+                                            float* lse, float rescale_threshold, hifa4_stream_t stream);
 
 /* The prefill forward with Smooth-QK and the Q quantization fused into the
  * attention kernel (the paper's Abstract para 2: Smooth-QK needs "only a

@@ -48,7 +48,8 @@ class Barrier:
 
 
 class Sim:
-    def __init__(self, nkt, NS, NSB, NH, rng, fused_q=False, relax_lag=None, two_issuers=False, kv_one=True):
+    def __init__(self, nkt, NS, NSB, NH, rng, fused_q=False, relax_lag=None, two_issuers=False, kv_one=True,
+                 qbias=False):
         self.nkt, self.NS, self.NSB, self.NH, self.rng = nkt, NS, NSB, NH, rng
         # a warp that does not rescale O in tile j waits for PV_{j - relax_lag},
         # or for no product at all (None: the kernel with one MMA-issuing
@@ -61,6 +62,11 @@ class Sim:
         # one barrier per K/V stage that completes when both copies landed
         # (the kernel's default), or one barrier per copy
         self.kv_one = kv_one
+        # the Q-Mean score terms ride on the K/V barrier; the softmax warps
+        # wait for it before reading them (and the TMA reloads a stage only
+        # after PV of its previous tile)
+        self.qbias = qbias
+        self.bias_stage = [None] * NS
         self.W = 4 * NH
         self.fused_q = fused_q
         B = Barrier
@@ -158,6 +164,11 @@ class Sim:
                 raise ProtocolError(f"warp {w} read S buffer {sb} holding tile {self.s_buf[sb]} for tile {j}")
             self.s_readers[sb].add(w)
             self.bars[f"SEMPTY{sb}"].arrive()
+            if self.qbias:
+                st = j % self.NS
+                yield from self.wait(f"KVFULL{st}", (j // self.NS) & 1, j // self.NS + 1)
+                if self.v_stage[st] != j:
+                    raise ProtocolError(f"warp {w} read the score terms of stage {st} holding {self.v_stage[st]}")
             if self.NH == 2:
                 self.xm[j & 1][w] = j
                 self.bars[f"XM{w & 3}"].arrive()
@@ -265,6 +276,15 @@ class Sim:
 def test_prefill_protocol_random_schedules(NH, NS, NSB, nkt, relax_lag, kv_one):
     for seed in range(40):
         Sim(nkt, NS, NSB, NH, random.Random(1000 * nkt + seed), relax_lag=relax_lag, kv_one=kv_one).run()
+
+
+@pytest.mark.parametrize("NH,NSB", [(1, 1), (2, 2)])
+@pytest.mark.parametrize("nkt", [1, 3, 7])
+def test_q_mean_terms_protocol(NH, NSB, nkt):
+    """The Q-Mean score terms travel with V on the stage's single K/V
+    barrier; a softmax warp reads stage j % NS only while it holds tile j."""
+    for seed in range(40):
+        Sim(nkt, 3, NSB, NH, random.Random(5000 * nkt + seed), qbias=True).run()
 
 
 @pytest.mark.parametrize("nkt", [2, 5, 9])

@@ -17,6 +17,7 @@ from bit_quantized_flashattention_smooth_b200 import workloads as W
     ("gemma2_prefill", (1, 16, 8, 8192, 256), torch.bfloat16),
     ("long_prefill", (8, 32, 8, 16384, 128), torch.bfloat16),
     ("split_decode", (64, 32, 8, 32768, 128), torch.bfloat16),
+    ("qwen3_qmean", (1, 32, 8, 4096, 128), torch.bfloat16),
 ])
 def test_workload_table(name, shape, dtype):
     w = W.WORKLOADS[name]
@@ -101,3 +102,20 @@ def test_prefill_recipe_uses_exact_rope(name):
     qn, kn = W.rope_neox(qn, w.theta), W.rope_neox(kn, w.theta)
     for a, b in ((q, qn), (k, kn), (v, vn)):
         assert torch.equal(a, torch.from_numpy(b).to(W.torch_dtype(w.dtype)))
+
+
+def test_q_offset_channels_carry_a_near_constant_mean():
+    """qwen3_qmean: +8 on Q channels 58-60 before RoPE; those pairs barely
+    rotate, so the channels keep a mean near 8 (the other channels near 0),
+    and K keeps qwen3_prefill's outliers on channels 61-63 / 125-127."""
+    w = W.WORKLOADS["qwen3_qmean"]
+    q, k, _ = W.make_prefill(w, N=512)
+    qf = q.float()
+    m = qf[..., 58:61].mean(dim=(0, 1, 2))
+    assert torch.all((m > 7.5) & (m < 8.5)), m
+    rest = [c for c in range(w.d) if c not in (58, 59, 60)]
+    assert qf[..., rest].mean(dim=(0, 1, 2)).abs().max() < 0.3
+    assert k.float()[..., [61, 62, 63]].mean() > 10.0
+    w0 = W.WORKLOADS["qwen3_prefill"]
+    q0, _, _ = W.make_prefill(w0, N=512)
+    assert q0.float()[..., 58:61].mean().abs() < 0.2
