@@ -479,6 +479,45 @@ def comparisons(res):
     return out
 
 
+def q_mean_comparison():
+    """The Q-Mean auxiliary (a reading: the pages name it only) on the
+    Q-offset workload and on qwen3 (no offsets), both formats: the time of each
+    stage (L2 flushed) and the deviation of the output from exact attention
+    (heads 0-3, by query-tile range), with and without the auxiliary."""
+    import bit_quantized_flashattention_smooth_b200 as h
+    out = []
+    for name in ("qwen3_qmean", "qwen3_prefill"):
+        w = W.WORKLOADS[name]
+        q, k, v = (t.cuda() for t in W.make_prefill(w))
+        s, inv = h.calibrate_smooth_qk(q[:, :, : w.n_cal], k[:, :, : w.n_cal], w.n_cal)
+        mu = h.calibrate_q_mean(q[:, :, : w.n_cal], s, w.n_cal)
+        scale = 1.0 / math.sqrt(w.d)
+        heads = list(range(4))
+        ex = exact_attention_rows(q, k, v, w.causal, scale, heads)
+        for fmt_name, fmt in (("nvfp4", h.NVFP4), ("mxfp4", h.MXFP4)):
+            z = h.alloc_qkv(w.B, w.Hq, w.Hkv, w.N, w.d, fmt)
+            o = torch.empty((w.B, w.Hq, w.N, w.d), device="cuda", dtype=W.torch_dtype(w.dtype))
+            rec = {"workload": name, "format": fmt_name}
+            h.quantize_qkv(q, k, v, s, inv, fmt, out=z)
+            rec["plain"] = {"quantize_ms": time_ms(lambda: h.quantize_qkv(q, k, v, s, inv, fmt, out=z), n=20),
+                            "attn_ms": time_ms(lambda: h.attn_fwd(z, scale, w.causal, h.PREORDER, w.block_n, out=o),
+                                               n=20)}
+            rec["plain"]["deviation"] = deviation_by_rows(o[0, heads], ex, w.N)
+            h.quantize_qkv(q, k, v, s, inv, fmt, out=z, q_mu=mu)
+            bias = h.q_mean_bias(z, mu)
+            rec["q_mean"] = {
+                "quantize_ms": time_ms(lambda: h.quantize_qkv(q, k, v, s, inv, fmt, out=z, q_mu=mu), n=20),
+                "bias_ms": time_ms(lambda: h.q_mean_bias(z, mu), n=20),
+                "attn_ms": time_ms(lambda: h.attn_fwd(z, scale, w.causal, h.PREORDER, w.block_n, out=o,
+                                                      qk_bias=bias), n=20)}
+            rec["q_mean"]["deviation"] = deviation_by_rows(o[0, heads], ex, w.N)
+            out.append(rec)
+            del z, o, bias
+        del q, k, v, ex
+        torch.cuda.empty_cache()
+    return out
+
+
 def traffic_record(kernel, workload, fmt, block_n, launch_path="fused"):
     """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
     one ncu capture, from profiles/traffic.json, if the kernel source still has
@@ -828,6 +867,10 @@ def main():
     torch.cuda.empty_cache()
     if rank == 0 and not args.no_configs:
         line["configs"] = measure_all_configs(args, pk, w.name)
+        try:
+            line["q_mean"] = q_mean_comparison()
+        except Exception as e:  # measurement only
+            line["q_mean"] = {"error": str(e)[:200]}
     if not args.no_decode:
         try:
             decode = run_decode(args)
