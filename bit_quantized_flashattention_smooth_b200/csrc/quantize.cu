@@ -81,7 +81,7 @@ __device__ __forceinline__ uint32_t quant_part(const float (&v)[8], uint32_t& pa
 // 32, and a CTA's rows on a multiple of ROWS), so every per-group address is
 // the lane's first one plus a constant: the scale byte moves by RPI * 16
 // bytes per group, the codes by RPI * D/2, the input by RPI * D values.
-template <int FMT, typename T, int D>
+template <int FMT, typename T, int D, bool QM>
 __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H, int G, int N, int Np,
                                                   const float* __restrict__ scale, const float* __restrict__ mu,
                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
@@ -112,15 +112,10 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
     const float4 a = s4[0], b = s4[1];
     sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w; sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
   }
-  // Q-Mean auxiliary: the head's calibration mean, subtracted after the
-  // smoothing multiply from real rows (negated here: x - mu = x + (-mu) exactly)
-  float nmu[8];
-  if (mu != nullptr) {
-    const float4* m4 = reinterpret_cast<const float4*>(mu + static_cast<int64_t>(bh % H) * D + ch * 8);
-    const float4 a = m4[0], b = m4[1];
-    nmu[0] = -a.x; nmu[1] = -a.y; nmu[2] = -a.z; nmu[3] = -a.w; nmu[4] = -b.x; nmu[5] = -b.y; nmu[6] = -b.z;
-    nmu[7] = -b.w;
-  }
+  // Q-Mean auxiliary: the head's calibration mean of this lane's 8 channels,
+  // subtracted after the smoothing multiply from real rows (re-read per row
+  // group from L1 rather than held in registers across the loop)
+  const float4* mu4 = QM ? reinterpret_cast<const float4*>(mu + static_cast<int64_t>(bh % H) * D + ch * 8) : nullptr;
   uint8_t* cdst = codes + (static_cast<int64_t>(bh) * Np + t0) * (D / 2) + ch * 4;
   uint8_t* sdst = sf + static_cast<int64_t>(bh) * sf_head_bytes + sf_word_offset(t0, blk / 4, WPR) + blk % 4;
 #pragma unroll
@@ -143,7 +138,10 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
         v[i + 1] = p2.y;
       }
     }
-    if (mu != nullptr && u * RPI < nvalid) {
+    if (QM && u * RPI < nvalid) {
+      // x - mu = x + (-mu) exactly: one packed add per pair
+      const float4 a = mu4[0], b = mu4[1];
+      const float nmu[8] = {-a.x, -a.y, -a.z, -a.w, -b.x, -b.y, -b.z, -b.w};
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
         const float2 d2 = fadd2(make_float2(v[i], v[i + 1]), make_float2(nmu[i], nmu[i + 1]));
@@ -283,7 +281,9 @@ struct QuantArgs {
   int nq_ctas, nk_ctas, nv_ctas;
 };
 
-template <int FMT, typename T, int D>
+// QM: the Q rows subtract the Q-Mean auxiliary (its own instantiation: the
+// plain quantizer carries none of it)
+template <int FMT, typename T, int D, bool QM>
 __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a) {
   __shared__ float inv_tab[128];
   if (FMT == HIFA4_NVFP4 && threadIdx.x < 128)
@@ -296,11 +296,11 @@ __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a)
     if (task < a.v_tasks)
       quantize_v_cols<FMT, T>(static_cast<const T*>(a.v), a.N, a.Np, a.d, a.vc, a.vs, a.sf_v_head, task, inv_tab);
   } else if (bid < a.nq_ctas) {
-    quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.s, a.q_mu, a.qc,
-                                 a.qs, a.sf_qk_head, bid, inv_tab);
+    quantize_rows_lpb<FMT, T, D, QM>(static_cast<const T*>(a.q), a.Hq, a.Hq / a.Hkv, a.N, a.Np, a.s, a.q_mu, a.qc,
+                                     a.qs, a.sf_qk_head, bid, inv_tab);
   } else if (bid < a.nq_ctas + a.nk_ctas) {
-    quantize_rows_lpb<FMT, T, D>(static_cast<const T*>(a.k), a.Hkv, 1, a.N, a.Np, a.inv_s, nullptr, a.kc, a.ks,
-                                 a.sf_qk_head, bid - a.nq_ctas, inv_tab);
+    quantize_rows_lpb<FMT, T, D, false>(static_cast<const T*>(a.k), a.Hkv, 1, a.N, a.Np, a.inv_s, nullptr, a.kc,
+                                        a.ks, a.sf_qk_head, bid - a.nq_ctas, inv_tab);
   }
 }
 
@@ -445,8 +445,14 @@ __global__ void q_mean_bias_kernel(const uint8_t* __restrict__ kc, const uint8_t
 template <typename T, int D>
 static void launch_quant_d(const QuantArgs& a, int fmt, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(a.nq_ctas + a.nk_ctas + a.nv_ctas);
-  if (fmt == HIFA4_NVFP4) quantize_qkv_kernel<HIFA4_NVFP4, T, D><<<grid, 256, 0, st>>>(a);
-  else quantize_qkv_kernel<HIFA4_MXFP4, T, D><<<grid, 256, 0, st>>>(a);
+  const bool qm = a.q_mu != nullptr;
+  if (fmt == HIFA4_NVFP4) {
+    if (qm) quantize_qkv_kernel<HIFA4_NVFP4, T, D, true><<<grid, 256, 0, st>>>(a);
+    else quantize_qkv_kernel<HIFA4_NVFP4, T, D, false><<<grid, 256, 0, st>>>(a);
+  } else {
+    if (qm) quantize_qkv_kernel<HIFA4_MXFP4, T, D, true><<<grid, 256, 0, st>>>(a);
+    else quantize_qkv_kernel<HIFA4_MXFP4, T, D, false><<<grid, 256, 0, st>>>(a);
+  }
 }
 template <typename T>
 static void launch_quant(const QuantArgs& a, int fmt, cudaStream_t st) {
