@@ -399,46 +399,52 @@ __global__ void calib_q_mean_kernel(const T* __restrict__ q, int B, int Hq, int 
 // The rank-one score term of the Q-Mean auxiliary: bias[b][hq][key] =
 // mu[hq] . K-hat[b][h(hq)][key] for every key of the padded rows (padding
 // keys have zero codes: bias 0), accumulated in fp64 (each product of an fp32
-// mu and an exact K-hat element is exact there) and rounded once to fp32.  One
-// thread per (b, kv head, key) decodes its K-hat row once (E2M1 x block
-// scale, exact in fp32) and serves the G query heads of the group.
-template <int FMT>
-__global__ void q_mean_bias_kernel(const uint8_t* __restrict__ kc, const uint8_t* __restrict__ ks,
-                                   const float* __restrict__ mu, int Hq, int Hkv, int Np, int d,
-                                   int64_t sf_head_bytes, float* __restrict__ bias) {
+// mu and an exact K-hat element is exact there; four interleaved partial sums)
+// and rounded once to fp32.  One thread per (b, q head, key), block by block:
+// the block's scale byte of the tiled layout, its codes as 32-bit words,
+// decoded in registers (E2M1 x block scale, exact in fp32); mu is staged in
+// shared memory already widened to fp64.
+template <int FMT, int D>
+__global__ void __launch_bounds__(128) q_mean_bias_kernel(const uint8_t* __restrict__ kc,
+                                                          const uint8_t* __restrict__ ks,
+                                                          const float* __restrict__ mu, int Hq, int Hkv, int Np,
+                                                          int64_t sf_head_bytes, float* __restrict__ bias) {
   constexpr int BETA = FMT == HIFA4_NVFP4 ? 16 : 32;
-  extern __shared__ float mu_sh[];                 // [G][d] of this kv head
-  const int G = Hq / Hkv;
-  const int bh = blockIdx.y;                       // b * Hkv + kv head
-  const int kvh = bh % Hkv, b = bh / Hkv;
-  for (int i = threadIdx.x; i < G * d; i += blockDim.x) mu_sh[i] = mu[(kvh * G) * d + i];
+  constexpr int NB = D / BETA;                     // blocks per row
+  constexpr int NKC = (NB + 3) / 4;                // scale words per row
+  __shared__ double mu_sh[D];
+  const int bhq = blockIdx.y;                      // b * Hq + q head
+  const int hq = bhq % Hq, b = bhq / Hq;
+  const int bh = b * Hkv + hq / (Hq / Hkv);        // its kv head's K-hat
+  for (int i = threadIdx.x; i < D; i += blockDim.x) mu_sh[i] = static_cast<double>(mu[hq * D + i]);
   __syncthreads();
   const int key = blockIdx.x * blockDim.x + threadIdx.x;
   if (key >= Np) return;
-  const uint8_t* row = kc + (static_cast<int64_t>(bh) * Np + key) * (d / 2);
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(kc + (static_cast<int64_t>(bh) * Np + key) * (D / 2));
   const uint8_t* sfh = ks + static_cast<int64_t>(bh) * sf_head_bytes;
-  const int nkc = (d / BETA + 3) / 4;
-  double acc[8];
-#pragma unroll
-  for (int g = 0; g < 8; ++g) acc[g] = 0.0;
-  for (int c0 = 0; c0 < d; c0 += BETA) {
-    const int blk = c0 / BETA;
-    const uint32_t sc = sfh[sf_word_offset(key, blk / 4, nkc) + blk % 4];
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 1
+  for (int blk = 0; blk < NB; ++blk) {
+    const uint32_t sc = sfh[sf_word_offset(key, blk / 4, NKC) + blk % 4];
     // UE4M3 value, or 2^(sc - 127) (code 0 is 2^-127, a subnormal)
     const float scale = FMT == HIFA4_NVFP4 ? ue4m3_to_f32(sc) : __uint_as_float(sc == 0 ? 0x00400000u : sc << 23);
-    for (int c = c0; c < c0 + BETA; ++c) {
-      const uint32_t code = (row[c / 2] >> (4 * (c & 1))) & 15u;
-      // E2M1 magnitude: exponent field e, mantissa bit m: 0.5 m for e = 0,
-      // else 2^(e-1) (1 + m/2)
-      const uint32_t e = (code >> 1) & 3u, m = code & 1u;
-      const float mag = e == 0 ? 0.5f * static_cast<float>(m) : __uint_as_float(((e + 126u) << 23) | (m << 22));
-      const float kv = __fmul_rn((code & 8u) ? -mag : mag, scale);
-      for (int g = 0; g < G && g < 8; ++g)
-        acc[g] = __fma_rn(static_cast<double>(mu_sh[g * d + c]), static_cast<double>(kv), acc[g]);
+#pragma unroll
+    for (int wi = 0; wi < BETA / 8; ++wi) {
+      const uint32_t wd = row[blk * (BETA / 8) + wi];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const int c = blk * BETA + 8 * wi + n;
+        const uint32_t code = (wd >> (4 * n)) & 15u;
+        // E2M1 magnitude: exponent field e, mantissa bit m: 0.5 m for e = 0,
+        // else 2^(e-1) (1 + m/2)
+        const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+        const float mag = e == 0 ? 0.5f * static_cast<float>(m) : __uint_as_float(((e + 126u) << 23) | (m << 22));
+        const float kv = __fmul_rn((code & 8u) ? -mag : mag, scale);
+        acc[n & 3] = __fma_rn(mu_sh[c], static_cast<double>(kv), acc[n & 3]);
+      }
     }
   }
-  for (int g = 0; g < G && g < 8; ++g)
-    bias[(static_cast<int64_t>(b) * Hq + kvh * G + g) * Np + key] = static_cast<float>(acc[g]);
+  bias[static_cast<int64_t>(bhq) * Np + key] = static_cast<float>((acc[0] + acc[1]) + (acc[2] + acc[3]));
 }
 
 // ---------------------------------------------------------- host launchers ---
@@ -510,12 +516,22 @@ hifa4_status q_mean_bias_launch(const uint8_t* kc, const uint8_t* ks, const floa
                                 int d, int fmt, float* bias, cudaStream_t st) {
   const int Np = static_cast<int>(pad128(N));
   const int64_t sf_head = static_cast<int64_t>(hifa4_scale_bytes(N, d, static_cast<hifa4_format>(fmt)));
-  const dim3 grid(static_cast<unsigned>(Np / 128), static_cast<unsigned>(B * Hkv));
-  const size_t smem = static_cast<size_t>(Hq / Hkv) * d * sizeof(float);
-  if (fmt == HIFA4_NVFP4)
-    q_mean_bias_kernel<HIFA4_NVFP4><<<grid, 128, smem, st>>>(kc, ks, mu, Hq, Hkv, Np, d, sf_head, bias);
-  else
-    q_mean_bias_kernel<HIFA4_MXFP4><<<grid, 128, smem, st>>>(kc, ks, mu, Hq, Hkv, Np, d, sf_head, bias);
+  const dim3 grid(static_cast<unsigned>(Np / 128), static_cast<unsigned>(B * Hq));
+  auto go = [&](auto fmt_tag, auto d_tag) {
+    constexpr int F = decltype(fmt_tag)::value, DD = decltype(d_tag)::value;
+    q_mean_bias_kernel<F, DD><<<grid, 128, 0, st>>>(kc, ks, mu, Hq, Hkv, Np, sf_head, bias);
+  };
+  using NV = std::integral_constant<int, HIFA4_NVFP4>;
+  using MX = std::integral_constant<int, HIFA4_MXFP4>;
+  if (fmt == HIFA4_NVFP4) {
+    if (d == 64) go(NV{}, std::integral_constant<int, 64>{});
+    else if (d == 128) go(NV{}, std::integral_constant<int, 128>{});
+    else go(NV{}, std::integral_constant<int, 256>{});
+  } else {
+    if (d == 64) go(MX{}, std::integral_constant<int, 64>{});
+    else if (d == 128) go(MX{}, std::integral_constant<int, 128>{});
+    else go(MX{}, std::integral_constant<int, 256>{});
+  }
   return launch_status("q_mean_bias");
 }
 
