@@ -96,6 +96,41 @@ def test_host_validation_without_gpu(L):
     assert L.hifa4_status_string(2) == b"unsupported configuration"
 
 
+def test_q_mean_entry_points_validate_on_the_host(L):
+    """The Q-Mean auxiliary's four entry points refuse bad arguments before
+    any launch: null or misaligned pointers, d = 256 in the forward, more
+    than 8 query heads per kv head for the score terms, bad calibration
+    counts."""
+    nul = None
+    fake = ctypes.c_void_p(16)
+    bad = ctypes.c_void_p(24)
+    # calibration: n_cal outside (0, ld_tok], null output
+    st = L.hifa4_calibrate_q_mean(fake, 0, 1, 4, 2, 0, 64, 128, nul, fake, nul)
+    assert st == 1 and b"n_cal" in L.hifa4_last_error()
+    st = L.hifa4_calibrate_q_mean(fake, 0, 1, 4, 2, 32, 64, 128, nul, nul, nul)
+    assert st == 1
+    # quantize with the mean: q_mu required and aligned
+    st = L.hifa4_quantize_qkv_qmean(fake, fake, fake, 0, 1, 4, 2, 128, 128, nul, nul, nul, 0, fake, fake, fake,
+                                    fake, fake, fake, nul)
+    assert st == 1 and b"q_mu" in L.hifa4_last_error()
+    st = L.hifa4_quantize_qkv_qmean(fake, fake, fake, 0, 1, 4, 2, 128, 128, nul, nul, bad, 0, fake, fake, fake,
+                                    fake, fake, fake, nul)
+    assert st == 1 and b"q_mu" in L.hifa4_last_error()
+    # score terms: at most 8 query heads per kv head
+    st = L.hifa4_q_mean_bias(fake, fake, fake, 1, 16, 1, 128, 128, 0, fake, nul)
+    assert st == 2 and b"8 query heads" in L.hifa4_last_error()
+    # forward: d = 256 refused, terms required and aligned
+    st = L.hifa4_attn_fwd_qmean(fake, fake, fake, fake, fake, fake, fake, 1, 2, 2, 128, 256, 0, 0.1, 1, 0, 128,
+                                fake, 0, nul, ctypes.c_float(0.0), nul)
+    assert st == 2 and b"d=256" in L.hifa4_last_error()
+    st = L.hifa4_attn_fwd_qmean(fake, fake, fake, fake, fake, fake, bad, 1, 2, 2, 128, 128, 0, 0.1, 1, 0, 128,
+                                fake, 0, nul, ctypes.c_float(0.0), nul)
+    assert st == 1 and b"aligned" in L.hifa4_last_error()
+    st = L.hifa4_attn_fwd_qmean(fake, fake, fake, fake, fake, fake, nul, 1, 2, 2, 128, 128, 0, 0.1, 1, 0, 128,
+                                fake, 0, nul, ctypes.c_float(0.0), nul)
+    assert st == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import bit_quantized_flashattention_smooth_b200 as h
     monkeypatch.setattr(h, "LIB_PATH", str(tmp_path / "missing.so"))
