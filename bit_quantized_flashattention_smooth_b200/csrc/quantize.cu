@@ -103,9 +103,16 @@ __device__ __forceinline__ void quantize_rows_lpb(const T* __restrict__ x, int H
   // all U loads in flight at once, kept packed (4 registers each) until their
   // row group is quantized; rows past N are zeros
   uint4 raw[U];
+  if (chunk * R::ROWS + R::ROWS <= N) {
+    // every row of the CTA is real (all CTAs but the last of a head): plain
+    // loads, no per-group selects
 #pragma unroll
-  for (int u = 0; u < U; ++u)
-    raw[u] = u * RPI < nvalid ? *reinterpret_cast<const uint4*>(src + u * RPI * D) : make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < U; ++u) raw[u] = *reinterpret_cast<const uint4*>(src + u * RPI * D);
+  } else {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      raw[u] = u * RPI < nvalid ? *reinterpret_cast<const uint4*>(src + u * RPI * D) : make_uint4(0u, 0u, 0u, 0u);
+  }
   float sv[8];
   if (scale != nullptr) {
     const float4* s4 = reinterpret_cast<const float4*>(scale + kvh * D + ch * 8);
@@ -217,8 +224,14 @@ __device__ __forceinline__ void quantize_v_cols(const T* __restrict__ v, int N, 
   const int nkc = Np / (4 * BETA);               // scale chunks per 128-row group of V^T
   uint32_t w[kVTok];
   const uint32_t* src = reinterpret_cast<const uint32_t*>(v + (head * N + t0) * static_cast<int64_t>(d) + c);
+  if (t0 + kVTok <= N) {
+    // a chunk of real tokens (all but the last chunk of a head): plain loads
 #pragma unroll
-  for (int i = 0; i < kVTok; ++i) w[i] = (t0 + i < N) ? src[static_cast<int64_t>(i) * (d / 2)] : 0u;
+    for (int i = 0; i < kVTok; ++i) w[i] = src[static_cast<int64_t>(i) * (d / 2)];
+  } else {
+#pragma unroll
+    for (int i = 0; i < kVTok; ++i) w[i] = (t0 + i < N) ? src[static_cast<int64_t>(i) * (d / 2)] : 0u;
+  }
   uint32_t codes0[kVTok / 8], codes1[kVTok / 8];
   uint32_t scw0 = 0, scw1 = 0;
 #pragma unroll
