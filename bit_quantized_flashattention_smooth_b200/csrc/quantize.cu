@@ -294,13 +294,38 @@ struct QuantArgs {
   int nq_ctas, nk_ctas, nv_ctas;
 };
 
+// fl32(1 / UE4M3(c)) for c = 1..127 (0 for c = 0), the element multiplier of
+// a block with scale code c: IEEE division evaluated by the compiler, the
+// same correctly rounded quotient __fdiv_rn gives on the device, so the
+// kernel only copies it into shared memory.
+struct InvScaleTable {
+  float v[128];
+};
+constexpr float ue4m3_value(int c) {
+  // (1 + m/8) 2^(e-7) for e > 0, m 2^-9 for e = 0 (powers of two exact)
+  const int e = (c >> 3) & 15, m = c & 7;
+  float p = 1.0f;
+  if (e == 0) {
+    for (int i = 0; i < 9; ++i) p *= 0.5f;
+    return static_cast<float>(m) * p;
+  }
+  for (int i = 0; i < 7 - e; ++i) p *= 0.5f;
+  for (int i = 0; i < e - 7; ++i) p *= 2.0f;
+  return (1.0f + static_cast<float>(m) / 8.0f) * p;
+}
+constexpr InvScaleTable make_inv_scale_table() {
+  InvScaleTable t{};
+  for (int c = 1; c < 128; ++c) t.v[c] = 1.0f / ue4m3_value(c);
+  return t;
+}
+__device__ const InvScaleTable kInvScale = make_inv_scale_table();
+
 // QM: the Q rows subtract the Q-Mean auxiliary (its own instantiation: the
 // plain quantizer carries none of it)
 template <int FMT, typename T, int D, bool QM>
 __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QuantArgs a) {
   __shared__ float inv_tab[128];
-  if (FMT == HIFA4_NVFP4 && threadIdx.x < 128)
-    inv_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __fdiv_rn(1.0f, ue4m3_to_f32(threadIdx.x));
+  if (FMT == HIFA4_NVFP4 && threadIdx.x < 128) inv_tab[threadIdx.x] = kInvScale.v[threadIdx.x];
   __syncthreads();
   // V tiles first (the longest CTAs start early), then Q rows, then K rows
   const int bid = static_cast<int>(blockIdx.x) - a.nv_ctas;
