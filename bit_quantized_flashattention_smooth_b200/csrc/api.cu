@@ -222,6 +222,9 @@ hifa4_status hifa4_q_mean_bias(const uint8_t* k_codes, const uint8_t* k_scales, 
   HIFA4_REQUIRE(B > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && N > 0, HIFA4_ERR_INVALID_ARG,
                 "q_mean_bias: bad shape B=%d Hq=%d Hkv=%d N=%d", B, Hq, Hkv, N);
   HIFA4_REQUIRE(Hq / Hkv <= 8, HIFA4_ERR_UNSUPPORTED, "q_mean_bias: at most 8 query heads per kv head");
+  HIFA4_REQUIRE(static_cast<int64_t>(B) * Hq <= 65535, HIFA4_ERR_UNSUPPORTED,
+                "q_mean_bias: B*Hq=%lld exceeds 65535 (one grid row per batch and query head)",
+                static_cast<long long>(B) * Hq);
   HIFA4_REQUIRE(valid_d(d), HIFA4_ERR_UNSUPPORTED, "q_mean_bias: d=%d not in {64,128,256}", d);
   return q_mean_bias_launch(k_codes, k_scales, q_mu, B, Hq, Hkv, N, d, fmt, bias_out,
                             static_cast<cudaStream_t>(stream));

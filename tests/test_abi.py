@@ -119,6 +119,8 @@ def test_q_mean_entry_points_validate_on_the_host(L):
     # score terms: at most 8 query heads per kv head
     st = L.hifa4_q_mean_bias(fake, fake, fake, 1, 16, 1, 128, 128, 0, fake, nul)
     assert st == 2 and b"8 query heads" in L.hifa4_last_error()
+    st = L.hifa4_q_mean_bias(fake, fake, fake, 4096, 32, 8, 128, 128, 0, fake, nul)
+    assert st == 2 and b"65535" in L.hifa4_last_error()
     # forward: d = 256 refused, terms required and aligned
     st = L.hifa4_attn_fwd_qmean(fake, fake, fake, fake, fake, fake, fake, 1, 2, 2, 128, 256, 0, 0.1, 1, 0, 128,
                                 fake, 0, nul, ctypes.c_float(0.0), nul)
